@@ -1,0 +1,336 @@
+// RoLA forward — CPU oracle (test infrastructure, NOT part of the product).
+//
+// Only the test-suite, the smoke check and the benchmark's CPU-baseline leg may
+// load this library.  It shares no code, header, table or constant with the
+// CUDA library: every quantity below is recomputed here from the definition with
+// plain loops and no blocking, fusion or reordering -- in double precision, except
+// the block selection, which is taken in fp32 (item 2 below).
+//
+// Sources (web pages about SparkDiffusion / RoLA; cited by page title and section):
+//   [README]  "AlibabaResearch/SparkDiffusion" (GitHub README mirror):
+//             - inference section: topk is a keep ratio (0.1/0.05/0.03 = 90/95/97 % sparsity);
+//             - sparse-finetuning section: RoLA adds proj_q, proj_k, gate_proj, gate_bias;
+//             - citation block: "RoLA: Rotary-Positioned Low-Rank Linear Attention",
+//               "RoPeSLR: 3D RoPE-driven Sparse-LowRank Attention".
+//   [NEWS]    "SparkDiffusion ... SparkWan" news article, section "What's New":
+//             RoLA = a sparse branch over high-energy query-key blocks plus a light
+//             low-rank path that restores global context.
+//   [BLOG]    "SparkDiffusion: 265x Faster Video Generation on Consumer GPUs via Sparse
+//             Attention & Distillation", section "RoLA: Preserving Global Context at
+//             Extreme Sparsity": block-sparse branch keeps the high-energy interactions,
+//             a low-rank linear branch with rotary positions recovers the dropped context.
+//
+// The pages fix only that structure.  The concrete operator this oracle computes
+// (each reading is listed again in the design notes of the repository):
+//   1. 64-token blocks of the flattened (t,h,w) token order; the last block may be short.
+//   2. Block energy s_ij = mean(q over block i) . mean(k over block j), no scale.  The
+//      selection is an integer decision taken from floating point, so it is taken in
+//      the precision of the GPU kernels (fp32), in a stated order: token sums in token
+//      order, one division by the count, a fused multiply-add chain over channels.
+//   3. Each query block keeps k = clamp(ceil(topk*nb - 1e-9), 1, nb) key blocks with the
+//      largest s_ij; equal scores rank the lower key-block index first; the kept list is
+//      stored in ascending order.
+//   4. Sparse branch: exact softmax attention of every query token of block i over all
+//      valid key tokens of its kept blocks, logits (q.k)*scale, scale = 1/sqrt(d) by default.
+//   5. Linear branch over ALL N keys: u = phi(q Wq_h), f = phi(k Wk_h), phi(x) = elu(x)+1;
+//      R(p) rotates the r/2 adjacent pairs (2c, 2c+1) by theta_c = pos_axis(c)(p) *
+//      base^(-c'/P_axis); numerator = (R(p_n) u_n)^T sum_m R(p_m) f_m v_m^T,
+//      denominator = u_n^T sum_m f_m (unrotated), O_lin = numerator / denominator.
+//   6. out = O_sparse + g_h * O_lin.
+//
+// Build: g++ -O3 -fopenmp -shared -fPIC (no -march, no fast-math: no FMA contraction).
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+constexpr int kBlock = 64;  // tokens per block (reading 1)
+
+}  // namespace
+
+extern "C" {
+
+// Problem description as the oracle sees it.  Plain struct, own definition.
+struct rola_oracle_shape {
+  int B, H, N, d, r;
+  int grid_t, grid_h, grid_w;     // grid_t*grid_h*grid_w == N
+  int pairs_t, pairs_h, pairs_w;  // rotary pairs per axis, sum == r/2
+  double rope_base;               // frequency base (10000)
+  double scale;                   // softmax logit scale
+  double topk;                    // keep ratio in (0, 1]
+};
+
+int rola_oracle_num_blocks(int N) { return (N + kBlock - 1) / kBlock; }
+
+// Reading 3 / [README] inference section: topk is the fraction of key blocks kept.
+int rola_oracle_keep_count(int nb, double topk) {
+  double x = std::ceil(topk * (double)nb - 1e-9);
+  int k = (int)x;
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return k;
+}
+
+// Positions of the flattened (t, h, w) grid: token n = (t*grid_h + y)*grid_w + x.
+// pos is [N][3] = (t, y, x).
+void rola_oracle_positions(const rola_oracle_shape* s, double* pos) {
+  for (int n = 0; n < s->N; ++n) {
+    int x = n % s->grid_w;
+    int y = (n / s->grid_w) % s->grid_h;
+    int t = n / (s->grid_w * s->grid_h);
+    pos[3 * n + 0] = t;
+    pos[3 * n + 1] = y;
+    pos[3 * n + 2] = x;
+  }
+}
+
+// Mean of x over the valid tokens of each block (reading 2), in the precision the
+// selection decision is taken in (fp32): the tokens of the block are added one after
+// the other in token order into an fp32 sum, then the sum is divided by the count
+// (one IEEE fp32 division).  x: [B, N, H, d] (float values), xbar: [B, H, nb, d].
+void rola_oracle_pool(const rola_oracle_shape* s, const float* x, float* xbar) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d;
+  const int nb = rola_oracle_num_blocks(N);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int i = 0; i < nb; ++i) {
+        int n0 = i * kBlock, n1 = std::min(N, n0 + kBlock);
+        float* o = xbar + (((size_t)b * H + h) * nb + i) * d;
+        for (int c = 0; c < d; ++c) {
+          volatile float acc = 0.0f;  // volatile: one rounding per addition, in order
+          for (int n = n0; n < n1; ++n) acc = acc + x[(((size_t)b * N + n) * H + h) * d + c];
+          o[c] = acc / (float)(n1 - n0);
+        }
+      }
+}
+
+// Block energy s_ij = qbar_i . kbar_j (reading 2) in fp32: a chain of fused
+// multiply-adds over the channels in order 0..d-1, starting from 0.
+static float block_score(const float* qb, const float* kb, int d) {
+  float acc = 0.0f;
+  for (int c = 0; c < d; ++c) acc = std::fmaf(qb[c], kb[c], acc);
+  return acc;
+}
+
+// Top-k with lowest-index tie-break, ascending lists (reading 3).
+// col_idx: [B, H, nb, k].  kth: the k-th largest score of each row.  next: the
+// (k+1)-th largest (-inf when k == nb).  amax: max_j |s_ij|.  All per row [B, H, nb].
+void rola_oracle_select(const rola_oracle_shape* s, const float* qbar, const float* kbar,
+                        int32_t* col_idx, double* kth, double* next, double* amax) {
+  const int B = s->B, H = s->H, d = s->d;
+  const int nb = rola_oracle_num_blocks(s->N);
+  const int k = rola_oracle_keep_count(nb, s->topk);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      std::vector<float> sc(nb);
+      std::vector<int> order(nb);
+      const float* Qb = qbar + ((size_t)b * H + h) * nb * d;
+      const float* Kb = kbar + ((size_t)b * H + h) * nb * d;
+      for (int i = 0; i < nb; ++i) {
+        double m = 0.0;
+        for (int j = 0; j < nb; ++j) {
+          sc[j] = block_score(Qb + (size_t)i * d, Kb + (size_t)j * d, d);
+          m = std::max(m, std::fabs((double)sc[j]));
+        }
+        for (int j = 0; j < nb; ++j) order[j] = j;
+        std::sort(order.begin(), order.end(), [&](int a, int c) {
+          if (sc[a] != sc[c]) return sc[a] > sc[c];
+          return a < c;
+        });
+        size_t row = ((size_t)b * H + h) * nb + i;
+        kth[row] = sc[order[k - 1]];
+        next[row] = (k < nb) ? (double)sc[order[k]] : -std::numeric_limits<double>::infinity();
+        amax[row] = m;
+        std::vector<int> kept(order.begin(), order.begin() + k);
+        std::sort(kept.begin(), kept.end());
+        for (int t = 0; t < k; ++t) col_idx[row * k + t] = kept[t];
+      }
+    }
+}
+
+// phi(x) = elu(x) + 1 (alpha = 1): x + 1 for x > 0, exp(x) otherwise (reading 5).
+static double phi(double x) { return x > 0.0 ? x + 1.0 : std::exp(x); }
+
+// Axis and in-axis index of rotary pair c: pairs are ordered t, then h, then w.
+static void pair_axis(const rola_oracle_shape* s, int c, int* axis, int* cprime, int* count) {
+  if (c < s->pairs_t) {
+    *axis = 0; *cprime = c; *count = s->pairs_t;
+  } else if (c < s->pairs_t + s->pairs_h) {
+    *axis = 1; *cprime = c - s->pairs_t; *count = s->pairs_h;
+  } else {
+    *axis = 2; *cprime = c - s->pairs_t - s->pairs_h; *count = s->pairs_w;
+  }
+}
+
+// y = R(p) x for one position p (3 coordinates), x, y of length r.
+// Pair (2c, 2c+1) is turned counter-clockwise by theta_c.
+static void rotate(const rola_oracle_shape* s, const double* p, const double* x, double* y) {
+  for (int c = 0; c < s->r / 2; ++c) {
+    int axis, cp, cnt;
+    pair_axis(s, c, &axis, &cp, &cnt);
+    double theta = p[axis] * std::pow(s->rope_base, -(double)cp / (double)cnt);
+    double cs = std::cos(theta), sn = std::sin(theta);
+    y[2 * c] = cs * x[2 * c] - sn * x[2 * c + 1];
+    y[2 * c + 1] = sn * x[2 * c] + cs * x[2 * c + 1];
+  }
+}
+
+// phi(x_n W_h) for one token row x (length d), W: [H, d, r] (float values).
+static void feature(const rola_oracle_shape* s, const float* xrow, const float* W, int h,
+                    double* out) {
+  const int d = s->d, r = s->r;
+  for (int a = 0; a < r; ++a) {
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += (double)xrow[c] * (double)W[((size_t)h * d + c) * r + a];
+    out[a] = phi(acc);
+  }
+}
+
+// Linear-branch state over all N keys (reading 5):
+//   S_h = sum_m R(p_m) phi(k_m Wk_h) v_m^T   -> S: [B, H, r, d]
+//   z_h = sum_m phi(k_m Wk_h)                -> z: [B, H, r]
+// pos: [N][3] positions (any values; the grid helper gives the default ones).
+void rola_oracle_linear_state(const rola_oracle_shape* s, const float* k, const float* v,
+                              const float* Wk, const double* pos, double* S, double* z) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d, r = s->r;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      std::vector<double> f(r), fr(r);
+      double* Sh = S + ((size_t)b * H + h) * r * d;
+      double* zh = z + ((size_t)b * H + h) * r;
+      for (int a = 0; a < r * d; ++a) Sh[a] = 0.0;
+      for (int a = 0; a < r; ++a) zh[a] = 0.0;
+      for (int m = 0; m < N; ++m) {
+        const float* km = k + (((size_t)b * N + m) * H + h) * d;
+        const float* vm = v + (((size_t)b * N + m) * H + h) * d;
+        feature(s, km, Wk, h, f.data());
+        rotate(s, pos + 3 * (size_t)m, f.data(), fr.data());
+        for (int a = 0; a < r; ++a) {
+          zh[a] += f[a];
+          for (int c = 0; c < d; ++c) Sh[(size_t)a * d + c] += fr[a] * (double)vm[c];
+        }
+      }
+    }
+}
+
+// Output of the listed query blocks.  blocks: nrows triples (b, h, i).
+// For each listed block, rows [0, 64) of the three outputs (each [nrows][64][d]) hold
+//   sparse: O_sparse, lin: O_lin, out: O_sparse + g_h * O_lin
+// for the valid tokens of the block; rows past N are left at 0.
+void rola_oracle_attend_blocks(const rola_oracle_shape* s, const float* q, const float* k,
+                               const float* v, const float* Wq, const double* g,
+                               const int32_t* col_idx, const double* S, const double* z,
+                               const double* pos, int nrows, const int32_t* blocks,
+                               double* sparse, double* lin, double* out) {
+  const int H = s->H, N = s->N, d = s->d, r = s->r;
+  const int nb = rola_oracle_num_blocks(N);
+  const int kk = rola_oracle_keep_count(nb, s->topk);
+#pragma omp parallel for schedule(dynamic)
+  for (int t = 0; t < nrows; ++t) {
+    const int b = blocks[3 * t], h = blocks[3 * t + 1], i = blocks[3 * t + 2];
+    const int32_t* L = col_idx + (((size_t)b * H + h) * nb + i) * kk;
+    const double* Sh = S + ((size_t)b * H + h) * r * d;
+    const double* zh = z + ((size_t)b * H + h) * r;
+    std::vector<int> keys;
+    for (int a = 0; a < kk; ++a)
+      for (int m = L[a] * kBlock; m < std::min(N, (L[a] + 1) * kBlock); ++m) keys.push_back(m);
+    std::vector<double> logit(keys.size()), u(r), ur(r);
+    double* os = sparse + (size_t)t * kBlock * d;
+    double* ol = lin + (size_t)t * kBlock * d;
+    double* oo = out + (size_t)t * kBlock * d;
+    std::memset(os, 0, sizeof(double) * kBlock * d);
+    std::memset(ol, 0, sizeof(double) * kBlock * d);
+    std::memset(oo, 0, sizeof(double) * kBlock * d);
+    for (int n = i * kBlock; n < std::min(N, (i + 1) * kBlock); ++n) {
+      const int row = n - i * kBlock;
+      const float* qn = q + (((size_t)b * N + n) * H + h) * d;
+      // Sparse branch: exact softmax over the kept keys (reading 4).
+      double mx = -std::numeric_limits<double>::infinity();
+      for (size_t a = 0; a < keys.size(); ++a) {
+        const float* km = k + (((size_t)b * N + keys[a]) * H + h) * d;
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += (double)qn[c] * (double)km[c];
+        logit[a] = acc * s->scale;
+        mx = std::max(mx, logit[a]);
+      }
+      double den = 0.0;
+      for (size_t a = 0; a < keys.size(); ++a) {
+        logit[a] = std::exp(logit[a] - mx);
+        den += logit[a];
+      }
+      for (size_t a = 0; a < keys.size(); ++a) {
+        const float* vm = v + (((size_t)b * N + keys[a]) * H + h) * d;
+        double w = logit[a] / den;
+        for (int c = 0; c < d; ++c) os[(size_t)row * d + c] += w * (double)vm[c];
+      }
+      // Linear branch (reading 5).
+      feature(s, qn, Wq, h, u.data());
+      rotate(s, pos + 3 * (size_t)n, u.data(), ur.data());
+      double lden = 0.0;
+      for (int a = 0; a < r; ++a) lden += u[a] * zh[a];
+      for (int c = 0; c < d; ++c) {
+        double num = 0.0;
+        for (int a = 0; a < r; ++a) num += ur[a] * Sh[(size_t)a * d + c];
+        ol[(size_t)row * d + c] = num / lden;
+      }
+      // Combination (reading 6).
+      for (int c = 0; c < d; ++c)
+        oo[(size_t)row * d + c] = os[(size_t)row * d + c] + g[h] * ol[(size_t)row * d + c];
+    }
+  }
+}
+
+// Whole forward pass: out [B, N, H, d] (double) and col_idx [B, H, nb, k].
+void rola_oracle_forward(const rola_oracle_shape* s, const float* q, const float* k,
+                         const float* v, const float* Wq, const float* Wk, const double* g,
+                         double* out, int32_t* col_idx) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d, r = s->r;
+  const int nb = rola_oracle_num_blocks(N);
+  std::vector<float> qbar((size_t)B * H * nb * d), kbar((size_t)B * H * nb * d);
+  std::vector<double> kth((size_t)B * H * nb), nxt((size_t)B * H * nb), amax((size_t)B * H * nb);
+  std::vector<double> pos((size_t)N * 3), S((size_t)B * H * r * d), z((size_t)B * H * r);
+  rola_oracle_pool(s, q, qbar.data());
+  rola_oracle_pool(s, k, kbar.data());
+  rola_oracle_select(s, qbar.data(), kbar.data(), col_idx, kth.data(), nxt.data(), amax.data());
+  rola_oracle_positions(s, pos.data());
+  rola_oracle_linear_state(s, k, v, Wk, pos.data(), S.data(), z.data());
+  std::vector<int32_t> blocks;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int i = 0; i < nb; ++i) {
+        blocks.push_back(b); blocks.push_back(h); blocks.push_back(i);
+      }
+  const int nrows = B * H * nb;
+  std::vector<double> os((size_t)nrows * kBlock * d), ol((size_t)nrows * kBlock * d),
+      oo((size_t)nrows * kBlock * d);
+  rola_oracle_attend_blocks(s, q, k, v, Wq, g, col_idx, S.data(), z.data(), pos.data(), nrows,
+                            blocks.data(), os.data(), ol.data(), oo.data());
+  for (int t = 0; t < nrows; ++t) {
+    const int b = blocks[3 * t], h = blocks[3 * t + 1], i = blocks[3 * t + 2];
+    for (int n = i * kBlock; n < std::min(N, (i + 1) * kBlock); ++n)
+      for (int c = 0; c < d; ++c)
+        out[(((size_t)b * N + n) * H + h) * d + c] =
+            oo[((size_t)t * kBlock + (n - i * kBlock)) * d + c];
+  }
+}
+
+int rola_oracle_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+}  // extern "C"
