@@ -1,0 +1,329 @@
+"""Benchmark of the RoLA attention forward on B200.
+
+One step = one whole forward pass (block pooling + top-k selection, linear state,
+sparse attention with the fused linear epilogue) over the Wan2.1-14B-720P-shaped
+workload (B=1, H=40, N=75600 = 21x45x80, d=128, r=32, topk=0.03, bf16) with the
+inputs resident in HBM.  The metric is kept-block TFLOP/s: the algorithmic FLOPs of
+the sparse branch, 4*d*c_i*c_j summed over every kept (query block i, key block j)
+pair (c = valid tokens of a block), divided by the step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rola|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent forward of the
+same workload (different seed), no collective on the data path ("scaling": "weak");
+the time is the max over ranks.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "RoLA fwd kept-block TFLOP/s at Wan2.1-14B-720P shape, 1xB200"
+UNIT = "TFLOP/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kept_block_flops(col: torch.Tensor, N: int, d: int) -> int:
+    """4*d*c_i*c_j over every kept pair; col is [B, H, nb, k] int32 on the device."""
+    B, H, nb, k = col.shape
+    c = torch.full((nb,), 64, dtype=torch.int64, device=col.device)
+    c[-1] = N - 64 * (nb - 1)
+    kept = c[col.long()].sum(-1)                 # [B, H, nb] sum_j c_j
+    return int((kept * c.view(1, 1, nb)).sum().item()) * 4 * d
+
+
+def linear_epilogue_flops(w) -> int:
+    """Query-side linear branch inside the attention kernel: u = q Wq and num = (R u) S."""
+    return 4 * w.B * w.H * w.N * w.d * w.r
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def oracle_sample(w, seconds_hint=20.0, heads=1, seed=0):
+    """Times the oracle as it stands on a bounded sample of workload ``w``: ``heads`` heads
+    with their full pooling, selection and linear state, attention on a seeded set of
+    query blocks; the time is extrapolated to the full head."""
+    import numpy as np
+    import oracle as O
+    sub = synth.custom(w.name + "_sample", B=w.B, H=heads, N=w.N, d=w.d, r=w.r, topk=w.topk,
+                       grid=w.grid, dtype=w.dtype, dist=w.dist)
+    inp = synth.make_inputs(sub, seed=seed, device="cpu")
+    h = {k: v.float().numpy() for k, v in inp.items()}
+    s = O.make_shape(sub.B, sub.H, sub.N, sub.d, sub.r, sub.topk, grid=sub.grid)
+    t0 = time.perf_counter()
+    qbar, kbar = O.pool(s, h["q"]), O.pool(s, h["k"])
+    col, *_ = O.select(s, qbar, kbar)
+    S, z = O.linear_state(s, h["k"], h["v"], h["Wk"])
+    t_pre = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    nblk = max(8, min(w.nb, int(8 * O.threads())))
+    idx = sorted(set(rng.choice(w.nb, size=nblk, replace=False).tolist()))
+    blocks = np.array([(0, hh, i) for hh in range(heads) for i in idx], dtype=np.int32)
+    t1 = time.perf_counter()
+    O.attend_blocks(s, h["q"], h["k"], h["v"], h["Wq"], h["g"], col, S, z, blocks)
+    t_att = time.perf_counter() - t1
+    t_head = t_pre + t_att * (w.nb / len(idx))
+    c = np.full(w.nb, 64, dtype=np.int64)
+    c[-1] = w.N - 64 * (w.nb - 1)
+    flops = 4 * w.d * int((c[col[0]].sum(-1) * c[None, :]).sum())   # all heads of the sample
+    return {"value": flops / t_head / 1e12, "seconds": t_pre + t_att, "cores": O.threads(),
+            "sample": (f"{heads} of {w.H} heads: full pooling, block selection and linear state; "
+                       f"sparse+linear attention on {len(idx)} of {w.nb} query blocks, "
+                       f"time extrapolated to the whole head(s)")}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="wan21_14b_720p")
+    ap.add_argument("--impl", default="rola", choices=["rola", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = dist_env()
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        samp = None
+        for it in range(args.warmup + args.steps):
+            r = oracle_sample(w, seed=it)
+            if it >= args.warmup:
+                vals.append(r["value"])
+                samp = r
+        v = statistics.median(vals)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N,
+                                                "d": w.d, "r": w.r, "topk": w.topk},
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": samp["cores"], "kind": "oracle",
+                                 "sample": samp["sample"]},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import sparse_rank_attention_b200 as rola
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rola.load()
+    inp = synth.make_inputs(w, seed=rank, device=dev)
+    plan = rola.Plan.for_workload(w, device=dev)
+    out = torch.empty_like(inp["q"])
+    q, k, v, Wq, Wk, g = (inp[x] for x in ("q", "k", "v", "Wq", "Wk", "g"))
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        plan.select_blocks(q, k)
+        if evs:
+            evs[1].record(stream)
+        plan.linear_state(k, v, Wk)
+        if evs:
+            evs[2].record(stream)
+        plan.attend(q, k, v, Wq, g, out)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert plan.poll_status() == 0
+    flops = kept_block_flops(plan.block_lists(), w.N, w.d)
+    att_flops = flops + linear_epilogue_flops(w)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = t0.elapsed_time(t1)
+    ms_total_max = max_over_ranks(ms_total, ws)
+    ms_step = ms_total_max / args.steps
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    assert plan.poll_status() == 0
+    value = ws * flops / (ms_step * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    att_ms = stage_ms[2]
+    achieved = att_flops / (att_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": "attend (sparse branch + fused linear epilogue)",
+            "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)"}
+    pool_bytes = 2 * w.B * w.N * w.H * w.d * 2
+    stages = {"select_blocks_ms": stage_ms[0], "linear_state_ms": stage_ms[1], "attend_ms": stage_ms[2],
+              "select_blocks_pool_read_GBs": pool_bytes / (stage_ms[0] * 1e-3) / 1e9}
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        hWq, hWk, hg = (x.cpu().pin_memory() for x in (Wq, Wk, g))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dWq, dWk, dg = torch.empty_like(Wq), torch.empty_like(Wk), torch.empty_like(g)
+        e_steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (dWq, hWq), (dWk, hWk), (dg, hg)):
+                dst.copy_(src, non_blocking=True)
+            plan.forward(dq, dk, dv, dWq, dWk, dg, out)
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b), ws) / e_steps
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hWq, hWk, hg))
+        e2e = {"value": ws * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(w)
+        cpu = {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+               "sample": r["sample"], "seconds": r["seconds"]}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype != "fp8" else "fp8",
+                "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "grid": list(w.grid),
+                           "d": w.d, "r": w.r, "topk": w.topk, "kept_blocks_per_row": plan.k,
+                           "blocks": plan.nb, "kept_block_tflop": flops / 1e12,
+                           "l2": "inputs (3 x 774 MB) larger than L2 (126 MB); no flush",
+                           "parallelism": f"replicas x{ws} (independent forward per GPU)"},
+                "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 5 * args.steps, "clocks": clk.summary()}
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

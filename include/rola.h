@@ -1,0 +1,161 @@
+/*
+ * rola.h — C ABI of the RoLA attention forward library for NVIDIA B200 (sm_100a).
+ *
+ * RoLA ("Rotary-Positioned Low-Rank Linear Attention", the sparse attention module of
+ * SparkDiffusion) has two branches:
+ *   - a block-sparse softmax branch that keeps, for every 64-token query block, the
+ *     top-k fraction of key blocks by block energy;
+ *   - a rank-r linear-attention branch with rotary (3D) positions over all keys, which
+ *     restores the global context the sparse branch drops.
+ * Sources: web page "SparkDiffusion: 265x Faster Video Generation on Consumer GPUs via
+ * Sparse Attention & Distillation", section "RoLA: Preserving Global Context at Extreme
+ * Sparsity"; news article on SparkDiffusion / SparkWan, section "What's New"; the
+ * "AlibabaResearch/SparkDiffusion" README (inference section: topk is a keep ratio;
+ * sparse-finetuning section: proj_q, proj_k, gate_proj, gate_bias; citation block:
+ * RoLA and "RoPeSLR: 3D RoPE-driven Sparse-LowRank Attention").
+ *
+ * The pages fix only that structure.  The operator computed here, for every batch b
+ * and head h (nb = ceil(N/64) blocks, the last one possibly short):
+ *   1. qbar_i, kbar_j: fp32 means over the valid tokens of each 64-token block
+ *      (token-order fp32 sums, one IEEE division by the count).
+ *   2. s_ij = qbar_i . kbar_j as an fp32 fused multiply-add chain over channels 0..d-1.
+ *      k = clamp(ceil(topk*nb - 1e-9), 1, nb) blocks with the largest s_ij are kept per
+ *      query block; equal scores keep the lower key-block index.  Lists are ascending.
+ *   3. O_sparse = softmax((q.k) * scale) v over the valid keys of the kept blocks.
+ *   4. u = phi(q Wq_h), f = phi(k Wk_h), phi(x) = elu(x) + 1.  R(p) turns rotary pair
+ *      (2c, 2c+1) by theta_c = pos_axis(c) * base^(-c'/P_axis) (pairs ordered t, h, w).
+ *      S_h = sum_m R(p_m) f_m v_m^T (r x d), z_h = sum_m f_m over all N keys;
+ *      O_lin = (R(p_n) u_n)^T S_h / (u_n^T z_h).
+ *   5. out = O_sparse + g_h * O_lin, rounded once to the output type.
+ *
+ * Layouts (all row-major, contiguous, device memory owned by the caller):
+ *   q, k, v, out : [B, N, H, d]  (fp32 for ROLA_F32, bf16 for ROLA_BF16 and ROLA_FP8_E4M3)
+ *   Wq, Wk       : [H, d, r]     (same element type as q)
+ *   g            : [H] fp32
+ *   workspace    : rola_workspace_size() bytes, 256-byte aligned, borrowed by the plan.
+ * Every pointer must be 16-byte aligned; out must not overlap any input.
+ *
+ * Errors: every call returns a rola_status; nothing is thrown across the ABI.  Invalid
+ * arguments are rejected on the host before any launch.  Calls are asynchronous on the
+ * given stream and never synchronise, except rola_poll_device_status.  Device-side
+ * waits are bounded: a wait that runs out records ROLA_ERR_DEVICE_TIMEOUT in a status
+ * word in the workspace, and the kernel returns; rola_poll_device_status reports it.
+ * The library never allocates device memory.
+ */
+#ifndef ROLA_H_
+#define ROLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ROLA_API __attribute__((visibility("default")))
+#else
+#define ROLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 means the legacy default stream. */
+typedef struct CUstream_st* rola_stream_t;
+
+typedef enum {
+  ROLA_OK = 0,
+  ROLA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or parameter            */
+  ROLA_ERR_UNSUPPORTED = 2,     /* valid in principle, not built (e.g. d not 64/128)   */
+  ROLA_ERR_WORKSPACE = 3,       /* workspace missing, misaligned or too small          */
+  ROLA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed                */
+  ROLA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out (see poll)       */
+  ROLA_ERR_DEVICE_BOUNDS = 6    /* a device-side index check failed (see poll)         */
+} rola_status;
+
+typedef enum {
+  ROLA_F32 = 0,       /* fp32 in/out, fp32 arithmetic (correctness configuration)       */
+  ROLA_BF16 = 1,      /* bf16 in/out, bf16 tensor-core products, fp32 accumulation      */
+  ROLA_FP8_E4M3 = 2   /* bf16 in/out; q, k, v quantised inside to e4m3 with one absmax */
+                      /* scale per (b, h, 64-token block); fp8 tensor-core products     */
+} rola_dtype;
+
+typedef struct {
+  int B, H, N, d, r;             /* batch, heads, tokens, head dim (64|128), rank (16|32)   */
+  int block;                     /* tokens per block; must be 64                            */
+  double topk;                   /* keep ratio in (0, 1]                                    */
+  int grid_t, grid_h, grid_w;    /* latent grid, product == N; (1, 1, N) for 1D positions   */
+  int rope_pairs_t, rope_pairs_h, rope_pairs_w; /* rotary pairs per axis, sum == r/2;      */
+                                 /* all 0 = default: 1D grid -> all on w; else h = w =      */
+                                 /* floor(r/6), t = r/2 - 2*floor(r/6)                      */
+  double rope_base;              /* rotary frequency base, > 1 (10000)                      */
+  float softmax_scale;           /* logit scale; 0 = 1/sqrt(d)                              */
+  rola_dtype dtype;
+} rola_params;
+
+typedef struct rola_plan_s* rola_plan_t;
+
+/* Fills *p with defaults: B=H=1, N=0, d=128, r=32, block 64, topk 0.1, grid (1,1,0),
+ * default rotary split, base 10000, scale 0 (1/sqrt(d)), ROLA_BF16. */
+ROLA_API rola_status rola_params_default(rola_params* p);
+
+/* Number of 64-token blocks nb and kept blocks per query block k for *p. */
+ROLA_API rola_status rola_keep_count(const rola_params* p, int* nb, int* k);
+
+/* Bytes of device workspace a plan for *p needs (pooled means, block lists, linear
+ * state, rotary table, fp8 copies, status word). */
+ROLA_API rola_status rola_workspace_size(const rola_params* p, size_t* bytes);
+
+/* Validates *p and binds it to `workspace` (device memory of at least
+ * rola_workspace_size bytes, 256-byte aligned).  Host-only: no launch, no allocation
+ * on the device.  The plan borrows the workspace until rola_plan_destroy. */
+ROLA_API rola_status rola_plan(const rola_params* p, void* workspace, size_t workspace_bytes,
+                      rola_plan_t* plan);
+
+ROLA_API void rola_plan_destroy(rola_plan_t plan);
+
+/* Steps 1-2 (block pooling, block scores, top-k): writes the block lists into the
+ * workspace.  In ROLA_FP8_E4M3 mode also writes the e4m3 copies of q and k with their
+ * per-block scales.  Reads q, k [B, N, H, d]. */
+ROLA_API rola_status rola_select_blocks(rola_plan_t plan, const void* q, const void* k,
+                               rola_stream_t stream);
+
+/* Step 4, key side: S_h, z_h over all N keys into the workspace (fixed-order, run-to-run
+ * deterministic reduction).  In ROLA_FP8_E4M3 mode also writes the e4m3 copy of v. */
+ROLA_API rola_status rola_linear_state(rola_plan_t plan, const void* k, const void* v, const void* Wk,
+                              rola_stream_t stream);
+
+/* Steps 3-5: sparse attention over the kept blocks with the linear branch and the
+ * combination fused into its epilogue; writes out [B, N, H, d] once.  Uses the block
+ * lists and the state the two calls above left in the workspace. */
+ROLA_API rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const void* v,
+                        const void* Wq, const float* g, void* out, rola_stream_t stream);
+
+/* The whole forward pass: rola_select_blocks, rola_linear_state, rola_attend. */
+ROLA_API rola_status rola_forward(rola_plan_t plan, const void* q, const void* k, const void* v,
+                         const void* Wq, const void* Wk, const float* g, void* out,
+                         rola_stream_t stream);
+
+/* Inspection (tests): copy, on `stream`, the block lists [B, H, nb, k] int32 (CSR column
+ * indices; row i of (b, h) starts at ((b*H + h)*nb + i)*k), the pooled means [B, H, nb, d]
+ * fp32, or the linear state S [B, H, r, d] and z [B, H, r] fp32 into caller buffers. */
+ROLA_API rola_status rola_get_block_lists(rola_plan_t plan, int32_t* col_idx, rola_stream_t stream);
+ROLA_API rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_stream_t stream);
+ROLA_API rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device status word: ROLA_OK, or
+ * ROLA_ERR_DEVICE_TIMEOUT / ROLA_ERR_DEVICE_BOUNDS if a kernel recorded one. */
+ROLA_API rola_status rola_poll_device_status(rola_plan_t plan, rola_stream_t stream);
+
+/* Debug hooks for tests of the failure path.  ROLA_DEBUG_STALL_WAIT makes the next
+ * rola_attend wait on a barrier that nothing arrives on, with a wait limit of
+ * `limit_us` microseconds; the kernel then records ROLA_ERR_DEVICE_TIMEOUT and returns.
+ * 0 clears all hooks. */
+#define ROLA_DEBUG_STALL_WAIT 1
+ROLA_API rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us);
+
+ROLA_API const char* rola_status_string(rola_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROLA_H_ */

@@ -1,0 +1,246 @@
+"""RoLA attention forward on NVIDIA B200 (sm_100a): thin Python binding of librola.so.
+
+RoLA ("Rotary-Positioned Low-Rank Linear Attention", the sparse attention module of
+SparkDiffusion) adds a rank-r linear-attention branch with 3D rotary positions to a
+block-sparse softmax branch that keeps the top-k fraction of 64-token key blocks per
+query block.  The operator, its layouts and error rules are documented in
+``include/rola.h``; every step runs in the library's CUDA kernels.  This module only
+marshals torch tensors (device memory, the current stream) into the C ABI.
+
+Layouts: q, k, v, out [B, N, H, d]; Wq, Wk [H, d, r]; g [H] fp32 — contiguous, on the
+same CUDA device.  fp32 tensors select the fp32 configuration, bf16 tensors the bf16 one;
+``dtype="fp8"`` takes bf16 tensors and quantises inside.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librola.so")
+
+ROLA_F32, ROLA_BF16, ROLA_FP8_E4M3 = 0, 1, 2
+DTYPES = {"f32": ROLA_F32, "bf16": ROLA_BF16, "fp8": ROLA_FP8_E4M3}
+ROLA_DEBUG_STALL_WAIT = 1
+
+STATUS = {0: "ROLA_OK", 1: "ROLA_ERR_INVALID_ARG", 2: "ROLA_ERR_UNSUPPORTED",
+          3: "ROLA_ERR_WORKSPACE", 4: "ROLA_ERR_CUDA", 5: "ROLA_ERR_DEVICE_TIMEOUT",
+          6: "ROLA_ERR_DEVICE_BOUNDS"}
+
+EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rola_plan",
+           "rola_plan_destroy", "rola_select_blocks", "rola_linear_state", "rola_attend",
+           "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
+           "rola_poll_device_status", "rola_set_debug", "rola_status_string")
+
+
+class RolaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({_lib_status_string(code)})")
+
+
+class RolaParams(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+        ("d", ctypes.c_int), ("r", ctypes.c_int), ("block", ctypes.c_int),
+        ("topk", ctypes.c_double),
+        ("grid_t", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+        ("rope_pairs_t", ctypes.c_int), ("rope_pairs_h", ctypes.c_int),
+        ("rope_pairs_w", ctypes.c_int),
+        ("rope_base", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load librola.so; raises if it has not been built (no fallback path exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m sparse_rank_attention_b200.build` "
+            "(or __graft_entry__.build()). There is no CPU or PyTorch fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    pp = ctypes.POINTER(RolaParams)
+    i32 = ctypes.c_int
+    for name, args in {
+        "rola_params_default": [pp],
+        "rola_keep_count": [pp, ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "rola_workspace_size": [pp, ctypes.POINTER(ctypes.c_size_t)],
+        "rola_plan": [pp, P, ctypes.c_size_t, ctypes.POINTER(P)],
+        "rola_select_blocks": [P, P, P, P],
+        "rola_linear_state": [P, P, P, P, P],
+        "rola_attend": [P, P, P, P, P, P, P, P],
+        "rola_forward": [P, P, P, P, P, P, P, P, P],
+        "rola_get_block_lists": [P, P, P],
+        "rola_get_pooled": [P, P, P, P],
+        "rola_get_linear_state": [P, P, P, P],
+        "rola_poll_device_status": [P, P],
+        "rola_set_debug": [P, i32, i32],
+    }.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = i32
+    lib.rola_plan_destroy.argtypes = [P]
+    lib.rola_plan_destroy.restype = None
+    lib.rola_status_string.argtypes = [i32]
+    lib.rola_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _lib_status_string(code: int) -> str:
+    try:
+        return load().rola_status_string(code).decode()
+    except Exception:  # noqa: BLE001 - message only
+        return "?"
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise RolaError(code, where)
+
+
+def make_params(B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
+                softmax_scale=0.0, dtype="bf16") -> RolaParams:
+    p = RolaParams()
+    load().rola_params_default(ctypes.byref(p))
+    grid = tuple(grid) if grid is not None else (1, 1, N)
+    p.B, p.H, p.N, p.d, p.r = B, H, N, d, r
+    p.topk = float(topk)
+    p.grid_t, p.grid_h, p.grid_w = grid
+    p.rope_pairs_t, p.rope_pairs_h, p.rope_pairs_w = pairs
+    p.rope_base = float(rope_base)
+    p.softmax_scale = float(softmax_scale)
+    p.dtype = DTYPES[dtype] if isinstance(dtype, str) else int(dtype)
+    return p
+
+
+def keep_count(params: RolaParams) -> tuple[int, int]:
+    nb, k = ctypes.c_int(), ctypes.c_int()
+    _check(load().rola_keep_count(ctypes.byref(params), ctypes.byref(nb), ctypes.byref(k)),
+           "rola_keep_count")
+    return nb.value, k.value
+
+
+def workspace_size(params: RolaParams) -> int:
+    n = ctypes.c_size_t()
+    _check(load().rola_workspace_size(ctypes.byref(params), ctypes.byref(n)), "rola_workspace_size")
+    return n.value
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Plan:
+    """A rola_plan bound to a workspace tensor allocated here with torch."""
+
+    def __init__(self, B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
+                 softmax_scale=0.0, dtype="bf16", device="cuda"):
+        self.params = make_params(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype)
+        self.dtype = dtype
+        self.nb, self.k = keep_count(self.params)
+        self.workspace_bytes = workspace_size(self.params)
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device)
+        h = ctypes.c_void_p()
+        _check(load().rola_plan(ctypes.byref(self.params), _ptr(self.workspace),
+                                self.workspace_bytes, ctypes.byref(h)), "rola_plan")
+        self._h = h
+
+    @classmethod
+    def for_workload(cls, w, device="cuda"):
+        return cls(w.B, w.H, w.N, w.d, w.r, w.topk, w.grid, w.pairs, dtype=w.dtype, device=device)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load().rola_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+    # ---- steps
+    def select_blocks(self, q, k, stream=None):
+        _check(load().rola_select_blocks(self._h, _ptr(q), _ptr(k), _stream(stream)),
+               "rola_select_blocks")
+
+    def linear_state(self, k, v, Wk, stream=None):
+        _check(load().rola_linear_state(self._h, _ptr(k), _ptr(v), _ptr(Wk), _stream(stream)),
+               "rola_linear_state")
+
+    def attend(self, q, k, v, Wq, g, out, stream=None):
+        _check(load().rola_attend(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(Wq), _ptr(g),
+                                  _ptr(out), _stream(stream)), "rola_attend")
+        return out
+
+    def forward(self, q, k, v, Wq, Wk, g, out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        _check(load().rola_forward(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(Wq), _ptr(Wk),
+                                   _ptr(g), _ptr(out), _stream(stream)), "rola_forward")
+        return out
+
+    # ---- inspection
+    def block_lists(self, stream=None) -> torch.Tensor:
+        p = self.params
+        t = torch.empty((p.B, p.H, self.nb, self.k), dtype=torch.int32, device=self.workspace.device)
+        _check(load().rola_get_block_lists(self._h, _ptr(t), _stream(stream)), "rola_get_block_lists")
+        return t
+
+    def pooled(self, stream=None):
+        p = self.params
+        qb = torch.empty((p.B, p.H, self.nb, p.d), dtype=torch.float32, device=self.workspace.device)
+        kb = torch.empty_like(qb)
+        _check(load().rola_get_pooled(self._h, _ptr(qb), _ptr(kb), _stream(stream)), "rola_get_pooled")
+        return qb, kb
+
+    def state(self, stream=None):
+        p = self.params
+        S = torch.empty((p.B, p.H, p.r, p.d), dtype=torch.float32, device=self.workspace.device)
+        z = torch.empty((p.B, p.H, p.r), dtype=torch.float32, device=self.workspace.device)
+        _check(load().rola_get_linear_state(self._h, _ptr(S), _ptr(z), _stream(stream)),
+               "rola_get_linear_state")
+        return S, z
+
+    def poll_status(self, stream=None) -> int:
+        """Synchronises the stream; returns the device status code (0 = ok), clearing it."""
+        return load().rola_poll_device_status(self._h, _stream(stream))
+
+    def set_debug(self, flags: int, limit_us: int = 0):
+        _check(load().rola_set_debug(self._h, flags, limit_us), "rola_set_debug")
+
+
+def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
+            softmax_scale=0.0, dtype=None, out=None):
+    """One-shot RoLA forward (builds a plan and workspace for this call)."""
+    B, N, H, d = q.shape
+    r = Wq.shape[-1]
+    if dtype is None:
+        dtype = "f32" if q.dtype == torch.float32 else "bf16"
+    plan = Plan(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype, q.device)
+    try:
+        return plan.forward(q, k, v, Wq, Wk, g, out)
+    finally:
+        torch.cuda.current_stream().synchronize()
+        plan.close()
+
+
+__all__ = ["Plan", "forward", "load", "make_params", "keep_count", "workspace_size", "RolaError",
+           "RolaParams", "EXPORTS", "LIB_PATH", "ROLA_DEBUG_STALL_WAIT"]

@@ -1,0 +1,321 @@
+// C ABI of the RoLA forward library: argument checks, workspace layout, launch order.
+// The operator, layouts, ownership and error rules are stated in include/rola.h.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "rola_internal.cuh"
+
+namespace {
+
+using rola::Dims;
+using rola::Workspace;
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxBlocks = 2800;  // scores of a row tile must fit shared memory
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Default rotary split: 1D grid -> every pair on w; else h = w = floor(P/3), t the rest.
+void default_pairs(const rola_params& p, int* pt, int* ph, int* pw) {
+  const int P = p.r / 2;
+  if (p.grid_t == 1 && p.grid_h == 1) {
+    *pt = 0; *ph = 0; *pw = P;
+  } else {
+    const int hw = P / 3;
+    *pt = P - 2 * hw; *ph = hw; *pw = hw;
+  }
+}
+
+int keep_count(int nb, double topk) {
+  double x = std::ceil(topk * (double)nb - 1e-9);
+  int k = (int)x;
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return k;
+}
+
+rola_status check_params(const rola_params* p) {
+  if (!p) return ROLA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1) return ROLA_ERR_INVALID_ARG;
+  if (p->block != rola::kBlock) return ROLA_ERR_UNSUPPORTED;
+  if (p->d != 64 && p->d != 128) return ROLA_ERR_UNSUPPORTED;
+  if (p->r != 16 && p->r != 32) return ROLA_ERR_UNSUPPORTED;
+  if (!(p->topk > 0.0 && p->topk <= 1.0)) return ROLA_ERR_INVALID_ARG;
+  if (p->grid_t < 1 || p->grid_h < 1 || p->grid_w < 1) return ROLA_ERR_INVALID_ARG;
+  if ((long long)p->grid_t * p->grid_h * p->grid_w != p->N) return ROLA_ERR_INVALID_ARG;
+  const int sp = p->rope_pairs_t + p->rope_pairs_h + p->rope_pairs_w;
+  if (p->rope_pairs_t < 0 || p->rope_pairs_h < 0 || p->rope_pairs_w < 0) return ROLA_ERR_INVALID_ARG;
+  if (sp != 0 && sp != p->r / 2) return ROLA_ERR_INVALID_ARG;
+  if (!(p->rope_base > 1.0) || !std::isfinite(p->rope_base)) return ROLA_ERR_INVALID_ARG;
+  if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return ROLA_ERR_INVALID_ARG;
+  if (p->dtype != ROLA_F32 && p->dtype != ROLA_BF16 && p->dtype != ROLA_FP8_E4M3)
+    return ROLA_ERR_INVALID_ARG;
+  if (p->dtype == ROLA_FP8_E4M3) return ROLA_ERR_UNSUPPORTED;
+  const int nb = (p->N + rola::kBlock - 1) / rola::kBlock;
+  if (nb > kMaxBlocks) return ROLA_ERR_UNSUPPORTED;
+  if ((long long)p->B * p->H * nb > (1ll << 31) / 64) return ROLA_ERR_UNSUPPORTED;
+  return ROLA_OK;
+}
+
+Dims make_dims(const rola_params& p) {
+  Dims dm{};
+  dm.B = p.B; dm.H = p.H; dm.N = p.N; dm.d = p.d; dm.r = p.r;
+  dm.nb = (p.N + rola::kBlock - 1) / rola::kBlock;
+  dm.k = keep_count(dm.nb, p.topk);
+  dm.gt = p.grid_t; dm.gh = p.grid_h; dm.gw = p.grid_w;
+  if (p.rope_pairs_t + p.rope_pairs_h + p.rope_pairs_w == 0) {
+    default_pairs(p, &dm.pt, &dm.ph, &dm.pw);
+  } else {
+    dm.pt = p.rope_pairs_t; dm.ph = p.rope_pairs_h; dm.pw = p.rope_pairs_w;
+  }
+  dm.rope_off_h = dm.gt * dm.pt;
+  dm.rope_off_w = dm.rope_off_h + dm.gh * dm.ph;
+  dm.nchunk = (p.N + rola::kStateChunk - 1) / rola::kStateChunk;
+  dm.scale = p.softmax_scale > 0.f ? p.softmax_scale : (float)(1.0 / std::sqrt((double)p.d));
+  dm.rope_base = p.rope_base;
+  return dm;
+}
+
+// Carves the workspace; with base == nullptr only the size is computed.
+size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* r = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return r;
+  };
+  const size_t BH = (size_t)dm.B * dm.H;
+  Workspace w{};
+  w.status = reinterpret_cast<int*>(take(kAlign));
+  w.rope = reinterpret_cast<float2*>(take(sizeof(float2) * (size_t)(dm.rope_off_w + dm.gw * dm.pw)));
+  w.qbar = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * dm.d));
+  w.kbar = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * dm.d));
+  w.col_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * dm.nb * dm.k));
+  w.S_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r * dm.d));
+  w.z_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r));
+  w.S = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r * dm.d));
+  w.z = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r));
+  w.S_bf = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
+  if (p.dtype == ROLA_FP8_E4M3) {
+    const size_t elems = (size_t)dm.B * dm.N * dm.H * dm.d;
+    w.q8 = reinterpret_cast<uint8_t*>(take(elems));
+    w.k8 = reinterpret_cast<uint8_t*>(take(elems));
+    w.v8 = reinterpret_cast<uint8_t*>(take(elems));
+    w.sq = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb));
+    w.sk = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb));
+    w.sv = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb));
+  }
+  if (ws) *ws = w;
+  return off;
+}
+
+rola_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA; }
+
+// Zeroes the device status word the first time a plan issues work.
+rola_status ensure_status_word(rola_plan_t plan, cudaStream_t st) {
+  if (plan->status_ready) return ROLA_OK;
+  cudaError_t e = cudaMemsetAsync(plan->ws.status, 0, kAlign, st);
+  if (e != cudaSuccess) return ROLA_ERR_CUDA;
+  plan->status_ready = true;
+  return ROLA_OK;
+}
+
+size_t elem_size(rola_dtype dt) { return dt == ROLA_F32 ? 4 : 2; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+rola_status rola_params_default(rola_params* p) {
+  if (!p) return ROLA_ERR_INVALID_ARG;
+  std::memset(p, 0, sizeof(*p));
+  p->B = 1; p->H = 1; p->N = 0; p->d = 128; p->r = 32;
+  p->block = rola::kBlock;
+  p->topk = 0.1;
+  p->grid_t = 1; p->grid_h = 1; p->grid_w = 0;
+  p->rope_base = 10000.0;
+  p->softmax_scale = 0.f;
+  p->dtype = ROLA_BF16;
+  return ROLA_OK;
+}
+
+rola_status rola_keep_count(const rola_params* p, int* nb, int* k) {
+  rola_status s = check_params(p);
+  if (s != ROLA_OK) return s;
+  if (!nb || !k) return ROLA_ERR_INVALID_ARG;
+  const Dims dm = make_dims(*p);
+  *nb = dm.nb;
+  *k = dm.k;
+  return ROLA_OK;
+}
+
+rola_status rola_workspace_size(const rola_params* p, size_t* bytes) {
+  rola_status s = check_params(p);
+  if (s != ROLA_OK) return s;
+  if (!bytes) return ROLA_ERR_INVALID_ARG;
+  *bytes = carve(*p, make_dims(*p), nullptr, nullptr);
+  return ROLA_OK;
+}
+
+rola_status rola_plan(const rola_params* p, void* workspace, size_t workspace_bytes,
+                      rola_plan_t* plan) {
+  rola_status s = check_params(p);
+  if (s != ROLA_OK) return s;
+  if (!plan) return ROLA_ERR_INVALID_ARG;
+  *plan = nullptr;
+  const Dims dm = make_dims(*p);
+  const size_t need = carve(*p, dm, nullptr, nullptr);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      workspace_bytes < need)
+    return ROLA_ERR_WORKSPACE;
+  rola_plan_s* pl = new (std::nothrow) rola_plan_s();
+  if (!pl) return ROLA_ERR_INVALID_ARG;
+  pl->p = *p;
+  pl->dm = dm;
+  carve(*p, dm, static_cast<char*>(workspace), &pl->ws);
+  pl->ws_base = workspace;
+  pl->ws_bytes = workspace_bytes;
+  *plan = pl;
+  return ROLA_OK;
+}
+
+void rola_plan_destroy(rola_plan_t plan) { delete plan; }
+
+rola_status rola_select_blocks(rola_plan_t plan, const void* q, const void* k,
+                               rola_stream_t stream) {
+  if (!plan || !q || !k || !aligned16(q) || !aligned16(k)) return ROLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rola_status s = ensure_status_word(plan, st);
+  if (s != ROLA_OK) return s;
+  cudaError_t e = rola::launch_pool(plan->dm, plan->p.dtype, q, k, plan->ws, st);
+  if (e != cudaSuccess) return ROLA_ERR_CUDA;
+  return cuda_status(rola::launch_select(plan->dm, plan->ws, st));
+}
+
+rola_status rola_linear_state(rola_plan_t plan, const void* k, const void* v, const void* Wk,
+                              rola_stream_t stream) {
+  if (!plan || !k || !v || !Wk || !aligned16(k) || !aligned16(v) || !aligned16(Wk))
+    return ROLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rola_status s = ensure_status_word(plan, st);
+  if (s != ROLA_OK) return s;
+  if (!plan->rope_ready) {
+    if (rola::launch_rope_table(plan->dm, plan->ws, st) != cudaSuccess) return ROLA_ERR_CUDA;
+    plan->rope_ready = true;
+  }
+  return cuda_status(rola::launch_linear_state(plan->dm, plan->p.dtype, k, v, Wk, plan->ws, st));
+}
+
+rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const void* v,
+                        const void* Wq, const float* g, void* out, rola_stream_t stream) {
+  if (!plan || !q || !k || !v || !Wq || !g || !out) return ROLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(Wq) || !aligned16(g) ||
+      !aligned16(out))
+    return ROLA_ERR_INVALID_ARG;
+  const rola_params& p = plan->p;
+  const size_t act = (size_t)p.B * p.N * p.H * p.d * elem_size(p.dtype);
+  if (overlaps(out, act, q, act) || overlaps(out, act, k, act) || overlaps(out, act, v, act))
+    return ROLA_ERR_INVALID_ARG;
+  if (!plan->rope_ready) return ROLA_ERR_INVALID_ARG;  // rola_linear_state must run first
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rola_status s = ensure_status_word(plan, st);
+  if (s != ROLA_OK) return s;
+  cudaError_t e;
+  if (p.dtype == ROLA_F32)
+    e = rola::launch_attend_f32(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
+  else
+    e = rola::launch_attend_bf16_warpmma(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
+  return cuda_status(e);
+}
+
+rola_status rola_forward(rola_plan_t plan, const void* q, const void* k, const void* v,
+                         const void* Wq, const void* Wk, const float* g, void* out,
+                         rola_stream_t stream) {
+  if (!plan || !q || !k || !v || !Wq || !Wk || !g || !out) return ROLA_ERR_INVALID_ARG;
+  const rola_params& p = plan->p;
+  const size_t act = (size_t)p.B * p.N * p.H * p.d * elem_size(p.dtype);
+  if (overlaps(out, act, q, act) || overlaps(out, act, k, act) || overlaps(out, act, v, act))
+    return ROLA_ERR_INVALID_ARG;
+  if (!aligned16(Wq) || !aligned16(Wk) || !aligned16(g) || !aligned16(out))
+    return ROLA_ERR_INVALID_ARG;
+  rola_status s = rola_select_blocks(plan, q, k, stream);
+  if (s != ROLA_OK) return s;
+  s = rola_linear_state(plan, k, v, Wk, stream);
+  if (s != ROLA_OK) return s;
+  return rola_attend(plan, q, k, v, Wq, g, out, stream);
+}
+
+rola_status rola_get_block_lists(rola_plan_t plan, int32_t* col_idx, rola_stream_t stream) {
+  if (!plan || !col_idx) return ROLA_ERR_INVALID_ARG;
+  const Dims& dm = plan->dm;
+  const size_t bytes = sizeof(int32_t) * (size_t)dm.B * dm.H * dm.nb * dm.k;
+  return cuda_status(cudaMemcpyAsync(col_idx, plan->ws.col_idx, bytes, cudaMemcpyDeviceToDevice,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_stream_t stream) {
+  if (!plan || !qbar || !kbar) return ROLA_ERR_INVALID_ARG;
+  const Dims& dm = plan->dm;
+  const size_t bytes = sizeof(float) * (size_t)dm.B * dm.H * dm.nb * dm.d;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(qbar, plan->ws.qbar, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  return cuda_status(cudaMemcpyAsync(kbar, plan->ws.kbar, bytes, cudaMemcpyDeviceToDevice, st));
+}
+
+rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream) {
+  if (!plan || !S || !z) return ROLA_ERR_INVALID_ARG;
+  const Dims& dm = plan->dm;
+  const size_t BH = (size_t)dm.B * dm.H;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(S, plan->ws.S, sizeof(float) * BH * dm.r * dm.d, cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  return cuda_status(
+      cudaMemcpyAsync(z, plan->ws.z, sizeof(float) * BH * dm.r, cudaMemcpyDeviceToDevice, st));
+}
+
+rola_status rola_poll_device_status(rola_plan_t plan, rola_stream_t stream) {
+  if (!plan) return ROLA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!plan->status_ready) return ROLA_OK;
+  int word = 0;
+  if (cudaMemcpyAsync(&word, plan->ws.status, sizeof(int), cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return ROLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ROLA_ERR_CUDA;
+  if (word == 0) return ROLA_OK;
+  if (cudaMemsetAsync(plan->ws.status, 0, sizeof(int), st) != cudaSuccess) return ROLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ROLA_ERR_CUDA;
+  return word == ROLA_ERR_DEVICE_TIMEOUT ? ROLA_ERR_DEVICE_TIMEOUT : ROLA_ERR_DEVICE_BOUNDS;
+}
+
+rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us) {
+  if (!plan || flags < 0 || limit_us < 0) return ROLA_ERR_INVALID_ARG;
+  plan->debug_flags = flags;
+  plan->debug_limit_us = limit_us;
+  return ROLA_OK;
+}
+
+const char* rola_status_string(rola_status s) {
+  switch (s) {
+    case ROLA_OK: return "ok";
+    case ROLA_ERR_INVALID_ARG: return "invalid argument";
+    case ROLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ROLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ROLA_ERR_CUDA: return "CUDA runtime error";
+    case ROLA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case ROLA_ERR_DEVICE_BOUNDS: return "a device-side index check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

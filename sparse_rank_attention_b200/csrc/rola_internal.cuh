@@ -1,0 +1,106 @@
+// Internal declarations of the RoLA forward library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "rola.h"
+
+namespace rola {
+
+constexpr int kBlock = 64;         // tokens per block
+constexpr int kStateChunk = 2048;  // tokens per linear-state partial sum
+
+// Device status word values (mirror rola_status codes).
+constexpr int kDevOk = 0;
+constexpr int kDevTimeout = ROLA_ERR_DEVICE_TIMEOUT;
+constexpr int kDevBounds = ROLA_ERR_DEVICE_BOUNDS;
+
+// Everything a kernel needs to know about the problem, passed by value.
+struct Dims {
+  int B, H, N, d, r;
+  int nb, k;                  // blocks, kept blocks per query block
+  int gt, gh, gw;             // latent grid
+  int pt, ph, pw;             // rotary pairs per axis
+  int rope_off_h, rope_off_w; // table offsets of the h and w axes (t starts at 0)
+  int nchunk;                 // linear-state partial sums per (b, h)
+  float scale;                // softmax logit scale
+  double rope_base;
+};
+
+// Device pointers carved out of the caller's workspace.
+struct Workspace {
+  int* status;        // [64] ints; status[0] = first recorded device error
+  float2* rope;       // (cos, sin) per (axis position, pair)
+  float* qbar;        // [B, H, nb, d]
+  float* kbar;        // [B, H, nb, d]
+  int32_t* col_idx;   // [B, H, nb, k]
+  float* S_part;      // [B, H, nchunk, r, d]
+  float* z_part;      // [B, H, nchunk, r]
+  float* S;           // [B, H, r, d]
+  float* z;           // [B, H, r]
+  __nv_bfloat16* S_bf;  // [B, H, r, d] bf16 copy (tensor-core operand of the epilogue)
+  uint8_t* q8;        // [B, N, H, d] e4m3 (fp8 mode)
+  uint8_t* k8;
+  uint8_t* v8;
+  float* sq;          // [B, H, nb] e4m3 scales (fp8 mode)
+  float* sk;
+  float* sv;
+};
+
+}  // namespace rola
+
+struct rola_plan_s {
+  rola_params p;
+  rola::Dims dm;
+  rola::Workspace ws;
+  void* ws_base;
+  size_t ws_bytes;
+  int debug_flags;
+  int debug_limit_us;
+  bool status_ready;  // status word zeroed on the device
+  bool rope_ready;    // rotary table written
+};
+
+namespace rola {
+
+// ---- launchers (each returns cudaGetLastError() of its launch) ----
+cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void* k,
+                        const Workspace& ws, cudaStream_t st);
+cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_rope_table(const Dims& dm, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_linear_state(const Dims& dm, rola_dtype dt, const void* k, const void* v,
+                                const void* Wk, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_attend_f32(const Dims& dm, const void* q, const void* k, const void* v,
+                              const void* Wq, const float* g, void* out, const Workspace& ws,
+                              cudaStream_t st);
+cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void* k,
+                                       const void* v, const void* Wq, const float* g, void* out,
+                                       const Workspace& ws, cudaStream_t st);
+size_t select_smem_bytes(const Dims& dm);
+
+// ---- device helpers ----
+__device__ __forceinline__ void record_status(int* status, int code) {
+  atomicCAS(status, kDevOk, code);
+}
+
+// Rotary cos/sin of pair c for token n.
+__device__ __forceinline__ float2 rope_cs(const Dims& dm, const float2* __restrict__ rope, int n,
+                                          int c) {
+  if (c < dm.pt) {
+    int t = n / (dm.gh * dm.gw);
+    return rope[t * dm.pt + c];
+  } else if (c < dm.pt + dm.ph) {
+    int y = (n / dm.gw) % dm.gh;
+    return rope[dm.rope_off_h + y * dm.ph + (c - dm.pt)];
+  } else {
+    int x = n % dm.gw;
+    return rope[dm.rope_off_w + x * dm.pw + (c - dm.pt - dm.ph)];
+  }
+}
+
+// phi(x) = elu(x) + 1.
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+}  // namespace rola

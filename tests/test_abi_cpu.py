@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry
+point, and its host-side logic (parameter checks, keep count, workspace sizing,
+plan creation) behaves as include/rola.h states."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_rank_attention_b200 as rola
+from sparse_rank_attention_b200 import build as rbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    rbuild.build()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "rola.h")).read()
+    return sorted(set(re.findall(r"ROLA_API\s+[\w\s\*]+?\b(rola_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 15
+    lib = rola.load()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(rola.EXPORTS)
+
+
+def _params(**kw):
+    base = dict(B=1, H=2, N=1000, d=64, r=16, topk=0.25)
+    base.update(kw)
+    return rola.make_params(**base)
+
+
+def test_keep_count_and_blocks():
+    assert rola.keep_count(_params(N=32760, topk=0.10, d=128, r=32)) == (512, 52)
+    assert rola.keep_count(_params(N=75600, topk=0.03, d=128, r=32)) == (1182, 36)
+    assert rola.keep_count(_params(N=32760, topk=0.05)) == (512, 26)
+    assert rola.keep_count(_params(N=6400, topk=0.07)) == (100, 7)
+    assert rola.keep_count(_params(N=64, topk=0.01)) == (1, 1)
+    assert rola.keep_count(_params(N=1000, topk=1.0)) == (16, 16)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(r=8), 2), (dict(N=0), 1), (dict(topk=0.0), 1), (dict(topk=1.5), 1),
+    (dict(grid=(2, 2, 7)), 1), (dict(pairs=(1, 1, 1)), 1), (dict(pairs=(-1, 5, 4)), 1),
+    (dict(rope_base=1.0), 1), (dict(softmax_scale=-1.0), 1), (dict(dtype=7), 1),
+    (dict(N=64 * 3000), 2),
+])
+def test_invalid_params_rejected(kw, code):
+    p = _params(**kw)
+    n = ctypes.c_size_t()
+    assert rola.load().rola_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code
+
+
+def test_block_size_must_be_64():
+    p = _params()
+    p.block = 32
+    n = ctypes.c_size_t()
+    assert rola.load().rola_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 2
+
+
+def test_workspace_size_grows_with_problem():
+    a = rola.workspace_size(_params(N=1024))
+    b = rola.workspace_size(_params(N=4096))
+    assert 0 < a < b and a % 256 == 0
+
+
+def test_plan_checks_workspace_without_touching_device():
+    lib = rola.load()
+    p = _params()
+    need = rola.workspace_size(p)
+    h = ctypes.c_void_p()
+    assert lib.rola_plan(ctypes.byref(p), None, need, ctypes.byref(h)) == 3
+    assert lib.rola_plan(ctypes.byref(p), ctypes.c_void_p(0x1000 + 16), need, ctypes.byref(h)) == 3
+    assert lib.rola_plan(ctypes.byref(p), ctypes.c_void_p(0x100000), need - 1, ctypes.byref(h)) == 3
+    # a well-formed (never dereferenced) address: plan creation is host-only
+    assert lib.rola_plan(ctypes.byref(p), ctypes.c_void_p(0x100000), need, ctypes.byref(h)) == 0
+    # null and misaligned tensors are rejected before any launch
+    assert lib.rola_select_blocks(h, None, ctypes.c_void_p(0x2000), None) == 1
+    assert lib.rola_select_blocks(h, ctypes.c_void_p(0x2008), ctypes.c_void_p(0x2000), None) == 1
+    assert lib.rola_attend(h, *[ctypes.c_void_p(0x4000)] * 6, None) == 1   # out overlaps q
+    assert lib.rola_set_debug(h, -1, 0) == 1
+    lib.rola_plan_destroy(h)
+
+
+def test_status_strings():
+    lib = rola.load()
+    for c in range(7):
+        assert lib.rola_status_string(c)
+    assert lib.rola_status_string(0) == b"ok"
