@@ -68,7 +68,9 @@ typedef enum {
   ROLA_ERR_WORKSPACE = 3,       /* workspace missing, misaligned or too small          */
   ROLA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed                */
   ROLA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out (see poll)       */
-  ROLA_ERR_DEVICE_BOUNDS = 6    /* a device-side index check failed (see poll)         */
+  ROLA_ERR_DEVICE_BOUNDS = 6,   /* a device-side index check failed (see poll)         */
+  ROLA_ERR_RANGE = 7            /* an input value is non-finite or, for v in ROLA_BF16, */
+                                /* outside +-65504 (v is carried in fp16; see poll)     */
 } rola_status;
 
 typedef enum {

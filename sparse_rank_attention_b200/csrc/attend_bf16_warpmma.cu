@@ -9,6 +9,10 @@
 // One CTA per (b, h, 64-token query block), 4 warps x 16 query rows:
 //   for each kept key block j (ascending):  S = Q K_j^T, online softmax, O += P V_j
 //   epilogue: u = phi(Q Wq), den = u.z, num = (R u) S_h, out = O/l + g * num/den
+// Precision: Q K^T in bf16 (exact products, fp32 sums); the softmax weights P are
+// rounded to fp16 and multiplied with the fp16 copy of v (bf16 P would cost up to
+// ~1e-3 absolute on peaked rows); R u and S_h enter the epilogue products as bf16
+// hi + lo pairs (three products), so the linear branch keeps ~fp32 accuracy.
 // K_j / V_j are double-buffered with cp.async; out is staged in shared memory and
 // written with 16-byte stores, once.
 #include "rola_internal.cuh"
@@ -22,26 +26,28 @@ struct AttSmem {
   static constexpr int DP = D + 8;            // padded row, bf16 elements
   static constexpr int kTile = kBlock * DP;
   static constexpr int kWq = RK * DP;         // WqT [r][d]
-  static constexpr int kS = RK * DP;          // S_h [r][d]
-  static constexpr size_t bytes = sizeof(__nv_bfloat16) * (5 * kTile + kWq + kS) + sizeof(float) * RK;
+  static constexpr int kS = RK * DP;          // S_h [r][d] (hi and lo)
+  static constexpr size_t bytes = sizeof(__nv_bfloat16) * (5 * kTile + kWq + 2 * kS) + sizeof(float) * RK;
 };
 
 template <int D, int RK>
 __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ Wq,
+    const __half* __restrict__ v, const __nv_bfloat16* __restrict__ Wq,
     const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Dims dm,
-    const int32_t* __restrict__ col_idx, const __nv_bfloat16* __restrict__ S_bf,
-    const float* __restrict__ z, const float2* __restrict__ rope, int* __restrict__ status) {
+    const int32_t* __restrict__ col_idx, const __nv_bfloat16* __restrict__ S_hi,
+    const __nv_bfloat16* __restrict__ S_lo, const float* __restrict__ z,
+    const float2* __restrict__ rope, int* __restrict__ status) {
   using L = AttSmem<D, RK>;
   constexpr int DP = L::DP;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   __nv_bfloat16* sK = sQ + L::kTile;          // [2][tile]
-  __nv_bfloat16* sV = sK + 2 * L::kTile;      // [2][tile]
-  __nv_bfloat16* sW = sV + 2 * L::kTile;
-  __nv_bfloat16* sS = sW + L::kWq;
-  float* sz = reinterpret_cast<float*>(sS + L::kS);
+  __half* sV = reinterpret_cast<__half*>(sK + 2 * L::kTile);      // [2][tile] fp16
+  __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(sV + 2 * L::kTile);
+  __nv_bfloat16* sS = sW + L::kWq;        // S_hi
+  __nv_bfloat16* sSl = sS + L::kS;        // S_lo
+  float* sz = reinterpret_cast<float*>(sSl + L::kS);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, t4 = lane & 3, quad = lane >> 3;
@@ -50,7 +56,7 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
   const size_t rs = (size_t)dm.H * D;
   const __nv_bfloat16* qb = q + (size_t)b * dm.N * rs + (size_t)h * D;
   const __nv_bfloat16* kb = k + (size_t)b * dm.N * rs + (size_t)h * D;
-  const __nv_bfloat16* vb = v + (size_t)b * dm.N * rs + (size_t)h * D;
+  const __half* vb = v + (size_t)b * dm.N * rs + (size_t)h * D;
   const int32_t* Lst = col_idx + ((size_t)bh * dm.nb + i) * dm.k;
   constexpr int VPR = D / 8;  // 16-byte vectors per row
 
@@ -62,7 +68,8 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
   }
   for (int e = tid; e < RK * VPR; e += 128) {
     const int a = e / VPR, cv = e % VPR;
-    cp_async16(smem_u32(sS + a * DP + cv * 8), S_bf + ((size_t)bh * RK + a) * D + cv * 8, 16);
+    cp_async16(smem_u32(sS + a * DP + cv * 8), S_hi + ((size_t)bh * RK + a) * D + cv * 8, 16);
+    cp_async16(smem_u32(sSl + a * DP + cv * 8), S_lo + ((size_t)bh * RK + a) * D + cv * 8, 16);
   }
   cp_async_commit();
   for (int e = tid; e < D * RK; e += 128) {
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     }
     __syncthreads();
     const __nv_bfloat16* tK = sK + stage * L::kTile;
-    const __nv_bfloat16* tV = sV + stage * L::kTile;
+    const __half* tV = sV + stage * L::kTile;
 
     float s[8][4];
 #pragma unroll
@@ -176,17 +183,17 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      pa[0] = pack_f16(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_f16(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_f16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_f16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int nt = 0; nt < D / 8; nt += 2) {
         uint32_t bf[4];
         ldsm_x4_t(smem_u32(tV + (kk * 16 + (quad & 1) * 8 + (lane & 7)) * DP + (nt + (quad >> 1)) * 8),
                   bf[0], bf[1], bf[2], bf[3]);
-        mma_bf16(o[nt], pa, bf);
-        mma_bf16(o[nt + 1], pa, bf + 2);
+        mma_f16(o[nt], pa, bf);
+        mma_f16(o[nt + 1], pa, bf + 2);
       }
     }
     __syncthreads();
@@ -244,24 +251,29 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
       u[nt][2 * hh + 1] = cs.y * x0 + cs.x * x1;
     }
   }
-  uint32_t ua[RK / 16][4];
+  uint32_t ua[RK / 16][4], ul[RK / 16][4];
 #pragma unroll
   for (int kk = 0; kk < RK / 16; ++kk) {
-    ua[kk][0] = pack_bf16(u[2 * kk][0], u[2 * kk][1]);
-    ua[kk][1] = pack_bf16(u[2 * kk][2], u[2 * kk][3]);
-    ua[kk][2] = pack_bf16(u[2 * kk + 1][0], u[2 * kk + 1][1]);
-    ua[kk][3] = pack_bf16(u[2 * kk + 1][2], u[2 * kk + 1][3]);
+    split_bf16(u[2 * kk][0], u[2 * kk][1], ua[kk][0], ul[kk][0]);
+    split_bf16(u[2 * kk][2], u[2 * kk][3], ua[kk][1], ul[kk][1]);
+    split_bf16(u[2 * kk + 1][0], u[2 * kk + 1][1], ua[kk][2], ul[kk][2]);
+    split_bf16(u[2 * kk + 1][2], u[2 * kk + 1][3], ua[kk][3], ul[kk][3]);
   }
 #pragma unroll
   for (int nt = 0; nt < D / 8; nt += 2) {
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < RK / 16; ++kk) {
-      uint32_t bf[4];
-      ldsm_x4_t(smem_u32(sS + (kk * 16 + (quad & 1) * 8 + (lane & 7)) * DP + (nt + (quad >> 1)) * 8),
-                bf[0], bf[1], bf[2], bf[3]);
+      uint32_t bf[4], bl[4];
+      const int off = (kk * 16 + (quad & 1) * 8 + (lane & 7)) * DP + (nt + (quad >> 1)) * 8;
+      ldsm_x4_t(smem_u32(sS + off), bf[0], bf[1], bf[2], bf[3]);
+      ldsm_x4_t(smem_u32(sSl + off), bl[0], bl[1], bl[2], bl[3]);
       mma_bf16(acc[0], ua[kk], bf);
       mma_bf16(acc[1], ua[kk], bf + 2);
+      mma_bf16(acc[0], ua[kk], bl);
+      mma_bf16(acc[1], ua[kk], bl + 2);
+      mma_bf16(acc[0], ul[kk], bf);
+      mma_bf16(acc[1], ul[kk], bf + 2);
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t)
@@ -294,8 +306,8 @@ cudaError_t launch_bf16(const Dims& dm, const void* q, const void* k, const void
   dim3 grid(dm.nb, dm.B * dm.H);
   attend_bf16_kernel<D, RK><<<grid, 128, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(Wq), g,
-      static_cast<__nv_bfloat16*>(out), dm, ws.col_idx, ws.S_bf, ws.z, ws.rope, ws.status);
+      ws.v16, static_cast<const __nv_bfloat16*>(Wq), g, static_cast<__nv_bfloat16*>(out), dm,
+      ws.col_idx, ws.S_hi, ws.S_lo, ws.z, ws.rope, ws.status);
   return cudaGetLastError();
 }
 

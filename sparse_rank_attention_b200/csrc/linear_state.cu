@@ -48,27 +48,32 @@ struct LSSmem {
   static constexpr int RP = RK + 8;
   static constexpr int kW = RK * DP;          // WkT [r][d]
   static constexpr int kTileElems = kLSTile * DP;
-  static constexpr int kF = kLSTile * RP;     // rotated features [tok][r]
-  static constexpr size_t bytes = sizeof(__nv_bfloat16) * (kW + 4 * kTileElems + kF) +
+  static constexpr int kF = kLSTile * RP;     // rotated features [tok][r] (hi and lo parts)
+  static constexpr size_t bytes = sizeof(__nv_bfloat16) * (kW + 4 * kTileElems + 2 * kF) +
                                   sizeof(float) * 4 * RK;
 };
 
 // grid: x = chunk, y = b*H + h; 128 threads (4 warps).
 //   A: F = K_tile Wk       (warp w: tokens 16w..16w+15, all r)       mma m16n8k16
-//   B: phi, z, rotation    (in registers; rotary pairs are adjacent accumulator columns)
-//   C: S += R(F)^T V_tile  (warp w: d columns [w*D/4, (w+1)*D/4))    mma m16n8k16
+//   B: phi, z, rotation    (in registers; rotary pairs are adjacent accumulator columns);
+//      the rotated features are split into bf16 hi + lo parts (F = hi + lo to ~2^-17)
+//   C: S += R(F)^T V_tile  (warp w: d columns [w*D/4, (w+1)*D/4))    2 x mma m16n8k16
+// The kernel also writes the fp16 copy of v that the attention kernel multiplies the
+// fp16 softmax weights with, and flags values outside the fp16 range.
 template <int D, int RK>
 __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin,
     const __nv_bfloat16* __restrict__ Wk, Dims dm, const float2* __restrict__ rope,
-    float* __restrict__ S_part, float* __restrict__ z_part) {
+    float* __restrict__ S_part, float* __restrict__ z_part, __half* __restrict__ v16,
+    int* __restrict__ status) {
   using L = LSSmem<D, RK>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   __nv_bfloat16* sK = sW + L::kW;                     // [2][tile]
   __nv_bfloat16* sV = sK + 2 * L::kTileElems;         // [2][tile]
-  __nv_bfloat16* sF = sV + 2 * L::kTileElems;
-  float* sZ = reinterpret_cast<float*>(sF + L::kF);   // [4][RK]
+  __nv_bfloat16* sF = sV + 2 * L::kTileElems;       // hi part
+  __nv_bfloat16* sFl = sF + L::kF;                    // lo part
+  float* sZ = reinterpret_cast<float*>(sFl + L::kF);  // [4][RK]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
@@ -128,6 +133,30 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* tK = sK + stage * L::kTileElems;
     const __nv_bfloat16* tV = sV + stage * L::kTileElems;
 
+    // fp16 copy of the V tile (+ range check)
+    {
+      constexpr int kVecPerRow = D / 8;
+      const int n0 = n_begin + tile * kLSTile;
+      bool bad = false;
+      for (int e = tid; e < kLSTile * kVecPerRow; e += 128) {
+        const int rr = e / kVecPerRow, cv = e % kVecPerRow, n = n0 + rr;
+        if (n >= n_end) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(tV + rr * L::DP + cv * 8);
+        const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        uint4 packed;
+        __half2* dst = reinterpret_cast<__half2*>(&packed);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(src[t]);
+          bad |= !(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f);
+          dst[t] = __floats2half2_rn(f.x, f.y);
+        }
+        *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n) * row_stride + (size_t)h * D + cv * 8) =
+            packed;
+      }
+      if (bad) record_status(status, kDevRange);
+    }
+
     // A: F = K Wk
     float f[NT_F][4];
 #pragma unroll
@@ -165,7 +194,11 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
         const float2 cs = ok ? rope_cs(dm, rope, n, nt * 4 + t4) : make_float2(1.f, 0.f);
         const float y0 = cs.x * x0 - cs.y * x1;
         const float y1 = cs.y * x0 + cs.x * x1;
-        *reinterpret_cast<uint32_t*>(sF + row * L::RP + nt * 8 + 2 * t4) = pack_bf16(y0, y1);
+        const uint32_t hi = pack_bf16(y0, y1);
+        const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+        *reinterpret_cast<uint32_t*>(sF + row * L::RP + nt * 8 + 2 * t4) = hi;
+        *reinterpret_cast<uint32_t*>(sFl + row * L::RP + nt * 8 + 2 * t4) =
+            pack_bf16(y0 - hf.x, y1 - hf.y);
       }
     }
     __syncthreads();
@@ -174,11 +207,13 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
 #pragma unroll
     for (int kk = 0; kk < kLSTile / 16; ++kk) {
       const int q = lane >> 3;
-      uint32_t af[MT_S][4];
+      uint32_t af[MT_S][4], al[MT_S][4];
 #pragma unroll
-      for (int mt = 0; mt < MT_S; ++mt)
-        ldsm_x4_t(smem_u32(sF + (kk * 16 + (q >> 1) * 8 + (lane & 7)) * L::RP + mt * 16 + (q & 1) * 8),
-                  af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+      for (int mt = 0; mt < MT_S; ++mt) {
+        const int off = (kk * 16 + (q >> 1) * 8 + (lane & 7)) * L::RP + mt * 16 + (q & 1) * 8;
+        ldsm_x4_t(smem_u32(sF + off), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+        ldsm_x4_t(smem_u32(sFl + off), al[mt][0], al[mt][1], al[mt][2], al[mt][3]);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT_S; nt += 2) {
         uint32_t bf[4];
@@ -189,6 +224,8 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
         for (int mt = 0; mt < MT_S; ++mt) {
           mma_bf16(sacc[mt][nt], af[mt], bf);
           mma_bf16(sacc[mt][nt + 1], af[mt], bf + 2);
+          mma_bf16(sacc[mt][nt], al[mt], bf);
+          mma_bf16(sacc[mt][nt + 1], al[mt], bf + 2);
         }
       }
     }
@@ -298,10 +335,11 @@ __global__ void __launch_bounds__(128) linear_state_f32_kernel(
   if (tid < RK) z_part[((size_t)bh * dm.nchunk + chunk) * RK + tid] = zacc;
 }
 
-// Adds the chunk partials in chunk order; writes S (fp32), its bf16 copy and z.
+// Adds the chunk partials in chunk order; writes S (fp32), its bf16 hi/lo split and z.
 __global__ void state_reduce_kernel(Dims dm, const float* __restrict__ S_part,
                                     const float* __restrict__ z_part, float* __restrict__ S,
-                                    __nv_bfloat16* __restrict__ S_bf, float* __restrict__ z) {
+                                    __nv_bfloat16* __restrict__ S_hi,
+                                    __nv_bfloat16* __restrict__ S_lo, float* __restrict__ z) {
   const int bh = blockIdx.y;
   const int rd = dm.r * dm.d;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -310,7 +348,9 @@ __global__ void state_reduce_kernel(Dims dm, const float* __restrict__ S_part,
     float acc = 0.f;
     for (int c = 0; c < dm.nchunk; ++c) acc += p[(size_t)c * rd];
     S[(size_t)bh * rd + e] = acc;
-    S_bf[(size_t)bh * rd + e] = __float2bfloat16_rn(acc);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+    S_hi[(size_t)bh * rd + e] = hi;
+    S_lo[(size_t)bh * rd + e] = __float2bfloat16_rn(acc - __bfloat162float(hi));
   } else if (e < rd + dm.r) {
     const int a = e - rd;
     const float* p = z_part + (size_t)bh * dm.nchunk * dm.r + a;
@@ -335,7 +375,8 @@ cudaError_t launch_ls(const Dims& dm, rola_dtype dt, const void* k, const void* 
     if (e != cudaSuccess) return e;
     linear_state_bf16_kernel<D, RK><<<grid, 128, smem, st>>>(
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part);
+        static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.v16,
+        ws.status);
   }
   return cudaGetLastError();
 }
@@ -359,7 +400,8 @@ cudaError_t launch_linear_state(const Dims& dm, rola_dtype dt, const void* k, co
   if (e != cudaSuccess) return e;
   const int rd = dm.r * dm.d + dm.r;
   dim3 grid((rd + 255) / 256, dm.B * dm.H);
-  state_reduce_kernel<<<grid, 256, 0, st>>>(dm, ws.S_part, ws.z_part, ws.S, ws.S_bf, ws.z);
+  state_reduce_kernel<<<grid, 256, 0, st>>>(dm, ws.S_part, ws.z_part, ws.S, ws.S_hi, ws.S_lo,
+                                            ws.z);
   return cudaGetLastError();
 }
 

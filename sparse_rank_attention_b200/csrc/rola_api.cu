@@ -98,7 +98,10 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   w.z_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r));
   w.S = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r * dm.d));
   w.z = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r));
-  w.S_bf = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
+  w.S_hi = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
+  w.S_lo = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
+  if (p.dtype == ROLA_BF16)
+    w.v16 = reinterpret_cast<__half*>(take(sizeof(__half) * (size_t)dm.B * dm.N * dm.H * dm.d));
   if (p.dtype == ROLA_FP8_E4M3) {
     const size_t elems = (size_t)dm.B * dm.N * dm.H * dm.d;
     w.q8 = reinterpret_cast<uint8_t*>(take(elems));
@@ -231,7 +234,10 @@ rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const vo
   cudaError_t e;
   if (p.dtype == ROLA_F32)
     e = rola::launch_attend_f32(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
-  else
+  else if (p.d == 128)
+    e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, Wq, g, out, plan->debug_flags,
+                                  plan->debug_limit_us, st);
+  else  // head dim 64: the transposed tcgen05 tile needs d = 128 rows
     e = rola::launch_attend_bf16_warpmma(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
   return cuda_status(e);
 }
@@ -295,7 +301,8 @@ rola_status rola_poll_device_status(rola_plan_t plan, rola_stream_t stream) {
   if (word == 0) return ROLA_OK;
   if (cudaMemsetAsync(plan->ws.status, 0, sizeof(int), st) != cudaSuccess) return ROLA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return ROLA_ERR_CUDA;
-  return word == ROLA_ERR_DEVICE_TIMEOUT ? ROLA_ERR_DEVICE_TIMEOUT : ROLA_ERR_DEVICE_BOUNDS;
+  if (word == ROLA_ERR_DEVICE_TIMEOUT || word == ROLA_ERR_RANGE) return (rola_status)word;
+  return ROLA_ERR_DEVICE_BOUNDS;
 }
 
 rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us) {
@@ -314,6 +321,7 @@ const char* rola_status_string(rola_status s) {
     case ROLA_ERR_CUDA: return "CUDA runtime error";
     case ROLA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
     case ROLA_ERR_DEVICE_BOUNDS: return "a device-side index check failed";
+    case ROLA_ERR_RANGE: return "an input value is outside the supported range";
   }
   return "unknown status";
 }

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "rola.h"
@@ -16,6 +17,7 @@ constexpr int kStateChunk = 2048;  // tokens per linear-state partial sum
 constexpr int kDevOk = 0;
 constexpr int kDevTimeout = ROLA_ERR_DEVICE_TIMEOUT;
 constexpr int kDevBounds = ROLA_ERR_DEVICE_BOUNDS;
+constexpr int kDevRange = ROLA_ERR_RANGE;
 
 // Everything a kernel needs to know about the problem, passed by value.
 struct Dims {
@@ -40,7 +42,9 @@ struct Workspace {
   float* z_part;      // [B, H, nchunk, r]
   float* S;           // [B, H, r, d]
   float* z;           // [B, H, r]
-  __nv_bfloat16* S_bf;  // [B, H, r, d] bf16 copy (tensor-core operand of the epilogue)
+  __nv_bfloat16* S_hi;  // [B, H, r, d] bf16(S)            } S = S_hi + S_lo to ~2^-17:
+  __nv_bfloat16* S_lo;  // [B, H, r, d] bf16(S - S_hi)     } tensor-core operands of the epilogue
+  __half* v16;          // [B, N, H, d] fp16 copy of v (bf16 and fp8-free paths: PV operand)
   uint8_t* q8;        // [B, N, H, d] e4m3 (fp8 mode)
   uint8_t* k8;
   uint8_t* v8;
@@ -78,6 +82,9 @@ cudaError_t launch_attend_f32(const Dims& dm, const void* q, const void* k, cons
 cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void* k,
                                        const void* v, const void* Wq, const float* g, void* out,
                                        const Workspace& ws, cudaStream_t st);
+cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
+                                const void* Wq, const float* g, void* out, int debug_flags,
+                                int debug_limit_us, cudaStream_t st);
 size_t select_smem_bytes(const Dims& dm);
 
 // ---- device helpers ----

