@@ -336,10 +336,13 @@ __global__ void __launch_bounds__(128) linear_state_f32_kernel(
 }
 
 // Adds the chunk partials in chunk order; writes S (fp32), its bf16 hi/lo split and z.
+// With d = 128 it also writes S^T hi | lo as the attention epilogue's tensor-core operand
+// image: MN-major, 128-byte swizzle, box c = channels 64c..64c+63, rank rows of 128 bytes.
 __global__ void state_reduce_kernel(Dims dm, const float* __restrict__ S_part,
                                     const float* __restrict__ z_part, float* __restrict__ S,
                                     __nv_bfloat16* __restrict__ S_hi,
-                                    __nv_bfloat16* __restrict__ S_lo, float* __restrict__ z) {
+                                    __nv_bfloat16* __restrict__ S_lo, float* __restrict__ z,
+                                    uint8_t* __restrict__ simg) {
   const int bh = blockIdx.y;
   const int rd = dm.r * dm.d;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -349,8 +352,16 @@ __global__ void state_reduce_kernel(Dims dm, const float* __restrict__ S_part,
     for (int c = 0; c < dm.nchunk; ++c) acc += p[(size_t)c * rd];
     S[(size_t)bh * rd + e] = acc;
     const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
     S_hi[(size_t)bh * rd + e] = hi;
-    S_lo[(size_t)bh * rd + e] = __float2bfloat16_rn(acc - __bfloat162float(hi));
+    S_lo[(size_t)bh * rd + e] = lo;
+    if (simg != nullptr) {
+      const int a = e / dm.d, dd = e % dm.d, c = dd >> 6, col = dd & 63;
+      uint8_t* im = simg + (size_t)bh * 4 * dm.r * 128;
+      const size_t off = (size_t)(c * dm.r + a) * 128 + (((col >> 3) ^ (a & 7)) << 4) + (col & 7) * 2;
+      *reinterpret_cast<__nv_bfloat16*>(im + off) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(im + 2 * dm.r * 128 + off) = lo;
+    }
   } else if (e < rd + dm.r) {
     const int a = e - rd;
     const float* p = z_part + (size_t)bh * dm.nchunk * dm.r + a;
@@ -401,7 +412,7 @@ cudaError_t launch_linear_state(const Dims& dm, rola_dtype dt, const void* k, co
   const int rd = dm.r * dm.d + dm.r;
   dim3 grid((rd + 255) / 256, dm.B * dm.H);
   state_reduce_kernel<<<grid, 256, 0, st>>>(dm, ws.S_part, ws.z_part, ws.S, ws.S_hi, ws.S_lo,
-                                            ws.z);
+                                            ws.z, ws.simg);
   return cudaGetLastError();
 }
 

@@ -6,7 +6,7 @@
 // the fraction of key blocks kept).  Block size, pooling rule and tie-break are this
 // library's reading: 64-token blocks, fp32 means, lowest key-block index wins a tie.
 //
-// Both kernels reproduce a stated fp32 order exactly, so the block lists are bit-exact:
+// The kernels reproduce a stated fp32 order exactly, so the block lists are bit-exact:
 //   qbar = (fp32 sum of the block's tokens in token order) / count   (IEEE division)
 //   s_ij = fma chain over channels 0..d-1 starting from 0
 #include "rola_internal.cuh"
@@ -80,161 +80,166 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, cons
   for (int e = 0; e < EPV; ++e) dst[e] = __fdiv_rn(acc[e], fc);
 }
 
-// ------------------------------------------------------------------ scores + top-k
+// ------------------------------------------------------------------ block scores
 
-constexpr int kSelThreads = 256;
-constexpr int kKeyChunk = 64;
-constexpr int kKTStride = kKeyChunk + 4;  // padded row of the transposed key chunk
+constexpr int kTS = 128;  // score tile: 128 query blocks x 128 key blocks
+constexpr int kKC = 32;   // channels staged per step
 
-__host__ __device__ inline int select_rows_per_cta(int nb) { return nb <= 1300 ? 32 : 16; }
-
-__host__ __device__ inline size_t select_smem(int R, int d, int nb) {
-  const int nbp = (nb + kKeyChunk - 1) / kKeyChunk * kKeyChunk;
-  return sizeof(float) * ((size_t)R * (d + 1) + (size_t)d * kKTStride + (size_t)R * nbp) +
-         sizeof(uint32_t) * 256 * (kSelThreads / 32);
+// grid: x = key-block tile, y = query-block tile, z = b*H + h; 256 threads, 8x8 scores each.
+// s_ij accumulates q_i[c] * k_j[c] with fmaf in channel order 0..d-1 (the stated order).
+__global__ void __launch_bounds__(256) score_kernel(Dims dm, const float* __restrict__ qbar,
+                                                    const float* __restrict__ kbar,
+                                                    float* __restrict__ scores, int nbp) {
+  __shared__ __align__(16) float As[kKC][kTS + 4];
+  __shared__ __align__(16) float Bs[kKC][kTS + 4];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int i0 = blockIdx.y * kTS, j0 = blockIdx.x * kTS, bh = blockIdx.z;
+  const int nb = dm.nb, d = dm.d;
+  const float* qb = qbar + (size_t)bh * nb * d;
+  const float* kb = kbar + (size_t)bh * nb * d;
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+  for (int c0 = 0; c0 < d; c0 += kKC) {
+    __syncthreads();
+    for (int e = tid; e < kTS * kKC; e += 256) {
+      const int r = e / kKC, c = e % kKC;
+      As[c][r] = (i0 + r < nb) ? qb[(size_t)(i0 + r) * d + c0 + c] : 0.f;
+      Bs[c][r] = (j0 + r < nb) ? kb[(size_t)(j0 + r) * d + c0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kKC; ++c) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[c][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[c][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(av[a], bv[e], acc[a][e]);
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + ty * 8 + a;
+    if (i >= nb) continue;
+    float* row = scores + ((size_t)bh * nb + i) * nbp + j0 + tx * 8;
+    if (j0 + tx * 8 + 8 <= nbp) {
+      *reinterpret_cast<float4*>(row) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+      *reinterpret_cast<float4*>(row + 4) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (j0 + tx * 8 + e < nbp) row[e] = acc[a][e];
+    }
+  }
 }
 
-// grid: x = row tiles of R query blocks, y = b*H + h.
-// Phase 1: scores of R query blocks against all key blocks into shared memory.
-// Phase 2: one warp per row: 4-pass 8-bit radix select of the k-th largest score,
-// then one pass in index order emits the kept indices (ties -> lower index).
-template <int R>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(Dims dm, const float* __restrict__ qbar,
-                                                             const float* __restrict__ kbar,
-                                                             int32_t* __restrict__ col_idx,
-                                                             int* __restrict__ status) {
-  constexpr int RPT = R / 16;  // rows per thread in phase 1
-  extern __shared__ float smem[];
-  const int d = dm.d, nb = dm.nb, kk = dm.k;
-  const int nbp = (nb + kKeyChunk - 1) / kKeyChunk * kKeyChunk;
-  float* qs = smem;                         // [R][d+1]
-  float* kT = qs + R * (d + 1);             // [d][kKTStride]
-  float* sc = kT + d * kKTStride;           // [R][nbp]
-  uint32_t* hist_all = reinterpret_cast<uint32_t*>(sc + R * nbp);  // [8][256]
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const int row0 = blockIdx.x * R;
-  const float* qsrc = qbar + (size_t)bh * nb * d;
-  const float* ksrc = kbar + (size_t)bh * nb * d;
+// ------------------------------------------------------------------ top-k per row
 
-  for (int e = tid; e < R * d; e += kSelThreads) {
-    const int rr = e / d, c = e % d;
-    qs[rr * (d + 1) + c] = (row0 + rr < nb) ? qsrc[(size_t)(row0 + rr) * d + c] : 0.f;
-  }
-  const int rg = tid / 16, kg = tid % 16;
-  for (int j0 = 0; j0 < nb; j0 += kKeyChunk) {
-    __syncthreads();
-    for (int e = tid; e < kKeyChunk * d; e += kSelThreads) {
-      const int jj = e / d, c = e % d;
-      kT[c * kKTStride + jj] = (j0 + jj < nb) ? ksrc[(size_t)(j0 + jj) * d + c] : 0.f;
-    }
-    __syncthreads();
-    float acc[RPT][4];
-#pragma unroll
-    for (int a = 0; a < RPT; ++a)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[a][e] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < d; ++c) {
-      const float4 kv = *reinterpret_cast<const float4*>(&kT[c * kKTStride + kg * 4]);
-#pragma unroll
-      for (int a = 0; a < RPT; ++a) {
-        const float qv = qs[(rg * RPT + a) * (d + 1) + c];
-        acc[a][0] = fmaf(qv, kv.x, acc[a][0]);
-        acc[a][1] = fmaf(qv, kv.y, acc[a][1]);
-        acc[a][2] = fmaf(qv, kv.z, acc[a][2]);
-        acc[a][3] = fmaf(qv, kv.w, acc[a][3]);
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < RPT; ++a)
-      *reinterpret_cast<float4*>(&sc[(rg * RPT + a) * nbp + j0 + kg * 4]) =
-          make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-  }
-  __syncthreads();
+constexpr int kTopkWarps = 8;
 
-  uint32_t* hist = hist_all + warp * 256;
+__host__ __device__ inline size_t topk_smem(int nbp) {
+  return sizeof(uint32_t) * ((size_t)kTopkWarps * nbp + 256 * kTopkWarps);
+}
+
+// One warp per row (b, h, i): 4-pass 8-bit radix select of the k-th largest score, then
+// one pass in index order emits the kept block indices (ties -> lower index).
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const float* __restrict__ scores,
+                                                               int nbp, int32_t* __restrict__ col_idx,
+                                                               int* __restrict__ status) {
+  extern __shared__ uint32_t tsm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kTopkWarps + warp;
+  const long long nrows = (long long)dm.B * dm.H * dm.nb;
+  if (row >= nrows) return;
+  const int nb = dm.nb, kk = dm.k;
+  uint32_t* key = tsm + warp * nbp;
+  uint32_t* hist = tsm + kTopkWarps * nbp + warp * 256;
+  const float* src = scores + row * nbp;
   const unsigned full = 0xffffffffu;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int rr = warp; rr < R; rr += kSelThreads / 32) {
-    const int i = row0 + rr;
-    if (i >= nb) break;
-    uint32_t* key = reinterpret_cast<uint32_t*>(sc + rr * nbp);
-    // Order-preserving map float -> uint32 (both zeros map to the key of +0).
-    for (int j = lane; j < nb; j += 32) {
-      float f = sc[rr * nbp + j];
-      if (f == 0.f) f = 0.f;
-      const uint32_t u = __float_as_uint(f);
-      key[j] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    }
+  // Order-preserving map float -> uint32 (both zeros map to the key of +0).
+  for (int j = lane; j < nb; j += 32) {
+    float f = src[j];
+    if (f == 0.f) f = 0.f;
+    const uint32_t u = __float_as_uint(f);
+    key[j] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+  __syncwarp();
+  uint32_t prefix = 0, pmask = 0;
+  int need = kk;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int bb = lane; bb < 256; bb += 32) hist[bb] = 0;
     __syncwarp();
-    uint32_t prefix = 0, pmask = 0;
-    int need = kk;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int bb = lane; bb < 256; bb += 32) hist[bb] = 0;
-      __syncwarp();
-      for (int j = lane; j < nb; j += 32) {
-        const uint32_t u = key[j];
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      int cntv[8], local = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {  // lane owns bins 255-8*lane-e, in descending order
-        cntv[e] = (int)hist[255 - 8 * lane - e];
-        local += cntv[e];
-      }
-      int incl = local;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(full, incl, off);
-        if (lane >= off) incl += t;
-      }
-      const int excl = incl - local;
-      const unsigned hit = __ballot_sync(full, excl < need && need <= incl);
-      const int src = hit ? (__ffs(hit) - 1) : 0;
-      int digit = 0, above = 0;
-      if (lane == src) {
-        int c = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (c + cntv[e] >= need) {
-            digit = 255 - 8 * lane - e;
-            above = c;
-            break;
-          }
-          c += cntv[e];
-        }
-      }
-      digit = __shfl_sync(full, digit, src);
-      above = __shfl_sync(full, above, src);
-      need -= above;
-      prefix |= (uint32_t)digit << shift;
-      pmask |= 255u << shift;
-      __syncwarp();
-    }
-    // prefix is the k-th largest key; `need` elements equal to it are kept.
-    int32_t* out = col_idx + ((size_t)bh * nb + i) * kk;
-    int written = 0, eqseen = 0;
+    // Lanes with equal digits are merged first (__match_any_sync), so a bin shared by
+    // most keys (e.g. the exponent byte in the first pass) costs one atomic per step.
     for (int j0 = 0; j0 < nb; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t u = (j < nb) ? key[j] : 0u;
-      const bool gt = (j < nb) && u > prefix;
-      const bool eq = (j < nb) && u == prefix;
-      const unsigned beq = __ballot_sync(full, eq);
-      const bool keep = gt || (eq && eqseen + __popc(beq & lt_mask) < need);
-      const unsigned bk = __ballot_sync(full, keep);
-      const int pos = written + __popc(bk & lt_mask);
-      if (keep) {
-        if (pos < kk) out[pos] = j;
-      }
-      written += __popc(bk);
-      eqseen += __popc(beq);
+      const uint32_t u = j < nb ? key[j] : 0u;
+      const uint32_t digit = (j < nb && (u & pmask) == prefix) ? ((u >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(full, digit);
+      if (digit != 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
     }
-    if (lane == 0 && written != kk) record_status(status, kDevBounds);
+    __syncwarp();
+    int cntv[8], local = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {  // lane owns bins 255-8*lane-e, in descending order
+      cntv[e] = (int)hist[255 - 8 * lane - e];
+      local += cntv[e];
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(full, incl, off);
+      if (lane >= off) incl += t;
+    }
+    const int excl = incl - local;
+    const unsigned hit = __ballot_sync(full, excl < need && need <= incl);
+    const int srcl = hit ? (__ffs(hit) - 1) : 0;
+    int digit = 0, above = 0;
+    if (lane == srcl) {
+      int c = excl;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (c + cntv[e] >= need) {
+          digit = 255 - 8 * lane - e;
+          above = c;
+          break;
+        }
+        c += cntv[e];
+      }
+    }
+    digit = __shfl_sync(full, digit, srcl);
+    above = __shfl_sync(full, above, srcl);
+    need -= above;
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 255u << shift;
     __syncwarp();
   }
+  // prefix is the k-th largest key; `need` elements equal to it are kept.
+  int32_t* out = col_idx + row * kk;
+  int written = 0, eqseen = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t u = (j < nb) ? key[j] : 0u;
+    const bool gt = (j < nb) && u > prefix;
+    const bool eq = (j < nb) && u == prefix;
+    const unsigned beq = __ballot_sync(full, eq);
+    const bool keep = gt || (eq && eqseen + __popc(beq & lt_mask) < need);
+    const unsigned bk = __ballot_sync(full, keep);
+    const int pos = written + __popc(bk & lt_mask);
+    if (keep && pos < kk) out[pos] = j;
+    written += __popc(bk);
+    eqseen += __popc(beq);
+  }
+  if (lane == 0 && written != kk) record_status(status, kDevBounds);
 }
 
 }  // namespace
@@ -255,26 +260,22 @@ cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void
   return cudaGetLastError();
 }
 
-size_t select_smem_bytes(const Dims& dm) {
-  return select_smem(select_rows_per_cta(dm.nb), dm.d, dm.nb);
-}
+int score_row_stride(const Dims& dm) { return (dm.nb + 3) / 4 * 4; }
+
+size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm)); }
 
 cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) {
-  const int R = select_rows_per_cta(dm.nb);
-  const size_t smem = select_smem(R, dm.d, dm.nb);
-  dim3 grid((dm.nb + R - 1) / R, dm.B * dm.H);
-  cudaError_t e;
-  if (R == 32) {
-    e = cudaFuncSetAttribute(select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<32><<<grid, kSelThreads, smem, st>>>(dm, ws.qbar, ws.kbar, ws.col_idx, ws.status);
-  } else {
-    e = cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<16><<<grid, kSelThreads, smem, st>>>(dm, ws.qbar, ws.kbar, ws.col_idx, ws.status);
-  }
+  const int nbp = score_row_stride(dm);
+  dim3 g1((dm.nb + kTS - 1) / kTS, (dm.nb + kTS - 1) / kTS, dm.B * dm.H);
+  score_kernel<<<g1, 256, 0, st>>>(dm, ws.qbar, ws.kbar, ws.scores, nbp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = topk_smem(nbp);
+  e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long rows = (long long)dm.B * dm.H * dm.nb;
+  topk_kernel<<<(unsigned)((rows + kTopkWarps - 1) / kTopkWarps), kTopkWarps * 32, smem, st>>>(
+      dm, ws.scores, nbp, ws.col_idx, ws.status);
   return cudaGetLastError();
 }
 

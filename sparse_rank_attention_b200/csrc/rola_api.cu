@@ -12,7 +12,7 @@ using rola::Dims;
 using rola::Workspace;
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxBlocks = 2800;  // scores of a row tile must fit shared memory
+constexpr int kMaxBlocks = 6000;  // one score row per warp must fit shared memory
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -94,6 +94,7 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   w.qbar = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * dm.d));
   w.kbar = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * dm.d));
   w.col_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * dm.nb * dm.k));
+  w.scores = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * rola::score_row_stride(dm)));
   w.S_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r * dm.d));
   w.z_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r));
   w.S = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r * dm.d));
@@ -102,6 +103,11 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   w.S_lo = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
   if (p.dtype == ROLA_BF16)
     w.v16 = reinterpret_cast<__half*>(take(sizeof(__half) * (size_t)dm.B * dm.N * dm.H * dm.d));
+  if (p.dtype != ROLA_F32 && p.d == 128) {
+    w.simg = reinterpret_cast<uint8_t*>(take(BH * 4 * dm.r * 128));
+    w.uimg = reinterpret_cast<uint8_t*>(take(BH * dm.nb * 2 * dm.r * 128));
+    w.gden = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * 64));
+  }
   if (p.dtype == ROLA_FP8_E4M3) {
     const size_t elems = (size_t)dm.B * dm.N * dm.H * dm.d;
     w.q8 = reinterpret_cast<uint8_t*>(take(elems));
@@ -234,9 +240,12 @@ rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const vo
   cudaError_t e;
   if (p.dtype == ROLA_F32)
     e = rola::launch_attend_f32(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
-  else if (p.d == 128)
-    e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, Wq, g, out, plan->debug_flags,
-                                  plan->debug_limit_us, st);
+  else if (p.d == 128) {
+    e = rola::launch_query_features(plan->dm, q, Wq, g, plan->ws, st);
+    if (e == cudaSuccess)
+      e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, plan->debug_flags,
+                                    plan->debug_limit_us, st);
+  }
   else  // head dim 64: the transposed tcgen05 tile needs d = 128 rows
     e = rola::launch_attend_bf16_warpmma(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
   return cuda_status(e);

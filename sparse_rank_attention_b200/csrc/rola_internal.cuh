@@ -38,6 +38,7 @@ struct Workspace {
   float* qbar;        // [B, H, nb, d]
   float* kbar;        // [B, H, nb, d]
   int32_t* col_idx;   // [B, H, nb, k]
+  float* scores;      // [B, H, nb, nbp] block scores (nbp = nb rounded up to 4)
   float* S_part;      // [B, H, nchunk, r, d]
   float* z_part;      // [B, H, nchunk, r]
   float* S;           // [B, H, r, d]
@@ -45,6 +46,9 @@ struct Workspace {
   __nv_bfloat16* S_hi;  // [B, H, r, d] bf16(S)            } S = S_hi + S_lo to ~2^-17:
   __nv_bfloat16* S_lo;  // [B, H, r, d] bf16(S - S_hi)     } tensor-core operands of the epilogue
   __half* v16;          // [B, N, H, d] fp16 copy of v (bf16 and fp8-free paths: PV operand)
+  uint8_t* simg;        // [B, H] S_h^T hi|lo as 128-byte-swizzled MN-major operand images
+  uint8_t* uimg;        // [B, H, nb] (R u)^T hi|lo images ([r rows][64 tokens], swizzled)
+  float* gden;          // [B, H, nb, 64] g_h / (u . z_h) per query token
   uint8_t* q8;        // [B, N, H, d] e4m3 (fp8 mode)
   uint8_t* k8;
   uint8_t* v8;
@@ -83,9 +87,11 @@ cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void
                                        const void* v, const void* Wq, const float* g, void* out,
                                        const Workspace& ws, cudaStream_t st);
 cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
-                                const void* Wq, const float* g, void* out, int debug_flags,
-                                int debug_limit_us, cudaStream_t st);
+                                void* out, int debug_flags, int debug_limit_us, cudaStream_t st);
+cudaError_t launch_query_features(const Dims& dm, const void* q, const void* Wq, const float* g,
+                                  const Workspace& ws, cudaStream_t st);
 size_t select_smem_bytes(const Dims& dm);
+int score_row_stride(const Dims& dm);
 
 // ---- device helpers ----
 __device__ __forceinline__ void record_status(int* status, int code) {

@@ -13,12 +13,6 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -49,29 +43,56 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait with a suspend-time hint: a waiting thread sleeps until the phase completes
+// (or the hint elapses) instead of polling and taking issue slots from its neighbours.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for phase `parity` of `bar`.  Gives up when *abort is set by another
-// thread, or after limit_ns of wall time (then sets *abort and records `timeout_code`).
+// thread, or after limit_cycles SM clock cycles (then sets *abort and records
+// ROLA_ERR_DEVICE_TIMEOUT in the status word).
 struct WaitCtl {
   volatile int* abort;
   int* status;
-  unsigned long long limit_ns;
+  unsigned long long limit_cycles;
 };
 
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w,
-                                       bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 15u) == 0) {
-      if (honour_abort && *w.abort) return false;
-      if (globaltimer() - t0 > w.limit_ns) {
-        *w.abort = 1;
-        atomicCAS(w.status, 0, 5 /* ROLA_ERR_DEVICE_TIMEOUT */);
-        return false;
-      }
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& w,
+                                            bool honour_abort) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;   // sleeps up to 0.2 ms
+    if (honour_abort && *w.abort) return false;
+    if ((unsigned long long)(clock64() - t0) > w.limit_cycles) {
+      *w.abort = 1;
+      atomicCAS(w.status, 0, 5 /* ROLA_ERR_DEVICE_TIMEOUT */);
+      return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w,
+                                          bool honour_abort = true) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, w, honour_abort);
 }
 
 // ------------------------------------------------------------------ fences / barriers
@@ -108,6 +129,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int 
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
       "%4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// Contiguous global -> shared copy (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
 }
 

@@ -51,7 +51,7 @@ def test_keep_count_and_blocks():
     (dict(d=96), 2), (dict(r=8), 2), (dict(N=0), 1), (dict(topk=0.0), 1), (dict(topk=1.5), 1),
     (dict(grid=(2, 2, 7)), 1), (dict(pairs=(1, 1, 1)), 1), (dict(pairs=(-1, 5, 4)), 1),
     (dict(rope_base=1.0), 1), (dict(softmax_scale=-1.0), 1), (dict(dtype=7), 1),
-    (dict(N=64 * 3000), 2),
+    (dict(N=64 * 7000), 2),
 ])
 def test_invalid_params_rejected(kw, code):
     p = _params(**kw)
