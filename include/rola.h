@@ -136,6 +136,24 @@ ROLA_API rola_status rola_forward(rola_plan_t plan, const void* q, const void* k
                          const void* Wq, const void* Wk, const float* g, void* out,
                          rola_stream_t stream);
 
+/* Steps 1-2 without any device allocation and without a plan or workspace (no
+ * counterpart on the pages: this is a deployment variant of rola_select_blocks).
+ * It is meant for callers that cannot allocate device memory at the point of the call
+ * and have no workspace to lend -- code running inside a host framework whose pool owns
+ * all device memory, or latency-critical paths where cudaMalloc's implicit device
+ * synchronisation is not acceptable.  Writes the block lists [B, H, nb, k] int32 to the
+ * caller's `col_idx` (q, k and col_idx as for rola_select_blocks; all 16-byte aligned).
+ * Scratch: one 16 MiB array inside the library, which every GPU that loads the library
+ * holds until the process exits; problems whose pooled means and block scores need more
+ * (about 256 + 8*B*H*nb*d + 4*B*H*nb*ceil4(nb) bytes) are rejected with
+ * ROLA_ERR_WORKSPACE before any launch.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array: calls that overlap on the GPU
+ * (other streams, other host threads) race and must be serialised by the caller.
+ * Device-side index checks of this variant are not reported. */
+ROLA_API rola_status rola_select_blocks_noalloc(const rola_params* p, const void* q, const void* k,
+                                                int32_t* col_idx, rola_stream_t stream);
+
 /* Inspection (tests): copy, on `stream`, the block lists [B, H, nb, k] int32 (CSR column
  * indices; row i of (b, h) starts at ((b*H + h)*nb + i)*k), the pooled means [B, H, nb, d]
  * fp32, or the linear state S [B, H, r, d] and z [B, H, r] fp32 into caller buffers. */

@@ -27,12 +27,13 @@ ROLA_DEBUG_STALL_WAIT = 1
 
 STATUS = {0: "ROLA_OK", 1: "ROLA_ERR_INVALID_ARG", 2: "ROLA_ERR_UNSUPPORTED",
           3: "ROLA_ERR_WORKSPACE", 4: "ROLA_ERR_CUDA", 5: "ROLA_ERR_DEVICE_TIMEOUT",
-          6: "ROLA_ERR_DEVICE_BOUNDS"}
+          6: "ROLA_ERR_DEVICE_BOUNDS", 7: "ROLA_ERR_RANGE"}
 
 EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rola_plan",
            "rola_plan_destroy", "rola_select_blocks", "rola_linear_state", "rola_attend",
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
-           "rola_poll_device_status", "rola_set_debug", "rola_status_string")
+           "rola_poll_device_status", "rola_set_debug", "rola_status_string",
+           "rola_select_blocks_noalloc")
 
 
 class RolaError(RuntimeError):
@@ -84,6 +85,7 @@ def load() -> ctypes.CDLL:
         "rola_get_linear_state": [P, P, P, P],
         "rola_poll_device_status": [P, P],
         "rola_set_debug": [P, i32, i32],
+        "rola_select_blocks_noalloc": [pp, P, P, P, P],
     }.items():
         f = getattr(lib, name)
         f.argtypes = args
@@ -227,6 +229,13 @@ class Plan:
         _check(load().rola_set_debug(self._h, flags, limit_us), "rola_set_debug")
 
 
+def select_blocks_noalloc(params: RolaParams, q, k, col_idx, stream=None) -> int:
+    """Block selection into the caller's col_idx [B,H,nb,k] int32 with no device allocation
+    (the library's own fixed scratch); returns the rola_status code."""
+    return load().rola_select_blocks_noalloc(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(col_idx),
+                                             _stream(stream))
+
+
 def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
             softmax_scale=0.0, dtype=None, out=None):
     """One-shot RoLA forward (builds a plan and workspace for this call)."""
@@ -242,5 +251,5 @@ def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=1000
         plan.close()
 
 
-__all__ = ["Plan", "forward", "load", "make_params", "keep_count", "workspace_size", "RolaError",
+__all__ = ["Plan", "forward", "select_blocks_noalloc", "load", "make_params", "keep_count", "workspace_size", "RolaError",
            "RolaParams", "EXPORTS", "LIB_PATH", "ROLA_DEBUG_STALL_WAIT"]

@@ -9,6 +9,8 @@
 // The kernels reproduce a stated fp32 order exactly, so the block lists are bit-exact:
 //   qbar = (fp32 sum of the block's tokens in token order) / count   (IEEE division)
 //   s_ij = fma chain over channels 0..d-1 starting from 0
+#include <mutex>
+
 #include "rola_internal.cuh"
 
 namespace rola {
@@ -277,6 +279,68 @@ cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) 
   topk_kernel<<<(unsigned)((rows + kTopkWarps - 1) / kTopkWarps), kTopkWarps * 32, smem, st>>>(
       dm, ws.scores, nbp, ws.col_idx, ws.status);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// Block selection for callers that cannot allocate device memory and have no workspace
+// to lend.  Its scratch (status word, pooled means, block scores) lives in one file-scope
+// device array of kSelectScratchBytes; every GPU that loads this library holds that array
+// until the process exits.  In host code `g_select_scratch` only names a host-side
+// stand-in, so its device address is looked up with cudaGetSymbolAddress, once per device
+// (on the first call made with that device current), and passed to the kernels.
+
+namespace {
+
+constexpr size_t kSelectScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_select_scratch[kSelectScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+size_t select_noalloc_bytes(const Dims& dm) {
+  const size_t BH = (size_t)dm.B * dm.H;
+  return 256 + 2 * align256(sizeof(float) * BH * dm.nb * dm.d) +
+         align256(sizeof(float) * BH * dm.nb * score_row_stride(dm));
+}
+
+size_t select_noalloc_capacity() { return kSelectScratchBytes; }
+
+cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, const void* k,
+                                  int32_t* col_idx, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_select_scratch);
+      if (e != cudaSuccess) return e;
+      g_scratch_addr[dev] = ptr;
+    }
+    base = static_cast<char*>(g_scratch_addr[dev]);
+  }
+  const size_t BH = (size_t)dm.B * dm.H;
+  Workspace w{};
+  w.status = reinterpret_cast<int*>(base);
+  w.qbar = reinterpret_cast<float*>(base + 256);
+  w.kbar = reinterpret_cast<float*>(base + 256 + align256(sizeof(float) * BH * dm.nb * dm.d));
+  w.scores = reinterpret_cast<float*>(base + 256 + 2 * align256(sizeof(float) * BH * dm.nb * dm.d));
+  w.col_idx = col_idx;
+  // The array keeps the previous call's contents: the status word must start at zero.
+  e = cudaMemsetAsync(w.status, 0, 256, st);
+  if (e != cudaSuccess) return e;
+  e = launch_pool(dm, dt, q, k, w, st);
+  if (e != cudaSuccess) return e;
+  return launch_select(dm, w, st);
 }
 
 }  // namespace rola

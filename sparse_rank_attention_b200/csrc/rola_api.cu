@@ -268,6 +268,18 @@ rola_status rola_forward(rola_plan_t plan, const void* q, const void* k, const v
   return rola_attend(plan, q, k, v, Wq, g, out, stream);
 }
 
+rola_status rola_select_blocks_noalloc(const rola_params* p, const void* q, const void* k,
+                                       int32_t* col_idx, rola_stream_t stream) {
+  rola_status s = check_params(p);
+  if (s != ROLA_OK) return s;
+  if (!q || !k || !col_idx || !aligned16(q) || !aligned16(k) || !aligned16(col_idx))
+    return ROLA_ERR_INVALID_ARG;
+  const Dims dm = make_dims(*p);
+  if (rola::select_noalloc_bytes(dm) > rola::select_noalloc_capacity()) return ROLA_ERR_WORKSPACE;
+  return cuda_status(rola::select_blocks_noalloc(dm, p->dtype, q, k, col_idx,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rola_status rola_get_block_lists(rola_plan_t plan, int32_t* col_idx, rola_stream_t stream) {
   if (!plan || !col_idx) return ROLA_ERR_INVALID_ARG;
   const Dims& dm = plan->dm;

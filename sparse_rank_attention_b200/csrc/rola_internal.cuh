@@ -92,6 +92,10 @@ cudaError_t launch_query_features(const Dims& dm, const void* q, const void* Wq,
                                   const Workspace& ws, cudaStream_t st);
 size_t select_smem_bytes(const Dims& dm);
 int score_row_stride(const Dims& dm);
+size_t select_noalloc_bytes(const Dims& dm);
+size_t select_noalloc_capacity();
+cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, const void* k,
+                                  int32_t* col_idx, cudaStream_t st);
 
 // ---- device helpers ----
 __device__ __forceinline__ void record_status(int* status, int code) {
