@@ -19,9 +19,10 @@
 // 128 lanes and rescales O^T.  Per-query sums l stay per thread (partials over that
 // thread's keys) until the end.
 //
-// Roles (192 threads): warp 0 = TMA producers (lane 0: Q and the K ring, lane 1: the V
-// ring, lane 2: the epilogue operands), warp 1 = MMA issuers (lane 0: Q K^T, lane 1:
-// P V; warp 1 also owns TMEM), warps 2-5 = softmax and epilogue.  K pairs are
+// Roles (256 threads, one role per warp so that a sleeping wait never holds another
+// role back): warp 0 = TMA producer of Q and the K ring, warp 1 = Q K^T issuer (and TMEM
+// owner), warps 2-5 = softmax and epilogue, warp 6 = P V issuer, warp 7 = producer of
+// the epilogue operands and the V ring.  K pairs are
 // triple-buffered (freed when their QK is done), V pairs double-buffered, S^T
 // triple-buffered in TMEM, so QK runs up to two pairs ahead of the softmax warps.
 //
@@ -45,29 +46,29 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kSBufs = 3;         // S^T buffers at columns 0, 64, 128
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 192;   // O^T
 constexpr uint32_t kColNum = 0;   // epilogue: num^T (reuses S buffer 0)
 
-constexpr int kKStages = 3;                // K pairs: freed as soon as their QK is done
+constexpr int kKStages = 2;                // K pairs: freed as soon as their QK is done
 constexpr int kVStages = 2;                // V pairs: freed after their PV
 constexpr uint32_t kPairBytes = 32768;     // one [128 keys][128 d] 16-bit pair (2 boxes)
 constexpr uint32_t kBoxKV = 16384;         // one [128][64] box of a pair
 constexpr uint32_t kOffQ = 0;                                    // 2 boxes [64 q][64 d] bf16
 constexpr uint32_t kOffK = 16384;                                // K ring
 constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;        // V ring (fp16)
-constexpr uint32_t kOffP = kOffV + kVStages * kPairBytes;        // P^T [128 keys][64 q] fp16
-constexpr uint32_t kOffSimg = kOffP + 16384;                     // S_h^T hi | lo images (<= 16 KB)
+constexpr uint32_t kOffP = kOffV + kVStages * kPairBytes;        // 2 x P^T [128 keys][64 q] fp16
+constexpr uint32_t kOffSimg = kOffP + 2 * 16384;                 // S_h^T hi | lo images (<= 16 KB)
 constexpr uint32_t kOffUimg = kOffSimg + 16384;                  // (R u)^T hi | lo images (<= 8 KB)
 constexpr uint32_t kOffGden = kOffUimg + 8192;                   // g/den per query (256 B)
 constexpr uint32_t kOffCtl = kOffGden + 256;
 
 struct Ctl {
   uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[kSBufs], s_empty[kSBufs], p_full, pv_done, ep_full, ep_bar, drain_bar, stall_bar;
+  uint64_t s_full[kSBufs], s_empty[kSBufs], p_full[2], pv_done[2], ep_full, ep_bar, drain_bar, stall_bar;
   uint32_t tmem_base;
   int abort;
   alignas(16) float m_used[64];
@@ -205,8 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       mbar_init(bar(ctl->s_full[s]), 1);
       mbar_init(bar(ctl->s_empty[s]), 128);
     }
-    mbar_init(bar(ctl->p_full), 128);
-    mbar_init(bar(ctl->pv_done), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ctl->p_full[s]), 128);
+      mbar_init(bar(ctl->pv_done[s]), 1);
+    }
     mbar_init(bar(ctl->ep_full), 1);
     mbar_init(bar(ctl->ep_bar), 1);
     mbar_init(bar(ctl->drain_bar), 2);
@@ -263,32 +266,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       mbar_wait(bar(ctl->q_full), 0, wc, false);
       for (int it = (issued > kKStages ? issued - kKStages : 0); it < issued; ++it)
         mbar_wait(bar(ctl->k_full[it % kKStages]), (it / kKStages) & 1, wc, false);
-    } else if (lane == 1) {        // the V ring
-      tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int it = 0; it < npairs; ++it) {
-        const int s = it % kVStages;
-        if (it >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((it / kVStages) - 1) & 1, wc)) break;
-        int j1, j2;
-        pair_blocks(it, j1, j2);
-        const uint32_t st = sbase + kOffV + s * kPairBytes;
-        mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
-        for (int c = 0; c < 2; ++c) {
-          tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
-          tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
-        }
-        issued = it + 1;
-      }
-      for (int it = (issued > kVStages ? issued - kVStages : 0); it < issued; ++it)
-        mbar_wait(bar(ctl->v_full[it % kVStages]), (it / kVStages) & 1, wc, false);
-    } else if (lane == 2) {        // epilogue operands: S_h^T and (R u)^T images, g/den
-      tma_prefetch_desc(&tm_out);
-      const uint32_t sbytes = 4 * RK * 128, ubytes = 2 * RK * 128;
-      mbar_expect_tx(bar(ctl->ep_full), sbytes + ubytes + 256);
-      bulk_load(sbase + kOffSimg, simg + (size_t)bh * sbytes, sbytes, bar(ctl->ep_full));
-      bulk_load(sbase + kOffUimg, uimg + ((size_t)bh * dm.nb + i) * ubytes, ubytes, bar(ctl->ep_full));
-      bulk_load(sbase + kOffGden, gden + ((size_t)bh * dm.nb + i) * 64, 256, bar(ctl->ep_full));
-      mbar_wait(bar(ctl->ep_full), 0, wc, false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuers
@@ -311,24 +288,56 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
       mma_commit(bar(ctl->drain_bar));       // no MMA may run when TMEM is freed
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
-    } else if (lane == 1) {        // O^T += V_pair^T P^T
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ P V issuer
+    if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_f16(0, 128, 64, 1, 1);
-      const uint64_t db = sdesc_sw128(sbase + kOffP, 8192, 1024);
       for (int t = 0; t < npairs; ++t) {
-        const int s = t % kVStages;
+        const int s = t % kVStages, pb = t & 1;
         if (!mbar_wait(bar(ctl->v_full[s]), (t / kVStages) & 1, wc)) break;
-        if (!mbar_wait(bar(ctl->p_full), t & 1, wc)) break;
+        if (!mbar_wait(bar(ctl->p_full[pb]), (t >> 1) & 1, wc)) break;
+        const uint64_t db = sdesc_sw128(sbase + kOffP + pb * 16384, 8192, 1024);
         tc_fence_after();
         // descriptors advance by 2048 bytes (16 K-rows) per step: +128 in the address field
         const uint64_t da = sdesc_sw128(sbase + kOffV + s * kPairBytes, kBoxKV, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_f16_ss(tmem + kColO, da + 128 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
-        mma_commit(bar(ctl->pv_done));
+        mma_commit(bar(ctl->pv_done[pb]));
         mma_commit(bar(ctl->v_empty[s]));
       }
       mma_commit(bar(ctl->drain_bar));
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
+    }
+  } else if (warp == 7) {
+    // ------------------------------------------------------------ epilogue operands + V ring
+    if (lane == 0) {
+      const int xh = h * 128;
+      tma_prefetch_desc(&tm_out);
+      const uint32_t sbytes = 4 * RK * 128, ubytes = 2 * RK * 128;
+      mbar_expect_tx(bar(ctl->ep_full), sbytes + ubytes + 256);
+      bulk_load(sbase + kOffSimg, simg + (size_t)bh * sbytes, sbytes, bar(ctl->ep_full));
+      bulk_load(sbase + kOffUimg, uimg + ((size_t)bh * dm.nb + i) * ubytes, ubytes, bar(ctl->ep_full));
+      bulk_load(sbase + kOffGden, gden + ((size_t)bh * dm.nb + i) * 64, 256, bar(ctl->ep_full));
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int it = 0; it < npairs; ++it) {
+        const int s = it % kVStages;
+        if (it >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((it / kVStages) - 1) & 1, wc)) break;
+        int j1, j2;
+        pair_blocks(it, j1, j2);
+        const uint32_t st = sbase + kOffV + s * kPairBytes;
+        mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
+          tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
+        }
+        issued = it + 1;
+      }
+      for (int it = (issued > kVStages ? issued - kVStages : 0); it < issued; ++it)
+        mbar_wait(bar(ctl->v_full[it % kVStages]), (it / kVStages) & 1, wc, false);
+      mbar_wait(bar(ctl->ep_full), 0, wc, false);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -399,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         if (it > 0) {
 #pragma unroll
           for (int q = 0; q < 64; ++q) lp[q] *= ctl->fac[q];
-          fail |= !mbar_wait(bar(ctl->pv_done), (it - 1) & 1, wc);
+          fail |= !mbar_wait(bar(ctl->pv_done[(it - 1) & 1]), ((it - 1) >> 1) & 1, wc);
           tc_fence_after();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -424,16 +433,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         lp[q + 1] += p1;
         pw[q >> 1] = pack_half2(p0, p1);
       }
-      if (it > 0 && !fail) fail |= !mbar_wait(bar(ctl->pv_done), (it - 1) & 1, wc);
-      st_row_sw128(sP, t, pw);
+      if (it > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[it & 1]), ((it - 2) >> 1) & 1, wc);
+      st_row_sw128(sP + (it & 1) * 16384, t, pw);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(ctl->p_full));
+      mbar_arrive(bar(ctl->p_full[it & 1]));
     }
 
     // ------------------------------------------------------------ epilogue
     if (!named_vote_or(1, 128, fail)) {
-      fail |= !mbar_wait(bar(ctl->pv_done), (npairs - 1) & 1, wc);
+      fail |= !mbar_wait(bar(ctl->pv_done[(npairs - 1) & 1]), ((npairs - 1) >> 1) & 1, wc);
     }
     if (!named_vote_or(1, 128, fail)) {
       tc_fence_after();
