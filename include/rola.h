@@ -77,7 +77,11 @@ typedef enum {
   ROLA_F32 = 0,       /* fp32 in/out, fp32 arithmetic (correctness configuration)       */
   ROLA_BF16 = 1,      /* bf16 in/out, bf16 tensor-core products, fp32 accumulation      */
   ROLA_FP8_E4M3 = 2   /* bf16 in/out; q, k, v quantised inside to e4m3 with one absmax */
-                      /* scale per (b, h, 64-token block); fp8 tensor-core products     */
+                      /* scale per (b, h, 64-token block) (scale = absmax/448, 1 when   */
+                      /* absmax = 0; round to nearest even, saturating); fp8 tensor-core */
+                      /* products, fp32 softmax; P is e4m3 too.  Block lists come from  */
+                      /* the bf16 inputs, so they equal the ROLA_BF16 lists.  d = 128    */
+                      /* only (ROLA_ERR_UNSUPPORTED otherwise).                          */
 } rola_dtype;
 
 typedef struct {
@@ -127,7 +131,8 @@ ROLA_API rola_status rola_linear_state(rola_plan_t plan, const void* k, const vo
 
 /* Steps 3-5: sparse attention over the kept blocks with the linear branch and the
  * combination fused into its epilogue; writes out [B, N, H, d] once.  Uses the block
- * lists and the state the two calls above left in the workspace. */
+ * lists and the state the two calls above left in the workspace (in ROLA_FP8_E4M3 mode
+ * also their e4m3 copies of q, k, v, which must come from the same q, k, v). */
 ROLA_API rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const void* v,
                         const void* Wq, const float* g, void* out, rola_stream_t stream);
 
@@ -160,6 +165,14 @@ ROLA_API rola_status rola_select_blocks_noalloc(const rola_params* p, const void
 ROLA_API rola_status rola_get_block_lists(rola_plan_t plan, int32_t* col_idx, rola_stream_t stream);
 ROLA_API rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_stream_t stream);
 ROLA_API rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream);
+
+/* Inspection (tests), ROLA_FP8_E4M3 plans only (ROLA_ERR_INVALID_ARG otherwise): copy the
+ * e4m3 copies q8, k8, v8 [B, N, H, d] (one byte per element, OCP E4M3 encoding) and their
+ * scales sq, sk, sv [B, H, nb] fp32 (value = decoded byte * scale of its (b, h, block))
+ * into caller device buffers on `stream`.  q8/k8/sq/sk are written by
+ * rola_select_blocks, v8/sv by rola_linear_state. */
+ROLA_API rola_status rola_get_fp8_copies(rola_plan_t plan, uint8_t* q8, uint8_t* k8, uint8_t* v8,
+                                         float* sq, float* sk, float* sv, rola_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the device status word: ROLA_OK, or
  * ROLA_ERR_DEVICE_TIMEOUT / ROLA_ERR_DEVICE_BOUNDS if a kernel recorded one. */

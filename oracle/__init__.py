@@ -66,6 +66,9 @@ def _load():
             lib.rola_oracle_attend_blocks.argtypes = [sp] + [P] * 9 + [ctypes.c_int, P, P, P, P]
             lib.rola_oracle_forward.argtypes = [sp] + [P] * 8
             lib.rola_oracle_threads.restype = ctypes.c_int
+            lib.rola_oracle_e4m3_encode.argtypes = [P, P, ctypes.c_size_t]
+            lib.rola_oracle_e4m3_decode.argtypes = [P, P, ctypes.c_size_t]
+            lib.rola_oracle_quantize_blocks.argtypes = [sp, P, P, P]
             _lib = lib
     return _lib
 
@@ -173,6 +176,41 @@ def attend_blocks(s: Shape, q, k, v, Wq, g, col_idx, S, z, blocks, pos=None):
     _load().rola_oracle_attend_blocks(ctypes.byref(s), _p(q), _p(k), _p(v), _p(Wq), _p(g), _p(col_idx),
                                       _p(S), _p(z), _p(pos), n, _p(blocks), _p(sp), _p(li), _p(out))
     return sp, li, out
+
+
+def e4m3_encode(y) -> np.ndarray:
+    """e4m3 codes (uint8) of float32 values: nearest, ties to even, saturating at 448."""
+    y = _f32(y)
+    out = np.zeros(y.shape, dtype=np.uint8)
+    _load().rola_oracle_e4m3_encode(_p(y), _p(out), y.size)
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values (float64) of e4m3 codes; the two NaN codes decode to NaN."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.zeros(codes.shape, dtype=np.float64)
+    _load().rola_oracle_e4m3_decode(_p(codes), _p(out), codes.size)
+    return out
+
+
+def quantize_blocks(s: Shape, x):
+    """Per-(b, h, 64-token block) e4m3 quantisation of x [B,N,H,d].
+
+    Returns (codes uint8 [B,N,H,d], scales float32 [B,H,nb]); scale = absmax/448 (1 if 0).
+    """
+    x = _f32(x)
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    scales = np.zeros((s.B, s.H, num_blocks(s.N)), dtype=np.float32)
+    _load().rola_oracle_quantize_blocks(ctypes.byref(s), _p(x), _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequantize_blocks(s: Shape, codes, scales) -> np.ndarray:
+    """codes * scale of their (b, h, block), float64 [B,N,H,d]."""
+    val = e4m3_decode(codes)
+    rep = np.repeat(np.asarray(scales, dtype=np.float64), BLOCK, axis=2)[:, :, :s.N]   # [B,H,N]
+    return val * rep.transpose(0, 2, 1)[..., None]
 
 
 def forward(s: Shape, q, k, v, Wq, Wk, g):

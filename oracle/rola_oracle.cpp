@@ -325,6 +325,87 @@ void rola_oracle_forward(const rola_oracle_shape* s, const float* q, const float
   }
 }
 
+// ------------------------------------------------------------------ fp8 (e4m3) variant
+//
+// OCP 8-bit floating point, E4M3 flavour: 1 sign bit, 4 exponent bits (bias 7), 3
+// mantissa bits.  Exponent field 0 holds subnormals m/8 * 2^-6; fields 1..15 hold
+// (1 + m/8) * 2^(e-7), except field 15 with mantissa 7, which is NaN.  There are no
+// infinities; the largest finite magnitude is 448 (field 15, mantissa 6).
+//
+// Encoding of a finite float y: round |y| to the nearest representable magnitude, ties
+// to the even mantissa; magnitudes above 448 saturate to 448.  Written from the format
+// definition: within the binade [2^E, 2^(E+1)) (E >= -6) the spacing is 2^(E-3); below
+// 2^-6 it is the subnormal spacing 2^-9.
+static uint8_t e4m3_encode(float y) {
+  const uint8_t sign = std::signbit(y) ? 0x80 : 0x00;
+  const double a = std::fabs((double)y);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int E = (int)std::floor(std::log2(a));
+  // log2 of a double can land one off near powers of two: correct it exactly.
+  while (std::ldexp(1.0, E) > a) --E;
+  while (std::ldexp(1.0, E + 1) <= a) ++E;
+  if (E < -6) E = -6;                                // subnormal range shares 2^-9 spacing
+  const double step = std::ldexp(1.0, E - 3);
+  const double n = a / step;                         // exact: a power-of-two division
+  double r = std::floor(n);
+  const double frac = n - r;
+  if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;
+  const double v = r * step;                         // the rounded magnitude (<= 448)
+  if (v < std::ldexp(1.0, -6)) return sign | (uint8_t)(v / std::ldexp(1.0, -9));   // subnormal
+  int Ev = (int)std::floor(std::log2(v));
+  while (std::ldexp(1.0, Ev) > v) --Ev;
+  while (std::ldexp(1.0, Ev + 1) <= v) ++Ev;
+  const int mant = (int)((v / std::ldexp(1.0, Ev) - 1.0) * 8.0);
+  return sign | (uint8_t)(((Ev + 7) << 3) | mant);
+}
+
+static double e4m3_decode(uint8_t c) {
+  const double sgn = (c & 0x80) ? -1.0 : 1.0;
+  const int e = (c >> 3) & 0xF, m = c & 7;
+  if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+  if (e == 0) return sgn * std::ldexp((double)m / 8.0, -6);
+  return sgn * std::ldexp(1.0 + m / 8.0, e - 7);
+}
+
+void rola_oracle_e4m3_encode(const float* y, uint8_t* code, size_t n) {
+  for (size_t e = 0; e < n; ++e) code[e] = e4m3_encode(y[e]);
+}
+
+void rola_oracle_e4m3_decode(const uint8_t* code, double* y, size_t n) {
+  for (size_t e = 0; e < n; ++e) y[e] = e4m3_decode(code[e]);
+}
+
+// Per-(b, h, 64-token block) quantisation of x [B, N, H, d] (float values) to e4m3:
+// absmax over the block's valid tokens and all d channels; scale = absmax / 448 (1 when
+// absmax = 0); code = encode(x * (1 / scale)).  The integer codes are decided from
+// floating point, so this is done in the precision the kernels use: the division, the
+// reciprocal and the product are each one fp32 operation rounded to nearest.
+// codes: [B, N, H, d]; scales: [B, H, nb].
+void rola_oracle_quantize_blocks(const rola_oracle_shape* s, const float* x, uint8_t* codes,
+                                 float* scales) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d;
+  const int nb = rola_oracle_num_blocks(N);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int i = 0; i < nb; ++i) {
+        const int n0 = i * kBlock, n1 = std::min(N, n0 + kBlock);
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+          for (int c = 0; c < d; ++c) amax = std::max(amax, std::fabs(x[(((size_t)b * N + n) * H + h) * d + c]));
+        volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        volatile float inv = 1.0f / scale;
+        scales[((size_t)b * H + h) * nb + i] = scale;
+        for (int n = n0; n < n1; ++n)
+          for (int c = 0; c < d; ++c) {
+            const size_t at = (((size_t)b * N + n) * H + h) * d + c;
+            volatile float y = x[at] * inv;
+            codes[at] = e4m3_encode(y);
+          }
+      }
+}
+
 int rola_oracle_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

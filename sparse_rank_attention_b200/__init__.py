@@ -33,7 +33,7 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_plan_destroy", "rola_select_blocks", "rola_linear_state", "rola_attend",
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
-           "rola_select_blocks_noalloc")
+           "rola_select_blocks_noalloc", "rola_get_fp8_copies")
 
 
 class RolaError(RuntimeError):
@@ -86,6 +86,7 @@ def load() -> ctypes.CDLL:
         "rola_poll_device_status": [P, P],
         "rola_set_debug": [P, i32, i32],
         "rola_select_blocks_noalloc": [pp, P, P, P, P],
+        "rola_get_fp8_copies": [P, P, P, P, P, P, P, P],
     }.items():
         f = getattr(lib, name)
         f.argtypes = args
@@ -220,6 +221,16 @@ class Plan:
         _check(load().rola_get_linear_state(self._h, _ptr(S), _ptr(z), _stream(stream)),
                "rola_get_linear_state")
         return S, z
+
+    def fp8_copies(self, stream=None):
+        """(q8, k8, v8) uint8 [B,N,H,d] e4m3 codes and (sq, sk, sv) fp32 [B,H,nb] scales."""
+        p = self.params
+        dev = self.workspace.device
+        codes = [torch.empty((p.B, p.N, p.H, p.d), dtype=torch.uint8, device=dev) for _ in range(3)]
+        scales = [torch.empty((p.B, p.H, self.nb), dtype=torch.float32, device=dev) for _ in range(3)]
+        _check(load().rola_get_fp8_copies(self._h, *[_ptr(t) for t in codes + scales], _stream(stream)),
+               "rola_get_fp8_copies")
+        return codes, scales
 
     def poll_status(self, stream=None) -> int:
         """Synchronises the stream; returns the device status code (0 = ok), clearing it."""

@@ -37,6 +37,7 @@
 // leave their loops, in-flight MMAs and TMA copies are drained and TMEM is freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp8.h>
 
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -55,16 +56,26 @@ constexpr uint32_t kColNum = 0;   // epilogue: num^T (reuses S buffer 0)
 
 constexpr int kKStages = 2;                // K pairs: freed as soon as their QK is done
 constexpr int kVStages = 2;                // V pairs: freed after their PV
-constexpr uint32_t kPairBytes = 32768;     // one [128 keys][128 d] 16-bit pair (2 boxes)
-constexpr uint32_t kBoxKV = 16384;         // one [128][64] box of a pair
-constexpr uint32_t kOffQ = 0;                                    // 2 boxes [64 q][64 d] bf16
-constexpr uint32_t kOffK = 16384;                                // K ring
-constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;        // V ring (fp16)
-constexpr uint32_t kOffP = kOffV + kVStages * kPairBytes;        // 2 x P^T [128 keys][64 q] fp16
-constexpr uint32_t kOffSimg = kOffP + 2 * 16384;                 // S_h^T hi | lo images (<= 16 KB)
-constexpr uint32_t kOffUimg = kOffSimg + 16384;                  // (R u)^T hi | lo images (<= 8 KB)
-constexpr uint32_t kOffGden = kOffUimg + 8192;                   // g/den per query (256 B)
-constexpr uint32_t kOffCtl = kOffGden + 256;
+
+// Shared-memory geometry.  16-bit path: a tile row of 128 channels is two 128-byte
+// swizzle boxes (channels 0-63, 64-127); fp8 path: one 128-byte box.  P^T is fp16 in
+// 128-byte rows (SW128) or e4m3 in 64-byte rows (SW64).
+template <bool FP8>
+struct Geo {
+  static constexpr uint32_t kEl = FP8 ? 1 : 2;                   // bytes per q/k/v element
+  static constexpr uint32_t kQBytes = 64 * 128 * kEl;             // Q tile
+  static constexpr uint32_t kPairBytes = 128 * 128 * kEl;         // K or V pair
+  static constexpr uint32_t kBoxKV = FP8 ? 16384 : 16384;         // channel-box stride in a pair
+  static constexpr uint32_t kPBytes = FP8 ? 8192 : 16384;         // one P^T buffer
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = 16384;                         // K ring (1024-aligned)
+  static constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;  // V ring
+  static constexpr uint32_t kOffP = kOffV + kVStages * kPairBytes;  // 2 x P^T (also out staging)
+  static constexpr uint32_t kOffSimg = kOffP + 2 * 16384;           // S_h^T hi | lo (<= 16 KB)
+  static constexpr uint32_t kOffUimg = kOffSimg + 16384;            // (R u)^T hi | lo (<= 8 KB)
+  static constexpr uint32_t kOffGden = kOffUimg + 8192;             // g/den per query (256 B)
+  static constexpr uint32_t kOffCtl = kOffGden + 256;
+};
 
 struct Ctl {
   uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
@@ -75,8 +86,10 @@ struct Ctl {
   alignas(16) float fac[64];
   float red[4][64];
   alignas(16) float linv[64];
+  float vref[4];     // fp8: per-warp partial max of the kept blocks' V scales
 };
-constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;
+template <bool FP8>
+constexpr size_t smem_bytes() { return Geo<FP8>::kOffCtl + sizeof(Ctl) + 1024; }
 
 
 // Reduce 64 per-lane values over the 32 lanes of a warp; lane l receives the results
@@ -173,13 +186,36 @@ __device__ __forceinline__ void st_row_sw128(uint8_t* tile, int row, const uint3
   }
 }
 
-template <int RK>
+// Writes one 64-byte row (64 e4m3 values as 16 packed words) of a SW64 tile: 16-byte
+// chunk c of row `row` goes to chunk position c ^ ((row / 2) % 4).
+__device__ __forceinline__ void st_row_sw64(uint8_t* tile, int row, const uint32_t* w) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+    *reinterpret_cast<uint4*>(tile + row * 64 + ((c ^ ((row >> 1) & 3)) << 4)) = v;
+  }
+}
+
+// Four floats to four e4m3 bytes (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+template <int RK, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out, Dims dm,
     const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ simg,
-    const uint8_t* __restrict__ uimg, const float* __restrict__ gden, int* __restrict__ status,
-    int debug_flags, unsigned long long limit_cycles, unsigned long long debug_limit_cycles) {
+    const uint8_t* __restrict__ uimg, const float* __restrict__ gden,
+    const float* __restrict__ sq, const float* __restrict__ sk, const float* __restrict__ sv,
+    int* __restrict__ status, int debug_flags, unsigned long long limit_cycles,
+    unsigned long long debug_limit_cycles) {
+  using G = Geo<FP8>;
+  constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV, kOffP = G::kOffP;
+  constexpr uint32_t kOffSimg = G::kOffSimg, kOffUimg = G::kOffUimg, kOffGden = G::kOffGden;
+  constexpr uint32_t kOffCtl = G::kOffCtl, kPairBytes = G::kPairBytes, kBoxKV = G::kBoxKV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(base + kOffCtl);
@@ -245,9 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     if (lane == 0) {               // Q and the K ring
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      mbar_expect_tx(bar(ctl->q_full), 16384);
+      mbar_expect_tx(bar(ctl->q_full), G::kQBytes);
       tma_load_3d(sbase + kOffQ, &tm_q, xh, i * 64, b, bar(ctl->q_full));
-      tma_load_3d(sbase + kOffQ + 8192, &tm_q, xh + 64, i * 64, b, bar(ctl->q_full));
+      if (!FP8) tma_load_3d(sbase + kOffQ + 8192, &tm_q, xh + 64, i * 64, b, bar(ctl->q_full));
       int issued = 0;
       for (int it = 0; it < npairs; ++it) {
         const int s = it % kKStages;
@@ -256,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         pair_blocks(it, j1, j2);
         const uint32_t st = sbase + kOffK + s * kPairBytes;
         mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
           tma_load_3d(st + c * kBoxKV, &tm_k, xh + 64 * c, j1 * 64, b, bar(ctl->k_full[s]));
           tma_load_3d(st + c * kBoxKV + 8192, &tm_k, xh + 64 * c, j2 * 64, b, bar(ctl->k_full[s]));
         }
@@ -270,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {               // S^T = K_pair Q^T
-      constexpr uint32_t idesc_qk = idesc_f16(1, 128, 64, 0, 0);
+      constexpr uint32_t idesc_qk = FP8 ? idesc_f8(128, 64, 0, 0) : idesc_f16(1, 128, 64, 0, 0);
       bool ok = mbar_wait(bar(ctl->q_full), 0, wc);
       const uint64_t dq = sdesc_sw128(sbase + kOffQ, 16, 1024);
       for (int it = 0; ok && it < npairs; ++it) {
@@ -279,10 +315,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         if (it >= kSBufs && !mbar_wait(bar(ctl->s_empty[sb]), ((it / kSBufs) - 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t da = sdesc_sw128(sbase + kOffK + ks * kPairBytes, 16, 1024);
+        if constexpr (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
-          mma_f16_ss(tmem + kColS + 64 * sb, da + (((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4),
-                     dq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)   // 32 e4m3 channels (32 B) per step, one box
+            mma_f8_ss(tmem + kColS + 64 * sb, da + ((kk * 32) >> 4), dq + ((kk * 32) >> 4), idesc_qk, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
+            mma_f16_ss(tmem + kColS + 64 * sb, da + (((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4),
+                       dq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+        }
         mma_commit(bar(ctl->s_full[sb]));
         mma_commit(bar(ctl->k_empty[ks]));
       }
@@ -292,18 +334,25 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   } else if (warp == 6) {
     // ------------------------------------------------------------ P V issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_pv = idesc_f16(0, 128, 64, 1, 1);
+      constexpr uint32_t idesc_pv = FP8 ? idesc_f8(128, 64, 1, 1) : idesc_f16(0, 128, 64, 1, 1);
       for (int t = 0; t < npairs; ++t) {
         const int s = t % kVStages, pb = t & 1;
         if (!mbar_wait(bar(ctl->v_full[s]), (t / kVStages) & 1, wc)) break;
         if (!mbar_wait(bar(ctl->p_full[pb]), (t >> 1) & 1, wc)) break;
-        const uint64_t db = sdesc_sw128(sbase + kOffP + pb * 16384, 8192, 1024);
+        const uint64_t db = FP8 ? sdesc_sw64(sbase + kOffP + pb * G::kPBytes, 4096, 512)
+                                : sdesc_sw128(sbase + kOffP + pb * G::kPBytes, 8192, 1024);
         tc_fence_after();
         // descriptors advance by 2048 bytes (16 K-rows) per step: +128 in the address field
         const uint64_t da = sdesc_sw128(sbase + kOffV + s * kPairBytes, kBoxKV, 1024);
+        if constexpr (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ss(tmem + kColO, da + 128 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys per step: V rows of 128 B, P rows of 64 B
+            mma_f8_ss(tmem + kColO, da + 256 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ss(tmem + kColO, da + 128 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+        }
         mma_commit(bar(ctl->pv_done[pb]));
         mma_commit(bar(ctl->v_empty[s]));
       }
@@ -329,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         pair_blocks(it, j1, j2);
         const uint32_t st = sbase + kOffV + s * kPairBytes;
         mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
           tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
           tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
         }
@@ -355,6 +404,38 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
 #pragma unroll
     for (int q = 0; q < 64; ++q) lp[q] = 0.f;
 
+    // fp8: the scores carry sq_i * sk_j, P carries sv_j / vref and the output vref, where
+    // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
+    const size_t sbase_idx = (size_t)bh * dm.nb;
+    float sqi = 1.f, vref = 1.f;
+    if constexpr (FP8) {
+      sqi = __ldg(sq + sbase_idx + i);
+      float mx = 0.f;
+      for (int e = t; e < kk_list; e += 128) {
+        const int j = __ldg(L + e);
+        if (j >= 0 && j < dm.nb) mx = fmaxf(mx, __ldg(sv + sbase_idx + j));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) ctl->vref[wq] = mx;
+      named_sync(1, 128);
+      vref = fmaxf(fmaxf(ctl->vref[0], ctl->vref[1]), fmaxf(ctl->vref[2], ctl->vref[3]));
+      if (!(vref > 0.f)) vref = 1.f;
+    }
+    // This thread's key block for pair `it` (-1: the padding half of an odd list) and,
+    // for fp8, its K and V scales, fetched one pair ahead.
+    auto key_block = [&](int it) {
+      return (t < 64) ? __ldg(L + 2 * it) : ((2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : -1);
+    };
+    int jb_next = key_block(0);
+    float sk_next = 1.f, sv_next = 1.f;
+    if constexpr (FP8) {
+      if (jb_next >= 0 && jb_next < dm.nb) {
+        sk_next = __ldg(sk + sbase_idx + jb_next);
+        sv_next = __ldg(sv + sbase_idx + jb_next);
+      }
+    }
+
     for (int it = 0; it < npairs; ++it) {
       const int sb = it % kSBufs;
       const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (it / kSBufs) & 1, wc);
@@ -367,19 +448,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       tmem_wait_ld();
       tc_fence_before();
       if (ok) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
-      const int jb = (t < 64) ? __ldg(L + 2 * it)
-                              : ((2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : -1);
+      const int jb = jb_next;
+      const float skj = sk_next, svj = sv_next;
+      if (it + 1 < npairs) {
+        jb_next = key_block(it + 1);
+        if constexpr (FP8) {
+          if (jb_next >= 0 && jb_next < dm.nb) {
+            sk_next = __ldg(sk + sbase_idx + jb_next);
+            sv_next = __ldg(sv + sbase_idx + jb_next);
+          }
+        }
+      }
       const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
+      const float slt = FP8 ? sl2 * sqi * skj : sl2;
       const float4* m4 = reinterpret_cast<const float4*>(ctl->m_used);
       float dmax = -INFINITY;
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const float4 m = m4[q4];
-        x[4 * q4 + 0] = fmaf(x[4 * q4 + 0], sl2, -m.x);
-        x[4 * q4 + 1] = fmaf(x[4 * q4 + 1], sl2, -m.y);
-        x[4 * q4 + 2] = fmaf(x[4 * q4 + 2], sl2, -m.z);
-        x[4 * q4 + 3] = fmaf(x[4 * q4 + 3], sl2, -m.w);
+        x[4 * q4 + 0] = fmaf(x[4 * q4 + 0], slt, -m.x);
+        x[4 * q4 + 1] = fmaf(x[4 * q4 + 1], slt, -m.y);
+        x[4 * q4 + 2] = fmaf(x[4 * q4 + 2], slt, -m.z);
+        x[4 * q4 + 3] = fmaf(x[4 * q4 + 3], slt, -m.w);
       }
       if (!valid) {
 #pragma unroll
@@ -423,18 +514,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         }
         named_sync(1, 128);                          // red[0] is rewritten next time
       }
-      // P = 2^x (fp16) and the per-thread partial row sums
+      // P = 2^x (fp16, or e4m3 times sv_j / vref) and the per-thread partial row sums
       uint32_t pw[32];
+      if constexpr (FP8) {
+        const float pf = svj / vref;
 #pragma unroll
-      for (int q = 0; q < 64; q += 2) {
-        const float p0 = ex2_approx(x[q]);
-        const float p1 = ex2_approx(x[q + 1]);
-        lp[q] += p0;
-        lp[q + 1] += p1;
-        pw[q >> 1] = pack_half2(p0, p1);
+        for (int q = 0; q < 64; q += 4) {
+          const float p0 = ex2_approx(x[q]), p1 = ex2_approx(x[q + 1]);
+          const float p2 = ex2_approx(x[q + 2]), p3 = ex2_approx(x[q + 3]);
+          lp[q] += p0;
+          lp[q + 1] += p1;
+          lp[q + 2] += p2;
+          lp[q + 3] += p3;
+          pw[q >> 2] = pack_e4m3x4(p0 * pf, p1 * pf, p2 * pf, p3 * pf);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; q += 2) {
+          const float p0 = ex2_approx(x[q]);
+          const float p1 = ex2_approx(x[q + 1]);
+          lp[q] += p0;
+          lp[q + 1] += p1;
+          pw[q >> 1] = pack_half2(p0, p1);
+        }
       }
       if (it > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[it & 1]), ((it - 2) >> 1) & 1, wc);
-      st_row_sw128(sP + (it & 1) * 16384, t, pw);
+      if constexpr (FP8)
+        st_row_sw64(sP + (it & 1) * G::kPBytes, t, pw);
+      else
+        st_row_sw128(sP + (it & 1) * G::kPBytes, t, pw);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(ctl->p_full[it & 1]));
@@ -451,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       ctl->red[wq][2 * lane] = ls.x;
       ctl->red[wq][2 * lane + 1] = ls.y;
       named_sync(1, 128);
-      if (t < 64) ctl->linv[t] = 1.f / (ctl->red[0][t] + ctl->red[1][t] + ctl->red[2][t] + ctl->red[3][t]);
+      if (t < 64) ctl->linv[t] = vref / (ctl->red[0][t] + ctl->red[1][t] + ctl->red[2][t] + ctl->red[3][t]);
       if (t == 0) {
         fail |= !mbar_wait(bar(ctl->ep_full), 0, wc);
         tc_fence_after();
@@ -528,53 +636,63 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B, N, H*128] 16-bit tensor as a 3D map with [64 tokens x 64 channels] boxes.
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, const Dims& dm,
+// [B, N, H*128] tensor as a 3D map with [64 tokens x 128 bytes] boxes (64 channels of a
+// 16-bit type, 128 of an 8-bit one).
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, const Dims& dm,
               CUtensorMapSwizzle sw) {
   auto enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t HD = (cuuint64_t)dm.H * dm.d;
   cuuint64_t dims[3] = {HD, (cuuint64_t)dm.N, (cuuint64_t)dm.B};
-  cuuint64_t strides[2] = {HD * 2, HD * 2 * (cuuint64_t)dm.N};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint64_t strides[2] = {HD * el_bytes, HD * el_bytes * (cuuint64_t)dm.N};
+  cuuint32_t box[3] = {128 / el_bytes, 64, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
 
-size_t attend_sm100_smem_bytes() { return kSmemBytes; }
-
-cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
-                                void* out, int debug_flags, int debug_limit_us, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+template <int RK, bool FP8>
+cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to, const Dims& dm, const Workspace& ws, int debug_flags,
+                           int debug_limit_us, cudaStream_t st) {
   // Wait limits in SM clock cycles: 2e9 cycles is 1 s at 2 GHz (longer at lower clocks).
   const unsigned long long limit_cycles = 2000000000ull;
   const unsigned long long dlimit = (unsigned long long)(debug_limit_us > 0 ? debug_limit_us : 1000) * 2000ull;
+  constexpr size_t smem = smem_bytes<FP8>();
+  cudaError_t e = cudaFuncSetAttribute(attend_sm100_kernel<RK, FP8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(dm.nb, dm.B * dm.H);
-  cudaError_t e;
-  if (dm.r == 32) {
-    e = cudaFuncSetAttribute(attend_sm100_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attend_sm100_kernel<32><<<grid, kThreads, kSmemBytes, st>>>(
-        tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.status, debug_flags,
-        limit_cycles, dlimit);
-  } else {
-    e = cudaFuncSetAttribute(attend_sm100_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attend_sm100_kernel<16><<<grid, kThreads, kSmemBytes, st>>>(
-        tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.status, debug_flags,
-        limit_cycles, dlimit);
-  }
+  attend_sm100_kernel<RK, FP8><<<grid, kThreads, smem, st>>>(
+      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status,
+      debug_flags, limit_cycles, dlimit);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attend_sm100_smem_bytes(bool fp8) { return fp8 ? smem_bytes<true>() : smem_bytes<false>(); }
+
+cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
+                                void* out, bool fp8, int debug_flags, int debug_limit_us, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, to;
+  bool ok;
+  if (fp8)
+    ok = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.q8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.k8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.v8, dm, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
+  if (fp8)
+    return dm.r == 32 ? launch_variant<32, true>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st)
+                      : launch_variant<16, true>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st);
+  return dm.r == 32 ? launch_variant<32, false>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st)
+                    : launch_variant<16, false>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st);
 }
 
 }  // namespace rola

@@ -12,6 +12,8 @@
 #include "rola_internal.cuh"
 #include "warp_mma.cuh"
 
+#include <cuda_fp8.h>
+
 namespace rola {
 namespace {
 
@@ -60,12 +62,12 @@ struct LSSmem {
 //   C: S += R(F)^T V_tile  (warp w: d columns [w*D/4, (w+1)*D/4))    2 x mma m16n8k16
 // The kernel also writes the fp16 copy of v that the attention kernel multiplies the
 // fp16 softmax weights with, and flags values outside the fp16 range.
-template <int D, int RK>
+template <int D, int RK, bool FP8>
 __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin,
     const __nv_bfloat16* __restrict__ Wk, Dims dm, const float2* __restrict__ rope,
     float* __restrict__ S_part, float* __restrict__ z_part, __half* __restrict__ v16,
-    int* __restrict__ status) {
+    uint8_t* __restrict__ v8, float* __restrict__ sv, int* __restrict__ status) {
   using L = LSSmem<D, RK>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem_raw);
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* tK = sK + stage * L::kTileElems;
     const __nv_bfloat16* tV = sV + stage * L::kTileElems;
 
-    // fp16 copy of the V tile (+ range check)
-    {
+    if constexpr (!FP8) {
+      // fp16 copy of the V tile (+ range check)
       constexpr int kVecPerRow = D / 8;
       const int n0 = n_begin + tile * kLSTile;
       bool bad = false;
@@ -155,6 +157,42 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
             packed;
       }
       if (bad) record_status(status, kDevRange);
+    } else {
+      // e4m3 copy of the V tile: the tile is one 64-token block; scale = absmax / 448.
+      constexpr int kVecPerRow = D / 8;
+      const int n0 = n_begin + tile * kLSTile;
+      float amax = 0.f;
+      for (int e = tid; e < kLSTile * kVecPerRow; e += 128) {
+        const int rr = e / kVecPerRow, cv = e % kVecPerRow;
+        if (n0 + rr >= n_end) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(tV + rr * L::DP + cv * 8);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[t] << 16)), fabsf(__uint_as_float(w[t] & 0xffff0000u))));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      if (lane == 0) sZ[warp] = amax;   // sZ is free until the end of the chunk loop
+      __syncthreads();
+      amax = fmaxf(fmaxf(sZ[0], sZ[1]), fmaxf(sZ[2], sZ[3]));
+      __syncthreads();
+      const float scale = amax > 0.f ? amax / 448.f : 1.f, inv = 1.f / scale;
+      if (tid == 0) sv[(size_t)bh * dm.nb + n0 / kLSTile] = scale;
+      for (int e = tid; e < kLSTile * kVecPerRow; e += 128) {
+        const int rr = e / kVecPerRow, cv = e % kVecPerRow, n = n0 + rr;
+        if (n >= n_end) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(tV + rr * L::DP + cv * 8);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t o[2] = {0, 0};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = make_float2(__uint_as_float(w[t] << 16) * inv, __uint_as_float(w[t] & 0xffff0000u) * inv);
+          o[t >> 1] |= (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3) << (16 * (t & 1));
+        }
+        *reinterpret_cast<uint2*>(v8 + ((size_t)b * dm.N + n) * row_stride + (size_t)h * D + cv * 8) =
+            make_uint2(o[0], o[1]);
+      }
     }
 
     // A: F = K Wk
@@ -381,13 +419,23 @@ cudaError_t launch_ls(const Dims& dm, rola_dtype dt, const void* k, const void* 
         dm, ws.rope, ws.S_part, ws.z_part);
   } else {
     const size_t smem = LSSmem<D, RK>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(linear_state_bf16_kernel<D, RK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    linear_state_bf16_kernel<D, RK><<<grid, 128, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.v16,
-        ws.status);
+    if (dt == ROLA_FP8_E4M3) {
+      cudaError_t e = cudaFuncSetAttribute(linear_state_bf16_kernel<D, RK, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      linear_state_bf16_kernel<D, RK, true><<<grid, 128, smem, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, nullptr, ws.v8,
+          ws.sv, ws.status);
+    } else {
+      cudaError_t e = cudaFuncSetAttribute(linear_state_bf16_kernel<D, RK, false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      linear_state_bf16_kernel<D, RK, false><<<grid, 128, smem, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.v16, nullptr,
+          nullptr, ws.status);
+    }
   }
   return cudaGetLastError();
 }

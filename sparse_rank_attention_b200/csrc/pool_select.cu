@@ -9,6 +9,8 @@
 // The kernels reproduce a stated fp32 order exactly, so the block lists are bit-exact:
 //   qbar = (fp32 sum of the block's tokens in token order) / count   (IEEE division)
 //   s_ij = fma chain over channels 0..d-1 starting from 0
+#include <cuda_fp8.h>
+
 #include <mutex>
 
 #include "rola_internal.cuh"
@@ -29,6 +31,8 @@ struct PoolTraits<float> {
     acc[2] = acc[2] + __uint_as_float(v.z);
     acc[3] = acc[3] + __uint_as_float(v.w);
   }
+  __device__ static float absmax(const uint4&) { return 0.f; }        // fp8 takes bf16 only
+  __device__ static uint2 to_e4m3(const uint4&, float) { return make_uint2(0, 0); }
 };
 template <>
 struct PoolTraits<__nv_bfloat16> {
@@ -41,14 +45,38 @@ struct PoolTraits<__nv_bfloat16> {
       acc[2 * e + 1] = acc[2 * e + 1] + __uint_as_float(w[e] & 0xffff0000u);
     }
   }
+  __device__ static float absmax(const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[e] << 16)), fabsf(__uint_as_float(w[e] & 0xffff0000u))));
+    return m;
+  }
+  // 8 bf16 values times `inv`, rounded to e4m3 (nearest, saturating), in element order.
+  __device__ static uint2 to_e4m3(const uint4& v, float inv) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = make_float2(__uint_as_float(w[e] << 16) * inv, __uint_as_float(w[e] & 0xffff0000u) * inv);
+      const uint32_t pair = (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+      out[e >> 1] |= pair << (16 * (e & 1));
+    }
+    return make_uint2(out[0], out[1]);
+  }
 };
 
 // grid: x = vector-column tiles of 128 threads over H*d, y = block i, z = 2*b + tensor.
 // One thread owns one 16-byte column vector and adds the block's tokens in order.
-template <typename T>
+// With FP8 (bf16 inputs only) the same CTA also quantises the block to e4m3: per
+// (b, h, block) scale = absmax / 448 (1 if the block is all zero), x8 = RN-sat(x / scale).
+template <typename T, bool FP8>
 __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                    Dims dm, float* __restrict__ qbar,
-                                                   float* __restrict__ kbar) {
+                                                   float* __restrict__ kbar, uint8_t* __restrict__ q8,
+                                                   uint8_t* __restrict__ k8, float* __restrict__ sq,
+                                                   float* __restrict__ sk) {
   constexpr int EPV = PoolTraits<T>::kEPV;
   constexpr int kBatch = 8;
   const int tensor = blockIdx.z & 1, b = blockIdx.z >> 1;
@@ -56,30 +84,52 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, cons
   float* __restrict__ xb = tensor ? kbar : qbar;
   const int HD = dm.H * dm.d;
   const int vcol = blockIdx.x * blockDim.x + threadIdx.x;
-  if (vcol * EPV >= HD) return;
+  const bool active = vcol * EPV < HD;
+  if (!FP8 && !active) return;
   const int i = blockIdx.y;
   const int n0 = i * kBlock, cnt = min(dm.N - n0, kBlock);
   const uint4* __restrict__ src =
       reinterpret_cast<const uint4*>(x + ((size_t)b * dm.N + n0) * HD) + vcol;
   const size_t vstride = (size_t)HD / EPV;
   float acc[EPV];
+  float amax = 0.f;
 #pragma unroll
   for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
-  for (int t0 = 0; t0 < cnt; t0 += kBatch) {
-    uint4 buf[kBatch];
+  if (active) {
+    for (int t0 = 0; t0 < cnt; t0 += kBatch) {
+      uint4 buf[kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (t0 + u < cnt) buf[u] = __ldg(src + (size_t)(t0 + u) * vstride);
+      for (int u = 0; u < kBatch; ++u)
+        if (t0 + u < cnt) buf[u] = __ldg(src + (size_t)(t0 + u) * vstride);
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (t0 + u < cnt) PoolTraits<T>::add(acc, buf[u]);
+      for (int u = 0; u < kBatch; ++u)
+        if (t0 + u < cnt) {
+          PoolTraits<T>::add(acc, buf[u]);
+          if (FP8) amax = fmaxf(amax, PoolTraits<T>::absmax(buf[u]));
+        }
+    }
+    const int c0 = vcol * EPV;
+    const int h = c0 / dm.d, ch = c0 % dm.d;
+    float* dst = xb + (((size_t)b * dm.H + h) * dm.nb + i) * dm.d + ch;
+    const float fc = (float)cnt;
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) dst[e] = __fdiv_rn(acc[e], fc);
   }
-  const int c0 = vcol * EPV;
-  const int h = c0 / dm.d, ch = c0 % dm.d;
-  float* dst = xb + (((size_t)b * dm.H + h) * dm.nb + i) * dm.d + ch;
-  const float fc = (float)cnt;
-#pragma unroll
-  for (int e = 0; e < EPV; ++e) dst[e] = __fdiv_rn(acc[e], fc);
+  if constexpr (FP8) {
+    // a head's d channels are d/8 consecutive threads (16 for d = 128, 8 for d = 64)
+    const int per_head = dm.d / EPV;
+    for (int off = 1; off < per_head; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (!active) return;
+    const int h = vcol * EPV / dm.d;
+    const float scale = amax > 0.f ? amax / 448.f : 1.f;
+    const float inv = 1.f / scale;
+    if ((vcol % per_head) == 0) (tensor ? sk : sq)[((size_t)b * dm.H + h) * dm.nb + i] = scale;
+    uint8_t* dst8 = (tensor ? k8 : q8) + ((size_t)b * dm.N + n0) * HD + (size_t)vcol * EPV;
+    for (int t = 0; t < cnt; ++t) {
+      const uint4 v = __ldg(src + (size_t)t * vstride);
+      *reinterpret_cast<uint2*>(dst8 + (size_t)t * HD) = PoolTraits<T>::to_e4m3(v, inv);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ block scores
@@ -251,13 +301,19 @@ cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void
   const int HD = dm.H * dm.d;
   if (dt == ROLA_F32) {
     dim3 grid((HD / 4 + 127) / 128, dm.nb, 2 * dm.B);
-    pool_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(q),
-                                             static_cast<const float*>(k), dm, ws.qbar, ws.kbar);
+    pool_kernel<float, false><<<grid, 128, 0, st>>>(static_cast<const float*>(q),
+                                                    static_cast<const float*>(k), dm, ws.qbar,
+                                                    ws.kbar, nullptr, nullptr, nullptr, nullptr);
+  } else if (dt == ROLA_FP8_E4M3) {
+    dim3 grid((HD / 8 + 127) / 128, dm.nb, 2 * dm.B);
+    pool_kernel<__nv_bfloat16, true><<<grid, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), dm, ws.qbar,
+        ws.kbar, ws.q8, ws.k8, ws.sq, ws.sk);
   } else {
     dim3 grid((HD / 8 + 127) / 128, dm.nb, 2 * dm.B);
-    pool_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                     static_cast<const __nv_bfloat16*>(k), dm,
-                                                     ws.qbar, ws.kbar);
+    pool_kernel<__nv_bfloat16, false><<<grid, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), dm, ws.qbar,
+        ws.kbar, nullptr, nullptr, nullptr, nullptr);
   }
   return cudaGetLastError();
 }
@@ -338,7 +394,8 @@ cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, 
   // The array keeps the previous call's contents: the status word must start at zero.
   e = cudaMemsetAsync(w.status, 0, 256, st);
   if (e != cudaSuccess) return e;
-  e = launch_pool(dm, dt, q, k, w, st);
+  // The selection does not depend on the fp8 copies; pool as for bf16 inputs.
+  e = launch_pool(dm, dt == ROLA_FP8_E4M3 ? ROLA_BF16 : dt, q, k, w, st);
   if (e != cudaSuccess) return e;
   return launch_select(dm, w, st);
 }

@@ -53,7 +53,7 @@ rola_status check_params(const rola_params* p) {
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return ROLA_ERR_INVALID_ARG;
   if (p->dtype != ROLA_F32 && p->dtype != ROLA_BF16 && p->dtype != ROLA_FP8_E4M3)
     return ROLA_ERR_INVALID_ARG;
-  if (p->dtype == ROLA_FP8_E4M3) return ROLA_ERR_UNSUPPORTED;
+  if (p->dtype == ROLA_FP8_E4M3 && p->d != 128) return ROLA_ERR_UNSUPPORTED;  // tcgen05 tile only
   const int nb = (p->N + rola::kBlock - 1) / rola::kBlock;
   if (nb > kMaxBlocks) return ROLA_ERR_UNSUPPORTED;
   if ((long long)p->B * p->H * nb > (1ll << 31) / 64) return ROLA_ERR_UNSUPPORTED;
@@ -243,8 +243,8 @@ rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const vo
   else if (p.d == 128) {
     e = rola::launch_query_features(plan->dm, q, Wq, g, plan->ws, st);
     if (e == cudaSuccess)
-      e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, plan->debug_flags,
-                                    plan->debug_limit_us, st);
+      e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, p.dtype == ROLA_FP8_E4M3,
+                                    plan->debug_flags, plan->debug_limit_us, st);
   }
   else  // head dim 64: the transposed tcgen05 tile needs d = 128 rows
     e = rola::launch_attend_bf16_warpmma(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
@@ -296,6 +296,22 @@ rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_str
   if (cudaMemcpyAsync(qbar, plan->ws.qbar, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return ROLA_ERR_CUDA;
   return cuda_status(cudaMemcpyAsync(kbar, plan->ws.kbar, bytes, cudaMemcpyDeviceToDevice, st));
+}
+
+rola_status rola_get_fp8_copies(rola_plan_t plan, uint8_t* q8, uint8_t* k8, uint8_t* v8, float* sq,
+                                float* sk, float* sv, rola_stream_t stream) {
+  if (!plan || !q8 || !k8 || !v8 || !sq || !sk || !sv) return ROLA_ERR_INVALID_ARG;
+  if (plan->p.dtype != ROLA_FP8_E4M3) return ROLA_ERR_INVALID_ARG;
+  const Dims& dm = plan->dm;
+  const size_t elems = (size_t)dm.B * dm.N * dm.H * dm.d;
+  const size_t sbytes = sizeof(float) * (size_t)dm.B * dm.H * dm.nb;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const struct { void* dst; const void* src; size_t n; } copies[6] = {
+      {q8, plan->ws.q8, elems}, {k8, plan->ws.k8, elems}, {v8, plan->ws.v8, elems},
+      {sq, plan->ws.sq, sbytes}, {sk, plan->ws.sk, sbytes}, {sv, plan->ws.sv, sbytes}};
+  for (const auto& c : copies)
+    if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return ROLA_ERR_CUDA;
+  return ROLA_OK;
 }
 
 rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream) {

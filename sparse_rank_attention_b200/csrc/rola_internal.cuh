@@ -87,7 +87,7 @@ cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void
                                        const void* v, const void* Wq, const float* g, void* out,
                                        const Workspace& ws, cudaStream_t st);
 cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
-                                void* out, int debug_flags, int debug_limit_us, cudaStream_t st);
+                                void* out, bool fp8, int debug_flags, int debug_limit_us, cudaStream_t st);
 cudaError_t launch_query_features(const Dims& dm, const void* q, const void* Wq, const float* g,
                                   const Workspace& ws, cudaStream_t st);
 size_t select_smem_bytes(const Dims& dm);

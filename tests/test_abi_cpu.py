@@ -95,3 +95,23 @@ def test_status_strings():
     for c in range(7):
         assert lib.rola_status_string(c)
     assert lib.rola_status_string(0) == b"ok"
+
+
+def test_fp8_configuration_host_rules():
+    lib = rola.load()
+    n = ctypes.c_size_t()
+    # the e4m3 path is the head-dim-128 tcgen05 kernel only
+    assert lib.rola_workspace_size(ctypes.byref(_params(d=64, dtype="fp8")), ctypes.byref(n)) == 2
+    p8 = _params(d=128, r=32, dtype="fp8")
+    pb = _params(d=128, r=32, dtype="bf16")
+    # fp8 carries three one-byte copies and three scale arrays instead of the fp16 copy of v
+    B, H, N, d = p8.B, p8.H, p8.N, p8.d
+    nb = (N + 63) // 64
+    extra = 3 * B * N * H * d + 3 * 4 * B * H * nb - 2 * B * N * H * d
+    assert abs(rola.workspace_size(p8) - rola.workspace_size(pb) - extra) <= 6 * 256
+    h = ctypes.c_void_p()
+    need = rola.workspace_size(pb)
+    assert lib.rola_plan(ctypes.byref(pb), ctypes.c_void_p(0x100000), need, ctypes.byref(h)) == 0
+    bufs = [ctypes.c_void_p(0x200000 + 0x10000 * j) for j in range(6)]
+    assert lib.rola_get_fp8_copies(h, *bufs, None) == 1      # not an fp8 plan
+    lib.rola_plan_destroy(h)
