@@ -139,37 +139,56 @@ def barrier(ws: int):
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def oracle_sample(w, seconds_hint=20.0, heads=1, seed=0):
-    """Times the oracle as it stands on a bounded sample of workload ``w``: ``heads`` heads
-    with their full pooling, selection and linear state, attention on a seeded set of
-    query blocks; the time is extrapolated to the full head."""
+def oracle_sample(w, seconds_hint=15.0, seed=0):
+    """Times the oracle as it stands on a bounded sample of workload ``w``, about
+    ``seconds_hint`` of CPU time: head after head (each with its full pooling, selection
+    and linear state), attention on a seeded set of query blocks that grows to the time
+    left; each head's time is extrapolated to all its query blocks."""
     import numpy as np
     import oracle as O
-    sub = synth.custom(w.name + "_sample", B=w.B, H=heads, N=w.N, d=w.d, r=w.r, topk=w.topk,
-                       grid=w.grid, dtype=w.dtype, dist=w.dist)
-    inp = synth.make_inputs(sub, seed=seed, device="cpu")
-    h = {k: v.float().numpy() for k, v in inp.items()}
-    s = O.make_shape(sub.B, sub.H, sub.N, sub.d, sub.r, sub.topk, grid=sub.grid)
-    t0 = time.perf_counter()
-    qbar, kbar = O.pool(s, h["q"]), O.pool(s, h["k"])
-    col, *_ = O.select(s, qbar, kbar)
-    S, z = O.linear_state(s, h["k"], h["v"], h["Wk"])
-    t_pre = time.perf_counter() - t0
-    rng = np.random.default_rng(seed)
-    nblk = max(8, min(w.nb, int(8 * O.threads())))
-    idx = sorted(set(rng.choice(w.nb, size=nblk, replace=False).tolist()))
-    blocks = np.array([(0, hh, i) for hh in range(heads) for i in idx], dtype=np.int32)
-    t1 = time.perf_counter()
-    O.attend_blocks(s, h["q"], h["k"], h["v"], h["Wq"], h["g"], col, S, z, blocks)
-    t_att = time.perf_counter() - t1
-    t_head = t_pre + t_att * (w.nb / len(idx))
-    c = np.full(w.nb, 64, dtype=np.int64)
-    c[-1] = w.N - 64 * (w.nb - 1)
-    flops = 4 * w.d * int((c[col[0]].sum(-1) * c[None, :]).sum())   # all heads of the sample
-    return {"value": flops / t_head / 1e12, "seconds": t_pre + t_att, "cores": O.threads(),
-            "sample": (f"{heads} of {w.H} heads: full pooling, block selection and linear state; "
-                       f"sparse+linear attention on {len(idx)} of {w.nb} query blocks, "
-                       f"time extrapolated to the whole head(s)")}
+    start = time.perf_counter()
+    t_sum = flops_sum = 0.0
+    heads = blocks_run = 0
+    for hh in range(w.H):
+        sub = synth.custom(w.name + "_sample", B=1, H=1, N=w.N, d=w.d, r=w.r, topk=w.topk,
+                           grid=w.grid, dtype=w.dtype, dist=w.dist)
+        inp = synth.make_inputs(sub, seed=1000 * seed + hh, device="cpu")
+        h = {k: v.float().numpy() for k, v in inp.items()}
+        s = O.make_shape(1, 1, sub.N, sub.d, sub.r, sub.topk, grid=sub.grid)
+        t0 = time.perf_counter()
+        qbar, kbar = O.pool(s, h["q"]), O.pool(s, h["k"])
+        col, *_ = O.select(s, qbar, kbar)
+        S, z = O.linear_state(s, h["k"], h["v"], h["Wk"])
+        t_pre = time.perf_counter() - t0
+        order = np.random.default_rng(seed + hh).permutation(w.nb)
+        n0 = max(8, min(w.nb, int(8 * O.threads())))
+
+        def run(sel):
+            blocks = np.array([(0, 0, i) for i in sorted(sel)], dtype=np.int32)
+            t = time.perf_counter()
+            O.attend_blocks(s, h["q"], h["k"], h["v"], h["Wq"], h["g"], col, S, z, blocks)
+            return time.perf_counter() - t
+
+        t_att = run(order[:n0].tolist())
+        left = seconds_hint - (time.perf_counter() - start)
+        n_more = max(0, min(w.nb - n0, int(left / (t_att / n0))))
+        if n_more > 0:
+            t_att += run(order[n0:n0 + n_more].tolist())
+        n = n0 + n_more
+        t_sum += t_pre + t_att * (w.nb / n)
+        c = np.full(w.nb, 64, dtype=np.int64)
+        c[-1] = w.N - 64 * (w.nb - 1)
+        flops_sum += 4 * w.d * int((c[col[0, 0]].sum(-1) * c).sum())
+        heads += 1
+        blocks_run += n
+        elapsed = time.perf_counter() - start
+        if elapsed >= 0.8 * seconds_hint or elapsed + t_pre + t_att * (w.nb / n) > 1.5 * seconds_hint:
+            break
+    return {"value": flops_sum / t_sum / 1e12, "seconds": time.perf_counter() - start,
+            "cores": O.threads(),
+            "sample": (f"{heads} of {w.H} heads, each with its full pooling, block selection and "
+                       f"linear state; sparse+linear attention on {blocks_run} of {heads * w.nb} "
+                       f"query blocks, each head's time extrapolated to all its blocks")}
 
 
 # ------------------------------------------------------------------ main
@@ -193,7 +212,7 @@ def main():
         vals = []
         samp = None
         for it in range(args.warmup + args.steps):
-            r = oracle_sample(w, seed=it)
+            r = oracle_sample(w, seconds_hint=max(2.0, 150.0 / (args.warmup + args.steps)), seed=it)
             if it >= args.warmup:
                 vals.append(r["value"])
                 samp = r
@@ -312,7 +331,7 @@ def main():
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        r = oracle_sample(w)
+        r = oracle_sample(w, seconds_hint=15.0)
         cpu = {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
                "sample": r["sample"], "seconds": r["seconds"]}
 

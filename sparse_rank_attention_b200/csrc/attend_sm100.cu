@@ -12,26 +12,27 @@
 // kept key blocks (M = 128 keys), and every MMA row does useful work:
 //   S^T [128 keys x 64 q]  = [K_j1; K_j2] Q_i^T            (bf16, K-major A and B)
 //   O^T [128 d x 64 q]    += [V_j1; V_j2]^T P^T            (fp16, MN-major A and B)
-// Thread t of the 4 softmax warps owns TMEM lane t: key t of the pair for S^T and
-// channel d = t for O^T.  The softmax max is per query (a TMEM column), so it is kept
-// lazily: each query's exponent offset m only moves when a new score exceeds it by
-// more than 8 (log2 units); that rare case takes an exact per-query max across the
-// 128 lanes and rescales O^T.  Per-query sums l stay per thread (partials over that
-// thread's keys) until the end.
+// The softmax runs in two independent groups of four warps; group g owns the query
+// columns [32g, 32g + 32) of S^T and O^T.  Thread t of a group owns TMEM lane t: key t of
+// the pair for S^T and channel d = t for O^T.  The softmax max is per query (a TMEM
+// column), so it is kept lazily: each query's exponent offset m only moves when a new
+// score exceeds it by more than 8 (log2 units); that rare case takes an exact per-query
+// max across the 128 lanes and rescales the group's O^T columns.  Per-query sums l stay
+// per thread (partials over that thread's keys) until the end.
 //
-// Roles (256 threads, one role per warp so that a sleeping wait never holds another
+// Roles (384 threads, one role per warp so that a sleeping wait never holds another
 // role back): warp 0 = TMA producer of Q and the K ring, warp 1 = Q K^T issuer (and TMEM
-// owner), warps 2-5 = softmax and epilogue, warp 6 = P V issuer, warp 7 = producer of
-// the epilogue operands and the V ring.  K pairs are
-// triple-buffered (freed when their QK is done), V pairs double-buffered, S^T
+// owner), warp 2 = P V issuer, warp 3 = producer of the epilogue operands and the V
+// ring, warps 4-11 = the two softmax groups (two softmax warps per SM sub-partition).
+// K and V pairs are double-buffered (K freed when its QK is done, V after its PV), S^T
 // triple-buffered in TMEM, so QK runs up to two pairs ahead of the softmax warps.
 //
 // Epilogue (per query block): num^T = S_h^T (R u)^T on the tensor cores, with S_h and
 // the rotated query features R u each as bf16 hi + lo (three MMAs); both operands, and
 // g/den per query, arrive as ready-made shared-memory images (state reduction and the
 // query-feature pre-pass write them) with one bulk copy issued in the prologue.
-// out = O/l + (g/den) num, staged in shared memory and written by one TMA store (rows
-// past N are clipped by the tensor map).
+// out = O/l + (g/den) num, staged in shared memory and written by TMA stores, one per
+// query group and channel half (rows past N are clipped by the tensor map).
 //
 // Every mbarrier wait is bounded (ROLA_ERR_DEVICE_TIMEOUT); on a timeout all roles
 // leave their loops, in-flight MMAs and TMA copies are drained and TMEM is freed.
@@ -47,7 +48,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: query columns 0-31, warps 8-11: columns 32-63
 constexpr uint32_t kTmemCols = 256;
 constexpr int kSBufs = 3;         // S^T buffers at columns 0, 64, 128
 constexpr uint32_t kColS = 0;
@@ -84,50 +86,13 @@ struct Ctl {
   int abort;
   alignas(16) float m_used[64];
   alignas(16) float fac[64];
-  float red[4][64];
+  alignas(16) float red[2][4][32];   // per query group: per-warp partial reductions
   alignas(16) float linv[64];
-  float vref[4];     // fp8: per-warp partial max of the kept blocks' V scales
+  float vref[2][4];  // fp8: per-warp partial max of the kept blocks' V scales
 };
 template <bool FP8>
 constexpr size_t smem_bytes() { return Geo<FP8>::kOffCtl + sizeof(Ctl) + 1024; }
 
-
-// Reduce 64 per-lane values over the 32 lanes of a warp; lane l receives the results
-// for entries 2l and 2l+1 (62 shuffles instead of 320).
-template <bool kMax>
-__device__ __forceinline__ float2 reduce_scatter64(const float* x, int lane) {
-  const unsigned full = 0xffffffffu;
-  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
-  float a[32], b[16], c[8], d[4];
-  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2, h1 = lane & 1;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const float mine = h16 ? x[32 + e] : x[e], send = h16 ? x[e] : x[32 + e];
-    a[e] = op(mine, __shfl_xor_sync(full, send, 16));
-  }
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float mine = h8 ? a[16 + e] : a[e], send = h8 ? a[e] : a[16 + e];
-    b[e] = op(mine, __shfl_xor_sync(full, send, 8));
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float mine = h4 ? b[8 + e] : b[e], send = h4 ? b[e] : b[8 + e];
-    c[e] = op(mine, __shfl_xor_sync(full, send, 4));
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float mine = h2 ? c[4 + e] : c[e], send = h2 ? c[e] : c[4 + e];
-    d[e] = op(mine, __shfl_xor_sync(full, send, 2));
-  }
-  float r[2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float mine = h1 ? d[2 + e] : d[e], send = h1 ? d[e] : d[2 + e];
-    r[e] = op(mine, __shfl_xor_sync(full, send, 1));
-  }
-  return make_float2(r[0], r[1]);
-}
 
 // 2^x on the special-function unit (ex2.approx: relative error ~2^-22, 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -176,23 +141,24 @@ __device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Writes one 128-byte row (64 16-bit values given as 32 packed words) of a
-// SW128 tile: 16-byte chunk c of row `row` goes to chunk position c ^ (row % 8).
-__device__ __forceinline__ void st_row_sw128(uint8_t* tile, int row, const uint32_t* w) {
+// Writes NC 16-byte chunks (4 packed words each), logical chunks c0 .. c0 + NC - 1 of
+// row `row` of a SW128 tile (128-byte rows): chunk c goes to position c ^ (row % 8).
+template <int NC>
+__device__ __forceinline__ void st_chunks_sw128(uint8_t* tile, int row, int c0, const uint32_t* w) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < NC; ++c) {
     uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-    *reinterpret_cast<uint4*>(tile + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+    *reinterpret_cast<uint4*>(tile + row * 128 + (((c0 + c) ^ (row & 7)) << 4)) = v;
   }
 }
 
-// Writes one 64-byte row (64 e4m3 values as 16 packed words) of a SW64 tile: 16-byte
-// chunk c of row `row` goes to chunk position c ^ ((row / 2) % 4).
-__device__ __forceinline__ void st_row_sw64(uint8_t* tile, int row, const uint32_t* w) {
+// The same for a SW64 tile (64-byte rows): chunk c goes to position c ^ ((row / 2) % 4).
+template <int NC>
+__device__ __forceinline__ void st_chunks_sw64(uint8_t* tile, int row, int c0, const uint32_t* w) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < NC; ++c) {
     uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-    *reinterpret_cast<uint4*>(tile + row * 64 + ((c ^ ((row >> 1) & 3)) << 4)) = v;
+    *reinterpret_cast<uint4*>(tile + row * 64 + (((c0 + c) ^ ((row >> 1) & 3)) << 4)) = v;
   }
 }
 
@@ -240,10 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(ctl->s_full[s]), 1);
-      mbar_init(bar(ctl->s_empty[s]), 128);
+      mbar_init(bar(ctl->s_empty[s]), 256);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(ctl->p_full[s]), 128);
+      mbar_init(bar(ctl->p_full[s]), 256);
       mbar_init(bar(ctl->pv_done[s]), 1);
     }
     mbar_init(bar(ctl->ep_full), 1);
@@ -254,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 2) {
+  if (warp == kSoftmaxWarp0) {
     ctl->m_used[lane] = 0.f;
     ctl->m_used[lane + 32] = 0.f;
   }
@@ -331,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       mma_commit(bar(ctl->drain_bar));       // no MMA may run when TMEM is freed
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
     }
-  } else if (warp == 6) {
+  } else if (warp == 2) {
     // ------------------------------------------------------------ P V issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = FP8 ? idesc_f8(128, 64, 1, 1) : idesc_f16(0, 128, 64, 1, 1);
@@ -359,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       mma_commit(bar(ctl->drain_bar));
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
     }
-  } else if (warp == 7) {
+  } else if (warp == 3) {
     // ------------------------------------------------------------ epilogue operands + V ring
     if (lane == 0) {
       const int xh = h * 128;
@@ -390,8 +356,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int wq = warp & 3;
+    // Two independent groups of four warps: group g owns query columns [32g, 32g + 32)
+    // of S^T and O^T (its own exponent offsets, sums, rescales and output rows), so two
+    // softmax warps share each SM sub-partition and hide each other's latencies.
+    const int g = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;                       // TMEM lane quadrant of this warp
     const int t = 32 * wq + lane;                  // TMEM lane: key of the pair / channel d
+    const int c0 = 32 * g;                         // first query column of the group
+    const uint32_t gbar = 1 + g;                   // the group's named barrier
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
     const float sl2 = dm.scale * 1.4426950408889634f;
     uint8_t* sP = base + kOffP;
@@ -400,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       WaitCtl dw{&ctl->abort, status, debug_limit_cycles};
       fail = !mbar_wait(bar(ctl->stall_bar), 0, dw);
     }
-    float lp[64];
+    float lp[32];
 #pragma unroll
-    for (int q = 0; q < 64; ++q) lp[q] = 0.f;
+    for (int q = 0; q < 32; ++q) lp[q] = 0.f;
 
     // fp8: the scores carry sq_i * sk_j, P carries sv_j / vref and the output vref, where
     // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
@@ -417,9 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) ctl->vref[wq] = mx;
-      named_sync(1, 128);
-      vref = fmaxf(fmaxf(ctl->vref[0], ctl->vref[1]), fmaxf(ctl->vref[2], ctl->vref[3]));
+      if (lane == 0) ctl->vref[g][wq] = mx;
+      named_sync(gbar, 128);
+      vref = fmaxf(fmaxf(ctl->vref[g][0], ctl->vref[g][1]), fmaxf(ctl->vref[g][2], ctl->vref[g][3]));
       if (!(vref > 0.f)) vref = 1.f;
     }
     // This thread's key block for pair `it` (-1: the padding half of an odd list) and,
@@ -442,9 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       fail |= !ok;
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads; invalid keys are masked after.
-      float x[64];
-      tmem_ld32(lane_addr + kColS + 64 * sb, x);
-      tmem_ld32(lane_addr + kColS + 64 * sb + 32, x + 32);
+      float x[32];
+      tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
       tmem_wait_ld();
       tc_fence_before();
       if (ok) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
@@ -462,10 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
       const float slt = FP8 ? sl2 * sqi * skj : sl2;
-      const float4* m4 = reinterpret_cast<const float4*>(ctl->m_used);
-      float dmax = -INFINITY;
+      const float4* m4 = reinterpret_cast<const float4*>(ctl->m_used + c0);
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
+      for (int q4 = 0; q4 < 8; ++q4) {
         const float4 m = m4[q4];
         x[4 * q4 + 0] = fmaf(x[4 * q4 + 0], slt, -m.x);
         x[4 * q4 + 1] = fmaf(x[4 * q4 + 1], slt, -m.y);
@@ -474,52 +444,67 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
       if (!valid) {
 #pragma unroll
-        for (int q = 0; q < 64; ++q) x[q] = -INFINITY;
+        for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
       }
+      float dmax = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 64; q += 4)
+      for (int q = 0; q < 32; q += 4)
         dmax = fmaxf(dmax, fmaxf(fmaxf(x[q], x[q + 1]), fmaxf(x[q + 2], x[q + 3])));
       // The first pair always sets the offsets; later pairs move them only when a score
       // exceeds its query's offset by more than 8 (P then stays within [0, 256]).
-      if (named_vote_or(1, 128, fail || it == 0 || dmax > 8.f)) {
-        if (named_vote_or(1, 128, fail)) break;
-        ctl->red[wq][lane] = reduce_scatter32<true>(x, lane);
-        ctl->red[wq][32 + lane] = reduce_scatter32<true>(x + 32, lane);
-        named_sync(1, 128);
-        if (t < 64) {
-          const float bm = fmaxf(fmaxf(ctl->red[0][t], ctl->red[1][t]), fmaxf(ctl->red[2][t], ctl->red[3][t]));
+      if (named_vote_or(gbar, 128, fail || it == 0 || dmax > 8.f)) {
+        if (named_vote_or(gbar, 128, fail)) break;
+        ctl->red[g][wq][lane] = reduce_scatter32<true>(x, lane);
+        named_sync(gbar, 128);
+        if (wq == 0) {                               // lane = query column c0 + lane
+          const float bm = fmaxf(fmaxf(ctl->red[g][0][lane], ctl->red[g][1][lane]),
+                                 fmaxf(ctl->red[g][2][lane], ctl->red[g][3][lane]));
           const float delta = it == 0 ? bm : fmaxf(bm, 0.f);
-          ctl->red[0][t] = delta;                    // reuse: shift of each query's offset
-          ctl->fac[t] = ex2_approx(-delta);
-          ctl->m_used[t] += delta;
+          ctl->red[g][0][lane] = delta;              // reuse: shift of each query's offset
+          ctl->fac[c0 + lane] = ex2_approx(-delta);
+          ctl->m_used[c0 + lane] += delta;
         }
-        named_sync(1, 128);
+        named_sync(gbar, 128);
+        const float4* d4 = reinterpret_cast<const float4*>(ctl->red[g][0]);
 #pragma unroll
-        for (int q = 0; q < 64; ++q) x[q] -= ctl->red[0][q];
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 dd = d4[q4];
+          x[4 * q4 + 0] -= dd.x;
+          x[4 * q4 + 1] -= dd.y;
+          x[4 * q4 + 2] -= dd.z;
+          x[4 * q4 + 3] -= dd.w;
+        }
         if (it > 0) {
+          const float4* f4 = reinterpret_cast<const float4*>(ctl->fac + c0);
+          float f[32];
 #pragma unroll
-          for (int q = 0; q < 64; ++q) lp[q] *= ctl->fac[q];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 ff = f4[q4];
+            f[4 * q4 + 0] = ff.x;
+            f[4 * q4 + 1] = ff.y;
+            f[4 * q4 + 2] = ff.z;
+            f[4 * q4 + 3] = ff.w;
+          }
+#pragma unroll
+          for (int q = 0; q < 32; ++q) lp[q] *= f[q];
           fail |= !mbar_wait(bar(ctl->pv_done[(it - 1) & 1]), ((it - 1) >> 1) & 1, wc);
           tc_fence_after();
+          float o[32];
+          tmem_ld32(lane_addr + kColO + c0, o);
+          tmem_wait_ld();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float o[32];
-            tmem_ld32(lane_addr + kColO + 32 * half, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) o[q] *= ctl->fac[32 * half + q];
-            tmem_st32(lane_addr + kColO + 32 * half, o);
-          }
+          for (int q = 0; q < 32; ++q) o[q] *= f[q];
+          tmem_st32(lane_addr + kColO + c0, o);
           tmem_wait_st();
         }
-        named_sync(1, 128);                          // red[0] is rewritten next time
+        named_sync(gbar, 128);                       // red[g][0] is rewritten next time
       }
       // P = 2^x (fp16, or e4m3 times sv_j / vref) and the per-thread partial row sums
-      uint32_t pw[32];
+      uint32_t pw[16];
       if constexpr (FP8) {
         const float pf = svj / vref;
 #pragma unroll
-        for (int q = 0; q < 64; q += 4) {
+        for (int q = 0; q < 32; q += 4) {
           const float p0 = ex2_approx(x[q]), p1 = ex2_approx(x[q + 1]);
           const float p2 = ex2_approx(x[q + 2]), p3 = ex2_approx(x[q + 3]);
           lp[q] += p0;
@@ -530,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < 64; q += 2) {
+        for (int q = 0; q < 32; q += 2) {
           const float p0 = ex2_approx(x[q]);
           const float p1 = ex2_approx(x[q + 1]);
           lp[q] += p0;
@@ -540,27 +525,28 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
       if (it > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[it & 1]), ((it - 2) >> 1) & 1, wc);
       if constexpr (FP8)
-        st_row_sw64(sP + (it & 1) * G::kPBytes, t, pw);
+        st_chunks_sw64<2>(sP + (it & 1) * G::kPBytes, t, 2 * g, pw);
       else
-        st_row_sw128(sP + (it & 1) * G::kPBytes, t, pw);
+        st_chunks_sw128<4>(sP + (it & 1) * G::kPBytes, t, 4 * g, pw);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(ctl->p_full[it & 1]));
     }
 
     // ------------------------------------------------------------ epilogue
-    if (!named_vote_or(1, 128, fail)) {
+    if (!named_vote_or(gbar, 128, fail)) {
+      // the last P V: also proves that both groups are done reading every S buffer
       fail |= !mbar_wait(bar(ctl->pv_done[(npairs - 1) & 1]), ((npairs - 1) >> 1) & 1, wc);
     }
-    if (!named_vote_or(1, 128, fail)) {
+    if (!named_vote_or(gbar, 128, fail)) {
       tc_fence_after();
-      // per-query sums l over the 128 threads
-      const float2 ls = reduce_scatter64<false>(lp, lane);
-      ctl->red[wq][2 * lane] = ls.x;
-      ctl->red[wq][2 * lane + 1] = ls.y;
-      named_sync(1, 128);
-      if (t < 64) ctl->linv[t] = vref / (ctl->red[0][t] + ctl->red[1][t] + ctl->red[2][t] + ctl->red[3][t]);
-      if (t == 0) {
+      // per-query sums l over the group's 128 threads
+      ctl->red[g][wq][lane] = reduce_scatter32<false>(lp, lane);
+      named_sync(gbar, 128);
+      if (wq == 0)
+        ctl->linv[c0 + lane] = vref / (ctl->red[g][0][lane] + ctl->red[g][1][lane] +
+                                       ctl->red[g][2][lane] + ctl->red[g][3][lane]);
+      if (g == 0 && t == 0) {
         fail |= !mbar_wait(bar(ctl->ep_full), 0, wc);
         tc_fence_after();
         constexpr uint32_t idesc_n = idesc_f16(1, 128, 64, 1, 1);
@@ -580,34 +566,33 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
       fail |= !mbar_wait(bar(ctl->ep_bar), 0, wc);
       fail |= !mbar_wait(bar(ctl->ep_full), 0, wc);     // g/den copy visible to every thread
-      if (!named_vote_or(1, 128, fail)) {
+      if (!named_vote_or(gbar, 128, fail)) {
         tc_fence_after();
-        // out^T[d = t][q] = O^T / l + (g / den) num^T -> staging [2 boxes][64 q][64 d]
+        // out^T[d = t][q] = O^T / l + (g / den) num^T -> staging [2 boxes][64 q][64 d],
+        // this group's rows c0 .. c0 + 31
         const float* gd = reinterpret_cast<const float*>(base + kOffGden);
         uint8_t* stg = base + kOffQ;
         __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(stg + (t >> 6) * 8192) + (t & 63);
+        float o[32], nm[32];
+        tmem_ld32(lane_addr + kColO + c0, o);
+        tmem_ld32(lane_addr + kColNum + c0, nm);
+        tmem_wait_ld();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float o[32], nm[32];
-          tmem_ld32(lane_addr + kColO + 32 * half, o);
-          tmem_ld32(lane_addr + kColNum + 32 * half, nm);
-          tmem_wait_ld();
-#pragma unroll
-          for (int qq4 = 0; qq4 < 8; ++qq4) {
-            const float4 li = reinterpret_cast<const float4*>(ctl->linv)[8 * half + qq4];
-            const float4 gg = reinterpret_cast<const float4*>(gd)[8 * half + qq4];
-            const int q0 = 32 * half + 4 * qq4, j = 4 * qq4;
-            col[(q0 + 0) * 64] = __float2bfloat16_rn(o[j + 0] * li.x + nm[j + 0] * gg.x);
-            col[(q0 + 1) * 64] = __float2bfloat16_rn(o[j + 1] * li.y + nm[j + 1] * gg.y);
-            col[(q0 + 2) * 64] = __float2bfloat16_rn(o[j + 2] * li.z + nm[j + 2] * gg.z);
-            col[(q0 + 3) * 64] = __float2bfloat16_rn(o[j + 3] * li.w + nm[j + 3] * gg.w);
-          }
+        for (int qq4 = 0; qq4 < 8; ++qq4) {
+          const float4 li = reinterpret_cast<const float4*>(ctl->linv + c0)[qq4];
+          const float4 gg = reinterpret_cast<const float4*>(gd + c0)[qq4];
+          const int q0 = c0 + 4 * qq4, j = 4 * qq4;
+          col[(q0 + 0) * 64] = __float2bfloat16_rn(o[j + 0] * li.x + nm[j + 0] * gg.x);
+          col[(q0 + 1) * 64] = __float2bfloat16_rn(o[j + 1] * li.y + nm[j + 1] * gg.y);
+          col[(q0 + 2) * 64] = __float2bfloat16_rn(o[j + 2] * li.z + nm[j + 2] * gg.z);
+          col[(q0 + 3) * 64] = __float2bfloat16_rn(o[j + 3] * li.w + nm[j + 3] * gg.w);
         }
         fence_proxy_async_smem();
-        named_sync(1, 128);
-        if (t == 0) {
-          tma_store_3d(&tm_out, h * 128, i * 64, b, sbase + kOffQ);
-          tma_store_3d(&tm_out, h * 128 + 64, i * 64, b, sbase + kOffQ + 8192);
+        named_sync(gbar, 128);
+        // rows at or past N are clipped by the tensor map; a box wholly past N is skipped
+        if (t == 0 && i * 64 + c0 < dm.N) {
+          tma_store_3d(&tm_out, h * 128, i * 64 + c0, b, sbase + kOffQ + c0 * 128);
+          tma_store_3d(&tm_out, h * 128 + 64, i * 64 + c0, b, sbase + kOffQ + 8192 + c0 * 128);
           tma_store_commit();
           tma_store_wait_read0();
         }
@@ -639,13 +624,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // [B, N, H*128] tensor as a 3D map with [64 tokens x 128 bytes] boxes (64 channels of a
 // 16-bit type, 128 of an 8-bit one).
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, const Dims& dm,
-              CUtensorMapSwizzle sw) {
+              CUtensorMapSwizzle sw, uint32_t box_rows = 64) {
   auto enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t HD = (cuuint64_t)dm.H * dm.d;
   cuuint64_t dims[3] = {HD, (cuuint64_t)dm.N, (cuuint64_t)dm.B};
   cuuint64_t strides[2] = {HD * el_bytes, HD * el_bytes * (cuuint64_t)dm.N};
-  cuuint32_t box[3] = {128 / el_bytes, 64, 1};
+  cuuint32_t box[3] = {128 / el_bytes, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -686,7 +671,8 @@ cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, co
     ok = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE);
+  // output: [32 tokens x 64 channels] boxes, one per query group and channel half
+  ok = ok && make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE, 32);
   if (!ok) return cudaErrorInvalidValue;
   if (fp8)
     return dm.r == 32 ? launch_variant<32, true>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st)

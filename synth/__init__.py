@@ -68,6 +68,8 @@ WORKLOADS = {
 for _t in (0.03, 0.05, 0.10, 0.25, 1.0):
     _n = f"wan21_14b_480p_topk{_t:g}"
     WORKLOADS[_n] = replace(WORKLOADS["wan21_14b_480p"], name=_n, topk=_t)
+WORKLOADS["wan21_14b_480p_fp8"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_480p_fp8",
+                                          dtype="fp8")
 WORKLOADS["wan21_14b_480p_dense_g0"] = replace(WORKLOADS["wan21_14b_480p"],
                                                name="wan21_14b_480p_dense_g0", topk=1.0,
                                                g_const=0.0)
