@@ -36,8 +36,8 @@ METRIC = "RoLA fwd kept-block TFLOP/s at Wan2.1-14B-720P shape, 1xB200"
 UNIT = "TFLOP/s"
 
 
-# pool, block scores, top-k | linear state, state reduction | query features, attention
-LAUNCHES_PER_STEP = 7
+# key/value pass, state reduction | query pass | block scores, top-k | attention
+LAUNCHES_PER_STEP = 6
 
 
 def load_peaks():
@@ -245,18 +245,8 @@ def main():
     q, k, v, Wq, Wk, g = (inp[x] for x in ("q", "k", "v", "Wq", "Wk", "g"))
     stream = torch.cuda.current_stream()
 
-    def step(evs=None):
-        if evs:
-            evs[0].record(stream)
-        plan.select_blocks(q, k)
-        if evs:
-            evs[1].record(stream)
-        plan.linear_state(k, v, Wk)
-        if evs:
-            evs[2].record(stream)
-        plan.attend(q, k, v, Wq, g, out)
-        if evs:
-            evs[3].record(stream)
+    def step():
+        plan.forward(q, k, v, Wq, Wk, g, out)
 
     for _ in range(args.warmup):
         step()
@@ -265,7 +255,7 @@ def main():
     flops = kept_block_flops(plan.block_lists(), w.N, w.d)
     att_flops = flops + linear_epilogue_flops(w)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    plan.profile_stages(True)      # events between the forward's stages (host call, untimed)
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
@@ -273,19 +263,21 @@ def main():
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for i in range(args.steps):
-            step(evs[i])
+            step()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(ws)
     ms_total = t0.elapsed_time(t1)
     ms_total_max = max_over_ranks(ms_total, ws)
     ms_step = ms_total_max / args.steps
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    stage_sum, ncalls = plan.stage_times()
+    plan.profile_stages(False)
+    stage_ms = [x / ncalls for x in stage_sum]
     assert plan.poll_status() == 0
     value = ws * flops / (ms_step * 1e-3) / 1e12
 
     peaks = load_peaks()
-    att_ms = stage_ms[2]
+    att_ms = stage_ms[-1]
     achieved = att_flops / (att_ms * 1e-3) / 1e12
     if w.dtype == "fp8":   # e4m3 products: the bf16 measurement times the nominal 4.5 / 2.25
         peak = 2.0 * peaks["bf16_tflops"]
@@ -296,9 +288,20 @@ def main():
     roof = {"bound": "tensor", "kernel": "attend (sparse branch + fused linear epilogue)",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": None, "peak_source": peak_src}
-    pool_bytes = 2 * w.B * w.N * w.H * w.d * 2
-    stages = {"select_blocks_ms": stage_ms[0], "linear_state_ms": stage_ms[1], "attend_ms": stage_ms[2],
-              "select_blocks_pool_read_GBs": pool_bytes / (stage_ms[0] * 1e-3) / 1e9}
+    act = w.B * w.N * w.H * w.d                     # elements of one activation tensor
+    nblk = w.B * w.H * plan.nb
+    if len(stage_ms) == 4:
+        # algorithmic HBM bytes: the key/value pass reads k, v and writes the fp16 copy of v
+        # (bf16) or the e4m3 k and v; the query pass reads q and writes the query-feature
+        # images, g/den, the q means (and e4m3 q)
+        kv_bytes = 2 * act * 2 + (2 * act if w.dtype == "fp8" else act * 2)
+        q_bytes = act * 2 + nblk * (2 * w.r * 128 + 64 * 4 + w.d * 4) + (act if w.dtype == "fp8" else 0)
+        stages = {"kv_pass_ms": stage_ms[0], "query_pass_ms": stage_ms[1], "select_ms": stage_ms[2],
+                  "attend_ms": stage_ms[3],
+                  "kv_pass_GBs": kv_bytes / (stage_ms[0] * 1e-3) / 1e9,
+                  "query_pass_GBs": q_bytes / (stage_ms[1] * 1e-3) / 1e9}
+    else:
+        stages = {"select_blocks_ms": stage_ms[0], "linear_state_ms": stage_ms[1], "attend_ms": stage_ms[2]}
 
     e2e = None
     if not args.no_e2e:

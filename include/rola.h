@@ -185,6 +185,24 @@ ROLA_API rola_status rola_poll_device_status(rola_plan_t plan, rola_stream_t str
 #define ROLA_DEBUG_STALL_WAIT 1
 ROLA_API rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us);
 
+/* Stage timing (no counterpart on the pages; a measurement aid).  With `enable` != 0 every
+ * later rola_forward on the plan records CUDA events on its stream between its stages
+ * (at most ROLA_PROFILE_CALLS calls are kept; later calls run unrecorded).  It does not
+ * change the work done.  Stages, for head dim 128 with bf16 or fp8 inputs:
+ *   0: key/value pass and state reduction (state, k means, v copy / e4m3 k and v)
+ *   1: query pass (q means, query features, e4m3 q)
+ *   2: block scores and top-k selection
+ *   3: attention (sparse branch with the fused linear epilogue)
+ * and for the other configurations: 0 selection, 1 linear state, 2 attention.
+ * Enabling creates the events (host call, synchronous); 0 destroys them.
+ * rola_get_stage_times synchronises on the last recorded event, writes into ms[s] the
+ * sum over the recorded calls of stage s's elapsed milliseconds (for s < max_stages),
+ * and reports the stage and call counts; it then clears the record. */
+#define ROLA_PROFILE_CALLS 64
+ROLA_API rola_status rola_profile_stages(rola_plan_t plan, int enable);
+ROLA_API rola_status rola_get_stage_times(rola_plan_t plan, float* ms, int max_stages, int* nstages,
+                                          int* ncalls);
+
 ROLA_API const char* rola_status_string(rola_status s);
 
 #ifdef __cplusplus

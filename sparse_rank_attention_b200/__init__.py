@@ -33,7 +33,8 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_plan_destroy", "rola_select_blocks", "rola_linear_state", "rola_attend",
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
-           "rola_select_blocks_noalloc", "rola_get_fp8_copies")
+           "rola_select_blocks_noalloc", "rola_get_fp8_copies", "rola_profile_stages",
+           "rola_get_stage_times")
 
 
 class RolaError(RuntimeError):
@@ -87,6 +88,9 @@ def load() -> ctypes.CDLL:
         "rola_set_debug": [P, i32, i32],
         "rola_select_blocks_noalloc": [pp, P, P, P, P],
         "rola_get_fp8_copies": [P, P, P, P, P, P, P, P],
+        "rola_profile_stages": [P, i32],
+        "rola_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32),
+                                 ctypes.POINTER(i32)],
     }.items():
         f = getattr(lib, name)
         f.argtypes = args
@@ -231,6 +235,18 @@ class Plan:
         _check(load().rola_get_fp8_copies(self._h, *[_ptr(t) for t in codes + scales], _stream(stream)),
                "rola_get_fp8_copies")
         return codes, scales
+
+    def profile_stages(self, enable: bool = True):
+        """Record CUDA events between the stages of later forward calls (see rola.h)."""
+        _check(load().rola_profile_stages(self._h, int(bool(enable))), "rola_profile_stages")
+
+    def stage_times(self) -> tuple[list[float], int]:
+        """(summed milliseconds per stage, number of recorded forward calls); clears the record."""
+        ms = (ctypes.c_float * 8)()
+        ns, nc = ctypes.c_int(), ctypes.c_int()
+        _check(load().rola_get_stage_times(self._h, ms, 8, ctypes.byref(ns), ctypes.byref(nc)),
+               "rola_get_stage_times")
+        return [ms[i] for i in range(ns.value)], nc.value
 
     def poll_status(self, stream=None) -> int:
         """Synchronises the stream; returns the device status code (0 = ok), clearing it."""

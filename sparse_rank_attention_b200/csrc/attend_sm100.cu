@@ -50,6 +50,7 @@ using namespace sm100;
 
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: query columns 0-31, warps 8-11: columns 32-63
+constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kSBufs = 3;         // S^T buffers at columns 0, 64, 128
 constexpr uint32_t kColS = 0;
@@ -206,10 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(bar(ctl->s_full[s]), 1);
-      mbar_init(bar(ctl->s_empty[s]), 256);
+      mbar_init(bar(ctl->s_empty[s]), kSoftmaxWarps);   // one arrive per softmax warp
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(ctl->p_full[s]), 256);
+      mbar_init(bar(ctl->p_full[s]), kSoftmaxWarps);
       mbar_init(bar(ctl->pv_done[s]), 1);
     }
     mbar_init(bar(ctl->ep_full), 1);
@@ -418,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
       tmem_wait_ld();
       tc_fence_before();
-      if (ok) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
       const int jb = jb_next;
       const float skj = sk_next, svj = sv_next;
       if (it + 1 < npairs) {
@@ -530,7 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         st_chunks_sw128<4>(sP + (it & 1) * G::kPBytes, t, 4 * g, pw);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(ctl->p_full[it & 1]));
+      __syncwarp();                                  // the warp's P rows and O^T rescale are done
+      if (lane == 0) mbar_arrive(bar(ctl->p_full[it & 1]));
     }
 
     // ------------------------------------------------------------ epilogue
@@ -609,34 +612,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// [B, N, H*128] tensor as a 3D map with [64 tokens x 128 bytes] boxes (64 channels of a
-// 16-bit type, 128 of an 8-bit one).
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, const Dims& dm,
-              CUtensorMapSwizzle sw, uint32_t box_rows = 64) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t HD = (cuuint64_t)dm.H * dm.d;
-  cuuint64_t dims[3] = {HD, (cuuint64_t)dm.N, (cuuint64_t)dm.B};
-  cuuint64_t strides[2] = {HD * el_bytes, HD * el_bytes * (cuuint64_t)dm.N};
-  cuuint32_t box[3] = {128 / el_bytes, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-
 template <int RK, bool FP8>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& to, const Dims& dm, const Workspace& ws, int debug_flags,
@@ -664,15 +639,15 @@ cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, co
   CUtensorMap tq, tk, tv, to;
   bool ok;
   if (fp8)
-    ok = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.q8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.k8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.v8, dm, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.q8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.k8, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws.v8, dm, CU_TENSOR_MAP_SWIZZLE_128B);
   else
-    ok = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B);
   // output: [32 tokens x 64 channels] boxes, one per query group and channel half
-  ok = ok && make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE, 32);
+  ok = ok && make_act_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE, 32);
   if (!ok) return cudaErrorInvalidValue;
   if (fp8)
     return dm.r == 32 ? launch_variant<32, true>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st)

@@ -7,8 +7,9 @@
 // positions restores global context); README sparse-finetuning section (proj_k);
 // citation block "RoPeSLR: 3D RoPE-driven Sparse-LowRank Attention" (3D rotary).
 //
-// Split-N: each CTA sums one 2048-token chunk into a partial; a second kernel adds the
-// partials in chunk order, so the result does not depend on scheduling.
+// Split-N: each CTA sums one chunk of tokens into a partial; a second kernel adds the
+// partials in chunk order, so the result does not depend on scheduling.  (For head dim
+// 128 with bf16 inputs the key/value pass computes the partials instead.)
 #include "rola_internal.cuh"
 #include "warp_mma.cuh"
 
@@ -81,8 +82,8 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
   const int g = lane >> 2, t4 = lane & 3;
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int b = bh / dm.H, h = bh % dm.H;
-  const int n_begin = chunk * kStateChunk;
-  const int n_end = min(dm.N, n_begin + kStateChunk);
+  const int n_begin = chunk * dm.chunk_tok;
+  const int n_end = min(dm.N, n_begin + dm.chunk_tok);
   const int ntiles = (n_end - n_begin + kLSTile - 1) / kLSTile;
   const size_t row_stride = (size_t)dm.H * D;  // elements between tokens
   const __nv_bfloat16* kbase = kin + ((size_t)b * dm.N) * row_stride + (size_t)h * D;
@@ -315,8 +316,8 @@ __global__ void __launch_bounds__(128) linear_state_f32_kernel(
   const int tid = threadIdx.x;
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int b = bh / dm.H, h = bh % dm.H;
-  const int n_begin = chunk * kStateChunk;
-  const int n_end = min(dm.N, n_begin + kStateChunk);
+  const int n_begin = chunk * dm.chunk_tok;
+  const int n_end = min(dm.N, n_begin + dm.chunk_tok);
   const size_t row_stride = (size_t)dm.H * D;
   for (int e = tid; e < D * RK; e += 128) sW[e / RK][e % RK] = Wk[(size_t)h * D * RK + e];
   constexpr int kPer = (RK * D + 127) / 128;
@@ -452,11 +453,16 @@ cudaError_t launch_rope_table(const Dims& dm, const Workspace& ws, cudaStream_t 
 cudaError_t launch_linear_state(const Dims& dm, rola_dtype dt, const void* k, const void* v,
                                 const void* Wk, const Workspace& ws, cudaStream_t st) {
   cudaError_t e;
-  if (dm.d == 128 && dm.r == 32) e = launch_ls<128, 32>(dm, dt, k, v, Wk, ws, st);
+  if (dm.d == 128 && dt != ROLA_F32) e = launch_kv_pass(dm, dt == ROLA_FP8_E4M3, k, v, Wk, ws, st);
+  else if (dm.d == 128 && dm.r == 32) e = launch_ls<128, 32>(dm, dt, k, v, Wk, ws, st);
   else if (dm.d == 128 && dm.r == 16) e = launch_ls<128, 16>(dm, dt, k, v, Wk, ws, st);
   else if (dm.d == 64 && dm.r == 32) e = launch_ls<64, 32>(dm, dt, k, v, Wk, ws, st);
   else e = launch_ls<64, 16>(dm, dt, k, v, Wk, ws, st);
   if (e != cudaSuccess) return e;
+  return launch_state_reduce(dm, ws, st);
+}
+
+cudaError_t launch_state_reduce(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   const int rd = dm.r * dm.d + dm.r;
   dim3 grid((rd + 255) / 256, dm.B * dm.H);
   state_reduce_kernel<<<grid, 256, 0, st>>>(dm, ws.S_part, ws.z_part, ws.S, ws.S_hi, ws.S_lo,

@@ -60,6 +60,28 @@ rola_status check_params(const rola_params* p) {
   return ROLA_OK;
 }
 
+// Tokens per linear-state partial.  The head-dim-128 key/value pass runs one CTA per SM
+// (148 SMs), so its chunk is chosen to fill the SMs in whole waves: the smallest
+// makespan (waves x blocks per chunk, plus one block of per-CTA overhead) over all
+// chunk lengths.  The other paths keep fixed 2048-token chunks.
+int state_chunk_tokens(const rola_params& p, int nb) {
+  if (!(p.d == 128 && p.dtype != ROLA_F32)) return rola::kStateChunk;
+  constexpr long long kSMs = 148;
+  const long long bh = (long long)p.B * p.H;
+  long long best_cost = -1;
+  int best = nb;
+  for (int cb = 1; cb <= nb; ++cb) {
+    const long long nchunk = (nb + cb - 1) / cb;
+    const long long waves = (bh * nchunk + kSMs - 1) / kSMs;
+    const long long cost = waves * (cb + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = cb;
+    }
+  }
+  return best * rola::kBlock;
+}
+
 Dims make_dims(const rola_params& p) {
   Dims dm{};
   dm.B = p.B; dm.H = p.H; dm.N = p.N; dm.d = p.d; dm.r = p.r;
@@ -73,7 +95,8 @@ Dims make_dims(const rola_params& p) {
   }
   dm.rope_off_h = dm.gt * dm.pt;
   dm.rope_off_w = dm.rope_off_h + dm.gh * dm.ph;
-  dm.nchunk = (p.N + rola::kStateChunk - 1) / rola::kStateChunk;
+  dm.chunk_tok = state_chunk_tokens(p, dm.nb);
+  dm.nchunk = (p.N + dm.chunk_tok - 1) / dm.chunk_tok;
   dm.scale = p.softmax_scale > 0.f ? p.softmax_scale : (float)(1.0 / std::sqrt((double)p.d));
   dm.rope_base = p.rope_base;
   return dm;
@@ -196,7 +219,64 @@ rola_status rola_plan(const rola_params* p, void* workspace, size_t workspace_by
   return ROLA_OK;
 }
 
-void rola_plan_destroy(rola_plan_t plan) { delete plan; }
+namespace {
+constexpr int kProfSlots = 5;   // events per recorded forward (at most 4 stages)
+
+void destroy_profile(rola_plan_t plan) {
+  if (!plan->prof_events) return;
+  for (int e = 0; e < ROLA_PROFILE_CALLS * kProfSlots; ++e)
+    if (plan->prof_events[e]) cudaEventDestroy(plan->prof_events[e]);
+  delete[] plan->prof_events;
+  plan->prof_events = nullptr;
+  plan->prof_calls = 0;
+}
+
+// Records the boundary event `k` of the current recorded call (no-op when not profiling).
+void mark(rola_plan_t plan, int slot, int k, cudaStream_t st) {
+  if (plan->prof_events && slot >= 0) cudaEventRecord(plan->prof_events[slot * kProfSlots + k], st);
+}
+}  // namespace
+
+void rola_plan_destroy(rola_plan_t plan) {
+  if (!plan) return;
+  destroy_profile(plan);
+  delete plan;
+}
+
+rola_status rola_profile_stages(rola_plan_t plan, int enable) {
+  if (!plan) return ROLA_ERR_INVALID_ARG;
+  destroy_profile(plan);
+  if (!enable) return ROLA_OK;
+  plan->prof_events = new (std::nothrow) cudaEvent_t[ROLA_PROFILE_CALLS * kProfSlots]();
+  if (!plan->prof_events) return ROLA_ERR_INVALID_ARG;
+  for (int e = 0; e < ROLA_PROFILE_CALLS * kProfSlots; ++e)
+    if (cudaEventCreate(&plan->prof_events[e]) != cudaSuccess) {
+      destroy_profile(plan);
+      return ROLA_ERR_CUDA;
+    }
+  plan->prof_calls = 0;
+  return ROLA_OK;
+}
+
+rola_status rola_get_stage_times(rola_plan_t plan, float* ms, int max_stages, int* nstages, int* ncalls) {
+  if (!plan || !plan->prof_events || !nstages || !ncalls || (max_stages > 0 && !ms)) return ROLA_ERR_INVALID_ARG;
+  const int calls = plan->prof_calls, ns = plan->prof_stages;
+  *nstages = ns;
+  *ncalls = calls;
+  for (int s = 0; s < max_stages; ++s) ms[s] = 0.f;
+  if (calls == 0) return ROLA_OK;
+  if (cudaEventSynchronize(plan->prof_events[(calls - 1) * kProfSlots + ns]) != cudaSuccess) return ROLA_ERR_CUDA;
+  for (int c = 0; c < calls; ++c)
+    for (int s = 0; s < ns && s < max_stages; ++s) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, plan->prof_events[c * kProfSlots + s], plan->prof_events[c * kProfSlots + s + 1]) !=
+          cudaSuccess)
+        return ROLA_ERR_CUDA;
+      ms[s] += t;
+    }
+  plan->prof_calls = 0;
+  return ROLA_OK;
+}
 
 rola_status rola_select_blocks(rola_plan_t plan, const void* q, const void* k,
                                rola_stream_t stream) {
@@ -241,7 +321,7 @@ rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const vo
   if (p.dtype == ROLA_F32)
     e = rola::launch_attend_f32(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
   else if (p.d == 128) {
-    e = rola::launch_query_features(plan->dm, q, Wq, g, plan->ws, st);
+    e = rola::launch_query_features(plan->dm, p.dtype == ROLA_FP8_E4M3, q, Wq, g, plan->ws, st);
     if (e == cudaSuccess)
       e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, p.dtype == ROLA_FP8_E4M3,
                                     plan->debug_flags, plan->debug_limit_us, st);
@@ -259,13 +339,42 @@ rola_status rola_forward(rola_plan_t plan, const void* q, const void* k, const v
   const size_t act = (size_t)p.B * p.N * p.H * p.d * elem_size(p.dtype);
   if (overlaps(out, act, q, act) || overlaps(out, act, k, act) || overlaps(out, act, v, act))
     return ROLA_ERR_INVALID_ARG;
-  if (!aligned16(Wq) || !aligned16(Wk) || !aligned16(g) || !aligned16(out))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(Wq) || !aligned16(Wk) || !aligned16(g) ||
+      !aligned16(out))
     return ROLA_ERR_INVALID_ARG;
-  rola_status s = rola_select_blocks(plan, q, k, stream);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int slot = -1;
+  if (plan->prof_events && plan->prof_calls < ROLA_PROFILE_CALLS) slot = plan->prof_calls++;
+  if (!(p.d == 128 && p.dtype != ROLA_F32)) {
+    plan->prof_stages = 3;
+    mark(plan, slot, 0, st);
+    rola_status s = rola_select_blocks(plan, q, k, stream);
+    if (s != ROLA_OK) return s;
+    mark(plan, slot, 1, st);
+    s = rola_linear_state(plan, k, v, Wk, stream);
+    if (s != ROLA_OK) return s;
+    mark(plan, slot, 2, st);
+    s = rola_attend(plan, q, k, v, Wq, g, out, stream);
+    mark(plan, slot, 3, st);
+    return s;
+  }
+  // Head dim 128, bf16 / fp8: each input is read once before the attention kernel.
+  //   key/value pass (state partials, k means, v copy / e4m3 k and v) -> state reduction
+  //   -> query pass (q means, query features, e4m3 q) -> block scores -> top-k -> attention
+  plan->prof_stages = 4;
+  mark(plan, slot, 0, st);
+  rola_status s = rola_linear_state(plan, k, v, Wk, stream);
   if (s != ROLA_OK) return s;
-  s = rola_linear_state(plan, k, v, Wk, stream);
-  if (s != ROLA_OK) return s;
-  return rola_attend(plan, q, k, v, Wq, g, out, stream);
+  mark(plan, slot, 1, st);
+  const bool fp8 = p.dtype == ROLA_FP8_E4M3;
+  cudaError_t e = rola::launch_query_features(plan->dm, fp8, q, Wq, g, plan->ws, st);
+  mark(plan, slot, 2, st);
+  if (e == cudaSuccess) e = rola::launch_select(plan->dm, plan->ws, st);
+  mark(plan, slot, 3, st);
+  if (e == cudaSuccess)
+    e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, fp8, plan->debug_flags, plan->debug_limit_us, st);
+  mark(plan, slot, 4, st);
+  return cuda_status(e);
 }
 
 rola_status rola_select_blocks_noalloc(const rola_params* p, const void* q, const void* k,

@@ -1,6 +1,7 @@
 // Internal declarations of the RoLA forward library (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -11,7 +12,7 @@
 namespace rola {
 
 constexpr int kBlock = 64;         // tokens per block
-constexpr int kStateChunk = 2048;  // tokens per linear-state partial sum
+constexpr int kStateChunk = 2048;  // tokens per linear-state partial sum (fp32 and d = 64 paths)
 
 // Device status word values (mirror rola_status codes).
 constexpr int kDevOk = 0;
@@ -26,6 +27,7 @@ struct Dims {
   int gt, gh, gw;             // latent grid
   int pt, ph, pw;             // rotary pairs per axis
   int rope_off_h, rope_off_w; // table offsets of the h and w axes (t starts at 0)
+  int chunk_tok;              // tokens per linear-state partial sum (a multiple of 64)
   int nchunk;                 // linear-state partial sums per (b, h)
   float scale;                // softmax logit scale
   double rope_base;
@@ -69,6 +71,10 @@ struct rola_plan_s {
   int debug_limit_us;
   bool status_ready;  // status word zeroed on the device
   bool rope_ready;    // rotary table written
+  // stage timing (rola_profile_stages): ROLA_PROFILE_CALLS x (stages + 1) events
+  cudaEvent_t* prof_events;
+  int prof_calls;     // forwards recorded since the last read
+  int prof_stages;    // stages of the recorded configuration
 };
 
 namespace rola {
@@ -88,8 +94,15 @@ cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void
                                        const Workspace& ws, cudaStream_t st);
 cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
                                 void* out, bool fp8, int debug_flags, int debug_limit_us, cudaStream_t st);
-cudaError_t launch_query_features(const Dims& dm, const void* q, const void* Wq, const float* g,
+cudaError_t launch_query_features(const Dims& dm, bool fp8, const void* q, const void* Wq, const float* g,
                                   const Workspace& ws, cudaStream_t st);
+cudaError_t launch_kv_pass(const Dims& dm, bool fp8, const void* k, const void* v, const void* Wk,
+                           const Workspace& ws, cudaStream_t st);
+cudaError_t launch_state_reduce(const Dims& dm, const Workspace& ws, cudaStream_t st);
+// TMA descriptor of a [B, N, H*d] activation tensor: boxes of box_rows tokens x 128
+// bytes (64 channels of a 16-bit type, 128 of an 8-bit one).  False if encoding fails.
+bool make_act_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, const Dims& dm,
+                  CUtensorMapSwizzle sw, uint32_t box_rows = 64);
 size_t select_smem_bytes(const Dims& dm);
 int score_row_stride(const Dims& dm);
 size_t select_noalloc_bytes(const Dims& dm);
@@ -115,6 +128,25 @@ __device__ __forceinline__ float2 rope_cs(const Dims& dm, const float2* __restri
     int x = n % dm.gw;
     return rope[dm.rope_off_w + x * dm.pw + (c - dm.pt - dm.ph)];
   }
+}
+
+// Rotary-table offsets of token n's t, h and w positions (one division chain per token).
+struct TokPos {
+  int t, y, x;
+};
+__device__ __forceinline__ TokPos token_pos(const Dims& dm, int n) {
+  const int hw = dm.gh * dm.gw;
+  const int t = n / hw, rem = n - t * hw;
+  const int y = rem / dm.gw;
+  return {t * dm.pt, dm.rope_off_h + y * dm.ph, dm.rope_off_w + (rem - y * dm.gw) * dm.pw};
+}
+
+// Rotary cos/sin of pair c at a token position (same values as rope_cs).
+__device__ __forceinline__ float2 rope_at(const Dims& dm, const float2* __restrict__ rope, const TokPos& p,
+                                          int c) {
+  if (c < dm.pt) return rope[p.t + c];
+  if (c < dm.pt + dm.ph) return rope[p.y + (c - dm.pt)];
+  return rope[p.x + (c - dm.pt - dm.ph)];
 }
 
 // phi(x) = elu(x) + 1.

@@ -75,15 +75,17 @@ struct WaitCtl {
   unsigned long long limit_cycles;
 };
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& w,
-                                            bool honour_abort) {
+// Slow path, out of line; arguments by value so that the call needs no stack frame.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                   int* status, unsigned long long limit_cycles,
+                                                   bool honour_abort) {
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;   // sleeps up to 0.2 ms
-    if (honour_abort && *w.abort) return false;
-    if ((unsigned long long)(clock64() - t0) > w.limit_cycles) {
-      *w.abort = 1;
-      atomicCAS(w.status, 0, 5 /* ROLA_ERR_DEVICE_TIMEOUT */);
+    if (honour_abort && *abort) return false;
+    if ((unsigned long long)(clock64() - t0) > limit_cycles) {
+      *abort = 1;
+      atomicCAS(status, 0, 5 /* ROLA_ERR_DEVICE_TIMEOUT */);
       return false;
     }
   }
@@ -92,7 +94,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w,
                                           bool honour_abort = true) {
   if (mbar_test_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, w, honour_abort);
+  return mbar_wait_slow(bar, parity, w.abort, w.status, w.limit_cycles, honour_abort);
 }
 
 // ------------------------------------------------------------------ fences / barriers
