@@ -18,8 +18,9 @@
 // flow through a 4-stage ring of TMA copies completing on mbarriers, so three tiles are in
 // flight while one is processed; rows past N arrive as zeros.
 // Per tile: warps 0-3 compute F = K Wk (mma.sync), phi, z and the rotation and store
-// the rotated features as bf16 hi + lo; warps 4-7 meanwhile pool k and write the copies
-// of v (or k and v in e4m3); then all 8 warps add F^T V into their 16 columns of S.
+// the rotated features as bf16 hi + lo; meanwhile warps 4-5 pool k (and write its e4m3
+// copy) and warps 6-7 write the copy of v; then all 8 warps add F^T V into their 16
+// columns of S.
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "warp_mma.cuh"
@@ -195,8 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1) kv_pass_kernel(
         const TokPos pos = token_pos(dm, valid ? n : 0);
 #pragma unroll
         for (int nt = 0; nt < NT_F; ++nt) {
-          const float x0 = valid ? phi(f[nt][2 * half]) : 0.f;
-          const float x1 = valid ? phi(f[nt][2 * half + 1]) : 0.f;
+          const float x0 = valid ? phi_fast(f[nt][2 * half]) : 0.f;
+          const float x1 = valid ? phi_fast(f[nt][2 * half + 1]) : 0.f;
           zacc[nt][0] += x0;
           zacc[nt][1] += x1;
           const float2 cs = valid ? rope_at(dm, rope, pos, nt * 4 + t4) : make_float2(1.f, 0.f);
@@ -208,64 +209,80 @@ __global__ void __launch_bounds__(kThreads, 1) kv_pass_kernel(
           *reinterpret_cast<uint32_t*>(sFl + row * L::RP + nt * 8 + 2 * t4) = lo;
         }
       }
-    } else {
-      // ---- pooling of k (column c, tokens in order), copies of v (and k)
-      const int c = tid - 128;                      // channel 0..127
+    } else if (warp < 6) {
+      // ---- pooling of k: thread = two adjacent channels, tokens added in order
+      const int cp = tid - 128;                     // channel pair 0..63
       const int blk = n0 / kTok;
-      float acc = 0.f, amk = 0.f, amv = 0.f;
+      float a0 = 0.f, a1 = 0.f, am = 0.f;
+      const uint8_t* col = pK + (cp >> 5) * 8192 + (cp & 3) * 4;   // box, word in chunk
+      const int ch = (cp >> 2) & 7;                                 // chunk within the box
       for (int r = 0; r < cnt; ++r) {
-        const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(pK + swz(r, c >> 3) + (c & 7) * 2));
-        acc = acc + x;
-        if (FP8) {
-          amk = fmaxf(amk, fabsf(x));
-          amv = fmaxf(amv, fabsf(__bfloat162float(
-                               *reinterpret_cast<const __nv_bfloat16*>(pV + swz(r, c >> 3) + (c & 7) * 2))));
-        }
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(col + r * 128 + ((ch ^ (r & 7)) << 4));
+        const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
+        a0 = a0 + x0;
+        a1 = a1 + x1;
+        if (FP8) am = fmaxf(am, fmaxf(fabsf(x0), fabsf(x1)));
       }
-      kbar[((size_t)bh * dm.nb + blk) * kD + c] = __fdiv_rn(acc, (float)cnt);
+      *reinterpret_cast<float2*>(kbar + ((size_t)bh * dm.nb + blk) * kD + 2 * cp) =
+          make_float2(__fdiv_rn(a0, (float)cnt), __fdiv_rn(a1, (float)cnt));
+      if constexpr (FP8) {
+        // e4m3 copy of the k tile: block scale from the max over the two warps
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) sRed[warp - 4] = am;
+        asm volatile("bar.sync 1, 64;" ::: "memory");
+        am = fmaxf(sRed[0], sRed[1]);
+        const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;
+        if (cp == 0) sk[(size_t)bh * dm.nb + blk] = sc;
+        for (int e = cp; e < cnt * 16; e += 64) {
+          const int r = e >> 4, cv = e & 15;
+          *reinterpret_cast<uint2*>(k8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+              e4m3x8(*reinterpret_cast<const uint4*>(pK + swz(r, cv)), inv);
+        }
+        asm volatile("bar.sync 1, 64;" ::: "memory");   // sRed is rewritten next tile
+      }
+    } else {
+      // ---- copy of v: fp16 (bf16 configuration) or e4m3 with its block scale (fp8)
+      const int tv = tid - 192;                     // 0..63
       if constexpr (!FP8) {
         bool bad = false;
-        for (int e = c; e < cnt * 16; e += 128) {
+        for (int e = tv; e < cnt * 16; e += 64) {
           const int r = e >> 4, cv = e & 15;
           const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(r, cv));
-          const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(&raw);
-          uint4 packed;
-          __half2* dst = reinterpret_cast<__half2*>(&packed);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float2 fv = __bfloat1622float2(src[u]);
-            bad |= !(fabsf(fv.x) <= 65504.f) || !(fabsf(fv.y) <= 65504.f);
-            dst[u] = __floats2half2_rn(fv.x, fv.y);
+            // |x| >= 65536 (bf16 0x4780 and up, inf, nan) does not fit fp16; below that
+            // every bf16 value rounds to fp16 within its range
+            bad |= ((w[u] & 0x7fffu) >= 0x4780u) || (((w[u] >> 16) & 0x7fffu) >= 0x4780u);
+            const __half2 hv = __floats2half2_rn(__uint_as_float(w[u] << 16), __uint_as_float(w[u] & 0xffff0000u));
+            o[u] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) = packed;
+          *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+              make_uint4(o[0], o[1], o[2], o[3]);
         }
         if (bad) record_status(status, kDevRange);
       } else {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          amk = fmaxf(amk, __shfl_xor_sync(0xffffffffu, amk, o));
-          amv = fmaxf(amv, __shfl_xor_sync(0xffffffffu, amv, o));
-        }
-        if (lane == 0) {
-          sRed[warp - 4] = amk;
-          sRed[4 + warp - 4] = amv;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        amk = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
-        amv = fmaxf(fmaxf(sRed[4], sRed[5]), fmaxf(sRed[6], sRed[7]));
-        const float sck = amk > 0.f ? amk / 448.f : 1.f, ink = 1.f / sck;
-        const float scv = amv > 0.f ? amv / 448.f : 1.f, inv = 1.f / scv;
-        if (c == 0) {
-          sk[(size_t)bh * dm.nb + blk] = sck;
-          sv[(size_t)bh * dm.nb + blk] = scv;
-        }
-        for (int e = c; e < cnt * 16; e += 128) {
+        float am = 0.f;
+        for (int e = tv; e < cnt * 16; e += 64) {
           const int r = e >> 4, cv = e & 15;
-          const size_t at = ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8;
-          *reinterpret_cast<uint2*>(k8 + at) = e4m3x8(*reinterpret_cast<const uint4*>(pK + swz(r, cv)), ink);
-          *reinterpret_cast<uint2*>(v8 + at) = e4m3x8(*reinterpret_cast<const uint4*>(pV + swz(r, cv)), inv);
+          am = fmaxf(am, absmax8(*reinterpret_cast<const uint4*>(pV + swz(r, cv))));
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // sRed is rewritten next tile
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) sRed[4 + warp - 6] = am;
+        asm volatile("bar.sync 2, 64;" ::: "memory");
+        am = fmaxf(sRed[4], sRed[5]);
+        const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;
+        const int blk = n0 / kTok;
+        if (tv == 0) sv[(size_t)bh * dm.nb + blk] = sc;
+        for (int e = tv; e < cnt * 16; e += 64) {
+          const int r = e >> 4, cv = e & 15;
+          *reinterpret_cast<uint2*>(v8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+              e4m3x8(*reinterpret_cast<const uint4*>(pV + swz(r, cv)), inv);
+        }
+        asm volatile("bar.sync 2, 64;" ::: "memory");
       }
     }
     __syncthreads();                 // sF complete

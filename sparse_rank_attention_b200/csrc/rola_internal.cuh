@@ -152,4 +152,12 @@ __device__ __forceinline__ float2 rope_at(const Dims& dm, const float2* __restri
 // phi(x) = elu(x) + 1.
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
+// The same with e^x for x <= 0 as 2^(x log2 e) on the special-function unit (relative
+// error ~2^-21: well inside what the bf16 paths keep of phi).
+__device__ __forceinline__ float phi_fast(float x) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * 1.4426950408889634f));
+  return x > 0.f ? x + 1.f : e;
+}
+
 }  // namespace rola
