@@ -51,11 +51,12 @@ using namespace sm100;
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: query columns 0-31, warps 8-11: columns 32-63
 constexpr int kSoftmaxWarps = 8;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;         // S^T buffers at columns 0, 64, 128
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 192;   // O^T
-constexpr uint32_t kColNum = 0;   // epilogue: num^T (reuses S buffer 0)
+constexpr uint32_t kColNum = 256; // epilogue: num^T (its own columns: the next tile's S^T
+                                  // are computed while a tile's epilogue runs)
 
 constexpr int kKStages = 2;                // K pairs: freed as soon as their QK is done
 constexpr int kVStages = 2;                // V pairs: freed after their PV
@@ -70,8 +71,9 @@ struct Geo {
   static constexpr uint32_t kPairBytes = 128 * 128 * kEl;         // K or V pair
   static constexpr uint32_t kBoxKV = FP8 ? 16384 : 16384;         // channel-box stride in a pair
   static constexpr uint32_t kPBytes = FP8 ? 8192 : 16384;         // one P^T buffer
-  static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = 16384;                         // K ring (1024-aligned)
+  static constexpr uint32_t kOffQ = 0;                             // 2 Q slots of 16 KB (each
+                                                                   // also its tile's out staging)
+  static constexpr uint32_t kOffK = 32768;                         // K ring (1024-aligned)
   static constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;  // V ring
   static constexpr uint32_t kOffP = kOffV + kVStages * kPairBytes;  // 2 x P^T (also out staging)
   static constexpr uint32_t kOffSimg = kOffP + 2 * 16384;           // S_h^T hi | lo (<= 16 KB)
@@ -81,7 +83,7 @@ struct Geo {
 };
 
 struct Ctl {
-  uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t q_full[2], q_free[2], k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[kSBufs], s_empty[kSBufs], p_full[2], pv_done[2], ep_full, ep_bar, drain_bar, stall_bar;
   uint32_t tmem_base;
   int abort;
@@ -188,15 +190,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   Ctl* ctl = reinterpret_cast<Ctl*>(base + kOffCtl);
   const uint32_t sbase = smem_addr(base);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / dm.H, h = bh % dm.H;
+  const int ntiles = dm.nb * dm.B * dm.H;        // tile = (b, h, query block i)
   const int kk_list = dm.k;
   const int npairs = (kk_list + 1) >> 1;
-  const int32_t* L = col_idx + ((size_t)bh * dm.nb + i) * kk_list;
   auto bar = [&](uint64_t& m) { return smem_addr(&m); };
+  // tile tau -> (b*H + h, i): consecutive tiles are consecutive query blocks of one head,
+  // so the CTAs working at one time share that head's key/value blocks in L2
+  auto tile_bh = [&](int tau) { return tau / dm.nb; };
+  auto list_of = [&](int tau) { return col_idx + (size_t)tau * kk_list; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(ctl->q_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ctl->q_full[s]), 1);
+      mbar_init(bar(ctl->q_free[s]), 2);                 // one arrive per softmax group
+    }
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(ctl->k_full[s]), 1);
       mbar_init(bar(ctl->k_empty[s]), 1);
@@ -221,10 +228,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == kSoftmaxWarp0) {
-    ctl->m_used[lane] = 0.f;
-    ctl->m_used[lane + 32] = 0.f;
-  }
   if (warp == 1) {
     tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
     tmem_relinquish();
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtl wc{&ctl->abort, status, limit_cycles};
-  auto pair_blocks = [&](int it, int& j1, int& j2) {
+  auto pair_blocks = [&](const int32_t* L, int it, int& j1, int& j2) {
     j1 = __ldg(L + 2 * it);
     j2 = (2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : j1;
     if (j1 < 0 || j1 >= dm.nb || j2 < 0 || j2 >= dm.nb) {
@@ -243,117 +246,161 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producers
-    const int xh = h * 128;
-    if (lane == 0) {               // Q and the K ring
+    // ------------------------------------------------------------ Q and the K ring
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      mbar_expect_tx(bar(ctl->q_full), G::kQBytes);
-      tma_load_3d(sbase + kOffQ, &tm_q, xh, i * 64, b, bar(ctl->q_full));
-      if (!FP8) tma_load_3d(sbase + kOffQ + 8192, &tm_q, xh + 64, i * 64, b, bar(ctl->q_full));
-      int issued = 0;
-      for (int it = 0; it < npairs; ++it) {
-        const int s = it % kKStages;
-        if (it >= kKStages && !mbar_wait(bar(ctl->k_empty[s]), ((it / kKStages) - 1) & 1, wc)) break;
-        int j1, j2;
-        pair_blocks(it, j1, j2);
-        const uint32_t st = sbase + kOffK + s * kPairBytes;
-        mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
-        for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
-          tma_load_3d(st + c * kBoxKV, &tm_k, xh + 64 * c, j1 * 64, b, bar(ctl->k_full[s]));
-          tma_load_3d(st + c * kBoxKV + 8192, &tm_k, xh + 64 * c, j2 * 64, b, bar(ctl->k_full[s]));
+      int nq = 0, gp = 0;               // Q tiles and K pairs issued
+      bool ok = true;
+      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x) {
+        const int bh = tile_bh(tau), i = tau - bh * dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        const int qb = nq & 1;
+        // the Q slot doubles as the output staging of the tile two back: wait for its store
+        if (nq >= 2 && !mbar_wait(bar(ctl->q_free[qb]), ((nq - 2) >> 1) & 1, wc)) break;
+        mbar_expect_tx(bar(ctl->q_full[qb]), G::kQBytes);
+        tma_load_3d(sbase + kOffQ + qb * 16384, &tm_q, xh, i * 64, b, bar(ctl->q_full[qb]));
+        if (!FP8) tma_load_3d(sbase + kOffQ + qb * 16384 + 8192, &tm_q, xh + 64, i * 64, b, bar(ctl->q_full[qb]));
+        ++nq;
+        for (int it = 0; it < npairs; ++it) {
+          const int s = gp % kKStages;
+          if (gp >= kKStages && !mbar_wait(bar(ctl->k_empty[s]), ((gp / kKStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + kOffK + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
+          for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_k, xh + 64 * c, j1 * 64, b, bar(ctl->k_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_k, xh + 64 * c, j2 * 64, b, bar(ctl->k_full[s]));
+          }
+          ++gp;
         }
-        issued = it + 1;
       }
       // Drain: every issued copy must land before the CTA leaves.
-      mbar_wait(bar(ctl->q_full), 0, wc, false);
-      for (int it = (issued > kKStages ? issued - kKStages : 0); it < issued; ++it)
-        mbar_wait(bar(ctl->k_full[it % kKStages]), (it / kKStages) & 1, wc, false);
+      for (int x = (nq > 2 ? nq - 2 : 0); x < nq; ++x) mbar_wait(bar(ctl->q_full[x & 1]), (x >> 1) & 1, wc, false);
+      for (int x = (gp > kKStages ? gp - kKStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->k_full[x % kKStages]), (x / kKStages) & 1, wc, false);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuers
-    if (lane == 0) {               // S^T = K_pair Q^T
+    // ------------------------------------------------------------ S^T = K_pair Q^T issuer
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = FP8 ? idesc_f8(128, 64, 0, 0) : idesc_f16(1, 128, 64, 0, 0);
-      bool ok = mbar_wait(bar(ctl->q_full), 0, wc);
-      const uint64_t dq = sdesc_sw128(sbase + kOffQ, 16, 1024);
-      for (int it = 0; ok && it < npairs; ++it) {
-        const int ks = it % kKStages, sb = it % kSBufs;
-        if (!mbar_wait(bar(ctl->k_full[ks]), (it / kKStages) & 1, wc)) { ok = false; break; }
-        if (it >= kSBufs && !mbar_wait(bar(ctl->s_empty[sb]), ((it / kSBufs) - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t da = sdesc_sw128(sbase + kOffK + ks * kPairBytes, 16, 1024);
-        if constexpr (FP8) {
+      int j = 0, gp = 0;
+      bool ok = true;
+      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x, ++j) {
+        const int qb = j & 1;
+        if (!mbar_wait(bar(ctl->q_full[qb]), (j >> 1) & 1, wc)) break;
+        const uint64_t dq = sdesc_sw128(sbase + kOffQ + qb * 16384, 16, 1024);
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int ks = gp % kKStages, sb = gp % kSBufs;
+          if (!mbar_wait(bar(ctl->k_full[ks]), (gp / kKStages) & 1, wc)) { ok = false; break; }
+          if (gp >= kSBufs && !mbar_wait(bar(ctl->s_empty[sb]), ((gp / kSBufs) - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = sdesc_sw128(sbase + kOffK + ks * kPairBytes, 16, 1024);
+          if constexpr (FP8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 32 e4m3 channels (32 B) per step, one box
-            mma_f8_ss(tmem + kColS + 64 * sb, da + ((kk * 32) >> 4), dq + ((kk * 32) >> 4), idesc_qk, kk > 0);
-        } else {
+            for (int kk = 0; kk < 4; ++kk)   // 32 e4m3 channels (32 B) per step, one box
+              mma_f8_ss(tmem + kColS + 64 * sb, da + ((kk * 32) >> 4), dq + ((kk * 32) >> 4), idesc_qk, kk > 0);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
-            mma_f16_ss(tmem + kColS + 64 * sb, da + (((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4),
-                       dq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+            for (int kk = 0; kk < 8; ++kk)   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
+              mma_f16_ss(tmem + kColS + 64 * sb, da + (((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4),
+                         dq + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+          }
+          mma_commit(bar(ctl->s_full[sb]));
+          mma_commit(bar(ctl->k_empty[ks]));
         }
-        mma_commit(bar(ctl->s_full[sb]));
-        mma_commit(bar(ctl->k_empty[ks]));
       }
       mma_commit(bar(ctl->drain_bar));       // no MMA may run when TMEM is freed
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ P V issuer
+    // ------------------------------------------------------------ O^T += V^T P^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = FP8 ? idesc_f8(128, 64, 1, 1) : idesc_f16(0, 128, 64, 1, 1);
-      for (int t = 0; t < npairs; ++t) {
-        const int s = t % kVStages, pb = t & 1;
-        if (!mbar_wait(bar(ctl->v_full[s]), (t / kVStages) & 1, wc)) break;
-        if (!mbar_wait(bar(ctl->p_full[pb]), (t >> 1) & 1, wc)) break;
-        const uint64_t db = FP8 ? sdesc_sw64(sbase + kOffP + pb * G::kPBytes, 4096, 512)
-                                : sdesc_sw128(sbase + kOffP + pb * G::kPBytes, 8192, 1024);
-        tc_fence_after();
-        // descriptors advance by 2048 bytes (16 K-rows) per step: +128 in the address field
-        const uint64_t da = sdesc_sw128(sbase + kOffV + s * kPairBytes, kBoxKV, 1024);
-        if constexpr (FP8) {
+      int gp = 0;
+      bool ok = true;
+      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x) {
+        for (int t = 0; t < npairs; ++t, ++gp) {
+          const int s = gp % kVStages, pb = gp & 1;
+          if (!mbar_wait(bar(ctl->v_full[s]), (gp / kVStages) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(bar(ctl->p_full[pb]), (gp >> 1) & 1, wc)) { ok = false; break; }
+          const uint64_t db = FP8 ? sdesc_sw64(sbase + kOffP + pb * G::kPBytes, 4096, 512)
+                                  : sdesc_sw128(sbase + kOffP + pb * G::kPBytes, 8192, 1024);
+          tc_fence_after();
+          // descriptors advance by 2048 bytes (16 K-rows) per step: +128 in the address field
+          const uint64_t da = sdesc_sw128(sbase + kOffV + s * kPairBytes, kBoxKV, 1024);
+          if constexpr (FP8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 32 keys per step: V rows of 128 B, P rows of 64 B
-            mma_f8_ss(tmem + kColO, da + 256 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
-        } else {
+            for (int kk = 0; kk < 4; ++kk)   // 32 keys per step: V rows of 128 B, P rows of 64 B
+              mma_f8_ss(tmem + kColO, da + 256 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_f16_ss(tmem + kColO, da + 128 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+            for (int kk = 0; kk < 8; ++kk)
+              mma_f16_ss(tmem + kColO, da + 128 * kk, db + 128 * kk, idesc_pv, (t > 0) || (kk > 0));
+          }
+          mma_commit(bar(ctl->pv_done[pb]));
+          mma_commit(bar(ctl->v_empty[s]));
         }
-        mma_commit(bar(ctl->pv_done[pb]));
-        mma_commit(bar(ctl->v_empty[s]));
       }
       mma_commit(bar(ctl->drain_bar));
       mbar_wait(bar(ctl->drain_bar), 0, wc, false);
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------ epilogue operands + V ring
+    // ------------------------------------------------------------ V ring + epilogue operands
     if (lane == 0) {
-      const int xh = h * 128;
+      tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_out);
       const uint32_t sbytes = 4 * RK * 128, ubytes = 2 * RK * 128;
-      mbar_expect_tx(bar(ctl->ep_full), sbytes + ubytes + 256);
-      bulk_load(sbase + kOffSimg, simg + (size_t)bh * sbytes, sbytes, bar(ctl->ep_full));
-      bulk_load(sbase + kOffUimg, uimg + ((size_t)bh * dm.nb + i) * ubytes, ubytes, bar(ctl->ep_full));
-      bulk_load(sbase + kOffGden, gden + ((size_t)bh * dm.nb + i) * 64, 256, bar(ctl->ep_full));
-      tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int it = 0; it < npairs; ++it) {
-        const int s = it % kVStages;
-        if (it >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((it / kVStages) - 1) & 1, wc)) break;
-        int j1, j2;
-        pair_blocks(it, j1, j2);
-        const uint32_t st = sbase + kOffV + s * kPairBytes;
-        mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
-        for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
-          tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
-          tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
+      int gp = 0, j = 0, nep = 0, prev_bh = -1;
+      bool ok = true;
+      // Epilogue operands of tile j go into single buffers once tile j - 1's epilogue is
+      // over (its output store has read the staging: everything before it is done too);
+      // S_h only when the head changes.
+      auto load_ep = [&](int tau) {
+        if (j >= 1 && !mbar_wait(bar(ctl->q_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, wc)) return false;
+        const int bh = tile_bh(tau);
+        const bool new_s = bh != prev_bh;
+        mbar_expect_tx(bar(ctl->ep_full), (new_s ? sbytes : 0) + ubytes + 256);
+        if (new_s) bulk_load(sbase + kOffSimg, simg + (size_t)bh * sbytes, sbytes, bar(ctl->ep_full));
+        bulk_load(sbase + kOffUimg, uimg + (size_t)tau * ubytes, ubytes, bar(ctl->ep_full));
+        bulk_load(sbase + kOffGden, gden + (size_t)tau * 64, 256, bar(ctl->ep_full));
+        prev_bh = bh;
+        ++nep;
+        return true;
+      };
+      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x, ++j) {
+        const int bh = tile_bh(tau), b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        bool ep_done = false;
+        for (int it = 0; it < npairs; ++it) {
+          if (it == kVStages) {            // the tile's first V pairs are on their way
+            if (!load_ep(tau)) { ok = false; break; }
+            ep_done = true;
+          }
+          const int s = gp % kVStages;
+          if (gp >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((gp / kVStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + kOffV + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
+          for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
+          }
+          ++gp;
         }
-        issued = it + 1;
+        if (ok && !ep_done && !load_ep(tau)) ok = false;
       }
-      for (int it = (issued > kVStages ? issued - kVStages : 0); it < issued; ++it)
-        mbar_wait(bar(ctl->v_full[it % kVStages]), (it / kVStages) & 1, wc, false);
-      mbar_wait(bar(ctl->ep_full), 0, wc, false);
+      for (int x = (gp > kVStages ? gp - kVStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->v_full[x % kVStages]), (x / kVStages) & 1, wc, false);
+      if (nep > 0) mbar_wait(bar(ctl->ep_full), (nep - 1) & 1, wc, false);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -373,6 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       WaitCtl dw{&ctl->abort, status, debug_limit_cycles};
       fail = !mbar_wait(bar(ctl->stall_bar), 0, dw);
     }
+    int gp = 0, j = 0;                             // pairs and tiles done by this CTA
+    for (int tau = blockIdx.x; tau < ntiles; tau += gridDim.x, ++j) {
+    if (named_vote_or(gbar, 128, fail)) break;
+    const int bh = tile_bh(tau), i = tau - bh * dm.nb, h = bh % dm.H;
+    const int b = bh / dm.H;
+    const int32_t* L = list_of(tau);
     float lp[32];
 #pragma unroll
     for (int q = 0; q < 32; ++q) lp[q] = 0.f;
@@ -385,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       sqi = __ldg(sq + sbase_idx + i);
       float mx = 0.f;
       for (int e = t; e < kk_list; e += 128) {
-        const int j = __ldg(L + e);
-        if (j >= 0 && j < dm.nb) mx = fmaxf(mx, __ldg(sv + sbase_idx + j));
+        const int jj = __ldg(L + e);
+        if (jj >= 0 && jj < dm.nb) mx = fmaxf(mx, __ldg(sv + sbase_idx + jj));
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -409,9 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
     }
 
-    for (int it = 0; it < npairs; ++it) {
-      const int sb = it % kSBufs;
-      const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (it / kSBufs) & 1, wc);
+    for (int it = 0; it < npairs; ++it, ++gp) {
+      const int sb = gp % kSBufs;
+      const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (gp / kSBufs) & 1, wc);
       fail |= !ok;
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads; invalid keys are masked after.
@@ -435,10 +488,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
       const float slt = FP8 ? sl2 * sqi * skj : sl2;
+      // (the first pair of a tile takes m = 0 and then its exact maxima)
       const float4* m4 = reinterpret_cast<const float4*>(ctl->m_used + c0);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 m = m4[q4];
+        const float4 m = it > 0 ? m4[q4] : make_float4(0.f, 0.f, 0.f, 0.f);
         x[4 * q4 + 0] = fmaf(x[4 * q4 + 0], slt, -m.x);
         x[4 * q4 + 1] = fmaf(x[4 * q4 + 1], slt, -m.y);
         x[4 * q4 + 2] = fmaf(x[4 * q4 + 2], slt, -m.z);
@@ -464,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           const float delta = it == 0 ? bm : fmaxf(bm, 0.f);
           ctl->red[g][0][lane] = delta;              // reuse: shift of each query's offset
           ctl->fac[c0 + lane] = ex2_approx(-delta);
-          ctl->m_used[c0 + lane] += delta;
+          ctl->m_used[c0 + lane] = it == 0 ? bm : ctl->m_used[c0 + lane] + delta;
         }
         named_sync(gbar, 128);
         const float4* d4 = reinterpret_cast<const float4*>(ctl->red[g][0]);
@@ -489,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           }
 #pragma unroll
           for (int q = 0; q < 32; ++q) lp[q] *= f[q];
-          fail |= !mbar_wait(bar(ctl->pv_done[(it - 1) & 1]), ((it - 1) >> 1) & 1, wc);
+          fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
           tc_fence_after();
           float o[32];
           tmem_ld32(lane_addr + kColO + c0, o);
@@ -525,21 +579,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           pw[q >> 1] = pack_half2(p0, p1);
         }
       }
-      if (it > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[it & 1]), ((it - 2) >> 1) & 1, wc);
+      // the P buffer was last read by the P V two pairs back (maybe in the previous tile)
+      if (gp > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1, wc);
       if constexpr (FP8)
-        st_chunks_sw64<2>(sP + (it & 1) * G::kPBytes, t, 2 * g, pw);
+        st_chunks_sw64<2>(sP + (gp & 1) * G::kPBytes, t, 2 * g, pw);
       else
-        st_chunks_sw128<4>(sP + (it & 1) * G::kPBytes, t, 4 * g, pw);
+        st_chunks_sw128<4>(sP + (gp & 1) * G::kPBytes, t, 4 * g, pw);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();                                  // the warp's P rows and O^T rescale are done
-      if (lane == 0) mbar_arrive(bar(ctl->p_full[it & 1]));
+      if (lane == 0) mbar_arrive(bar(ctl->p_full[gp & 1]));
     }
 
     // ------------------------------------------------------------ epilogue
     if (!named_vote_or(gbar, 128, fail)) {
       // the last P V: also proves that both groups are done reading every S buffer
-      fail |= !mbar_wait(bar(ctl->pv_done[(npairs - 1) & 1]), ((npairs - 1) >> 1) & 1, wc);
+      fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
     }
     if (!named_vote_or(gbar, 128, fail)) {
       tc_fence_after();
@@ -550,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         ctl->linv[c0 + lane] = vref / (ctl->red[g][0][lane] + ctl->red[g][1][lane] +
                                        ctl->red[g][2][lane] + ctl->red[g][3][lane]);
       if (g == 0 && t == 0) {
-        fail |= !mbar_wait(bar(ctl->ep_full), 0, wc);
+        fail |= !mbar_wait(bar(ctl->ep_full), j & 1, wc);
         tc_fence_after();
         constexpr uint32_t idesc_n = idesc_f16(1, 128, 64, 1, 1);
         const uint32_t sh = sbase + kOffSimg, sl = sh + 2 * RK * 128;
@@ -566,15 +621,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           mma_f16_ss(tmem + kColNum, ah, bld, idesc_n, true);
         }
         mma_commit(bar(ctl->ep_bar));
+        // wait without honouring an abort: the MMA must be over before TMEM can be freed
+        fail |= !mbar_wait(bar(ctl->ep_bar), j & 1, wc, false);
       }
-      fail |= !mbar_wait(bar(ctl->ep_bar), 0, wc);
-      fail |= !mbar_wait(bar(ctl->ep_full), 0, wc);     // g/den copy visible to every thread
+      fail |= !mbar_wait(bar(ctl->ep_bar), j & 1, wc);
+      fail |= !mbar_wait(bar(ctl->ep_full), j & 1, wc);     // g/den copy visible to every thread
       if (!named_vote_or(gbar, 128, fail)) {
         tc_fence_after();
         // out^T[d = t][q] = O^T / l + (g / den) num^T -> staging [2 boxes][64 q][64 d],
         // this group's rows c0 .. c0 + 31
         const float* gd = reinterpret_cast<const float*>(base + kOffGden);
-        uint8_t* stg = base + kOffQ;
+        uint8_t* stg = base + kOffQ + (j & 1) * 16384;   // the tile's Q slot
         __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(stg + (t >> 6) * 8192) + (t & 63);
         float o[32], nm[32];
         tmem_ld32(lane_addr + kColO + c0, o);
@@ -593,15 +650,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         fence_proxy_async_smem();
         named_sync(gbar, 128);
         // rows at or past N are clipped by the tensor map; a box wholly past N is skipped
-        if (t == 0 && i * 64 + c0 < dm.N) {
-          tma_store_3d(&tm_out, h * 128, i * 64 + c0, b, sbase + kOffQ + c0 * 128);
-          tma_store_3d(&tm_out, h * 128 + 64, i * 64 + c0, b, sbase + kOffQ + 8192 + c0 * 128);
-          tma_store_commit();
-          tma_store_wait_read0();
+        if (t == 0) {
+          const uint32_t src = sbase + kOffQ + (j & 1) * 16384 + c0 * 128;
+          if (i * 64 + c0 < dm.N) {
+            tma_store_3d(&tm_out, h * 128, i * 64 + c0, b, src);
+            tma_store_3d(&tm_out, h * 128 + 64, i * 64 + c0, b, src + 8192);
+            tma_store_commit();
+            tma_store_wait_read0();
+          }
+          mbar_arrive(bar(ctl->q_free[j & 1]));      // the Q slot may be refilled
         }
       }
     }
+    }   // tiles
   }
+
 
   tc_fence_before();
   __syncthreads();
@@ -623,7 +686,12 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
   cudaError_t e = cudaFuncSetAttribute(attend_sm100_kernel<RK, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(dm.nb, dm.B * dm.H);
+  // persistent: one CTA per SM, each walking the tiles tau = blockIdx.x + n * gridDim.x
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long ntiles = (long long)dm.nb * dm.B * dm.H;
+  dim3 grid((unsigned)(ntiles < sms ? ntiles : sms));
   attend_sm100_kernel<RK, FP8><<<grid, kThreads, smem, st>>>(
       tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status,
       debug_flags, limit_cycles, dlimit);
