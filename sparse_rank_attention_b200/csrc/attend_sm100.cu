@@ -57,6 +57,8 @@ constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 192;   // O^T
 constexpr uint32_t kColNum = 256; // epilogue: num^T (its own columns: the next tile's S^T
                                   // are computed while a tile's epilogue runs)
+constexpr uint32_t kColM = 384;   // exponent offsets m: every lane holds the 64 queries' m,
+                                  // read with S^T (tensor memory, not shared memory)
 
 constexpr int kKStages = 2;                // K pairs: freed as soon as their QK is done
 constexpr int kVStages = 2;                // V pairs: freed after their PV
@@ -87,7 +89,6 @@ struct Ctl {
   uint64_t s_full[kSBufs], s_empty[kSBufs], p_full[2], pv_done[2], ep_full, ep_bar, drain_bar, stall_bar;
   uint32_t tmem_base;
   int abort;
-  alignas(16) float m_used[64];
   alignas(16) float fac[64];
   alignas(16) float red[2][4][32];   // per query group: per-warp partial reductions
   alignas(16) float linv[64];
@@ -468,8 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       fail |= !ok;
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads; invalid keys are masked after.
-      float x[32];
+      float x[32], m[32];
       tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
+      if (it > 0) tmem_ld32(lane_addr + kColM + c0, m);   // (the first pair of a tile: m = 0)
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -488,15 +490,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
       const float slt = FP8 ? sl2 * sqi * skj : sl2;
-      // (the first pair of a tile takes m = 0 and then its exact maxima)
-      const float4* m4 = reinterpret_cast<const float4*>(ctl->m_used + c0);
+      if (it > 0) {
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 m = it > 0 ? m4[q4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        x[4 * q4 + 0] = fmaf(x[4 * q4 + 0], slt, -m.x);
-        x[4 * q4 + 1] = fmaf(x[4 * q4 + 1], slt, -m.y);
-        x[4 * q4 + 2] = fmaf(x[4 * q4 + 2], slt, -m.z);
-        x[4 * q4 + 3] = fmaf(x[4 * q4 + 3], slt, -m.w);
+        for (int q = 0; q < 32; ++q) x[q] = fmaf(x[q], slt, -m[q]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) x[q] *= slt;
       }
       if (!valid) {
 #pragma unroll
@@ -518,38 +517,48 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           const float delta = it == 0 ? bm : fmaxf(bm, 0.f);
           ctl->red[g][0][lane] = delta;              // reuse: shift of each query's offset
           ctl->fac[c0 + lane] = ex2_approx(-delta);
-          ctl->m_used[c0 + lane] = it == 0 ? bm : ctl->m_used[c0 + lane] + delta;
         }
         named_sync(gbar, 128);
+        // new offsets m + delta (m = 0 on a tile's first pair) into this lane's copy
+        if (it > 0) tmem_ld32(lane_addr + kColM + c0, m);
         const float4* d4 = reinterpret_cast<const float4*>(ctl->red[g][0]);
+        tmem_wait_ld();
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
           const float4 dd = d4[q4];
-          x[4 * q4 + 0] -= dd.x;
-          x[4 * q4 + 1] -= dd.y;
-          x[4 * q4 + 2] -= dd.z;
-          x[4 * q4 + 3] -= dd.w;
+          const float d[4] = {dd.x, dd.y, dd.z, dd.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = 4 * q4 + e;
+            x[q] -= d[e];
+            m[q] = it > 0 ? m[q] + d[e] : d[e];
+          }
         }
+        tmem_st32(lane_addr + kColM + c0, m);
+        tmem_wait_st();
         if (it > 0) {
           const float4* f4 = reinterpret_cast<const float4*>(ctl->fac + c0);
-          float f[32];
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             const float4 ff = f4[q4];
-            f[4 * q4 + 0] = ff.x;
-            f[4 * q4 + 1] = ff.y;
-            f[4 * q4 + 2] = ff.z;
-            f[4 * q4 + 3] = ff.w;
+            lp[4 * q4 + 0] *= ff.x;
+            lp[4 * q4 + 1] *= ff.y;
+            lp[4 * q4 + 2] *= ff.z;
+            lp[4 * q4 + 3] *= ff.w;
           }
-#pragma unroll
-          for (int q = 0; q < 32; ++q) lp[q] *= f[q];
           fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
           tc_fence_after();
           float o[32];
           tmem_ld32(lane_addr + kColO + c0, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] *= f[q];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 ff = f4[q4];
+            o[4 * q4 + 0] *= ff.x;
+            o[4 * q4 + 1] *= ff.y;
+            o[4 * q4 + 2] *= ff.z;
+            o[4 * q4 + 3] *= ff.w;
+          }
           tmem_st32(lane_addr + kColO + c0, o);
           tmem_wait_st();
         }
