@@ -123,12 +123,19 @@ def dist_env():
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Largest value of x over the ranks (the job's time is its slowest rank's)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: int, ms_per_step_max: float, ws: int) -> float:
+    """Whole-job throughput of ws independent replicas: all ranks' work over the slowest time."""
+    return ws * flops_per_rank / (ms_per_step_max * 1e-3) / 1e12
 
 
 def barrier(ws: int):
@@ -274,7 +281,7 @@ def main():
     plan.profile_stages(False)
     stage_ms = [x / ncalls for x in stage_sum]
     assert plan.poll_status() == 0
-    value = ws * flops / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(flops, ms_step, ws)
 
     peaks = load_peaks()
     att_ms = stage_ms[-1]
@@ -329,7 +336,7 @@ def main():
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), ws) / e_steps
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hWq, hWk, hg))
-        e2e = {"value": ws * flops / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": aggregate_tflops(flops, e_ms, ws), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
 
     cpu = None
