@@ -174,6 +174,13 @@ ROLA_API rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z,
 ROLA_API rola_status rola_get_fp8_copies(rola_plan_t plan, uint8_t* q8, uint8_t* k8, uint8_t* v8,
                                          float* sq, float* sk, float* sv, rola_stream_t stream);
 
+/* Inspection (tests): the number of query-block tiles whose output the last attention
+ * call recomputed in its careful pass (head dim 128, bf16 / fp8; 0 otherwise).  The fast
+ * pass fixes each tile's softmax offsets from its first pair of key blocks; a tile where a
+ * later score rises too far above them (P would leave fp16, or e4m3, range) is listed and
+ * recomputed with per-pair offset updates.  Synchronises `stream`; writes a host int. */
+ROLA_API rola_status rola_get_attend_redo_count(rola_plan_t plan, int* count, rola_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device status word: ROLA_OK, or
  * ROLA_ERR_DEVICE_TIMEOUT / ROLA_ERR_DEVICE_BOUNDS if a kernel recorded one. */
 ROLA_API rola_status rola_poll_device_status(rola_plan_t plan, rola_stream_t stream);

@@ -34,7 +34,7 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
            "rola_select_blocks_noalloc", "rola_get_fp8_copies", "rola_profile_stages",
-           "rola_get_stage_times")
+           "rola_get_stage_times", "rola_get_attend_redo_count")
 
 
 class RolaError(RuntimeError):
@@ -89,6 +89,7 @@ def load() -> ctypes.CDLL:
         "rola_select_blocks_noalloc": [pp, P, P, P, P],
         "rola_get_fp8_copies": [P, P, P, P, P, P, P, P],
         "rola_profile_stages": [P, i32],
+        "rola_get_attend_redo_count": [P, ctypes.POINTER(i32), P],
         "rola_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32),
                                  ctypes.POINTER(i32)],
     }.items():
@@ -247,6 +248,13 @@ class Plan:
         _check(load().rola_get_stage_times(self._h, ms, 8, ctypes.byref(ns), ctypes.byref(nc)),
                "rola_get_stage_times")
         return [ms[i] for i in range(ns.value)], nc.value
+
+    def attend_redo_count(self, stream=None) -> int:
+        """Tiles the last attention call recomputed in its careful pass (synchronises)."""
+        n = ctypes.c_int()
+        _check(load().rola_get_attend_redo_count(self._h, ctypes.byref(n), _stream(stream)),
+               "rola_get_attend_redo_count")
+        return n.value
 
     def poll_status(self, stream=None) -> int:
         """Synchronises the stream; returns the device status code (0 = ok), clearing it."""

@@ -174,14 +174,14 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return lo | (hi << 16);
 }
 
-template <int RK, bool FP8>
+template <int RK, bool FP8, bool CAREFUL>
 __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out, Dims dm,
     const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ simg,
     const uint8_t* __restrict__ uimg, const float* __restrict__ gden,
     const float* __restrict__ sq, const float* __restrict__ sk, const float* __restrict__ sv,
-    int* __restrict__ status, int debug_flags, unsigned long long limit_cycles,
+    int* __restrict__ status, int* __restrict__ redo, int debug_flags, unsigned long long limit_cycles,
     unsigned long long debug_limit_cycles) {
   using G = Geo<FP8>;
   constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV, kOffP = G::kOffP;
@@ -192,7 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   Ctl* ctl = reinterpret_cast<Ctl*>(base + kOffCtl);
   const uint32_t sbase = smem_addr(base);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = dm.nb * dm.B * dm.H;        // tile = (b, h, query block i)
+  // tile = (b, h, query block i).  The fast pass walks all tiles; the careful pass walks
+  // the tiles the fast pass listed in redo[1..redo[0]] (each listed at most twice).
+  const int ntiles_all = dm.nb * dm.B * dm.H;
+  const int ntiles = CAREFUL ? min(*reinterpret_cast<volatile int*>(redo), 2 * ntiles_all) : ntiles_all;
+  auto tile_at = [&](int idx) { return CAREFUL ? __ldg(redo + 1 + idx) : idx; };
   const int kk_list = dm.k;
   const int npairs = (kk_list + 1) >> 1;
   auto bar = [&](uint64_t& m) { return smem_addr(&m); };
@@ -254,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       tma_prefetch_desc(&tm_k);
       int nq = 0, gp = 0;               // Q tiles and K pairs issued
       bool ok = true;
-      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x) {
+      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x) {
+        const int tau = tile_at(idx);
         const int bh = tile_bh(tau), i = tau - bh * dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
         const int32_t* L = list_of(tau);
         const int qb = nq & 1;
@@ -292,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       constexpr uint32_t idesc_qk = FP8 ? idesc_f8(128, 64, 0, 0) : idesc_f16(1, 128, 64, 0, 0);
       int j = 0, gp = 0;
       bool ok = true;
-      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x, ++j) {
+      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x, ++j) {
+        const int tau = tile_at(idx);
         const int qb = j & 1;
         if (!mbar_wait(bar(ctl->q_full[qb]), (j >> 1) & 1, wc)) break;
         const uint64_t dq = sdesc_sw128(sbase + kOffQ + qb * 16384, 16, 1024);
@@ -325,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       constexpr uint32_t idesc_pv = FP8 ? idesc_f8(128, 64, 1, 1) : idesc_f16(0, 128, 64, 1, 1);
       int gp = 0;
       bool ok = true;
-      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x) {
+      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x) {
+        const int tau = tile_at(idx);
         for (int t = 0; t < npairs; ++t, ++gp) {
           const int s = gp % kVStages, pb = gp & 1;
           if (!mbar_wait(bar(ctl->v_full[s]), (gp / kVStages) & 1, wc)) { ok = false; break; }
@@ -374,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         ++nep;
         return true;
       };
-      for (int tau = blockIdx.x; ok && tau < ntiles; tau += gridDim.x, ++j) {
+      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x, ++j) {
+        const int tau = tile_at(idx);
         const int bh = tile_bh(tau), b = bh / dm.H, xh = (bh % dm.H) * 128;
         const int32_t* L = list_of(tau);
         bool ep_done = false;
@@ -423,7 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       fail = !mbar_wait(bar(ctl->stall_bar), 0, dw);
     }
     int gp = 0, j = 0;                             // pairs and tiles done by this CTA
-    for (int tau = blockIdx.x; tau < ntiles; tau += gridDim.x, ++j) {
+    bool overflow = false;                         // fast pass: this tile needs the careful pass
+    for (int idx = blockIdx.x; idx < ntiles; idx += gridDim.x, ++j) {
+    const int tau = tile_at(idx);
     if (named_vote_or(gbar, 128, fail)) break;
     const int bh = tile_bh(tau), i = tau - bh * dm.nb, h = bh % dm.H;
     const int b = bh / dm.H;
@@ -431,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     float lp[32];
 #pragma unroll
     for (int q = 0; q < 32; ++q) lp[q] = 0.f;
+    overflow = false;
 
     // fp8: the scores carry sq_i * sk_j, P carries sv_j / vref and the output vref, where
     // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
@@ -510,9 +521,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
 #pragma unroll
       for (int q = 0; q < 32; q += 4)
         dmax = fmaxf(dmax, fmaxf(fmaxf(x[q], x[q + 1]), fmaxf(x[q + 2], x[q + 3])));
-      // The first pair always sets the offsets; later pairs move them only when a score
-      // exceeds its query's offset by more than 8 (P then stays within [0, 256]).
-      if (named_vote_or(gbar, 128, fail || it == 0 || dmax > 8.f)) {
+      // The first pair of a tile sets the offsets (its exact column maxima).  Careful pass:
+      // later pairs move them when a score exceeds its query's offset by more than 8 (P
+      // then stays within [0, 256]), decided by a vote of the group on every pair.  Fast
+      // pass: no vote; a score more than kOverflow above its offset (P would leave the
+      // range of fp16, or of e4m3 after the V-scale factor) marks the tile, whose output
+      // the careful pass then recomputes.
+      bool slow;
+      if constexpr (CAREFUL) {
+        slow = named_vote_or(gbar, 128, fail || it == 0 || dmax > 8.f);
+      } else {
+        slow = it == 0;
+        if (!slow) overflow |= !(dmax <= (FP8 ? 8.f : 15.f));   // (NaN counts as overflow)
+      }
+      if (slow) {
         if (named_vote_or(gbar, 128, fail)) break;
         ctl->red[g][wq][lane] = reduce_scatter32<true>(x, lane);
         named_sync(gbar, 128);
@@ -606,6 +628,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     }
 
     // ------------------------------------------------------------ epilogue
+    if constexpr (!CAREFUL) {
+      if (named_vote_or(gbar, 128, overflow) && t == 0) {
+        const int slot = atomicAdd(redo, 1);
+        if (slot < 2 * ntiles_all) redo[1 + slot] = tau;
+      }
+    }
     if (!named_vote_or(gbar, 128, fail)) {
       // the last P V: also proves that both groups are done reading every S buffer
       fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
@@ -697,17 +725,27 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
   const unsigned long long limit_cycles = 2000000000ull;
   const unsigned long long dlimit = (unsigned long long)(debug_limit_us > 0 ? debug_limit_us : 1000) * 2000ull;
   constexpr size_t smem = smem_bytes<FP8>();
-  cudaError_t e = cudaFuncSetAttribute(attend_sm100_kernel<RK, FP8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(attend_sm100_kernel<RK, FP8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(attend_sm100_kernel<RK, FP8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)) != cudaSuccess)
+    return e;
   // persistent: one CTA per SM, each walking the tiles tau = blockIdx.x + n * gridDim.x
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const long long ntiles = (long long)dm.nb * dm.B * dm.H;
   dim3 grid((unsigned)(ntiles < sms ? ntiles : sms));
-  attend_sm100_kernel<RK, FP8><<<grid, kThreads, smem, st>>>(
-      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status,
+  // fast pass over every tile, then the careful pass over the tiles it listed (none, usually:
+  // its CTAs then exit at once)
+  if ((e = cudaMemsetAsync(ws.redo, 0, sizeof(int), st)) != cudaSuccess) return e;
+  attend_sm100_kernel<RK, FP8, false><<<grid, kThreads, smem, st>>>(
+      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status, ws.redo,
+      debug_flags, limit_cycles, dlimit);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attend_sm100_kernel<RK, FP8, true><<<grid, kThreads, smem, st>>>(
+      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status, ws.redo,
       debug_flags, limit_cycles, dlimit);
   return cudaGetLastError();
 }

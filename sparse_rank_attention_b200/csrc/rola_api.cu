@@ -127,6 +127,7 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   if (p.dtype == ROLA_BF16)
     w.v16 = reinterpret_cast<__half*>(take(sizeof(__half) * (size_t)dm.B * dm.N * dm.H * dm.d));
   if (p.dtype != ROLA_F32 && p.d == 128) {
+    w.redo = reinterpret_cast<int*>(take(sizeof(int) * (1 + 2 * BH * dm.nb)));
     w.simg = reinterpret_cast<uint8_t*>(take(BH * 4 * dm.r * 128));
     w.uimg = reinterpret_cast<uint8_t*>(take(BH * dm.nb * 2 * dm.r * 128));
     w.gden = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * 64));
@@ -421,6 +422,16 @@ rola_status rola_get_fp8_copies(rola_plan_t plan, uint8_t* q8, uint8_t* k8, uint
   for (const auto& c : copies)
     if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return ROLA_ERR_CUDA;
   return ROLA_OK;
+}
+
+rola_status rola_get_attend_redo_count(rola_plan_t plan, int* count, rola_stream_t stream) {
+  if (!plan || !count) return ROLA_ERR_INVALID_ARG;
+  *count = 0;
+  if (!plan->ws.redo) return ROLA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(count, plan->ws.redo, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(st));
 }
 
 rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream) {

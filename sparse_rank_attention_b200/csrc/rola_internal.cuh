@@ -54,6 +54,7 @@ struct Workspace {
   uint8_t* q8;        // [B, N, H, d] e4m3 (fp8 mode)
   uint8_t* k8;
   uint8_t* v8;
+  int* redo;          // [1 + 2*B*H*nb]: count, then the tiles the attention's careful pass redoes
   float* sq;          // [B, H, nb] e4m3 scales (fp8 mode)
   float* sk;
   float* sv;

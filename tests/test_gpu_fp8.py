@@ -34,8 +34,10 @@ def _all_blocks(w):
                     dtype=np.int32)
 
 
-def _check(w, seed, blocks=None, copies_full=True):
+def _check(w, seed, blocks=None, copies_full=True, modify=None):
     inp = synth.make_inputs(w, seed=seed, device="cuda")
+    if modify is not None:
+        inp = modify(inp)
     res = run_gpu(w, inp)
     assert res["status"] == 0
     (q8, k8, v8), (sq, sk, sv) = res["plan"].fp8_copies()
@@ -67,6 +69,7 @@ def _check(w, seed, blocks=None, copies_full=True):
     norm, worst = check_out_fp8(got, want, valid, w.name)
     diag, _ = check_out_fp8(got, want_q, valid, w.name + " (dequantised inputs)", tol=DIAG_TOL)
     print(f"PARITY {w.name} normwise={norm:.3e} worst_block={worst:.3e} vs_dequantised={diag:.3e}")
+    return res
 
 
 SMALL = [
@@ -105,3 +108,12 @@ def test_fp8_zero_block_scale_is_one():
 def test_fp8_wan_720p_sampled():
     w = synth.WORKLOADS["wan21_14b_720p_fp8"]
     _check(w, seed=0, blocks=sample_blocks(w, 3, 12, 0))
+
+
+def test_fp8_careful_pass_recomputes_overflowing_tiles():
+    """Later key blocks scaled up (by at most 1.8x): scores rise more than 8 (log2) above a
+    tile's first pair, so its e4m3 weights would saturate and the careful pass redoes it."""
+    from test_gpu_parity import _rising_keys
+    w = synth.custom("fp8_rising", B=1, H=2, N=4096, d=128, r=32, topk=0.25, grid=(4, 16, 64), dtype="fp8")
+    res = _check(w, seed=7, modify=lambda inp: _rising_keys(inp, w, top=0.8))
+    assert res["plan"].attend_redo_count() > 0

@@ -132,3 +132,31 @@ def _compare_sampled(w, n_heads=3, n_blocks=12, seed=0):
                                   "wan21_14b_480p_dense_g0", "wan21_14b_480p_topk0.25"])
 def test_wan_shapes_sampled(name):
     _compare_sampled(synth.WORKLOADS[name])
+
+
+def _rising_keys(inp, w, top=6.0):
+    """Scales key block j by 1 + top * j / nb: later kept blocks score far above the first
+    pair of each row, so the fast attention pass must hand tiles to the careful pass."""
+    nb = w.nb
+    scale = 1.0 + top * torch.arange(nb, device=inp["k"].device, dtype=torch.float32) / nb
+    per_tok = scale.repeat_interleave(64)[: w.N].view(1, w.N, 1, 1)
+    inp["k"] = (inp["k"].float() * per_tok).to(inp["k"].dtype)
+    return inp
+
+
+def test_careful_pass_recomputes_overflowing_tiles():
+    w = synth.custom("bf16_rising", B=1, H=2, N=4096, d=128, r=32, topk=0.25, grid=(4, 16, 64))
+    inp = _rising_keys(synth.make_inputs(w, seed=7, device="cuda"), w, top=1.5)
+    res = run_gpu(w, inp)
+    assert res["status"] == 0
+    assert res["plan"].attend_redo_count() > 0      # the careful pass ran on some tiles
+    h = host_inputs(inp)
+    out, _ = O.forward(shape_of(w), h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"])
+    r = check_out(np32(res["out"]).astype(np.float64), out, w.dtype, w.name)
+    print(f"PARITY {w.name} redo={res['plan'].attend_redo_count()} max_err={r[0]:.3e} rms={r[1]}")
+
+
+def test_fast_pass_alone_on_wan_like_inputs():
+    w = synth.custom("bf16_wan_like", B=1, H=2, N=4152, d=128, r=32, topk=0.1, grid=(2, 4, 519))
+    res = run_gpu(w, synth.make_inputs(w, seed=1, device="cuda"))
+    assert res["status"] == 0 and res["plan"].attend_redo_count() == 0
