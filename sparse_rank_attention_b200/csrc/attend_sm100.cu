@@ -61,8 +61,7 @@ constexpr uint32_t kColNum = 256; // epilogue: num^T (its own columns: the next 
 constexpr uint32_t kColM = 384;   // exponent offsets m: every lane holds the 64 queries' m,
                                   // read with S^T (tensor memory, not shared memory)
 
-constexpr int kKStages = 2;                // K pairs: freed as soon as their QK is done
-constexpr int kVStages = 2;                // V pairs: freed after their PV
+constexpr int kMaxStages = 4;              // ring-depth bound (barrier arrays)
 
 // Shared-memory geometry.  16-bit path: a tile row of 128 channels is two 128-byte
 // swizzle boxes (channels 0-63, 64-127); fp8 path: one 128-byte box.  P^T is fp16 in
@@ -74,6 +73,11 @@ struct Geo {
   static constexpr uint32_t kPairBytes = 128 * 128 * kEl;         // K or V pair
   static constexpr uint32_t kBoxKV = FP8 ? 16384 : 16384;         // channel-box stride in a pair
   static constexpr uint32_t kPBytes = FP8 ? 8192 : 16384;         // one P^T buffer
+  // K pairs are freed as soon as their QK is done, V pairs after their PV.  A pair's copy
+  // from L2 takes longer than a pair's work, so the rings are as deep as shared memory
+  // allows: 2 + 2 of 32 KB for 16-bit operands, 4 + 4 of 16 KB for e4m3.
+  static constexpr int kKStages = FP8 ? 4 : 2;
+  static constexpr int kVStages = FP8 ? 4 : 2;
   static constexpr uint32_t kOffQ = 0;                             // 2 Q slots of 16 KB (each
                                                                    // also its tile's out staging)
   static constexpr uint32_t kOffK = 32768;                         // K ring (1024-aligned)
@@ -86,7 +90,7 @@ struct Geo {
 };
 
 struct Ctl {
-  uint64_t q_full[2], q_free[2], k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t q_full[2], q_free[2], k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages];
   uint64_t s_full[kSBufs], s_empty[kSBufs], p_full[2], pv_done[2], ep_full, ep_bar, drain_bar, stall_bar;
   uint32_t tmem_base;
   int abort;
@@ -184,6 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     int* __restrict__ status, int* __restrict__ redo, int debug_flags, unsigned long long limit_cycles,
     unsigned long long debug_limit_cycles) {
   using G = Geo<FP8>;
+  constexpr int kKStages = G::kKStages, kVStages = G::kVStages;
+  static_assert(kKStages <= kMaxStages && kVStages <= kMaxStages, "ring depth");
   constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV, kOffP = G::kOffP;
   constexpr uint32_t kOffSimg = G::kOffSimg, kOffUimg = G::kOffUimg, kOffGden = G::kOffGden;
   constexpr uint32_t kOffCtl = G::kOffCtl, kPairBytes = G::kPairBytes, kBoxKV = G::kBoxKV;
