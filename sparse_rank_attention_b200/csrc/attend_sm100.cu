@@ -248,9 +248,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtl wc{&ctl->abort, status, limit_cycles};
-  auto pair_blocks = [&](const int32_t* L, int it, int& j1, int& j2) {
+  // The producers read a pair's key blocks before they wait for its ring slot (the list
+  // load then overlaps the wait) and check them after.
+  auto pair_read = [&](const int32_t* L, int it, int& j1, int& j2) {
     j1 = __ldg(L + 2 * it);
-    j2 = (2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : j1;
+    j2 = (2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : -2;
+  };
+  auto pair_check = [&](int& j1, int& j2) {
+    if (j2 == -2) j2 = j1;
     if (j1 < 0 || j1 >= dm.nb || j2 < 0 || j2 >= dm.nb) {
       atomicCAS(status, 0, kDevBounds);
       j1 = j2 = 0;
@@ -277,12 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         ++nq;
         for (int it = 0; it < npairs; ++it) {
           const int s = gp % kKStages;
+          int j1, j2;
+          pair_read(L, it, j1, j2);
           if (gp >= kKStages && !mbar_wait(bar(ctl->k_empty[s]), ((gp / kKStages) - 1) & 1, wc)) {
             ok = false;
             break;
           }
-          int j1, j2;
-          pair_blocks(L, it, j1, j2);
+          pair_check(j1, j2);
           const uint32_t st = sbase + kOffK + s * kPairBytes;
           mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
           for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
@@ -398,12 +404,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
             ep_done = true;
           }
           const int s = gp % kVStages;
+          int j1, j2;
+          pair_read(L, it, j1, j2);
           if (gp >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((gp / kVStages) - 1) & 1, wc)) {
             ok = false;
             break;
           }
-          int j1, j2;
-          pair_blocks(L, it, j1, j2);
+          pair_check(j1, j2);
           const uint32_t st = sbase + kOffV + s * kPairBytes;
           mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
           for (int c = 0; c < (FP8 ? 1 : 2); ++c) {
