@@ -341,9 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     // ------------------------------------------------------------ O^T += V^T P^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = FP8 ? idesc_f8(128, 64, 1, 1) : idesc_f16(0, 128, 64, 1, 1);
-      int gp = 0;
+      constexpr uint32_t idesc_n = idesc_f16(1, 128, 64, 1, 1);
+      const int t_num = npairs > 2 ? 2 : npairs - 1;   // the pair after which num^T is issued
+      int gp = 0, j = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x) {
+      for (int idx = blockIdx.x; ok && idx < ntiles; idx += gridDim.x, ++j) {
         const int tau = tile_at(idx);
         for (int t = 0; t < npairs; ++t, ++gp) {
           const int s = gp % kVStages, pb = gp & 1;
@@ -365,6 +367,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           }
           mma_commit(bar(ctl->pv_done[pb]));
           mma_commit(bar(ctl->v_empty[s]));
+          if (t == t_num) {
+            // num^T = S_h^T (R u)^T for the tile's epilogue, early: it needs only the
+            // epilogue operands (by now loaded), and both groups are past the previous
+            // tile's epilogue (they produced this tile's P), so its columns are free.
+            if (!mbar_wait(bar(ctl->ep_full), j & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sh = sbase + kOffSimg, sl = sh + 2 * RK * 128;
+            const uint32_t uh = sbase + kOffUimg, ul = uh + RK * 128;
+#pragma unroll
+            for (int kk = 0; kk < RK / 16; ++kk) {
+              const uint64_t ah = sdesc_sw128(sh + kk * 2048, RK * 128, 1024);
+              const uint64_t al = sdesc_sw128(sl + kk * 2048, RK * 128, 1024);
+              const uint64_t bhd = sdesc_sw128(uh + kk * 2048, 4096, 1024);
+              const uint64_t bld = sdesc_sw128(ul + kk * 2048, 4096, 1024);
+              mma_f16_ss(tmem + kColNum, ah, bhd, idesc_n, kk > 0);
+              mma_f16_ss(tmem + kColNum, al, bhd, idesc_n, true);
+              mma_f16_ss(tmem + kColNum, ah, bld, idesc_n, true);
+            }
+            mma_commit(bar(ctl->ep_bar));
+          }
         }
       }
       mma_commit(bar(ctl->drain_bar));
@@ -648,37 +670,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       }
     }
     if (!named_vote_or(gbar, 128, fail)) {
-      // the last P V: also proves that both groups are done reading every S buffer
-      fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
-    }
-    if (!named_vote_or(gbar, 128, fail)) {
-      tc_fence_after();
-      // per-query sums l over the group's 128 threads
+      // per-query sums l over the group's 128 threads (final once the last P is made)
       ctl->red[g][wq][lane] = reduce_scatter32<false>(lp, lane);
       named_sync(gbar, 128);
       if (wq == 0)
         ctl->linv[c0 + lane] = vref / (ctl->red[g][0][lane] + ctl->red[g][1][lane] +
                                        ctl->red[g][2][lane] + ctl->red[g][3][lane]);
-      if (g == 0 && t == 0) {
-        fail |= !mbar_wait(bar(ctl->ep_full), j & 1, wc);
-        tc_fence_after();
-        constexpr uint32_t idesc_n = idesc_f16(1, 128, 64, 1, 1);
-        const uint32_t sh = sbase + kOffSimg, sl = sh + 2 * RK * 128;
-        const uint32_t uh = sbase + kOffUimg, ul = uh + RK * 128;
-#pragma unroll
-        for (int kk = 0; kk < RK / 16; ++kk) {
-          const uint64_t ah = sdesc_sw128(sh + kk * 2048, RK * 128, 1024);
-          const uint64_t al = sdesc_sw128(sl + kk * 2048, RK * 128, 1024);
-          const uint64_t bhd = sdesc_sw128(uh + kk * 2048, 4096, 1024);
-          const uint64_t bld = sdesc_sw128(ul + kk * 2048, 4096, 1024);
-          mma_f16_ss(tmem + kColNum, ah, bhd, idesc_n, kk > 0);
-          mma_f16_ss(tmem + kColNum, al, bhd, idesc_n, true);
-          mma_f16_ss(tmem + kColNum, ah, bld, idesc_n, true);
-        }
-        mma_commit(bar(ctl->ep_bar));
-        // wait without honouring an abort: the MMA must be over before TMEM can be freed
-        fail |= !mbar_wait(bar(ctl->ep_bar), j & 1, wc, false);
-      }
+      // the tile's last P V (it also proves both groups are done with its S buffers), and
+      // num^T (issued by the P V issuer early in the tile)
+      fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
       fail |= !mbar_wait(bar(ctl->ep_bar), j & 1, wc);
       fail |= !mbar_wait(bar(ctl->ep_full), j & 1, wc);     // g/den copy visible to every thread
       if (!named_vote_or(gbar, 128, fail)) {
@@ -696,11 +696,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         for (int qq4 = 0; qq4 < 8; ++qq4) {
           const float4 li = reinterpret_cast<const float4*>(ctl->linv + c0)[qq4];
           const float4 gg = reinterpret_cast<const float4*>(gd + c0)[qq4];
-          const int q0 = c0 + 4 * qq4, j = 4 * qq4;
-          col[(q0 + 0) * 64] = __float2bfloat16_rn(o[j + 0] * li.x + nm[j + 0] * gg.x);
-          col[(q0 + 1) * 64] = __float2bfloat16_rn(o[j + 1] * li.y + nm[j + 1] * gg.y);
-          col[(q0 + 2) * 64] = __float2bfloat16_rn(o[j + 2] * li.z + nm[j + 2] * gg.z);
-          col[(q0 + 3) * 64] = __float2bfloat16_rn(o[j + 3] * li.w + nm[j + 3] * gg.w);
+          const int q0 = c0 + 4 * qq4, e = 4 * qq4;
+          col[(q0 + 0) * 64] = __float2bfloat16_rn(o[e + 0] * li.x + nm[e + 0] * gg.x);
+          col[(q0 + 1) * 64] = __float2bfloat16_rn(o[e + 1] * li.y + nm[e + 1] * gg.y);
+          col[(q0 + 2) * 64] = __float2bfloat16_rn(o[e + 2] * li.z + nm[e + 2] * gg.z);
+          col[(q0 + 3) * 64] = __float2bfloat16_rn(o[e + 3] * li.w + nm[e + 3] * gg.w);
         }
         fence_proxy_async_smem();
         named_sync(gbar, 128);
