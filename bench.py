@@ -36,8 +36,15 @@ METRIC = "RoLA fwd kept-block TFLOP/s at Wan2.1-14B-720P shape, 1xB200"
 UNIT = "TFLOP/s"
 
 
-# key/value pass, state reduction | query pass | block scores, top-k | attention
-LAUNCHES_PER_STEP = 6
+# key/value pass, state reduction | query pass | block scores, top-k | attention fast and
+# careful passes
+LAUNCHES_PER_STEP = 7
+
+# DRAM bytes (read + write) per launch of the attention kernel's fast pass, from
+# `dram__bytes_read.sum + dram__bytes_write.sum` of one ncu capture of the current kernel on the
+# 14B-480P workload, scaled to 720P by the token count (the streamed bytes grow with N); see
+# profiles/attend_sm100_wan21_14b_480p.md.  None where no capture of the current kernel exists.
+ATTEND_DRAM_BYTES = {"wan21_14b_720p": 1.507e9 * 75600 / 32760, "wan21_14b_480p": 1.507e9}
 
 
 def load_peaks():
@@ -294,7 +301,8 @@ def main():
         peak_src = f"{peaks['source']} bf16 burst (cuBLAS 8192^3)"
     roof = {"bound": "tensor", "kernel": "attend (sparse branch + fused linear epilogue)",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None, "peak_source": peak_src}
+            "frac": achieved / peak, "traffic": ATTEND_DRAM_BYTES.get(w.name), "traffic_unit": "bytes/launch",
+            "peak_source": peak_src}
     act = w.B * w.N * w.H * w.d                     # elements of one activation tensor
     nblk = w.B * w.H * plan.nb
     if len(stage_ms) == 4:
