@@ -32,7 +32,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kTok = 64;                     // tokens per tile = one block
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr int kThreads = 256;
 constexpr uint32_t kTileBytes = kTok * kD * 2;   // 16 KB, 64 rows of 256 bytes
 
@@ -79,7 +79,7 @@ __device__ __forceinline__ uint2 e4m3x8(const uint4& v, float inv) {
 }
 
 template <int RK, bool FP8>
-__global__ void __launch_bounds__(kThreads, 1) kv_pass_kernel(
+__global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __nv_bfloat16* __restrict__ Wk, Dims dm, const float2* __restrict__ rope,
     float* __restrict__ S_part, float* __restrict__ z_part, float* __restrict__ kbar,

@@ -66,7 +66,7 @@ rola_status check_params(const rola_params* p) {
 // chunk lengths.  The other paths keep fixed 2048-token chunks.
 int state_chunk_tokens(const rola_params& p, int nb) {
   if (!(p.d == 128 && p.dtype != ROLA_F32)) return rola::kStateChunk;
-  constexpr long long kSMs = 148;
+  constexpr long long kSMs = 2 * 148;   // CTA slots: two per SM
   const long long bh = (long long)p.B * p.H;
   long long best_cost = -1;
   int best = nb;
