@@ -135,39 +135,62 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, cons
 // ------------------------------------------------------------------ block scores
 
 constexpr int kTS = 128;  // score tile: 128 query blocks x 128 key blocks
-constexpr int kKC = 32;   // channels staged per step
+constexpr int kKC = 16;   // channels staged per step
 
 // grid: x = key-block tile, y = query-block tile, z = b*H + h; 256 threads, 8x8 scores each.
 // s_ij accumulates q_i[c] * k_j[c] with fmaf in channel order 0..d-1 (the stated order).
-__global__ void __launch_bounds__(256) score_kernel(Dims dm, const float* __restrict__ qbar,
-                                                    const float* __restrict__ kbar,
-                                                    float* __restrict__ scores, int nbp) {
-  __shared__ __align__(16) float As[kKC][kTS + 4];
-  __shared__ __align__(16) float Bs[kKC][kTS + 4];
+// The next 16-channel chunk is loaded into registers (float4 per row and channel quad)
+// while the current one is multiplied, then stored transposed into the other buffer.
+constexpr size_t kScoreSmem = sizeof(float) * 2 * 2 * kKC * (kTS + 4);
+
+__global__ void __launch_bounds__(256, 2) score_kernel(Dims dm, const float* __restrict__ qbar,
+                                                       const float* __restrict__ kbar,
+                                                       float* __restrict__ scores, int nbp) {
+  extern __shared__ __align__(16) float ssm[];
+  float (*As)[kKC][kTS + 4] = reinterpret_cast<float (*)[kKC][kTS + 4]>(ssm);
+  float (*Bs)[kKC][kTS + 4] = reinterpret_cast<float (*)[kKC][kTS + 4]>(ssm + 2 * kKC * (kTS + 4));
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int i0 = blockIdx.y * kTS, j0 = blockIdx.x * kTS, bh = blockIdx.z;
   const int nb = dm.nb, d = dm.d;
   const float* qb = qbar + (size_t)bh * nb * d;
   const float* kb = kbar + (size_t)bh * nb * d;
+  constexpr int kQuads = kKC / 4, kPer = kTS * kQuads / 256;   // float4 loads per thread
+  float4 ra[kPer], rb[kPer];
+  auto load = [&](int c0) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + 256 * u, r = e / kQuads, cq = e % kQuads;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      ra[u] = (i0 + r < nb) ? *reinterpret_cast<const float4*>(qb + (size_t)(i0 + r) * d + c0 + 4 * cq) : z;
+      rb[u] = (j0 + r < nb) ? *reinterpret_cast<const float4*>(kb + (size_t)(j0 + r) * d + c0 + 4 * cq) : z;
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + 256 * u, r = e / kQuads, c = 4 * (e % kQuads);
+      As[buf][c][r] = ra[u].x; As[buf][c + 1][r] = ra[u].y; As[buf][c + 2][r] = ra[u].z; As[buf][c + 3][r] = ra[u].w;
+      Bs[buf][c][r] = rb[u].x; Bs[buf][c + 1][r] = rb[u].y; Bs[buf][c + 2][r] = rb[u].z; Bs[buf][c + 3][r] = rb[u].w;
+    }
+  };
   float acc[8][8];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-  for (int c0 = 0; c0 < d; c0 += kKC) {
-    __syncthreads();
-    for (int e = tid; e < kTS * kKC; e += 256) {
-      const int r = e / kKC, c = e % kKC;
-      As[c][r] = (i0 + r < nb) ? qb[(size_t)(i0 + r) * d + c0 + c] : 0.f;
-      Bs[c][r] = (j0 + r < nb) ? kb[(size_t)(j0 + r) * d + c0 + c] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
+  const int nch = d / kKC;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int ch = 0; ch < nch; ++ch) {
+    const int buf = ch & 1;
+    if (ch + 1 < nch) load((ch + 1) * kKC);
+#pragma unroll 2
     for (int c = 0; c < kKC; ++c) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[c][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[c][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[c][tx * 8 + 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][c][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][c][tx * 8 + 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -175,6 +198,8 @@ __global__ void __launch_bounds__(256) score_kernel(Dims dm, const float* __rest
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(av[a], bv[e], acc[a][e]);
     }
+    if (ch + 1 < nch) store(buf ^ 1);   // the other buffer was last read before the barrier below
+    __syncthreads();
   }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
@@ -325,8 +350,10 @@ size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm)
 cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   const int nbp = score_row_stride(dm);
   dim3 g1((dm.nb + kTS - 1) / kTS, (dm.nb + kTS - 1) / kTS, dm.B * dm.H);
-  score_kernel<<<g1, 256, 0, st>>>(dm, ws.qbar, ws.kbar, ws.scores, nbp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+  if (e != cudaSuccess) return e;
+  score_kernel<<<g1, 256, kScoreSmem, st>>>(dm, ws.qbar, ws.kbar, ws.scores, nbp);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = topk_smem(nbp);
   e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
