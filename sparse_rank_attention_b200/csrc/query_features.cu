@@ -56,16 +56,22 @@ __global__ void __launch_bounds__(128) query_features_kernel(
   cp_async_wait<0>();
   __syncthreads();
 
-  // block mean of q: thread = channel, tokens added in order
+  // block mean of q: threads 0-63 own two adjacent channels each, tokens added in order
   {
-    const int c = tid;
-    float acc = 0.f, am = 0.f;
-    for (int r = 0; r < cnt; ++r) {
-      const float x = __bfloat162float(sQ[r * DP + c]);
-      acc = acc + x;
-      if (FP8) am = fmaxf(am, fabsf(x));
+    float am = 0.f;
+    if (tid < 64) {
+      float a0 = 0.f, a1 = 0.f;
+      const uint32_t* col = reinterpret_cast<const uint32_t*>(sQ) + tid;
+      for (int r = 0; r < cnt; ++r) {
+        const uint32_t w = col[r * (DP / 2)];
+        const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
+        a0 = a0 + x0;
+        a1 = a1 + x1;
+        if (FP8) am = fmaxf(am, fmaxf(fabsf(x0), fabsf(x1)));
+      }
+      *reinterpret_cast<float2*>(qbar + ((size_t)bh * dm.nb + i) * D + 2 * tid) =
+          make_float2(__fdiv_rn(a0, (float)cnt), __fdiv_rn(a1, (float)cnt));
     }
-    qbar[((size_t)bh * dm.nb + i) * D + c] = __fdiv_rn(acc, (float)cnt);
     if constexpr (FP8) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
@@ -120,7 +126,7 @@ __global__ void __launch_bounds__(128) query_features_kernel(
     float den = 0.f;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const float u0 = phi(f[nt][2 * half]), u1 = phi(f[nt][2 * half + 1]);
+      const float u0 = phi_fast(f[nt][2 * half]), u1 = phi_fast(f[nt][2 * half + 1]);
       const int a = nt * 8 + 2 * t4;
       den = fmaf(u0, sz[a], fmaf(u1, sz[a + 1], den));
       const float2 cs = ok ? rope_at(dm, rope, pos, nt * 4 + t4) : make_float2(1.f, 0.f);
