@@ -58,8 +58,9 @@ constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 192;   // O^T
 constexpr uint32_t kColNum = 256; // epilogue: num^T (its own columns: the next tile's S^T
                                   // are computed while a tile's epilogue runs)
-constexpr uint32_t kColM = 384;   // exponent offsets m: every lane holds the 64 queries' m,
-                                  // read with S^T (tensor memory, not shared memory)
+constexpr uint32_t kColM = 384;   // negated exponent offsets -m: every lane holds the 64
+                                  // queries' -m, read with S^T (tensor memory, not shared
+                                  // memory) and used as the addend of x = s * scale - m
 
 constexpr int kMaxStages = 4;              // ring-depth bound (barrier arrays)
 
@@ -123,6 +124,34 @@ __device__ __forceinline__ float ex2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(0.05508868f, fr, 0.24260405f), fr, 0.69327623f), fr, 0.99992895f);
   // t's low mantissa bits hold n; shifting by 23 drops the rest of t's bits
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Two fp32 lanes per instruction (the packed f32x2 operations of sm_100; each lane is
+// rounded exactly as its scalar counterpart): d = a * b + c, d += a, d *= b.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n .reg .b64 a, b, c, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n"
+      " mov.b64 c, {%6, %7};\n fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n .reg .b64 a, d;\n mov.b64 a, {%2, %3};\n mov.b64 d, {%0, %1};\n"
+      " add.rn.f32x2 d, d, a;\n mov.b64 {%0, %1}, d;\n}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float b0, float b1) {
+  asm("{\n .reg .b64 b, d;\n mov.b64 b, {%2, %3};\n mov.b64 d, {%0, %1};\n"
+      " mul.rn.f32x2 d, d, b;\n mov.b64 {%0, %1}, d;\n}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(b0), "f"(b1));
+}
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Reduce 32 per-lane values over the warp; lane l receives entry l (31 shuffles).
@@ -474,6 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const uint32_t gbar = 1 + g;                   // the group's named barrier
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
     const float sl2 = dm.scale * 1.4426950408889634f;
+    // fast pass: largest partial row sum (so largest P) a tile may reach, 2^15 for fp16 P
+    // and 2^8 for e4m3 P (whose V-scale factor is at most 1; e4m3 saturates at 448)
+    constexpr float kOverflow = FP8 ? 256.f : 32768.f;
     uint8_t* sP = base + kOffP;
     bool fail = false;
     if (debug_flags & ROLA_DEBUG_STALL_WAIT) {
@@ -481,7 +513,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       fail = !mbar_wait(bar(ctl->stall_bar), 0, dw);
     }
     int gp = 0, j = 0;                             // pairs and tiles done by this CTA
-    bool overflow = false;                         // fast pass: this tile needs the careful pass
     for (int idx = blockIdx.x; idx < ntiles; idx += gridDim.x, ++j) {
     const int tau = tile_at(idx);
     if (named_vote_or(gbar, 128, fail)) break;
@@ -491,7 +522,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     float lp[32];
 #pragma unroll
     for (int q = 0; q < 32; ++q) lp[q] = 0.f;
-    overflow = false;
 
     // fp8: the scores carry sq_i * sk_j, P carries sv_j / vref and the output vref, where
     // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
@@ -529,15 +559,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     // phases (exponentials and e4m3 packing on the special-function unit, the rest on the
     // other pipes) interleave; this measured faster for fp8 only.
     if (FP8 && g == 1) __nanosleep(kGroupOffsetNs);
+    bool s_seen = false;                           // the next pair's S was seen complete early
     for (int it = 0; it < npairs; ++it, ++gp) {
       const int sb = gp % kSBufs;
-      const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (gp / kSBufs) & 1, wc);
+      const bool ok = !fail && (s_seen || mbar_wait(bar(ctl->s_full[sb]), (gp / kSBufs) & 1, wc));
       fail |= !ok;
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads; invalid keys are masked after.
-      float x[32], m[32];
+      // mn = the queries' negated exponent offsets (the first pair of a tile: none yet).
+      float x[32], mn[32];
       tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
-      if (it > 0) tmem_ld32(lane_addr + kColM + c0, m);   // (the first pair of a tile: m = 0)
+      if (it > 0) tmem_ld32(lane_addr + kColM + c0, mn);
+      // The P buffer was last read by the P V two pairs back (maybe in the previous tile):
+      // its barrier is tested now and waited for only if that P V was not done yet.
+      const bool p_free = gp < 2 || mbar_test_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -558,31 +593,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       const float slt = FP8 ? sl2 * sqi * skj : sl2;
       if (it > 0) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) x[q] = fmaf(x[q], slt, -m[q]);
+        for (int q = 0; q < 32; q += 2) fma2(x[q], x[q + 1], x[q], x[q + 1], slt, slt, mn[q], mn[q + 1]);
       } else {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) x[q] *= slt;
+        for (int q = 0; q < 32; q += 2) mul2(x[q], x[q + 1], slt, slt);
       }
-      if (!valid) {
+      // keys past the end of the sequence and the padding half of an odd list (rare pairs)
+      if (__any_sync(0xffffffffu, !valid)) {
+        if (!valid) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
+          for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
+        }
       }
-      float dmax = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 32; q += 4)
-        dmax = fmaxf(dmax, fmaxf(fmaxf(x[q], x[q + 1]), fmaxf(x[q + 2], x[q + 3])));
       // The first pair of a tile sets the offsets (its exact column maxima).  Careful pass:
       // later pairs move them when a score exceeds its query's offset by more than 8 (P
       // then stays within [0, 256]), decided by a vote of the group on every pair.  Fast
-      // pass: no vote; a score more than kOverflow above its offset (P would leave the
-      // range of fp16, or of e4m3 after the V-scale factor) marks the tile, whose output
-      // the careful pass then recomputes.
+      // pass: no per-pair test; the tile's partial row sums bound every P it made, and a
+      // tile whose sums pass kOverflow (P may have left the range of fp16, or of e4m3
+      // after the V-scale factor) is recomputed by the careful pass.
       bool slow;
       if constexpr (CAREFUL) {
+        float dmax = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) dmax = max3f(dmax, x[q], x[q + 1]);
         slow = named_vote_or(gbar, 128, fail || it == 0 || dmax > 8.f);
       } else {
         slow = it == 0;
-        if (!slow) overflow |= !(dmax <= (FP8 ? 8.f : 15.f));   // (NaN counts as overflow)
       }
       if (slow) {
         if (named_vote_or(gbar, 128, fail)) break;
@@ -596,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           ctl->fac[c0 + lane] = ex2_approx(-delta);
         }
         named_sync(gbar, 128);
-        // new offsets m + delta (m = 0 on a tile's first pair) into this lane's copy
-        if (it > 0) tmem_ld32(lane_addr + kColM + c0, m);
+        // new negated offsets -(m + delta) (m = 0 on a tile's first pair) into this lane's copy
+        if (it > 0) tmem_ld32(lane_addr + kColM + c0, mn);
         const float4* d4 = reinterpret_cast<const float4*>(ctl->red[g][0]);
         tmem_wait_ld();
 #pragma unroll
@@ -608,10 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           for (int e = 0; e < 4; ++e) {
             const int q = 4 * q4 + e;
             x[q] -= d[e];
-            m[q] = it > 0 ? m[q] + d[e] : d[e];
+            mn[q] = it > 0 ? mn[q] - d[e] : -d[e];
           }
         }
-        tmem_st32(lane_addr + kColM + c0, m);
+        tmem_st32(lane_addr + kColM + c0, mn);
         tmem_wait_st();
         if (it > 0) {
           const float4* f4 = reinterpret_cast<const float4*>(ctl->fac + c0);
@@ -649,15 +685,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         for (int q = 0; q < 32; q += 4) {
           // a quarter of the exponentials on the FMA pipe (see ex2_poly)
           const bool poly = (q & 12) == 12;
-          const float p0 = poly ? ex2_poly(x[q]) : ex2_approx(x[q]);
-          const float p1 = poly ? ex2_poly(x[q + 1]) : ex2_approx(x[q + 1]);
-          const float p2 = poly ? ex2_poly(x[q + 2]) : ex2_approx(x[q + 2]);
-          const float p3 = poly ? ex2_poly(x[q + 3]) : ex2_approx(x[q + 3]);
-          lp[q] += p0;
-          lp[q + 1] += p1;
-          lp[q + 2] += p2;
-          lp[q + 3] += p3;
-          pw[q >> 2] = pack_e4m3x4(p0 * pf, p1 * pf, p2 * pf, p3 * pf);
+          float p0 = poly ? ex2_poly(x[q]) : ex2_approx(x[q]);
+          float p1 = poly ? ex2_poly(x[q + 1]) : ex2_approx(x[q + 1]);
+          float p2 = poly ? ex2_poly(x[q + 2]) : ex2_approx(x[q + 2]);
+          float p3 = poly ? ex2_poly(x[q + 3]) : ex2_approx(x[q + 3]);
+          add2(lp[q], lp[q + 1], p0, p1);
+          add2(lp[q + 2], lp[q + 3], p2, p3);
+          mul2(p0, p1, pf, pf);
+          mul2(p2, p3, pf, pf);
+          pw[q >> 2] = pack_e4m3x4(p0, p1, p2, p3);
         }
       } else {
 #pragma unroll
@@ -666,13 +702,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           const bool poly = (q & 6) == 6;
           const float p0 = poly ? ex2_poly(x[q]) : ex2_approx(x[q]);
           const float p1 = poly ? ex2_poly(x[q + 1]) : ex2_approx(x[q + 1]);
-          lp[q] += p0;
-          lp[q + 1] += p1;
+          add2(lp[q], lp[q + 1], p0, p1);
           pw[q >> 1] = pack_half2(p0, p1);
         }
       }
-      // the P buffer was last read by the P V two pairs back (maybe in the previous tile)
-      if (gp > 1 && !fail) fail |= !mbar_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1, wc);
+      // the next pair's S, tested before this pair's stores so that the test's latency
+      // overlaps them (a stale "not yet" only means a wait at the top of the loop)
+      s_seen = it + 1 < npairs && !fail &&
+               mbar_test_wait(bar(ctl->s_full[(gp + 1) % kSBufs]), ((gp + 1) / kSBufs) & 1);
+      if (!p_free && !fail) fail |= !mbar_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1, wc);
       if constexpr (FP8)
         st_chunks_sw64<2>(sP + (gp & 1) * G::kPBytes, t, 2 * g, pw);
       else
@@ -685,6 +723,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
 
     // ------------------------------------------------------------ epilogue
     if constexpr (!CAREFUL) {
+      // each P of the tile is at most its thread's partial row sum
+      bool overflow = false;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) overflow |= !(lp[q] <= kOverflow);   // (NaN counts too)
       if (named_vote_or(gbar, 128, overflow) && t == 0) {
         const int slot = atomicAdd(redo, 1);
         if (slot < 2 * ntiles_all) redo[1 + slot] = tau;
