@@ -189,10 +189,6 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 // Writes NC 16-byte chunks (4 packed words each), logical chunks c0 .. c0 + NC - 1 of
 // row `row` of a SW128 tile (128-byte rows): chunk c goes to position c ^ (row % 8).
@@ -541,19 +537,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       vref = fmaxf(fmaxf(ctl->vref[g][0], ctl->vref[g][1]), fmaxf(ctl->vref[g][2], ctl->vref[g][3]));
       if (!(vref > 0.f)) vref = 1.f;
     }
-    // This thread's key block for pair `it` (-1: the padding half of an odd list) and,
-    // for fp8, its K and V scales, fetched one pair ahead.
+    // The key block of this warp's half of each pair (warps 0-1 of a group hold the
+    // pair's first block, warps 2-3 its second; -1: the padding half of an odd list).
+    // fp8 (with the block's K and V scales, a chain of dependent loads): lane l holds
+    // those of pair 32c + l, loaded once per 32 pairs and broadcast by a shuffle.  16-bit
+    // path: one load per pair, a pair ahead (measured faster there).
+    const int half = t >> 6;
+    int lane_jb = -1;
+    float lane_sk = 1.f, lane_sv = 1.f;
+    auto stage_list = [&](int c) {
+      const int pr = 32 * c + lane, e = 2 * pr + half;
+      lane_jb = (pr < npairs && e < kk_list) ? __ldg(L + e) : -1;
+      if constexpr (FP8) {
+        const bool in = lane_jb >= 0 && lane_jb < dm.nb;
+        lane_sk = in ? __ldg(sk + sbase_idx + lane_jb) : 1.f;
+        lane_sv = in ? __ldg(sv + sbase_idx + lane_jb) : 1.f;
+      }
+    };
+    // keys of the last block past N (its rows come from the tensor map's zero fill)
+    const bool ragged_tail = (dm.N & 63) != 0;
     auto key_block = [&](int it) {
       return (t < 64) ? __ldg(L + 2 * it) : ((2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : -1);
     };
-    int jb_next = key_block(0);
-    float sk_next = 1.f, sv_next = 1.f;
-    if constexpr (FP8) {
-      if (jb_next >= 0 && jb_next < dm.nb) {
-        sk_next = __ldg(sk + sbase_idx + jb_next);
-        sv_next = __ldg(sv + sbase_idx + jb_next);
-      }
-    }
+    int jb_next = FP8 ? -1 : key_block(0);
 
     // fp8: the second group starts each tile a little later, so that the two groups'
     // phases (exponentials and e4m3 packing on the special-function unit, the rest on the
@@ -577,18 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       tc_fence_before();
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
-      const int jb = jb_next;
-      const float skj = sk_next, svj = sv_next;
-      if (it + 1 < npairs) {
-        jb_next = key_block(it + 1);
-        if constexpr (FP8) {
-          if (jb_next >= 0 && jb_next < dm.nb) {
-            sk_next = __ldg(sk + sbase_idx + jb_next);
-            sv_next = __ldg(sv + sbase_idx + jb_next);
-          }
-        }
+      int jb;                                        // uniform over the warp
+      float skj = 1.f, svj = 1.f;
+      if constexpr (FP8) {
+        if ((it & 31) == 0) stage_list(it >> 5);
+        jb = __shfl_sync(0xffffffffu, lane_jb, it & 31);
+        skj = __shfl_sync(0xffffffffu, lane_sk, it & 31);
+        svj = __shfl_sync(0xffffffffu, lane_sv, it & 31);
+      } else {
+        jb = jb_next;
+        if (it + 1 < npairs) jb_next = key_block(it + 1);
       }
-      const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
       const float slt = FP8 ? sl2 * sqi * skj : sl2;
       if (it > 0) {
@@ -599,7 +604,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         for (int q = 0; q < 32; q += 2) mul2(x[q], x[q + 1], slt, slt);
       }
       // keys past the end of the sequence and the padding half of an odd list (rare pairs)
-      if (__any_sync(0xffffffffu, !valid)) {
+      const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
+      bool any_invalid;
+      if constexpr (FP8)   // the test is uniform over the warp but for a failed wait
+        any_invalid = !ok || jb < 0 || jb >= dm.nb || (ragged_tail && jb == dm.nb - 1);
+      else
+        any_invalid = __any_sync(0xffffffffu, !valid);
+      if (any_invalid) {
         if (!valid) {
 #pragma unroll
           for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
