@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "rola_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace rola {
 namespace {
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(256, 2) score_kernel(Dims dm, const float* __r
   for (int ch = 0; ch < nch; ++ch) {
     const int buf = ch & 1;
     if (ch + 1 < nch) load((ch + 1) * kKC);
-#pragma unroll 2
+#pragma unroll 1
     for (int c = 0; c < kKC; ++c) {
       const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8]);
       const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8 + 4]);
@@ -193,10 +194,12 @@ __global__ void __launch_bounds__(256, 2) score_kernel(Dims dm, const float* __r
       const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][c][tx * 8 + 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      // two scores per packed f32x2 FMA (each rounded as fmaf: the chains stay exact)
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(av[a], bv[e], acc[a][e]);
+        for (int e = 0; e < 8; e += 2)
+          sm100::fma2(acc[a][e], acc[a][e + 1], av[a], av[a], bv[e], bv[e + 1], acc[a][e], acc[a][e + 1]);
     }
     if (ch + 1 < nch) store(buf ^ 1);   // the other buffer was last read before the barrier below
     __syncthreads();
@@ -220,13 +223,16 @@ __global__ void __launch_bounds__(256, 2) score_kernel(Dims dm, const float* __r
 // ------------------------------------------------------------------ top-k per row
 
 constexpr int kTopkWarps = 8;
+constexpr int kTopkCand = 256;   // keys left after the first digit, kept apart (if they fit)
 
 __host__ __device__ inline size_t topk_smem(int nbp) {
-  return sizeof(uint32_t) * ((size_t)kTopkWarps * nbp + 256 * kTopkWarps);
+  return sizeof(uint32_t) * ((size_t)kTopkWarps * (nbp + 256 + kTopkCand));
 }
 
 // One warp per row (b, h, i): 4-pass 8-bit radix select of the k-th largest score, then
-// one pass in index order emits the kept block indices (ties -> lower index).
+// one pass in index order emits the kept block indices (ties -> lower index).  The keys
+// whose first digit is the selected one are gathered after the first pass (when at most
+// kTopkCand), so that the other three passes read only them.
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const float* __restrict__ scores,
                                                                int nbp, int32_t* __restrict__ col_idx,
                                                                int* __restrict__ status) {
@@ -238,6 +244,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const fl
   const int nb = dm.nb, kk = dm.k;
   uint32_t* key = tsm + warp * nbp;
   uint32_t* hist = tsm + kTopkWarps * nbp + warp * 256;
+  uint32_t* cand = tsm + kTopkWarps * (nbp + 256) + warp * kTopkCand;
   const float* src = scores + row * nbp;
   const unsigned full = 0xffffffffu;
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -251,16 +258,37 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const fl
   __syncwarp();
   uint32_t prefix = 0, pmask = 0;
   int need = kk;
+  const uint32_t* src_keys = key;   // keys the passes read: all, then the gathered ones
+  int nsrc = nb;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
+    if (pass == 1) {
+      // gather the keys that still match the prefix, in any order (counts are all that
+      // the remaining passes take from them)
+      int nc = 0;
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t u = j < nb ? key[j] : 0u;
+        const bool in = j < nb && (u & pmask) == prefix;
+        const unsigned bin = __ballot_sync(full, in);
+        const int pos = nc + __popc(bin & lt_mask);
+        if (in && pos < kTopkCand) cand[pos] = u;
+        nc += __popc(bin);
+      }
+      if (nc <= kTopkCand) {
+        src_keys = cand;
+        nsrc = nc;
+      }
+      __syncwarp();
+    }
     for (int bb = lane; bb < 256; bb += 32) hist[bb] = 0;
     __syncwarp();
     // Lanes with equal digits are merged first (__match_any_sync), so a bin shared by
     // most keys (e.g. the exponent byte in the first pass) costs one atomic per step.
-    for (int j0 = 0; j0 < nb; j0 += 32) {
+    for (int j0 = 0; j0 < nsrc; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t u = j < nb ? key[j] : 0u;
-      const uint32_t digit = (j < nb && (u & pmask) == prefix) ? ((u >> shift) & 255u) : 256u;
+      const uint32_t u = j < nsrc ? src_keys[j] : 0u;
+      const uint32_t digit = (j < nsrc && (u & pmask) == prefix) ? ((u >> shift) & 255u) : 256u;
       const unsigned peers = __match_any_sync(full, digit);
       if (digit != 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
     }

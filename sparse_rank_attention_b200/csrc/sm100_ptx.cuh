@@ -97,6 +97,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   return mbar_wait_slow(bar, parity, w.abort, w.status, w.limit_cycles, honour_abort);
 }
 
+// ------------------------------------------------------------------ packed fp32
+
+// Two fp32 lanes per instruction (the packed f32x2 operations of sm_100; each lane is
+// rounded exactly as its scalar counterpart): d = a * b + c, d += a, d *= b.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n .reg .b64 a, b, c, d;\n mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %5};\n"
+      " mov.b64 c, {%6, %7};\n fma.rn.f32x2 d, a, b, c;\n mov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n .reg .b64 a, d;\n mov.b64 a, {%2, %3};\n mov.b64 d, {%0, %1};\n"
+      " add.rn.f32x2 d, d, a;\n mov.b64 {%0, %1}, d;\n}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float b0, float b1) {
+  asm("{\n .reg .b64 b, d;\n mov.b64 b, {%2, %3};\n mov.b64 d, {%0, %1};\n"
+      " mul.rn.f32x2 d, d, b;\n mov.b64 {%0, %1}, d;\n}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(b0), "f"(b1));
+}
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------------------------ fences / barriers
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
