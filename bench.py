@@ -216,6 +216,8 @@ def main():
     ap.add_argument("--impl", default="rola", choices=["rola", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--gate", default="head", choices=["head", "token"],
+                    help="gain of the linear branch per head (default) or per token and head")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     w = synth.WORKLOADS[args.workload]
@@ -254,7 +256,10 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     rola.load()
     inp = synth.make_inputs(w, seed=rank, device=dev)
-    plan = rola.Plan.for_workload(w, device=dev)
+    per_token = args.gate == "token"
+    if per_token:
+        inp["g"] = synth.make_gate(w, seed=100 + rank, device=dev)   # [B, N, H]
+    plan = rola.Plan.for_workload(w, device=dev, gate_per_token=per_token)
     out = torch.empty_like(inp["q"])
     q, k, v, Wq, Wk, g = (inp[x] for x in ("q", "k", "v", "Wq", "Wk", "g"))
     stream = torch.cuda.current_stream()
@@ -376,7 +381,7 @@ def main():
         assert plan.poll_status() == 0
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not per_token:
         r = oracle_sample(w, seconds_hint=15.0)
         cpu = {"value": r["value"], "unit": UNIT, "cores": r["cores"], "kind": "oracle",
                "sample": r["sample"], "seconds": r["seconds"]}
@@ -389,6 +394,7 @@ def main():
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "grid": list(w.grid),
                            "d": w.d, "r": w.r, "topk": w.topk, "kept_blocks_per_row": plan.k,
                            "blocks": plan.nb, "kept_block_tflop": flops / 1e12,
+                           "gate": "per-token" if per_token else "per-head",
                            "l2": "inputs (3 x 774 MB) larger than L2 (126 MB); no flush",
                            "parallelism": f"replicas x{ws} (independent forward per GPU)"},
                 "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,

@@ -95,12 +95,17 @@ typedef struct {
   double rope_base;              /* rotary frequency base, > 1 (10000)                      */
   float softmax_scale;           /* logit scale; 0 = 1/sqrt(d)                              */
   rola_dtype dtype;
+  int gate_per_token;            /* 0: the gain g is per head, g[H]; 1: per token and head, */
+                                 /* g[B, N, H] fp32 (an input-dependent gate, e.g. computed  */
+                                 /* from the layer input by the gate_proj / gate_bias        */
+                                 /* parameters the pages add, applied as out = O_sparse +   */
+                                 /* g[b, n, h] * O_lin)                                       */
 } rola_params;
 
 typedef struct rola_plan_s* rola_plan_t;
 
 /* Fills *p with defaults: B=H=1, N=0, d=128, r=32, block 64, topk 0.1, grid (1,1,0),
- * default rotary split, base 10000, scale 0 (1/sqrt(d)), ROLA_BF16. */
+ * default rotary split, base 10000, scale 0 (1/sqrt(d)), ROLA_BF16, per-head gain. */
 ROLA_API rola_status rola_params_default(rola_params* p);
 
 /* Number of 64-token blocks nb and kept blocks per query block k for *p. */
@@ -130,7 +135,8 @@ ROLA_API rola_status rola_linear_state(rola_plan_t plan, const void* k, const vo
                               rola_stream_t stream);
 
 /* Steps 3-5: sparse attention over the kept blocks with the linear branch and the
- * combination fused into its epilogue; writes out [B, N, H, d] once.  Uses the block
+ * combination fused into its epilogue; writes out [B, N, H, d] once.  g: fp32 gains,
+ * [H] or, with gate_per_token, [B, N, H] (device memory, 16-byte aligned).  Uses the block
  * lists and the state the two calls above left in the workspace (in ROLA_FP8_E4M3 mode
  * also their e4m3 copies of q, k, v, which must come from the same q, k, v). */
 ROLA_API rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const void* v,

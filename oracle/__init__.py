@@ -9,7 +9,8 @@ module builds that file with g++ when the shared object is missing or stale, and
 marshals numpy arrays in and out.  The definition it follows, and where each step
 comes from on the pages about SparkDiffusion / RoLA, is in the header of the C++ file.
 
-Shape conventions: q, k, v are [B, N, H, d]; Wq, Wk are [H, d, r]; g is [H].
+Shape conventions: q, k, v are [B, N, H, d]; Wq, Wk are [H, d, r]; g is [H], or [B, N, H]
+for a per-token gate (``make_shape(..., gate_per_token=True)``).
 """
 from __future__ import annotations
 
@@ -47,6 +48,7 @@ class Shape(ctypes.Structure):
         ("grid_t", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
         ("pairs_t", ctypes.c_int), ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int),
         ("rope_base", ctypes.c_double), ("scale", ctypes.c_double), ("topk", ctypes.c_double),
+        ("gate_per_token", ctypes.c_int),
     ]
 
 
@@ -87,7 +89,8 @@ def default_pairs(r: int, grid: tuple[int, int, int]) -> tuple[int, int, int]:
     return (P - 2 * hw, hw, hw)
 
 
-def make_shape(B, H, N, d, r, topk, grid=None, pairs=None, rope_base=10000.0, scale=None) -> Shape:
+def make_shape(B, H, N, d, r, topk, grid=None, pairs=None, rope_base=10000.0, scale=None,
+               gate_per_token=False) -> Shape:
     grid = tuple(grid) if grid is not None else (1, 1, N)
     assert grid[0] * grid[1] * grid[2] == N
     pairs = tuple(pairs) if pairs is not None and sum(pairs) > 0 else default_pairs(r, grid)
@@ -95,7 +98,7 @@ def make_shape(B, H, N, d, r, topk, grid=None, pairs=None, rope_base=10000.0, sc
     if scale is None or scale == 0:
         scale = 1.0 / math.sqrt(d)
     return Shape(B, H, N, d, r, grid[0], grid[1], grid[2], pairs[0], pairs[1], pairs[2],
-                 float(rope_base), float(scale), float(topk))
+                 float(rope_base), float(scale), float(topk), int(bool(gate_per_token)))
 
 
 def _f32(x) -> np.ndarray:
@@ -104,6 +107,13 @@ def _f32(x) -> np.ndarray:
 
 def _f64(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _gain(s: Shape, g) -> np.ndarray:
+    g = _f64(g)
+    want = s.B * s.N * s.H if s.gate_per_token else s.H
+    assert g.size == want, f"g has {g.size} values, the shape needs {want}"
+    return g
 
 
 def _p(a: np.ndarray):
@@ -167,7 +177,7 @@ def attend_blocks(s: Shape, q, k, v, Wq, g, col_idx, S, z, blocks, pos=None):
     [n, 64, d] float64; rows past N are zero.
     """
     q, k, v, Wq = _f32(q), _f32(k), _f32(v), _f32(Wq)
-    g = _f64(g); S = _f64(S); z = _f64(z)
+    g = _gain(s, g); S = _f64(S); z = _f64(z)
     col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
     blocks = np.ascontiguousarray(np.asarray(blocks, dtype=np.int32).reshape(-1, 3))
     pos = positions(s) if pos is None else _f64(pos)
@@ -216,7 +226,7 @@ def dequantize_blocks(s: Shape, codes, scales) -> np.ndarray:
 def forward(s: Shape, q, k, v, Wq, Wk, g):
     """Whole forward pass.  Returns (out [B,N,H,d] float64, col_idx [B,H,nb,k])."""
     q, k, v, Wq, Wk = _f32(q), _f32(k), _f32(v), _f32(Wq), _f32(Wk)
-    g = _f64(g)
+    g = _gain(s, g)
     nb = num_blocks(s.N)
     kk = keep_count(nb, s.topk)
     out = np.zeros((s.B, s.N, s.H, s.d))

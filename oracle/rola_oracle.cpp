@@ -66,6 +66,7 @@ struct rola_oracle_shape {
   double rope_base;               // frequency base (10000)
   double scale;                   // softmax logit scale
   double topk;                    // keep ratio in (0, 1]
+  int gate_per_token;             // g is [B][N][H] (a gain per token and head), else [H]
 };
 
 int rola_oracle_num_blocks(int N) { return (N + kBlock - 1) / kBlock; }
@@ -226,7 +227,10 @@ void rola_oracle_linear_state(const rola_oracle_shape* s, const float* k, const 
 
 // Output of the listed query blocks.  blocks: nrows triples (b, h, i).
 // For each listed block, rows [0, 64) of the three outputs (each [nrows][64][d]) hold
-//   sparse: O_sparse, lin: O_lin, out: O_sparse + g_h * O_lin
+//   sparse: O_sparse, lin: O_lin, out: O_sparse + g * O_lin
+// with g = g_h, or g_{n,h} of the token for a per-token gate (the gate_proj / gate_bias
+// parameters of the README's sparse-finetuning section make the gate input-dependent;
+// their values per token and head are an input here)
 // for the valid tokens of the block; rows past N are left at 0.
 void rola_oracle_attend_blocks(const rola_oracle_shape* s, const float* q, const float* k,
                                const float* v, const float* Wq, const double* g,
@@ -285,8 +289,9 @@ void rola_oracle_attend_blocks(const rola_oracle_shape* s, const float* q, const
         ol[(size_t)row * d + c] = num / lden;
       }
       // Combination (reading 6).
+      const double gn = s->gate_per_token ? g[((size_t)b * N + n) * H + h] : g[h];
       for (int c = 0; c < d; ++c)
-        oo[(size_t)row * d + c] = os[(size_t)row * d + c] + g[h] * ol[(size_t)row * d + c];
+        oo[(size_t)row * d + c] = os[(size_t)row * d + c] + gn * ol[(size_t)row * d + c];
     }
   }
 }

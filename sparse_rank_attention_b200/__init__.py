@@ -52,7 +52,7 @@ class RolaParams(ctypes.Structure):
         ("rope_pairs_t", ctypes.c_int), ("rope_pairs_h", ctypes.c_int),
         ("rope_pairs_w", ctypes.c_int),
         ("rope_base", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-        ("dtype", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("gate_per_token", ctypes.c_int),
     ]
 
 
@@ -117,7 +117,7 @@ def _check(code: int, where: str):
 
 
 def make_params(B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
-                softmax_scale=0.0, dtype="bf16") -> RolaParams:
+                softmax_scale=0.0, dtype="bf16", gate_per_token=False) -> RolaParams:
     p = RolaParams()
     load().rola_params_default(ctypes.byref(p))
     grid = tuple(grid) if grid is not None else (1, 1, N)
@@ -128,6 +128,7 @@ def make_params(B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000
     p.rope_base = float(rope_base)
     p.softmax_scale = float(softmax_scale)
     p.dtype = DTYPES[dtype] if isinstance(dtype, str) else int(dtype)
+    p.gate_per_token = int(bool(gate_per_token))
     return p
 
 
@@ -158,8 +159,9 @@ class Plan:
     """A rola_plan bound to a workspace tensor allocated here with torch."""
 
     def __init__(self, B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
-                 softmax_scale=0.0, dtype="bf16", device="cuda"):
-        self.params = make_params(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype)
+                 softmax_scale=0.0, dtype="bf16", device="cuda", gate_per_token=False):
+        self.params = make_params(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype,
+                                  gate_per_token)
         self.dtype = dtype
         self.nb, self.k = keep_count(self.params)
         self.workspace_bytes = workspace_size(self.params)
@@ -170,8 +172,9 @@ class Plan:
         self._h = h
 
     @classmethod
-    def for_workload(cls, w, device="cuda"):
-        return cls(w.B, w.H, w.N, w.d, w.r, w.topk, w.grid, w.pairs, dtype=w.dtype, device=device)
+    def for_workload(cls, w, device="cuda", gate_per_token=False):
+        return cls(w.B, w.H, w.N, w.d, w.r, w.topk, w.grid, w.pairs, dtype=w.dtype, device=device,
+                   gate_per_token=gate_per_token)
 
     def close(self):
         if getattr(self, "_h", None):
@@ -273,12 +276,14 @@ def select_blocks_noalloc(params: RolaParams, q, k, col_idx, stream=None) -> int
 
 def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
             softmax_scale=0.0, dtype=None, out=None):
-    """One-shot RoLA forward (builds a plan and workspace for this call)."""
+    """One-shot RoLA forward (builds a plan and workspace for this call).  g is [H], or
+    [B, N, H] for a per-token gate."""
     B, N, H, d = q.shape
     r = Wq.shape[-1]
     if dtype is None:
         dtype = "f32" if q.dtype == torch.float32 else "bf16"
-    plan = Plan(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype, q.device)
+    plan = Plan(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype, q.device,
+                gate_per_token=g.dim() > 1)
     try:
         return plan.forward(q, k, v, Wq, Wk, g, out)
     finally:

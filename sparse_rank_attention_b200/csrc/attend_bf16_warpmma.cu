@@ -4,7 +4,7 @@
 // Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
 // Preserving Global Context at Extreme Sparsity" (block-sparse softmax branch plus a
 // low-rank linear branch with rotary positions); README sparse-finetuning section
-// (proj_q, and the gate read here as a per-head gain g).
+// (proj_q, and the gate read here as a gain g per head or per token and head).
 //
 // One CTA per (b, h, 64-token query block), 4 warps x 16 query rows:
 //   for each kept key block j (ascending):  S = Q K_j^T, online softmax, O += P V_j
@@ -233,16 +233,15 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
       u[nt][e] = phi(u[nt][e]);
       den[e >> 1] += u[nt][e] * sz[nt * 8 + 2 * t4 + (e & 1)];
     }
-  const float gh = g[h];
   float coef[2];
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     float dd = den[hh];
     dd += __shfl_xor_sync(0xffffffffu, dd, 1);
     dd += __shfl_xor_sync(0xffffffffu, dd, 2);
-    coef[hh] = gh / dd;
     const int n = i * kBlock + 16 * warp + g8 + 8 * hh;
     const bool ok = n < dm.N;
+    coef[hh] = (ok ? g[gain_index(dm, b, n, h)] : 0.f) / dd;
 #pragma unroll
     for (int nt = 0; nt < NTU; ++nt) {
       const float2 cs = ok ? rope_cs(dm, rope, n, nt * 4 + t4) : make_float2(1.f, 0.f);

@@ -7,7 +7,8 @@
 // Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
 // Preserving Global Context at Extreme Sparsity" (block-sparse softmax branch plus a
 // low-rank linear branch with rotary positions); README sparse-finetuning section
-// (proj_q and the gate parameters; the gate is read here as a per-head gain g).
+// (proj_q and the gate parameters; the gate is read here as a gain g per head or per
+// token and head).
 #include "rola_internal.cuh"
 
 namespace rola {
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(64) attend_f32_kernel(
     ur[2 * c + 1] = cs.y * u[2 * c] + cs.x * u[2 * c + 1];
   }
   if (!valid) return;
-  const float gh = g[h];
+  const float gh = g[gain_index(dm, b, n, h)];
   const float inv_l = 1.f / l, inv_den = 1.f / den;
   float* ob = out + ((size_t)b * dm.N + n) * rs + (size_t)h * D;
 #pragma unroll

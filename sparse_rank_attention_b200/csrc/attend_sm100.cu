@@ -4,7 +4,7 @@
 // Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
 // Preserving Global Context at Extreme Sparsity" (block-sparse softmax branch plus a
 // low-rank linear branch with rotary positions); README sparse-finetuning section
-// (proj_q, and the gate read here as a per-head gain g).
+// (proj_q, and the gate read here as a gain g per head or per token and head).
 //
 // Why the transposed tile: tcgen05.mma needs M = 128 rows for full rate, but a query
 // block has 64 tokens and every query block keeps its own key blocks.  So the M side

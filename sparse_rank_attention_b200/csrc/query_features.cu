@@ -5,7 +5,8 @@
 //     all-zero block; code = RN-sat(x * (1 / scale)));
 //   * the query side of the linear branch (step 5):
 //       u_n = phi(q_n Wq_h)            (r values per token, phi = elu + 1)
-//       gden_n = g_h / (u_n . z_h)     (the gain over the unrotated normaliser)
+//       gden_n = g / (u_n . z_h)       (the gain over the unrotated normaliser; g = g_h,
+//                                       or g_{n,h} for a per-token gate)
 //       (R(p_n) u_n) split into bf16 hi + lo, stored transposed ([rank][64 tokens]) as the
 //       exact 128-byte-swizzled shared-memory image the attention epilogue multiplies
 //       with S_h on the tensor cores (one bulk copy there, no per-element work).
@@ -13,7 +14,7 @@
 // Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
 // Preserving Global Context at Extreme Sparsity" (high-energy block selection; low-rank
 // linear branch with rotary positions); README sparse-finetuning section (proj_q; the
-// gate read as a per-head gain).
+// gate read as a gain per head or per token and head).
 #include "rola_internal.cuh"
 #include "warp_mma.cuh"
 
@@ -116,12 +117,12 @@ __global__ void __launch_bounds__(128) query_features_kernel(
       mma_bf16(f[nt + 1], af, bf + 2);
     }
   }
-  const float gh = g[h];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int row = 16 * warp + g8 + 8 * half;     // token within the block
     const int n = i * kBlock + row;
     const bool ok = n < dm.N;
+    const float gh = ok ? g[gain_index(dm, b, n, h)] : 0.f;
     const TokPos pos = token_pos(dm, ok ? n : 0);
     float den = 0.f;
 #pragma unroll

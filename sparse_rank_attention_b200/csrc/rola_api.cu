@@ -54,6 +54,7 @@ rola_status check_params(const rola_params* p) {
   if (p->dtype != ROLA_F32 && p->dtype != ROLA_BF16 && p->dtype != ROLA_FP8_E4M3)
     return ROLA_ERR_INVALID_ARG;
   if (p->dtype == ROLA_FP8_E4M3 && p->d != 128) return ROLA_ERR_UNSUPPORTED;  // tcgen05 tile only
+  if (p->gate_per_token != 0 && p->gate_per_token != 1) return ROLA_ERR_INVALID_ARG;
   const int nb = (p->N + rola::kBlock - 1) / rola::kBlock;
   if (nb > kMaxBlocks) return ROLA_ERR_UNSUPPORTED;
   if ((long long)p->B * p->H * nb > (1ll << 31) / 64) return ROLA_ERR_UNSUPPORTED;
@@ -99,6 +100,7 @@ Dims make_dims(const rola_params& p) {
   dm.nchunk = (p.N + dm.chunk_tok - 1) / dm.chunk_tok;
   dm.scale = p.softmax_scale > 0.f ? p.softmax_scale : (float)(1.0 / std::sqrt((double)p.d));
   dm.rope_base = p.rope_base;
+  dm.gate_per_token = p.gate_per_token;
   return dm;
 }
 
@@ -177,6 +179,7 @@ rola_status rola_params_default(rola_params* p) {
   p->rope_base = 10000.0;
   p->softmax_scale = 0.f;
   p->dtype = ROLA_BF16;
+  p->gate_per_token = 0;
   return ROLA_OK;
 }
 

@@ -31,7 +31,13 @@ struct Dims {
   int nchunk;                 // linear-state partial sums per (b, h)
   float scale;                // softmax logit scale
   double rope_base;
+  int gate_per_token;         // gain g per token and head [B, N, H] (else per head [H])
 };
+
+// The gain of token n of (b, h): g[H], or g[B, N, H] for a per-token gate.
+__host__ __device__ inline size_t gain_index(const Dims& dm, int b, int n, int h) {
+  return dm.gate_per_token ? ((size_t)b * dm.N + n) * dm.H + h : (size_t)h;
+}
 
 // Device pointers carved out of the caller's workspace.
 struct Workspace {

@@ -137,4 +137,12 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> dict:
     return {"q": q, "k": k, "v": v, "Wq": Wq, "Wk": Wk, "g": g}
 
 
-__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs"]
+def make_gate(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """A per-token, per-head gate [B, N, H] (fp32, uniform in (0, 1), the range of a
+    sigmoid gate) for workload ``w``, from its own seeded stream."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.rand((w.B, w.N, w.H), generator=gen, device=device, dtype=torch.float32)
+
+
+__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs", "make_gate"]

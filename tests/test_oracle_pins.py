@@ -385,6 +385,34 @@ def test_zero_gain_gives_sparse_branch_and_gain_is_linear():
         np.testing.assert_allclose(out[t], sp[t] + gain[h] * li[t], atol=1e-13)
 
 
+def test_per_token_gate_equal_to_the_head_gain_reproduces_the_per_head_output():
+    B, N, H, d, r = 2, 200, 3, 16, 8
+    q, k, v, Wq, Wk, gain = _rand_inputs(B, N, H, d, r, seed=21)
+    s = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 100))
+    st = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 100), gate_per_token=True)
+    out_h, col_h = O.forward(s, q, k, v, Wq, Wk, gain)
+    g_tok = np.broadcast_to(gain, (B, N, H)).copy()
+    out_t, col_t = O.forward(st, q, k, v, Wq, Wk, g_tok)
+    np.testing.assert_array_equal(col_t, col_h)
+    np.testing.assert_array_equal(out_t, out_h)
+
+
+def test_per_token_gate_scales_each_tokens_linear_branch_by_its_own_gain():
+    # out = O_sparse + g[b, n, h] * O_lin: with random gains, out(g) - out(0) must be
+    # g[b, n, h] times out(1) - out(0) for every token of every batch entry and head (a
+    # gain read at a transposed index, or per head, fails this).
+    B, N, H, d, r = 2, 150, 3, 16, 8
+    q, k, v, Wq, Wk, _ = _rand_inputs(B, N, H, d, r, seed=22)
+    st = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 3, 50), gate_per_token=True)
+    g = _rng(23).uniform(0.0, 1.0, (B, N, H))
+    out_g, _ = O.forward(st, q, k, v, Wq, Wk, g)
+    out_0, _ = O.forward(st, q, k, v, Wq, Wk, np.zeros((B, N, H)))
+    out_1, _ = O.forward(st, q, k, v, Wq, Wk, np.ones((B, N, H)))
+    lin = out_1 - out_0
+    assert np.abs(lin).max() > 0.1
+    np.testing.assert_allclose(out_g - out_0, g[..., None] * lin, rtol=0, atol=1e-12)
+
+
 def test_forward_equals_composed_steps_and_lists_are_valid():
     B, N, H, d, r = 2, 330, 2, 16, 8
     q, k, v, Wq, Wk, gain = _rand_inputs(B, N, H, d, r, seed=15)
