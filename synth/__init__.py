@@ -70,6 +70,10 @@ for _t in (0.03, 0.05, 0.10, 0.25, 1.0):
     WORKLOADS[_n] = replace(WORKLOADS["wan21_14b_480p"], name=_n, topk=_t)
 WORKLOADS["wan21_14b_480p_fp8"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_480p_fp8",
                                           dtype="fp8")
+# Classifier-free guidance batch of the multi-step CFG sampler (the pages' teacher and
+# reference runs): the conditional and unconditional inputs as B = 2, 14B at 480P.
+WORKLOADS["wan21_14b_480p_cfg_b2"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_480p_cfg_b2",
+                                             B=2)
 WORKLOADS["wan21_14b_480p_dense_g0"] = replace(WORKLOADS["wan21_14b_480p"],
                                                name="wan21_14b_480p_dense_g0", topk=1.0,
                                                g_const=0.0)

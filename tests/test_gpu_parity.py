@@ -129,7 +129,8 @@ def _compare_sampled(w, n_heads=3, n_blocks=12, seed=0):
 
 
 @pytest.mark.parametrize("name", ["wan21_1p3b_480p", "wan21_14b_480p", "wan21_14b_720p",
-                                  "wan21_14b_480p_dense_g0", "wan21_14b_480p_topk0.25"])
+                                  "wan21_14b_480p_dense_g0", "wan21_14b_480p_topk0.25",
+                                  "wan21_14b_480p_cfg_b2"])
 def test_wan_shapes_sampled(name):
     _compare_sampled(synth.WORKLOADS[name])
 
