@@ -15,8 +15,9 @@
 // Layout of the work: a CTA owns one (b, h) and a chunk of whole 64-token blocks; the
 // chunk length is chosen on the host so that the CTAs fill the SMs in whole waves.  k and
 // v tiles (one block each: two TMA boxes of 64 tokens x 64 channels, 128-byte swizzle)
-// flow through a 4-stage ring of TMA copies completing on mbarriers, so three tiles are in
-// flight while one is processed; rows past N arrive as zeros.
+// flow through a 2-stage ring of TMA copies completing on mbarriers, so the next tile is in
+// flight while one is processed, with two CTAs per SM (two tiles in flight per SM); rows
+// past N arrive as zeros.
 // Per tile: warps 0-3 compute F = K Wk (mma.sync), phi, z and the rotation and store
 // the rotated features as bf16 hi + lo; meanwhile warps 4-5 pool k (and write its e4m3
 // copy) and warps 6-7 write the copy of v; then all 8 warps add F^T V into their 16
