@@ -135,6 +135,15 @@ def test_wan_shapes_sampled(name):
     _compare_sampled(synth.WORKLOADS[name])
 
 
+def test_longest_sequence_accepted_sampled():
+    """The largest block count the library accepts (6000 blocks: N = 384 000 tokens, one
+    head): every block list, mean and state entry, and sampled query blocks of the output."""
+    w = synth.custom("max_blocks_6000", B=1, H=1, N=6000 * 64, d=128, r=32, topk=0.01,
+                     grid=(20, 100, 192))
+    assert w.nb == 6000
+    _compare_sampled(w, n_heads=1, n_blocks=16, seed=3)
+
+
 def _rising_keys(inp, w, top=6.0):
     """Scales key block j by 1 + top * j / nb: later kept blocks score far above the first
     pair of each row, so the fast attention pass must hand tiles to the careful pass."""
