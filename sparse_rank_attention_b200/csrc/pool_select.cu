@@ -230,9 +230,11 @@ __host__ __device__ inline size_t topk_smem(int nbp) {
 }
 
 // One warp per row (b, h, i): 4-pass 8-bit radix select of the k-th largest score, then
-// one pass in index order emits the kept block indices (ties -> lower index).  The keys
-// whose first digit is the selected one are gathered after the first pass (when at most
-// kTopkCand), so that the other three passes read only them.
+// one pass in index order emits the kept block indices (ties -> lower index).  For
+// k <= 64 the select runs over few keys: the k-th largest of the 64 lane top-twos is a
+// lower bound of the answer, and only the keys at or above it (when at most kTopkCand)
+// are gathered and selected from.  Otherwise the first pass reads every key and the keys
+// still matching its digit are gathered for the other three.
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const float* __restrict__ scores,
                                                                int nbp, int32_t* __restrict__ col_idx,
                                                                int* __restrict__ status) {
@@ -248,47 +250,32 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const fl
   const float* src = scores + row * nbp;
   const unsigned full = 0xffffffffu;
   const unsigned lt_mask = (1u << lane) - 1u;
-  // Order-preserving map float -> uint32 (both zeros map to the key of +0).
+  // Order-preserving map float -> uint32 (both zeros map to the key of +0); each lane
+  // also keeps the two largest of its keys.
+  uint32_t top1 = 0, top2 = 0;
   for (int j = lane; j < nb; j += 32) {
     float f = src[j];
     if (f == 0.f) f = 0.f;
     const uint32_t u = __float_as_uint(f);
-    key[j] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t kj = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    key[j] = kj;
+    top2 = max(top2, min(top1, kj));
+    top1 = max(top1, kj);
   }
   __syncwarp();
-  uint32_t prefix = 0, pmask = 0;
-  int need = kk;
-  const uint32_t* src_keys = key;   // keys the passes read: all, then the gathered ones
-  int nsrc = nb;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (pass == 1) {
-      // gather the keys that still match the prefix, in any order (counts are all that
-      // the remaining passes take from them)
-      int nc = 0;
-      for (int j0 = 0; j0 < nb; j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t u = j < nb ? key[j] : 0u;
-        const bool in = j < nb && (u & pmask) == prefix;
-        const unsigned bin = __ballot_sync(full, in);
-        const int pos = nc + __popc(bin & lt_mask);
-        if (in && pos < kTopkCand) cand[pos] = u;
-        nc += __popc(bin);
-      }
-      if (nc <= kTopkCand) {
-        src_keys = cand;
-        nsrc = nc;
-      }
-      __syncwarp();
-    }
+
+  // One 8-bit radix step over keys[0, n) that match (prefix, pmask): picks the digit at
+  // `shift` of the need-th largest and updates prefix, pmask and need (the count still to
+  // take among keys equal to the prefix so far).  Lanes with equal digits are merged first
+  // (__match_any_sync), so a bin shared by most keys costs one atomic per step.
+  auto radix_step = [&](const uint32_t* keys, int n, int shift, uint32_t& prefix, uint32_t& pmask,
+                        int& need) {
     for (int bb = lane; bb < 256; bb += 32) hist[bb] = 0;
     __syncwarp();
-    // Lanes with equal digits are merged first (__match_any_sync), so a bin shared by
-    // most keys (e.g. the exponent byte in the first pass) costs one atomic per step.
-    for (int j0 = 0; j0 < nsrc; j0 += 32) {
+    for (int j0 = 0; j0 < n; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t u = j < nsrc ? src_keys[j] : 0u;
-      const uint32_t digit = (j < nsrc && (u & pmask) == prefix) ? ((u >> shift) & 255u) : 256u;
+      const uint32_t u = j < n ? keys[j] : 0u;
+      const uint32_t digit = (j < n && (u & pmask) == prefix) ? ((u >> shift) & 255u) : 256u;
       const unsigned peers = __match_any_sync(full, digit);
       if (digit != 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
     }
@@ -327,6 +314,51 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const fl
     prefix |= (uint32_t)digit << shift;
     pmask |= 255u << shift;
     __syncwarp();
+  };
+  // Gathers the keys that satisfy `in` into cand (in any order; counts are all the radix
+  // steps take from them).  Returns their number (those past kTopkCand are not stored).
+  auto gather = [&](auto in) {
+    int nc = 0;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t u = j < nb ? key[j] : 0u;
+      const bool take = j < nb && in(u);
+      const unsigned bin = __ballot_sync(full, take);
+      const int pos = nc + __popc(bin & lt_mask);
+      if (take && pos < kTopkCand) cand[pos] = u;
+      nc += __popc(bin);
+    }
+    __syncwarp();
+    return nc;
+  };
+
+  uint32_t prefix = 0, pmask = 0;
+  int need = kk;
+  bool done = false;
+  if (kk <= 64 && nb >= 64) {
+    // Bound from below: T = the kk-th largest of the 64 lane top-twos is a key with at least
+    // kk keys at or above it, so the kk-th largest key is >= T; the keys >= T (usually little
+    // more than kk) are gathered and the exact select runs over them alone.
+    cand[lane] = top1;
+    cand[32 + lane] = top2;
+    __syncwarp();
+    uint32_t tp = 0, tm = 0;
+    int tn = kk;
+    for (int pass = 0; pass < 4; ++pass) radix_step(cand, 64, 24 - 8 * pass, tp, tm, tn);
+    const int nc = gather([&](uint32_t u) { return u >= tp; });
+    if (nc <= kTopkCand) {
+      for (int pass = 0; pass < 4; ++pass) radix_step(cand, nc, 24 - 8 * pass, prefix, pmask, need);
+      done = true;
+    }
+  }
+  if (!done) {
+    // every key through the first digit; then the keys still matching it are gathered
+    // (when they fit) for the other three
+    radix_step(key, nb, 24, prefix, pmask, need);
+    const int nc = gather([&](uint32_t u) { return (u & pmask) == prefix; });
+    const uint32_t* src_keys = nc <= kTopkCand ? cand : key;
+    const int nsrc = nc <= kTopkCand ? nc : nb;
+    for (int pass = 1; pass < 4; ++pass) radix_step(src_keys, nsrc, 24 - 8 * pass, prefix, pmask, need);
   }
   // prefix is the k-th largest key; `need` elements equal to it are kept.
   int32_t* out = col_idx + row * kk;
