@@ -15,10 +15,13 @@
 // The softmax runs in two independent groups of four warps; group g owns the query
 // columns [32g, 32g + 32) of S^T and O^T.  Thread t of a group owns TMEM lane t: key t of
 // the pair for S^T and channel d = t for O^T.  The softmax max is per query (a TMEM
-// column), so it is kept lazily: each query's exponent offset m only moves when a new
-// score exceeds it by more than 8 (log2 units); that rare case takes an exact per-query
-// max across the 128 lanes and rescales the group's O^T columns.  Per-query sums l stay
-// per thread (partials over that thread's keys) until the end.
+// column spread over 128 lanes), so it is kept lazily.  Fast pass: each query's exponent
+// offset m is the exact column max of the tile's first pair and stays fixed; a tile whose
+// per-thread partial row sums (which bound every P it made) pass the range of P (2^15 for
+// fp16, 2^8 for e4m3) is listed for the careful pass, a second launch over the listed
+// tiles in which m moves whenever a score exceeds it by more than 8 (log2 units), by an
+// exact per-query max across the 128 lanes, rescaling the group's O^T columns and sums.
+// Per-query sums l stay per thread (partials over that thread's keys) until the end.
 //
 // Roles (384 threads, one role per warp so that a sleeping wait never holds another
 // role back): warp 0 = TMA producer of Q and the K ring, warp 1 = Q K^T issuer (and TMEM
