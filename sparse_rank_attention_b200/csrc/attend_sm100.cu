@@ -519,14 +519,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     // path: one load per pair, a pair ahead (measured faster there).
     const int half = t >> 6;
     int lane_jb = -1;
-    float lane_sk = 1.f, lane_sv = 1.f;
+    float lane_slt = sl2, lane_pf = 1.f;   // fp8: the pair's score scale and P factor
     auto stage_list = [&](int c) {
       const int pr = 32 * c + lane, e = 2 * pr + half;
       lane_jb = (pr < npairs && e < kk_list) ? __ldg(L + e) : -1;
       if constexpr (FP8) {
         const bool in = lane_jb >= 0 && lane_jb < dm.nb;
-        lane_sk = in ? __ldg(sk + sbase_idx + lane_jb) : 1.f;
-        lane_sv = in ? __ldg(sv + sbase_idx + lane_jb) : 1.f;
+        const float skb = in ? __ldg(sk + sbase_idx + lane_jb) : 1.f;
+        const float svb = in ? __ldg(sv + sbase_idx + lane_jb) : 1.f;
+        lane_slt = sl2 * sqi * skb;   // scale * log2(e) * sq_i * sk_j
+        lane_pf = svb / vref;         // sv_j / vref
       }
     };
     // keys of the last block past N (its rows come from the tensor map's zero fill)
@@ -559,18 +561,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(bar(ctl->s_empty[sb]));   // S is in registers: buffer free
       int jb;                                        // uniform over the warp
-      float skj = 1.f, svj = 1.f;
+      float slt = sl2, pf = 1.f;
       if constexpr (FP8) {
         if ((it & 31) == 0) stage_list(it >> 5);
         jb = __shfl_sync(0xffffffffu, lane_jb, it & 31);
-        skj = __shfl_sync(0xffffffffu, lane_sk, it & 31);
-        svj = __shfl_sync(0xffffffffu, lane_sv, it & 31);
+        slt = __shfl_sync(0xffffffffu, lane_slt, it & 31);
+        pf = __shfl_sync(0xffffffffu, lane_pf, it & 31);
       } else {
         jb = jb_next;
         if (it + 1 < npairs) jb_next = key_block(it + 1);
       }
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
-      const float slt = FP8 ? sl2 * sqi * skj : sl2;
       if (it > 0) {
 #pragma unroll
         for (int q = 0; q < 32; q += 2) fma2(x[q], x[q + 1], x[q], x[q + 1], slt, slt, mn[q], mn[q + 1]);
@@ -666,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       // P = 2^x (fp16, or e4m3 times sv_j / vref) and the per-thread partial row sums
       uint32_t pw[16];
       if constexpr (FP8) {
-        const float pf = svj / vref;
 #pragma unroll
         for (int q = 0; q < 32; q += 4) {
           // a quarter of the exponentials on the FMA pipe (see ex2_poly)
