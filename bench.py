@@ -45,7 +45,7 @@ LAUNCHES_PER_STEP = 7
 # 14B-480P workload, scaled to 720P by the token count (the streamed bytes grow with N); see
 # profiles/attend_sm100_wan21_14b_480p.md.  None where no capture of the current kernel exists.
 ATTEND_DRAM_BYTES = {"wan21_14b_720p": 1.519e9 * 75600 / 32760, "wan21_14b_480p": 1.519e9,
-                     "wan21_14b_720p_fp8": 0.9973e9 * 75600 / 32760, "wan21_14b_480p_fp8": 0.9973e9}
+                     "wan21_14b_720p_fp8": 0.9970e9 * 75600 / 32760, "wan21_14b_480p_fp8": 0.9970e9}
 
 
 def load_peaks():
