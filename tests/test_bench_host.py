@@ -59,3 +59,37 @@ def test_aggregate_counts_every_replica():
     # 2 replicas of 3.554 TFLOP each in 10 ms (the slowest rank) -> 710.8 TFLOP/s
     assert bench.aggregate_tflops(3_554_000_000_000, 10.0, 2) == pytest.approx(710.8)
     assert bench.aggregate_tflops(3_554_000_000_000, 10.0, 1) == pytest.approx(355.4)
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    env.update(env_extra or {})
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, cwd=root, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the oracle on the host and prints the same JSON
+    line as the library's arm (on a workload small enough for a unit test)."""
+    (line,) = _run_bench(["--impl", "reference", "--workload", "tiny_f32_h2_n1024", "--steps", "1",
+                          "--warmup", "1"])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["unit"] == "TFLOP/s" and line["config"]["workload"] == "tiny_f32_h2_n1024"
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == line["value"] and cpu["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    assert _run_bench(["--impl", "reference", "--workload", "tiny_f32_h2_n1024", "--steps", "1",
+                       "--warmup", "1"], {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
