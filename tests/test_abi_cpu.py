@@ -129,3 +129,20 @@ def test_fp8_configuration_host_rules():
     bufs = [ctypes.c_void_p(0x200000 + 0x10000 * j) for j in range(6)]
     assert lib.rola_get_fp8_copies(h, *bufs, None) == 1      # not an fp8 plan
     lib.rola_plan_destroy(h)
+
+
+def test_missing_library_fails_loudly_and_product_never_touches_the_oracle():
+    """No fallback: without librola.so the binding raises; and neither the package nor its
+    kernels import, link or read anything of the oracle (test infrastructure only)."""
+    import subprocess
+    import sys
+    code = ("import sparse_rank_attention_b200 as r; r.LIB_PATH = '/nonexistent/librola.so'; r._lib = None\n"
+            "try:\n    r.load()\nexcept RuntimeError as e:\n    print('raised', 'missing' in str(e))\n")
+    p = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120)
+    assert p.stdout.strip() == "raised True", p.stdout + p.stderr
+    pkg = os.path.join(ROOT, "sparse_rank_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert re.search(r"\boracle\b", text) is None, f"{f} mentions the oracle"
