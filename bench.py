@@ -8,6 +8,9 @@ the sparse branch, 4*d*c_i*c_j summed over every kept (query block i, key block 
 pair (c = valid tokens of a block), divided by the step time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rola|reference]
+                  [--gate head|token] [--no-e2e] [--no-cpu-baseline]
+
+``--gate token`` feeds a gain per token and head (g [B, N, H]) instead of per head.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs an independent forward of the
 same workload (different seed), no collective on the data path ("scaling": "weak");
