@@ -1,7 +1,9 @@
 """GPU parity of the per-token (input-dependent) gate against the CPU oracle.
 
 With ``gate_per_token`` the gain that scales the linear branch is read per token and head,
-g[B, N, H] (the values a gate built from the gate_proj / gate_bias parameters would give);
+g[B, N, H] (the values a gate built from the gate_proj / gate_bias parameters would give; the
+README's sparse-finetuning section on the SparkDiffusion page names them among RoLA's
+parameters without fixing their form);
 everything else is the per-head computation.  Each compute path (tcgen05 bf16 and fp8 at
 head dim 128, the head-dim-64 path, the fp32 path) is compared in full with the oracle at
 the same tolerances as the per-head tests, and a per-token gate equal to the per-head gains
