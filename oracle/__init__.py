@@ -9,8 +9,10 @@ module builds that file with g++ when the shared object is missing or stale, and
 marshals numpy arrays in and out.  The definition it follows, and where each step
 comes from on the pages about SparkDiffusion / RoLA, is in the header of the C++ file.
 
-Shape conventions: q, k, v are [B, N, H, d]; Wq, Wk are [H, d, r]; g is [H], or [B, N, H]
-for a per-token gate (``make_shape(..., gate_per_token=True)``).
+Shape conventions: q, k, v are [B, N, H, d]; Wq, Wk are [H, d, r]; g is [H] (a gain per
+head), [B, N, H] for a per-token gate (``make_shape(..., gate="token")``), or, for the gate
+computed from the query (``gate="proj"``), gate_proj [H, d] followed by gate_bias [H]
+(H*(d+1) values), the gain then being sigmoid(q . gate_proj_h + gate_bias_h).
 """
 from __future__ import annotations
 
@@ -48,7 +50,7 @@ class Shape(ctypes.Structure):
         ("grid_t", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
         ("pairs_t", ctypes.c_int), ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int),
         ("rope_base", ctypes.c_double), ("scale", ctypes.c_double), ("topk", ctypes.c_double),
-        ("gate_per_token", ctypes.c_int),
+        ("gate_mode", ctypes.c_int),
     ]
 
 
@@ -89,8 +91,14 @@ def default_pairs(r: int, grid: tuple[int, int, int]) -> tuple[int, int, int]:
     return (P - 2 * hw, hw, hw)
 
 
+GATES = {"head": 0, "token": 1, "proj": 2}
+
+
 def make_shape(B, H, N, d, r, topk, grid=None, pairs=None, rope_base=10000.0, scale=None,
-               gate_per_token=False) -> Shape:
+               gate_per_token=False, gate=None) -> Shape:
+    """gate: "head" (g [H]), "token" (g [B, N, H]) or "proj" (g = gate_proj [H, d] then
+    gate_bias [H]); ``gate_per_token=True`` is "token"."""
+    gate = gate or ("token" if gate_per_token else "head")
     grid = tuple(grid) if grid is not None else (1, 1, N)
     assert grid[0] * grid[1] * grid[2] == N
     pairs = tuple(pairs) if pairs is not None and sum(pairs) > 0 else default_pairs(r, grid)
@@ -98,7 +106,7 @@ def make_shape(B, H, N, d, r, topk, grid=None, pairs=None, rope_base=10000.0, sc
     if scale is None or scale == 0:
         scale = 1.0 / math.sqrt(d)
     return Shape(B, H, N, d, r, grid[0], grid[1], grid[2], pairs[0], pairs[1], pairs[2],
-                 float(rope_base), float(scale), float(topk), int(bool(gate_per_token)))
+                 float(rope_base), float(scale), float(topk), GATES[gate])
 
 
 def _f32(x) -> np.ndarray:
@@ -111,7 +119,7 @@ def _f64(x) -> np.ndarray:
 
 def _gain(s: Shape, g) -> np.ndarray:
     g = _f64(g)
-    want = s.B * s.N * s.H if s.gate_per_token else s.H
+    want = {0: s.H, 1: s.B * s.N * s.H, 2: s.H * (s.d + 1)}[s.gate_mode]
     assert g.size == want, f"g has {g.size} values, the shape needs {want}"
     return g
 

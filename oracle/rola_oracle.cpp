@@ -36,7 +36,10 @@
 //      R(p) rotates the r/2 adjacent pairs (2c, 2c+1) by theta_c = pos_axis(c)(p) *
 //      base^(-c'/P_axis); numerator = (R(p_n) u_n)^T sum_m R(p_m) f_m v_m^T,
 //      denominator = u_n^T sum_m f_m (unrotated), O_lin = numerator / denominator.
-//   6. out = O_sparse + g_h * O_lin.
+//   6. out = O_sparse + g * O_lin, with one of three gains: g_h per head; g_{n,h} per
+//      token and head, given; or the gate computed from the query, g_{n,h} =
+//      sigmoid(q_{n,h} . wg_h + bg_h), from the gate_proj (wg, [H][d]) and gate_bias (bg,
+//      [H]) parameters the README's sparse-finetuning section adds.
 //
 // Build: g++ -O3 -fopenmp -shared -fPIC (no -march, no fast-math: no FMA contraction).
 #include <algorithm>
@@ -66,7 +69,9 @@ struct rola_oracle_shape {
   double rope_base;               // frequency base (10000)
   double scale;                   // softmax logit scale
   double topk;                    // keep ratio in (0, 1]
-  int gate_per_token;             // g is [B][N][H] (a gain per token and head), else [H]
+  int gate_mode;                  // 0: g is [H] (a gain per head); 1: g is [B][N][H] (a gain
+                                  // per token and head); 2: g holds gate_proj [H][d] then
+                                  // gate_bias [H], and the gain is sigmoid(q . wg_h + bg_h)
 };
 
 int rola_oracle_num_blocks(int N) { return (N + kBlock - 1) / kBlock; }
@@ -225,13 +230,25 @@ void rola_oracle_linear_state(const rola_oracle_shape* s, const float* k, const 
     }
 }
 
+// The gain of token n of (b, h) (reading 6): g_h; g_{n,h} given per token; or the gate
+// from the query, sigmoid(q_n . wg_h + bg_h) (README sparse-finetuning section: gate_proj,
+// gate_bias), with the dot product and the sigmoid in double.
+static double gain(const rola_oracle_shape* s, const double* g, const float* qn, int b, int n, int h) {
+  if (s->gate_mode == 1) return g[((size_t)b * s->N + n) * s->H + h];
+  if (s->gate_mode == 2) {
+    const double* wg = g + (size_t)h * s->d;
+    double a = g[(size_t)s->H * s->d + h];
+    for (int c = 0; c < s->d; ++c) a += (double)qn[c] * wg[c];
+    return 1.0 / (1.0 + std::exp(-a));
+  }
+  return g[h];
+}
+
 // Output of the listed query blocks.  blocks: nrows triples (b, h, i).
 // For each listed block, rows [0, 64) of the three outputs (each [nrows][64][d]) hold
 //   sparse: O_sparse, lin: O_lin, out: O_sparse + g * O_lin
-// with g = g_h, or g_{n,h} of the token for a per-token gate (the gate_proj / gate_bias
-// parameters of the README's sparse-finetuning section make the gate input-dependent;
-// their values per token and head are an input here)
-// for the valid tokens of the block; rows past N are left at 0.
+// with g the gain of the token (see gain above), for the valid tokens of the block; rows
+// past N are left at 0.
 void rola_oracle_attend_blocks(const rola_oracle_shape* s, const float* q, const float* k,
                                const float* v, const float* Wq, const double* g,
                                const int32_t* col_idx, const double* S, const double* z,
@@ -289,7 +306,7 @@ void rola_oracle_attend_blocks(const rola_oracle_shape* s, const float* q, const
         ol[(size_t)row * d + c] = num / lden;
       }
       // Combination (reading 6).
-      const double gn = s->gate_per_token ? g[((size_t)b * N + n) * H + h] : g[h];
+      const double gn = gain(s, g, qn, b, n, h);
       for (int c = 0; c < d; ++c)
         oo[(size_t)row * d + c] = os[(size_t)row * d + c] + gn * ol[(size_t)row * d + c];
     }

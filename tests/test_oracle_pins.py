@@ -36,11 +36,6 @@ def _all_blocks(B, H, nb):
     return np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(nb)], np.int32)
 
 
-def _blocks_to_tokens(x, N):
-    """[B*H*nb, 64, d] block-major rows (b, h, i order) -> [B, N, H, d]."""
-    return x
-
-
 # ---------------------------------------------------------------- keep ratio (pages' table)
 
 def _golden_keep_ratio():
@@ -411,6 +406,67 @@ def test_per_token_gate_scales_each_tokens_linear_branch_by_its_own_gain():
     lin = out_1 - out_0
     assert np.abs(lin).max() > 0.1
     np.testing.assert_allclose(out_g - out_0, g[..., None] * lin, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- gate from the query
+# (README sparse-finetuning section: gate_proj, gate_bias; the gain is read as
+# sigmoid(q . gate_proj_h + gate_bias_h) per token and head)
+
+def _proj_gate(wg, bg):
+    """The "proj" gate's parameter buffer: gate_proj [H, d] then gate_bias [H]."""
+    return np.concatenate([np.asarray(wg, np.float64).ravel(), np.asarray(bg, np.float64)])
+
+
+def test_projected_gate_with_zero_weights_is_the_sigmoid_of_the_bias():
+    # wg = 0: the gain is sigmoid(bg_h) for every token.  With bg = ln 3 and ln(1/3) the
+    # gains are 3/4 and 1/4 (worked by hand: 1 / (1 + 1/3) and 1 / (1 + 3)), so the output
+    # equals the per-head-gain output with g = (3/4, 1/4).
+    B, N, H, d, r = 1, 200, 2, 16, 8
+    q, k, v, Wq, Wk, _ = _rand_inputs(B, N, H, d, r, seed=31)
+    s_head = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 100))
+    s_proj = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 100), gate="proj")
+    g = _proj_gate(np.zeros((H, d)), [math.log(3.0), math.log(1.0 / 3.0)])
+    out_p, col_p = O.forward(s_proj, q, k, v, Wq, Wk, g)
+    out_h, col_h = O.forward(s_head, q, k, v, Wq, Wk, np.array([0.75, 0.25]))
+    np.testing.assert_array_equal(col_p, col_h)
+    np.testing.assert_allclose(out_p, out_h, rtol=0, atol=1e-14)
+
+
+def test_projected_gate_limits_are_the_sparse_branch_and_the_unit_gain():
+    B, N, H, d, r = 1, 150, 2, 16, 8
+    q, k, v, Wq, Wk, _ = _rand_inputs(B, N, H, d, r, seed=32)
+    s_head = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 3, 50))
+    s_proj = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 3, 50), gate="proj")
+    wg = _rng(33).standard_normal((H, d)) * 0.1
+    out_off, _ = O.forward(s_proj, q, k, v, Wq, Wk, _proj_gate(wg, [-60.0, -60.0]))
+    out_on, _ = O.forward(s_proj, q, k, v, Wq, Wk, _proj_gate(wg, [60.0, 60.0]))
+    out_0, _ = O.forward(s_head, q, k, v, Wq, Wk, np.zeros(H))
+    out_1, _ = O.forward(s_head, q, k, v, Wq, Wk, np.ones(H))
+    np.testing.assert_allclose(out_off, out_0, rtol=0, atol=1e-12)   # sigmoid(-60) ~ 1e-26
+    np.testing.assert_allclose(out_on, out_1, rtol=0, atol=1e-12)
+
+
+def test_projected_gate_reads_each_heads_own_channel_of_its_own_query():
+    # gate_proj_h = alpha_h on one channel c_h (a different channel and weight per head):
+    # the gain of token n, head h is sigmoid(alpha_h * q[b, n, h, c_h] + bg_h), one product
+    # per token, so the output must equal the per-token-gate output with those gains.  A
+    # weight read transposed, from another head or another token fails this.
+    B, N, H, d, r = 2, 130, 3, 16, 8
+    q, k, v, Wq, Wk, _ = _rand_inputs(B, N, H, d, r, seed=34)
+    chans, alpha, bg = [3, 11, 0], [1.5, -0.7, 2.0], [0.2, -0.4, 0.1]
+    wg = np.zeros((H, d))
+    for h in range(H):
+        wg[h, chans[h]] = alpha[h]
+    s_proj = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 65), gate="proj")
+    s_tok = O.make_shape(B, H, N, d, r, 0.5, grid=(1, 2, 65), gate="token")
+    g_tok = np.zeros((B, N, H))
+    for h in range(H):
+        a = alpha[h] * q[:, :, h, chans[h]].astype(np.float64) + bg[h]
+        g_tok[:, :, h] = 1.0 / (1.0 + np.exp(-a))
+    out_p, _ = O.forward(s_proj, q, k, v, Wq, Wk, _proj_gate(wg, bg))
+    out_t, _ = O.forward(s_tok, q, k, v, Wq, Wk, g_tok)
+    np.testing.assert_allclose(out_p, out_t, rtol=0, atol=1e-13)
+    assert g_tok.std() > 0.1                       # the gains really differ per token
 
 
 def test_forward_equals_composed_steps_and_lists_are_valid():
