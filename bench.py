@@ -8,9 +8,13 @@ the sparse branch, 4*d*c_i*c_j summed over every kept (query block i, key block 
 pair (c = valid tokens of a block), divided by the step time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rola|reference]
-                  [--gate head|token] [--no-e2e] [--no-cpu-baseline]
+                  [--gate head|token] [--no-e2e] [--no-cpu-baseline] [--no-fp8]
 
-``--gate token`` feeds a gain per token and head (g [B, N, H]) instead of per head.
+``--gate token`` feeds a gain per token and head (g [B, N, H]) instead of per head;
+``--gate proj`` has the library compute it from the query (gate_proj, gate_bias).
+For a bf16 workload that has an fp8-e4m3 twin (the 720P and 480P 14B shapes), the same
+line also carries ``fp8``: the twin timed the same way on the same inputs (``--no-fp8``
+skips it).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs an independent forward of the
 same workload (different seed), no collective on the data path ("scaling": "weak");
@@ -45,8 +49,8 @@ LAUNCHES_PER_STEP = 7
 
 # DRAM bytes (read + write) per launch of the attention kernel's fast pass, from
 # `dram__bytes_read.sum + dram__bytes_write.sum` of one ncu capture of the current kernel on the
-# 14B-480P workload, scaled to 720P by the token count (the streamed bytes grow with N); see
-# profiles/attend_sm100_wan21_14b_480p.md.  None where no capture of the current kernel exists.
+# 14B-480P workload, scaled to 720P by the token count (the streamed bytes grow with N).  None
+# where no capture of the current kernel exists.
 ATTEND_DRAM_BYTES = {"wan21_14b_720p": 1.519e9 * 75600 / 32760, "wan21_14b_480p": 1.519e9,
                      "wan21_14b_720p_fp8": 0.9970e9 * 75600 / 32760, "wan21_14b_480p_fp8": 0.9970e9}
 
@@ -77,27 +81,74 @@ def linear_epilogue_flops(w) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed region, every
+    10 ms through NVML (the GPU found by its PCI bus id, so CUDA_VISIBLE_DEVICES does not
+    matter); ``nvidia-smi -lms 100`` when NVML is not usable."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.01):
         self.dev = device_index
+        self.period = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []       # (sm_mhz, max_mhz, reason bits)
+        self.lines = []
+
+    def _bus_id(self):
+        p = torch.cuda.get_device_properties(self.dev)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+
+    def _nvml_loop(self, nv, h):
+        import threading
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def __enter__(self):
         try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                h = nv.nvmlDeviceGetHandleByPciBusId(self._bus_id().encode())
+            except Exception:
+                h = nv.nvmlDeviceGetHandleByIndex(self.dev)
+            self._nv = nv
+            self._stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
+                ["nvidia-smi", f"--id={self._bus_id()}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self._nv.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -109,8 +160,14 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], None, set()
+        for s_mhz, m_mhz, bits in self.samples:
+            sm.append(s_mhz)
+            mx = m_mhz
+            for bit, name in self.REASONS.items():
+                if bits & bit:
+                    reasons.add(name)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
@@ -123,7 +180,8 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvml, 10 ms" if self.samples else "nvidia-smi, 100 ms"}
 
 
 def dist_env():
@@ -209,19 +267,72 @@ def oracle_sample(w, seconds_hint=15.0, seed=0):
                        f"query blocks, each head's time extrapolated to all its blocks")}
 
 
+# ------------------------------------------------------------------ device timing
+
+def measure(w, plan, step, steps, warmup, ws, dev):
+    """Times exactly ``steps`` calls of ``step`` (after ``warmup`` untimed ones) with CUDA
+    events on the launching stream, bracketed by a barrier and a synchronize on both
+    sides; the time is the max over ranks.  Stage times come from the library's own
+    events between the forward's stages, recorded in the same timed calls."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert plan.poll_status() == 0
+    flops = kept_block_flops(plan.block_lists(), w.N, w.d)
+    plan.profile_stages(True)      # events between the forward's stages (host call, untimed)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    stage_sum, ncalls = plan.stage_times()
+    plan.profile_stages(False)
+    assert plan.poll_status() == 0
+    return {"flops": flops, "ms_step": ms_total / steps, "stage_ms": [x / ncalls for x in stage_sum],
+            "clocks": clk.summary()}
+
+
+def roofline(w, stage_ms, flops):
+    """The attention kernel (kept-block + linear-epilogue FLOPs over its stage time) against
+    the measured dense tensor peak of its operand type."""
+    peaks = load_peaks()
+    att_ms = stage_ms[-1]
+    achieved = (flops + linear_epilogue_flops(w)) / (att_ms * 1e-3) / 1e12
+    if w.dtype == "fp8":   # e4m3 products: the bf16 measurement times the nominal 4.5 / 2.25
+        peak = 2.0 * peaks["bf16_tflops"]
+        peak_src = f"{peaks['source']} bf16 burst (cuBLAS 8192^3) x 2 (nominal fp8/bf16 ratio)"
+    else:
+        peak = peaks["bf16_tflops"]
+        peak_src = f"{peaks['source']} bf16 burst (cuBLAS 8192^3)"
+    return {"bound": "tensor", "kernel": "attend (sparse branch + fused linear epilogue)",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": ATTEND_DRAM_BYTES.get(w.name), "traffic_unit": "bytes/launch",
+            "peak_source": peak_src}
+
+
 # ------------------------------------------------------------------ main
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="wan21_14b_720p")
     ap.add_argument("--impl", default="rola", choices=["rola", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--gate", default="head", choices=["head", "token"],
-                    help="gain of the linear branch per head (default) or per token and head")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the fp8-e4m3 twin of a bf16 workload")
+    ap.add_argument("--gate", default="head", choices=["head", "token", "proj"],
+                    help="gain of the linear branch per head (default), per token and head, or "
+                         "computed from the query (sigmoid of q . gate_proj + gate_bias)")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     w = synth.WORKLOADS[args.workload]
@@ -232,7 +343,7 @@ def main():
         vals = []
         samp = None
         for it in range(args.warmup + args.steps):
-            r = oracle_sample(w, seconds_hint=max(2.0, 150.0 / (args.warmup + args.steps)), seed=it)
+            r = oracle_sample(w, seconds_hint=max(0.5, 150.0 / (args.warmup + args.steps)), seed=it)
             if it >= args.warmup:
                 vals.append(r["value"])
                 samp = r
@@ -260,10 +371,12 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     rola.load()
     inp = synth.make_inputs(w, seed=rank, device=dev)
-    per_token = args.gate == "token"
-    if per_token:
-        inp["g"] = synth.make_gate(w, seed=100 + rank, device=dev)   # [B, N, H]
-    plan = rola.Plan.for_workload(w, device=dev, gate_per_token=per_token)
+    per_token = args.gate != "head"
+    if args.gate == "token":
+        inp["g"] = synth.make_gate(w, seed=100 + rank, device=dev)        # [B, N, H]
+    elif args.gate == "proj":
+        inp["g"] = synth.make_gate_proj(w, seed=100 + rank, device=dev)   # [H*(d+1)]
+    plan = rola.Plan.for_workload(w, device=dev, gate=args.gate)
     out = torch.empty_like(inp["q"])
     q, k, v, Wq, Wk, g = (inp[x] for x in ("q", "k", "v", "Wq", "Wk", "g"))
     stream = torch.cuda.current_stream()
@@ -271,59 +384,29 @@ def main():
     def step():
         plan.forward(q, k, v, Wq, Wk, g, out)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert plan.poll_status() == 0
-    flops = kept_block_flops(plan.block_lists(), w.N, w.d)
-    att_flops = flops + linear_epilogue_flops(w)
-
-    plan.profile_stages(True)      # events between the forward's stages (host call, untimed)
-    barrier(ws)
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(args.steps):
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    ms_total = t0.elapsed_time(t1)
-    ms_total_max = max_over_ranks(ms_total, ws)
-    ms_step = ms_total_max / args.steps
-    stage_sum, ncalls = plan.stage_times()
-    plan.profile_stages(False)
-    stage_ms = [x / ncalls for x in stage_sum]
-    assert plan.poll_status() == 0
+    m = measure(w, plan, step, args.steps, args.warmup, ws, dev)
+    flops, ms_step, stage_ms, clk = m["flops"], m["ms_step"], m["stage_ms"], m["clocks"]
     value = aggregate_tflops(flops, ms_step, ws)
-
-    peaks = load_peaks()
-    att_ms = stage_ms[-1]
-    achieved = att_flops / (att_ms * 1e-3) / 1e12
-    if w.dtype == "fp8":   # e4m3 products: the bf16 measurement times the nominal 4.5 / 2.25
-        peak = 2.0 * peaks["bf16_tflops"]
-        peak_src = f"{peaks['source']} bf16 burst (cuBLAS 8192^3) x 2 (nominal fp8/bf16 ratio)"
-    else:
-        peak = peaks["bf16_tflops"]
-        peak_src = f"{peaks['source']} bf16 burst (cuBLAS 8192^3)"
-    roof = {"bound": "tensor", "kernel": "attend (sparse branch + fused linear epilogue)",
-            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": ATTEND_DRAM_BYTES.get(w.name), "traffic_unit": "bytes/launch",
-            "peak_source": peak_src}
+    roof = roofline(w, stage_ms, flops)
     act = w.B * w.N * w.H * w.d                     # elements of one activation tensor
     nblk = w.B * w.H * plan.nb
     if len(stage_ms) == 4:
-        # algorithmic HBM bytes: the key/value pass reads k, v and writes the fp16 copy of v
-        # (bf16) or the e4m3 k and v; the query pass reads q and writes the query-feature
-        # images, g/den, the q means (and e4m3 q)
-        kv_bytes = 2 * act * 2 + (2 * act if w.dtype == "fp8" else act * 2)
-        q_bytes = act * 2 + nblk * (2 * w.r * 128 + 64 * 4 + w.d * 4) + (act if w.dtype == "fp8" else 0)
+        # HBM bytes of the two passes.  The method's own bytes: each pass reads its inputs
+        # once (k and v; q).  The build's intermediates on top: the fp16 copy of v (bf16) or
+        # the e4m3 k and v (fp8) written by the key/value pass; the query-feature images,
+        # g/den, the q means (and e4m3 q) written by the query pass.
+        kv_method, q_method = 2 * act * 2, act * 2
+        kv_extra = 2 * act if w.dtype == "fp8" else act * 2
+        q_extra = nblk * (2 * w.r * 128 + 64 * 4 + w.d * 4) + (act if w.dtype == "fp8" else 0)
         stages = {"kv_pass_ms": stage_ms[0], "query_pass_ms": stage_ms[1], "select_ms": stage_ms[2],
                   "attend_ms": stage_ms[3],
-                  "kv_pass_GBs": kv_bytes / (stage_ms[0] * 1e-3) / 1e9,
-                  "query_pass_GBs": q_bytes / (stage_ms[1] * 1e-3) / 1e9}
+                  "pre_attention_ms": stage_ms[0] + stage_ms[1] + stage_ms[2],
+                  "kv_pass_GBs_method": kv_method / (stage_ms[0] * 1e-3) / 1e9,
+                  "query_pass_GBs_method": q_method / (stage_ms[1] * 1e-3) / 1e9,
+                  "passes_frac_hbm_method": (kv_method + q_method) / ((stage_ms[0] + stage_ms[1]) * 1e-3) / 1e9
+                  / load_peaks()["hbm_gbs"],
+                  "kv_pass_GBs_with_copies": (kv_method + kv_extra) / (stage_ms[0] * 1e-3) / 1e9,
+                  "query_pass_GBs_with_copies": (q_method + q_extra) / (stage_ms[1] * 1e-3) / 1e9}
     else:
         stages = {"select_blocks_ms": stage_ms[0], "linear_state_ms": stage_ms[1], "attend_ms": stage_ms[2]}
 
@@ -365,7 +448,7 @@ def main():
                 ev["out"][sl].record(s_out)
             issued[0] += 1
 
-        e_steps = max(4, min(args.steps, 8))
+        e_steps = max(20, min(args.steps, 40))
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
@@ -384,6 +467,26 @@ def main():
                             "while the next step computes (3 streams, double-buffered device tensors)"}
         assert plan.poll_status() == 0
 
+    fp8 = None
+    twin = synth.WORKLOADS.get(w.name + "_fp8")
+    if twin is not None and w.dtype == "bf16" and not args.no_fp8:
+        # the fp8-e4m3 twin on the same bf16 inputs: quantised inside the call, so the
+        # same step and the same timing rules; kept-block FLOPs are the same
+        plan8 = rola.Plan.for_workload(twin, device=dev, gate=args.gate)
+        out8 = torch.empty_like(out)
+
+        def step8():
+            plan8.forward(q, k, v, Wq, Wk, g, out8)
+
+        m8 = measure(twin, plan8, step8, args.steps, args.warmup, ws, dev)
+        s8 = m8["stage_ms"]
+        fp8 = {"workload": twin.name, "dtype": "fp8", "value": aggregate_tflops(m8["flops"], m8["ms_step"], ws),
+               "unit": UNIT, "ms_per_step": m8["ms_step"], "steps": args.steps, "warmup": args.warmup,
+               "stages": {"kv_pass_ms": s8[0], "query_pass_ms": s8[1], "select_ms": s8[2], "attend_ms": s8[3]},
+               "roofline": roofline(twin, s8, m8["flops"]), "clocks": m8["clocks"]}
+        plan8.close()
+        del out8
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not per_token:
         r = oracle_sample(w, seconds_hint=15.0)
@@ -398,11 +501,12 @@ def main():
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "grid": list(w.grid),
                            "d": w.d, "r": w.r, "topk": w.topk, "kept_blocks_per_row": plan.k,
                            "blocks": plan.nb, "kept_block_tflop": flops / 1e12,
-                           "gate": "per-token" if per_token else "per-head",
+                           "gate": {"head": "per-head", "token": "per-token",
+                                    "proj": "sigmoid(q . gate_proj + gate_bias)"}[args.gate],
                            "l2": "inputs (3 x 774 MB) larger than L2 (126 MB); no flush",
                            "parallelism": f"replicas x{ws} (independent forward per GPU)"},
-                "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk.summary()}
+                "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "fp8": fp8,
+                "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk}
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist

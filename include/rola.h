@@ -26,12 +26,13 @@
  *      (2c, 2c+1) by theta_c = pos_axis(c) * base^(-c'/P_axis) (pairs ordered t, h, w).
  *      S_h = sum_m R(p_m) f_m v_m^T (r x d), z_h = sum_m f_m over all N keys;
  *      O_lin = (R(p_n) u_n)^T S_h / (u_n^T z_h).
- *   5. out = O_sparse + g_h * O_lin, rounded once to the output type.
+ *   5. out = O_sparse + g * O_lin, rounded once to the output type; g per head, per token
+ *      and head, or sigmoid(q . wg_h + bg_h) from the query (rola_gate).
  *
  * Layouts (all row-major, contiguous, device memory owned by the caller):
  *   q, k, v, out : [B, N, H, d]  (fp32 for ROLA_F32, bf16 for ROLA_BF16 and ROLA_FP8_E4M3)
  *   Wq, Wk       : [H, d, r]     (same element type as q)
- *   g            : [H] fp32
+ *   g            : fp32, [H], [B, N, H] or [H*(d+1)] (rola_gate)
  *   workspace    : rola_workspace_size() bytes, 256-byte aligned, borrowed by the plan.
  * Every pointer must be 16-byte aligned; out must not overlap any input.
  *
@@ -84,6 +85,18 @@ typedef enum {
                       /* only (ROLA_ERR_UNSUPPORTED otherwise).                          */
 } rola_dtype;
 
+/* The gain g that scales the linear branch (out = O_sparse + g * O_lin).  The pages name
+ * gate_proj and gate_bias among RoLA's parameters (README, sparse-finetuning section)
+ * without their form; ROLA_GATE_QPROJ takes the plainest reading that fits this
+ * operator: a projection of each head's query to one logit, g = sigmoid(q . wg_h + bg_h). */
+typedef enum {
+  ROLA_GATE_HEAD = 0,   /* g: [H] fp32, one gain per head                                 */
+  ROLA_GATE_TOKEN = 1,  /* g: [B, N, H] fp32, one gain per token and head, given           */
+  ROLA_GATE_QPROJ = 2   /* g: fp32 gate_proj wg [H, d] followed by gate_bias bg [H]        */
+                        /* (H*(d+1) values); the gain of token n, head h is computed as     */
+                        /* sigmoid(sum_c q[b,n,h,c] * wg[h,c] + bg[h]) in fp32              */
+} rola_gate;
+
 typedef struct {
   int B, H, N, d, r;             /* batch, heads, tokens, head dim (64|128), rank (16|32)   */
   int block;                     /* tokens per block; must be 64                            */
@@ -95,17 +108,13 @@ typedef struct {
   double rope_base;              /* rotary frequency base, > 1 (10000)                      */
   float softmax_scale;           /* logit scale; 0 = 1/sqrt(d)                              */
   rola_dtype dtype;
-  int gate_per_token;            /* 0: the gain g is per head, g[H]; 1: per token and head, */
-                                 /* g[B, N, H] fp32 (an input-dependent gate, e.g. computed  */
-                                 /* from the layer input by the gate_proj / gate_bias        */
-                                 /* parameters the pages add, applied as out = O_sparse +   */
-                                 /* g[b, n, h] * O_lin)                                       */
+  rola_gate gate;                /* how the gain g is given (default ROLA_GATE_HEAD)        */
 } rola_params;
 
 typedef struct rola_plan_s* rola_plan_t;
 
 /* Fills *p with defaults: B=H=1, N=0, d=128, r=32, block 64, topk 0.1, grid (1,1,0),
- * default rotary split, base 10000, scale 0 (1/sqrt(d)), ROLA_BF16, per-head gain. */
+ * default rotary split, base 10000, scale 0 (1/sqrt(d)), ROLA_BF16, ROLA_GATE_HEAD. */
 ROLA_API rola_status rola_params_default(rola_params* p);
 
 /* Number of 64-token blocks nb and kept blocks per query block k for *p. */
@@ -135,8 +144,9 @@ ROLA_API rola_status rola_linear_state(rola_plan_t plan, const void* k, const vo
                               rola_stream_t stream);
 
 /* Steps 3-5: sparse attention over the kept blocks with the linear branch and the
- * combination fused into its epilogue; writes out [B, N, H, d] once.  g: fp32 gains,
- * [H] or, with gate_per_token, [B, N, H] (device memory, 16-byte aligned).  Uses the block
+ * combination fused into its epilogue; writes out [B, N, H, d] once.  g: fp32 gains [H],
+ * [B, N, H], or the gate's wg [H, d] and bg [H], as p->gate says (device memory, 16-byte
+ * aligned).  Uses the block
  * lists and the state the two calls above left in the workspace (in ROLA_FP8_E4M3 mode
  * also their e4m3 copies of q, k, v, which must come from the same q, k, v). */
 ROLA_API rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const void* v,
@@ -157,11 +167,15 @@ ROLA_API rola_status rola_forward(rola_plan_t plan, const void* q, const void* k
  * Scratch: one 16 MiB array inside the library, which every GPU that loads the library
  * holds until the process exits; problems whose pooled means and block scores need more
  * (about 256 + 8*B*H*nb*d + 4*B*H*nb*ceil4(nb) bytes) are rejected with
- * ROLA_ERR_WORKSPACE before any launch.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the array: calls that overlap on the GPU
- * (other streams, other host threads) race and must be serialised by the caller.
- * Device-side index checks of this variant are not reported. */
+ * ROLA_ERR_WORKSPACE before any launch.  col_idx must hold B*H*nb*k int32 and must not
+ * overlap q or k (ROLA_ERR_INVALID_ARG otherwise).  Every call made outside stream capture
+ * looks up the array's device address (cudaGetSymbolAddress) with the current device, so
+ * calls after a device reset see the reloaded array; a call made while `stream` is being
+ * captured reuses the address of the last uncaptured call on that device, so make at
+ * least one call before any capture (a first call under capture fails with ROLA_ERR_CUDA).
+ * All calls share the array: calls that overlap on the GPU (other streams, other host
+ * threads) race and must be serialised by the caller.  Device-side index checks of this
+ * variant are not reported. */
 ROLA_API rola_status rola_select_blocks_noalloc(const rola_params* p, const void* q, const void* k,
                                                 int32_t* col_idx, rola_stream_t stream);
 

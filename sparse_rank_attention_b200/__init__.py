@@ -24,6 +24,9 @@ LIB_PATH = os.path.join(_PKG, "librola.so")
 ROLA_F32, ROLA_BF16, ROLA_FP8_E4M3 = 0, 1, 2
 DTYPES = {"f32": ROLA_F32, "bf16": ROLA_BF16, "fp8": ROLA_FP8_E4M3}
 ROLA_DEBUG_STALL_WAIT = 1
+# how the gain of the linear branch is given (rola_gate): g [H], g [B, N, H], or the gate
+# computed from the query, g = gate_proj [H, d] followed by gate_bias [H]
+GATES = {"head": 0, "token": 1, "proj": 2}
 
 STATUS = {0: "ROLA_OK", 1: "ROLA_ERR_INVALID_ARG", 2: "ROLA_ERR_UNSUPPORTED",
           3: "ROLA_ERR_WORKSPACE", 4: "ROLA_ERR_CUDA", 5: "ROLA_ERR_DEVICE_TIMEOUT",
@@ -52,7 +55,7 @@ class RolaParams(ctypes.Structure):
         ("rope_pairs_t", ctypes.c_int), ("rope_pairs_h", ctypes.c_int),
         ("rope_pairs_w", ctypes.c_int),
         ("rope_base", ctypes.c_double), ("softmax_scale", ctypes.c_float),
-        ("dtype", ctypes.c_int), ("gate_per_token", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("gate", ctypes.c_int),
     ]
 
 
@@ -116,8 +119,15 @@ def _check(code: int, where: str):
         raise RolaError(code, where)
 
 
+def _gate(gate, gate_per_token) -> int:
+    if gate is None:
+        gate = "token" if gate_per_token else "head"
+    return GATES[gate] if isinstance(gate, str) else int(gate)
+
+
 def make_params(B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
-                softmax_scale=0.0, dtype="bf16", gate_per_token=False) -> RolaParams:
+                softmax_scale=0.0, dtype="bf16", gate_per_token=False, gate=None) -> RolaParams:
+    """rola_params; gate is "head", "token" or "proj" (``gate_per_token=True`` = "token")."""
     p = RolaParams()
     load().rola_params_default(ctypes.byref(p))
     grid = tuple(grid) if grid is not None else (1, 1, N)
@@ -128,7 +138,7 @@ def make_params(B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000
     p.rope_base = float(rope_base)
     p.softmax_scale = float(softmax_scale)
     p.dtype = DTYPES[dtype] if isinstance(dtype, str) else int(dtype)
-    p.gate_per_token = int(bool(gate_per_token))
+    p.gate = _gate(gate, gate_per_token)
     return p
 
 
@@ -159,9 +169,9 @@ class Plan:
     """A rola_plan bound to a workspace tensor allocated here with torch."""
 
     def __init__(self, B, H, N, d, r, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
-                 softmax_scale=0.0, dtype="bf16", device="cuda", gate_per_token=False):
+                 softmax_scale=0.0, dtype="bf16", device="cuda", gate_per_token=False, gate=None):
         self.params = make_params(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype,
-                                  gate_per_token)
+                                  gate_per_token, gate)
         self.dtype = dtype
         self.nb, self.k = keep_count(self.params)
         self.workspace_bytes = workspace_size(self.params)
@@ -172,9 +182,9 @@ class Plan:
         self._h = h
 
     @classmethod
-    def for_workload(cls, w, device="cuda", gate_per_token=False):
+    def for_workload(cls, w, device="cuda", gate_per_token=False, gate=None):
         return cls(w.B, w.H, w.N, w.d, w.r, w.topk, w.grid, w.pairs, dtype=w.dtype, device=device,
-                   gate_per_token=gate_per_token)
+                   gate_per_token=gate_per_token, gate=gate)
 
     def close(self):
         if getattr(self, "_h", None):
@@ -275,15 +285,16 @@ def select_blocks_noalloc(params: RolaParams, q, k, col_idx, stream=None) -> int
 
 
 def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=10000.0,
-            softmax_scale=0.0, dtype=None, out=None):
+            softmax_scale=0.0, dtype=None, out=None, gate=None):
     """One-shot RoLA forward (builds a plan and workspace for this call).  g is [H], or
-    [B, N, H] for a per-token gate."""
+    [B, N, H] for a per-token gate, or gate_proj [H, d] then gate_bias [H] with
+    ``gate="proj"``."""
     B, N, H, d = q.shape
     r = Wq.shape[-1]
     if dtype is None:
         dtype = "f32" if q.dtype == torch.float32 else "bf16"
     plan = Plan(B, H, N, d, r, topk, grid, pairs, rope_base, softmax_scale, dtype, q.device,
-                gate_per_token=g.dim() > 1)
+                gate_per_token=g.dim() > 1, gate=gate)
     try:
         return plan.forward(q, k, v, Wq, Wk, g, out)
     finally:
@@ -292,4 +303,4 @@ def forward(q, k, v, Wq, Wk, g, topk, grid=None, pairs=(0, 0, 0), rope_base=1000
 
 
 __all__ = ["Plan", "forward", "select_blocks_noalloc", "load", "make_params", "keep_count", "workspace_size", "RolaError",
-           "RolaParams", "EXPORTS", "LIB_PATH", "ROLA_DEBUG_STALL_WAIT"]
+           "RolaParams", "EXPORTS", "LIB_PATH", "ROLA_DEBUG_STALL_WAIT", "GATES"]

@@ -15,6 +15,8 @@
 // hi + lo pairs (three products), so the linear branch keeps ~fp32 accuracy.
 // K_j / V_j are double-buffered with cp.async; out is staged in shared memory and
 // written with 16-byte stores, once.
+#include <climits>
+
 #include "rola_internal.cuh"
 #include "warp_mma.cuh"
 
@@ -37,7 +39,7 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Dims dm,
     const int32_t* __restrict__ col_idx, const __nv_bfloat16* __restrict__ S_hi,
     const __nv_bfloat16* __restrict__ S_lo, const float* __restrict__ z,
-    const float2* __restrict__ rope, int* __restrict__ status) {
+    const float2* __restrict__ rope, const int* __restrict__ vexp, int* __restrict__ status) {
   using L = AttSmem<D, RK>;
   constexpr int DP = L::DP;
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -96,6 +98,16 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     }
     cp_async_commit();
   };
+
+  // v is carried in fp16 as v * 2^-vexp per key block: P of block j is scaled by
+  // 2^(vexp_j - eref) (at most 1) and the output by 2^eref, eref = the row's largest vexp
+  const int* ve = vexp + (size_t)bh * dm.nb;
+  int eref = INT_MIN;
+  for (int jj = 0; jj < dm.k; ++jj) {
+    const int j = Lst[jj];
+    if (j >= 0 && j < dm.nb) eref = max(eref, __ldg(ve + j));
+  }
+  if (eref == INT_MIN) eref = 0;
 
   int j_next = block_of(0);
   load_kv(j_next, 0);
@@ -180,6 +192,14 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
         o[nt][2 * hh + 1] *= corr;
       }
     }
+    const int ej = __ldg(ve + j);
+    if (ej != eref) {
+      const float fac = ldexpf(1.f, ej - eref);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] *= fac;
+    }
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t pa[4];
@@ -205,7 +225,7 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     float l = lrow[hh];
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    inv_l[hh] = 1.f / l;
+    inv_l[hh] = ldexpf(1.f / l, eref);
   }
 
   // ---- linear branch epilogue
@@ -241,7 +261,8 @@ __global__ void __launch_bounds__(128, 2) attend_bf16_kernel(
     dd += __shfl_xor_sync(0xffffffffu, dd, 2);
     const int n = i * kBlock + 16 * warp + g8 + 8 * hh;
     const bool ok = n < dm.N;
-    coef[hh] = (ok ? g[gain_index(dm, b, n, h)] : 0.f) / dd;
+    // the query row of token n is still in sQ (the output is staged there only later)
+    coef[hh] = (ok ? gate_value(dm, g, sQ + (16 * warp + g8 + 8 * hh) * DP, b, n, h) : 0.f) / dd;
 #pragma unroll
     for (int nt = 0; nt < NTU; ++nt) {
       const float2 cs = ok ? rope_cs(dm, rope, n, nt * 4 + t4) : make_float2(1.f, 0.f);
@@ -306,7 +327,7 @@ cudaError_t launch_bf16(const Dims& dm, const void* q, const void* k, const void
   attend_bf16_kernel<D, RK><<<grid, 128, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       ws.v16, static_cast<const __nv_bfloat16*>(Wq), g, static_cast<__nv_bfloat16*>(out), dm,
-      ws.col_idx, ws.S_hi, ws.S_lo, ws.z, ws.rope, ws.status);
+      ws.col_idx, ws.S_hi, ws.S_lo, ws.z, ws.rope, ws.vexp, ws.status);
   return cudaGetLastError();
 }
 

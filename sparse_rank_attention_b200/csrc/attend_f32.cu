@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(64) attend_f32_kernel(
     ur[2 * c + 1] = cs.y * u[2 * c] + cs.x * u[2 * c + 1];
   }
   if (!valid) return;
-  const float gh = g[gain_index(dm, b, n, h)];
+  const float gh = gate_value(dm, g, sQ + tid * (D + 1), b, n, h);
   const float inv_l = 1.f / l, inv_den = 1.f / den;
   float* ob = out + ((size_t)b * dm.N + n) * rs + (size_t)h * D;
 #pragma unroll

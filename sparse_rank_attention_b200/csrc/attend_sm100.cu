@@ -39,6 +39,7 @@
 //
 // Every mbarrier wait is bounded (ROLA_ERR_DEVICE_TIMEOUT); on a timeout all roles
 // leave their loops, in-flight MMAs and TMA copies are drained and TMEM is freed.
+#include <climits>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp8.h>
@@ -102,6 +103,7 @@ struct Ctl {
   alignas(16) float red[2][4][32];   // per query group: per-warp partial reductions
   alignas(16) float linv[64];
   float vref[2][4];  // fp8: per-warp partial max of the kept blocks' V scales
+  int emax[2][4], emin[2][4];  // 16-bit path: per-warp range of the kept blocks' v exponents
 };
 template <bool FP8>
 constexpr size_t smem_bytes() { return Geo<FP8>::kOffCtl + sizeof(Ctl) + 1024; }
@@ -200,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ simg,
     const uint8_t* __restrict__ uimg, const float* __restrict__ gden,
     const float* __restrict__ sq, const float* __restrict__ sk, const float* __restrict__ sv,
-    int* __restrict__ status, int* __restrict__ redo, int debug_flags, unsigned long long limit_cycles,
+    const int* __restrict__ vexp, int* __restrict__ status, int* __restrict__ redo, int debug_flags,
+    unsigned long long limit_cycles,
     unsigned long long debug_limit_cycles) {
   using G = Geo<FP8>;
   constexpr int kKStages = G::kKStages, kVStages = G::kVStages;
@@ -498,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
     const size_t sbase_idx = (size_t)bh * dm.nb;
     float sqi = 1.f, vref = 1.f;
+    int eref = 0;
     if constexpr (FP8) {
       sqi = __ldg(sq + sbase_idx + i);
       float mx = 0.f;
@@ -511,6 +515,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       named_sync(gbar, 128);
       vref = fmaxf(fmaxf(ctl->vref[g][0], ctl->vref[g][1]), fmaxf(ctl->vref[g][2], ctl->vref[g][3]));
       if (!(vref > 0.f)) vref = 1.f;
+    }
+    // 16-bit path: v is carried in fp16 as v * 2^-vexp per key block.  The output takes
+    // 2^eref / l (eref = the largest exponent of the row's kept blocks); a tile whose
+    // blocks do not all share one exponent is listed by the fast pass (its P would need a
+    // factor per pair) and redone by the careful pass, which scales each pair's P by
+    // 2^(vexp_j - eref) <= 1.  The fast pass gathers the exponents here and reads the
+    // group's range after its end-of-tile vote; the careful pass needs eref at once.
+    if constexpr (!FP8) {
+      int ex_hi = INT_MIN, ex_lo = INT_MAX;
+      for (int e = t; e < kk_list; e += 128) {
+        const int jj = __ldg(L + e);
+        if (jj >= 0 && jj < dm.nb) {
+          const int x = __ldg(vexp + sbase_idx + jj);
+          ex_hi = max(ex_hi, x);
+          ex_lo = min(ex_lo, x);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ex_hi = max(ex_hi, __shfl_xor_sync(0xffffffffu, ex_hi, o));
+        ex_lo = min(ex_lo, __shfl_xor_sync(0xffffffffu, ex_lo, o));
+      }
+      if (lane == 0) {
+        ctl->emax[g][wq] = ex_hi;
+        ctl->emin[g][wq] = ex_lo;
+      }
+      if constexpr (CAREFUL) {
+        named_sync(gbar, 128);
+        int er = max(max(ctl->emax[g][0], ctl->emax[g][1]), max(ctl->emax[g][2], ctl->emax[g][3]));
+        if (er == INT_MIN) er = 0;
+        eref = er;
+        vref = ldexpf(1.f, er);
+      }
     }
     // The key block of this warp's half of each pair (warps 0-1 of a group hold the
     // pair's first block, warps 2-3 its second; -1: the padding half of an odd list).
@@ -684,11 +721,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       } else {
         // every exponential on ex2 here (a quarter on the FMA pipe, as for fp8, measured
         // 1 % slower on this path)
+        float vf = 1.f;                    // careful pass: 2^(vexp_j - eref) of this pair
+        if constexpr (CAREFUL) {
+          if (jb >= 0 && jb < dm.nb) vf = ldexpf(1.f, __ldg(vexp + sbase_idx + jb) - eref);
+        }
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
-          const float p0 = ex2_approx(x[q]);
-          const float p1 = ex2_approx(x[q + 1]);
+          float p0 = ex2_approx(x[q]);
+          float p1 = ex2_approx(x[q + 1]);
           add2(lp[q], lp[q + 1], p0, p1);
+          if constexpr (CAREFUL) mul2(p0, p1, vf, vf);
           pw[q >> 1] = pack_half2(p0, p1);
         }
       }
@@ -713,7 +755,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       bool overflow = false;
 #pragma unroll
       for (int q = 0; q < 32; ++q) overflow |= !(lp[q] <= kOverflow);   // (NaN counts too)
-      if (named_vote_or(gbar, 128, overflow) && t == 0) {
+      const bool listed = named_vote_or(gbar, 128, overflow);
+      bool mixed = false;                  // 16-bit path: the kept blocks' v exponents differ
+      if constexpr (!FP8) {
+        const int hi = max(max(ctl->emax[g][0], ctl->emax[g][1]), max(ctl->emax[g][2], ctl->emax[g][3]));
+        const int lo = min(min(ctl->emin[g][0], ctl->emin[g][1]), min(ctl->emin[g][2], ctl->emin[g][3]));
+        mixed = hi != lo && hi != INT_MIN;
+        eref = hi == INT_MIN ? 0 : hi;
+        vref = ldexpf(1.f, eref);
+      }
+      if ((listed || mixed) && t == 0) {
         const int slot = atomicAdd(redo, 1);
         if (slot < 2 * ntiles_all) redo[1 + slot] = tau;
       }
@@ -803,12 +854,12 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
   // its CTAs then exit at once)
   if ((e = cudaMemsetAsync(ws.redo, 0, sizeof(int), st)) != cudaSuccess) return e;
   attend_sm100_kernel<RK, FP8, false><<<grid, kThreads, smem, st>>>(
-      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status, ws.redo,
-      debug_flags, limit_cycles, dlimit);
+      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.vexp, ws.status,
+      ws.redo, debug_flags, limit_cycles, dlimit);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attend_sm100_kernel<RK, FP8, true><<<grid, kThreads, smem, st>>>(
-      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.status, ws.redo,
-      debug_flags, limit_cycles, dlimit);
+      tq, tk, tv, to, dm, ws.col_idx, ws.simg, ws.uimg, ws.gden, ws.sq, ws.sk, ws.sv, ws.vexp, ws.status,
+      ws.redo, debug_flags, limit_cycles, dlimit);
   return cudaGetLastError();
 }
 

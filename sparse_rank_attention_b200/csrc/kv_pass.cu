@@ -2,9 +2,14 @@
 // and v computes everything the later steps need from them.
 //   * the linear-branch state partials over a chunk of tokens (split-N; step 4, key side)
 //       S_h += sum_m R(p_m) phi(k_m Wk_h) v_m^T,   z_h += sum_m phi(k_m Wk_h)
-//   * the block means of k (step 1, key side): fp32 sums in token order, one division
+//     with both contractions on the tcgen05 tensor cores, accumulating in tensor memory;
+//   * the block means of k (step 1, key side): fp32 sums in token order, one division;
 //   * bf16 configuration: the fp16 copy of v that the attention kernel multiplies the
-//     fp16 softmax weights with (values outside the fp16 range set ROLA_ERR_RANGE)
+//     fp16 softmax weights with.  Each (b, h, block) of v is carried as v * 2^-e with one
+//     power-of-two exponent e per block (0 for blocks whose largest |v| lies in
+//     [2^-6, 2^15), else the exponent that brings it into [2^14, 2^15)), so every finite
+//     bf16 value fits fp16 exactly as far as fp16's 11 bits allow; e goes to vexp.
+//     Non-finite v sets ROLA_ERR_RANGE;
 //   * fp8 configuration: the e4m3 copies of k and v with one scale per (b, h, block)
 //     (scale = absmax / 448, 1 for an all-zero block; code = RN-sat(x * (1 / scale))).
 //
@@ -13,29 +18,37 @@
 // linear branch with rotary positions); README sparse-finetuning section (proj_k).
 //
 // Layout of the work: a CTA owns one (b, h) and a chunk of whole 64-token blocks; the
-// chunk length is chosen on the host so that the CTAs fill the SMs in whole waves.  k and
-// v tiles (one block each: two TMA boxes of 64 tokens x 64 channels, 128-byte swizzle)
-// flow through a 2-stage ring of TMA copies completing on mbarriers, so the next tile is in
-// flight while one is processed, with two CTAs per SM (two tiles in flight per SM); rows
-// past N arrive as zeros.
-// Per tile: warps 0-3 compute F = K Wk (mma.sync), phi, z and the rotation and store
-// the rotated features as bf16 hi + lo; meanwhile warps 4-5 pool k (and write its e4m3
-// copy) and warps 6-7 write the copy of v; then all 8 warps add F^T V into their 16
-// columns of S.
+// chunk length is chosen on the host so that the CTAs fill the SMs in whole waves (two
+// CTAs per SM).  k and v tiles (one block each: two TMA boxes of 64 tokens x 64 channels,
+// 128-byte swizzle) flow through a 2-stage ring filled by a producer warp; rows past N
+// arrive as zeros.  Per tile:
+//   F = K Wk           one tcgen05 MMA chain, M = 64 tokens, N = r, K = 128 channels
+//                      (A = the k tile, B = Wk_h^T staged once per CTA), fp32 in TMEM;
+//   F~ = R(p) phi(F)   warps 0-3, one token and half of the r values per thread, stored
+//                      as bf16 hi + lo into a K-major operand image;
+//   S^T += V^T F~      M = 128 channels, N = r, K = 64 tokens (A = the v tile read
+//                      MN-major, B = the hi and lo images), accumulated in TMEM over the
+//                      whole chunk and read out once at its end;
+// while warps 4-5 pool k (and write its e4m3 copy) and warps 6-7 write the copy of v.
+// Every wait is bounded (ROLA_ERR_DEVICE_TIMEOUT).
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
-#include "warp_mma.cuh"
 
 #include <cuda_fp8.h>
 
 namespace rola {
 namespace {
 
+using namespace sm100;
+
 constexpr int kD = 128;
 constexpr int kTok = 64;                     // tokens per tile = one block
 constexpr int kStages = 2;
-constexpr int kThreads = 256;
-constexpr uint32_t kTileBytes = kTok * kD * 2;   // 16 KB, 64 rows of 256 bytes
+constexpr int kThreads = 288;                // warps 0-3 features, 4-5 k means, 6-7 v copy, 8 TMA
+constexpr uint32_t kTileBytes = kTok * kD * 2;   // 16 KB: two boxes of 64 rows x 128 bytes
+constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kColF = 0;                // F [64 tokens x r] (M = 64 layout)
+constexpr uint32_t kColS = 32;               // S^T [128 channels x r]
 
 // Byte offset of 16-byte chunk c (channels 8c .. 8c + 7, c = 0..15) of token row r in a
 // tile: box c / 8 (8 KB each), 128-byte rows, chunk position (c % 8) ^ (r % 8).
@@ -43,20 +56,31 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)((c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// Byte offset of element (row, col) of a K-major 128-byte-swizzled bf16 operand image
+// (rows of 64 elements; 8-row atoms of 1024 bytes).
+__device__ __forceinline__ uint32_t img_off(int row, int col) {
+  return (uint32_t)(row * 128 + ((((col >> 3) ^ row) & 7) << 4) + (col & 7) * 2);
+}
+
 template <int RK>
-struct KVSmem {
-  static constexpr int WP = RK + 8;          // Wk rows [d][r], padded (conflict-free ldmatrix)
-  static constexpr int RP = RK + 8;          // F rows [token][r], padded
-  static constexpr size_t offK = 0;
-  static constexpr size_t offV = offK + (size_t)kStages * kTileBytes;
-  static constexpr size_t offW = offV + (size_t)kStages * kTileBytes;
-  static constexpr size_t offF = offW + (size_t)kD * WP * 2;
-  static constexpr size_t offFl = offF + (size_t)kTok * RP * 2;
-  static constexpr size_t offZ = offFl + (size_t)kTok * RP * 2;   // [4][RK] fp32
-  static constexpr size_t offRed = offZ + (size_t)4 * RK * 4;      // [2][4] fp32
-  static constexpr size_t offBar = offRed + 2 * 4 * 4;              // full[kStages], abort flag
-  static constexpr size_t bytes = offBar + kStages * 8 + 16 + 1024;   // + alignment slack
+struct KVGeo {
+  static constexpr uint32_t offK = 0;                                // kStages k tiles
+  static constexpr uint32_t offV = offK + kStages * kTileBytes;      // kStages v tiles
+  static constexpr uint32_t offW = offV + kStages * kTileBytes;      // Wk_h^T: 2 boxes [r][64 ch]
+  static constexpr uint32_t offF = offW + 2 * RK * 128;              // F~ hi [r][64 tok], then lo
+  static constexpr uint32_t offCtl = offF + 2 * RK * 128;
 };
+
+struct KVCtl {
+  uint64_t full[kStages], freed[kStages], f_full, img_free, drain;
+  uint32_t tmem_base;
+  int abort;
+  float zred[4][32];
+  float red[8];
+};
+
+template <int RK>
+constexpr size_t kv_smem_bytes() { return KVGeo<RK>::offCtl + sizeof(KVCtl) + 1024; }
 
 __device__ __forceinline__ float absmax8(const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -79,141 +103,246 @@ __device__ __forceinline__ uint2 e4m3x8(const uint4& v, float inv) {
   return make_uint2(o[0], o[1]);
 }
 
+// (x0, x1) as packed bf16 pairs hi + lo with |x - hi - lo| <= 2^-16 |x|.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x0, x1);
+  const float2 bf = __bfloat1622float2(b);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - bf.x, x1 - bf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&b);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// 16 consecutive fp32 columns of TMEM lanes 0-15 of this warp's quadrant for threads
+// 0-15 and the next 16 columns of the same lanes for threads 16-31 (the M = 64 layout).
+__device__ __forceinline__ void tmem_ld16x2_x16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16], 16;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16x2_x8(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], 8;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane (all 32 lanes of the quadrant).
+__device__ __forceinline__ void tmem_ld32x32_x16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 template <int RK, bool FP8>
 __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __nv_bfloat16* __restrict__ Wk, Dims dm, const float2* __restrict__ rope,
     float* __restrict__ S_part, float* __restrict__ z_part, float* __restrict__ kbar,
-    __half* __restrict__ v16, uint8_t* __restrict__ k8, uint8_t* __restrict__ v8,
+    __half* __restrict__ v16, int* __restrict__ vexp, uint8_t* __restrict__ k8, uint8_t* __restrict__ v8,
     float* __restrict__ sk, float* __restrict__ sv, int* __restrict__ status) {
-  using L = KVSmem<RK>;
-  using namespace sm100;
+  using G = KVGeo<RK>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(smem);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  int* abort_flag = reinterpret_cast<int*>(smem + L::offBar + kStages * 8);
-  const __nv_bfloat16* sW = reinterpret_cast<const __nv_bfloat16*>(smem + L::offW);
-  __nv_bfloat16* sF = reinterpret_cast<__nv_bfloat16*>(smem + L::offF);
-  __nv_bfloat16* sFl = reinterpret_cast<__nv_bfloat16*>(smem + L::offFl);
-  float* sZ = reinterpret_cast<float*>(smem + L::offZ);
-  float* sRed = reinterpret_cast<float*>(smem + L::offRed);
+  const uint32_t sbase = smem_addr(smem);
+  KVCtl* ctl = reinterpret_cast<KVCtl*>(smem + G::offCtl);
+  auto bar = [&](uint64_t& m) { return smem_addr(&m); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g8 = lane >> 2, t4 = lane & 3;
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int b = bh / dm.H, h = bh % dm.H;
   const int n_begin = chunk * dm.chunk_tok;
   const int n_end = min(dm.N, n_begin + dm.chunk_tok);
   const int ntiles = n_end > n_begin ? (n_end - n_begin + kTok - 1) / kTok : 0;
   const size_t rs = (size_t)dm.H * kD;           // elements between tokens
+
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&full[s]), 1);
-    *abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(ctl->full[s]), 1);
+      mbar_init(bar(ctl->freed[s]), 5);   // the S^T MMAs' commit + warps 4-7
+    }
+    mbar_init(bar(ctl->f_full), 1);
+    mbar_init(bar(ctl->img_free), 1);
+    mbar_init(bar(ctl->drain), 1);
+    ctl->abort = 0;
     fence_barrier_init();
   }
+  // Wk_h^T as the K-major B operand of F = K Wk: row a (rank), channel c in box c / 64
+  for (int e = tid; e < kD * RK; e += kThreads) {
+    const int c = e / RK, a = e % RK;
+    *reinterpret_cast<__nv_bfloat16*>(smem + G::offW + (c >> 6) * (RK * 128) + img_off(a, c & 63)) =
+        Wk[((size_t)h * kD + c) * RK + a];
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
   __syncthreads();
-  const WaitCtl wc{abort_flag, status, 2000000000ull};
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtl wc{&ctl->abort, status, 2000000000ull};
 
-  // Wk_h [d][r] (contiguous in global) -> padded rows; part of the first copy group
-  for (int e = tid; e < kD * RK / 8; e += kThreads) {
-    const int c = e / (RK / 8), a8 = e % (RK / 8);
-    cp_async16(sbase + (uint32_t)(L::offW + (c * L::WP + a8 * 8) * 2), Wk + ((size_t)h * kD + c) * RK + a8 * 8, 16);
-  }
-  cp_async_commit();
-  // one thread issues the tile copies: 4 boxes (k, v x two channel halves) per tile
-  auto load_tile = [&](int t) {
-    const int s = t % kStages, n0 = n_begin + t * kTok;
-    const uint32_t bar = smem_u32(&full[s]);
-    mbar_expect_tx(bar, 2 * kTileBytes);
-    for (int c = 0; c < 2; ++c) {
-      tma_load_3d(sbase + (uint32_t)(L::offK + s * kTileBytes) + c * 8192, &tm_k, h * kD + 64 * c, n0, b, bar);
-      tma_load_3d(sbase + (uint32_t)(L::offV + s * kTileBytes) + c * 8192, &tm_v, h * kD + 64 * c, n0, b, bar);
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % kStages, n0 = n_begin + t * kTok;
+        if (t >= kStages && !mbar_wait(bar(ctl->freed[s]), ((t / kStages) - 1) & 1, wc)) break;
+        const uint32_t fb = bar(ctl->full[s]);
+        mbar_expect_tx(fb, 2 * kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + G::offK + s * kTileBytes + c * 8192, &tm_k, h * kD + 64 * c, n0, b, fb);
+          tma_load_3d(sbase + G::offV + s * kTileBytes + c * 8192, &tm_v, h * kD + 64 * c, n0, b, fb);
+        }
+        issued = t + 1;
+      }
+      // every issued copy must land before the CTA leaves
+      for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
+        mbar_wait(bar(ctl->full[t % kStages]), (t / kStages) & 1, wc, false);
     }
-  };
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    for (int t = 0; t < kStages - 1 && t < ntiles; ++t) load_tile(t);
-  }
-  cp_async_wait<0>();               // Wk (visible after the loop's first barrier)
-  int issued = ntiles < kStages - 1 ? ntiles : kStages - 1;
-
-  constexpr int NT_F = RK / 8;     // n-tiles of F (warps 0-3)
-  constexpr int MT_S = RK / 16;    // m-tiles of S
-  float sacc[MT_S][2][4];
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ features and the MMAs
+    const bool issuer = warp == 0 && lane == 0;
+    constexpr uint32_t idesc_f = idesc_f16(1, 64, RK, 0, 0);    // F = K Wk
+    constexpr uint32_t idesc_s = idesc_f16(1, 128, RK, 1, 0);   // S^T += V^T F~
+    constexpr int HR = RK / 2;                  // rank values per thread
+    const int row = 16 * warp + (lane & 15);    // token of the tile
+    const int a0 = (lane >> 4) * HR;            // first rank value of this thread
+    float zacc[HR];
 #pragma unroll
-  for (int a = 0; a < MT_S; ++a)
+    for (int a = 0; a < HR; ++a) zacc[a] = 0.f;
+    bool ok = true;
+    int done = 0;
+    for (int t = 0; t < ntiles && ok; ++t) {
+      const int s = t % kStages, n = n_begin + t * kTok + row;
+      if (issuer) {
+        ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t tk = sbase + G::offK + s * kTileBytes;
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+          for (int kk = 0; kk < kD / 16; ++kk)
+            mma_f16_ss(tmem + kColF, sdesc_sw128(tk + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                       sdesc_sw128(sbase + G::offW + (kk >> 2) * (RK * 128) + (kk & 3) * 32, 16, 1024), idesc_f,
+                       kk > 0);
+          mma_commit(bar(ctl->f_full));
+        }
+      }
+      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      ok = mbar_wait(bar(ctl->f_full), t & 1, wc);
+      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      tc_fence_after();
+      float f[HR];
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+      if constexpr (RK == 32) tmem_ld16x2_x16(lane_addr + kColF, f);
+      else tmem_ld16x2_x8(lane_addr + kColF, f);
+      tmem_wait_ld();
+      // phi, z, rotation (pairs a0/2 ..) and the hi / lo split; tokens past the chunk
+      // (or N) contribute nothing
+      const bool valid = n < n_end;
+      const TokPos pos = token_pos(dm, valid ? n : 0);
+      uint32_t hi[HR / 2], lo[HR / 2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[a][c][e] = 0.f;
-  float zacc[NT_F][2];
+      for (int p = 0; p < HR / 2; ++p) {
+        const float x0 = valid ? phi_fast(f[2 * p]) : 0.f;
+        const float x1 = valid ? phi_fast(f[2 * p + 1]) : 0.f;
+        zacc[2 * p] += x0;
+        zacc[2 * p + 1] += x1;
+        const float2 cs = valid ? rope_at(dm, rope, pos, a0 / 2 + p) : make_float2(1.f, 0.f);
+        split_bf16x2(cs.x * x0 - cs.y * x1, cs.y * x0 + cs.x * x1, hi[p], lo[p]);
+      }
+      // the previous tile's S^T MMAs read the images: wait for them before rewriting
+      if (t > 0) ok = mbar_wait(bar(ctl->img_free), (t - 1) & 1, wc);
+      if (ok) {
 #pragma unroll
-  for (int a = 0; a < NT_F; ++a) zacc[a][0] = zacc[a][1] = 0.f;
-
-  int consumed = 0;
-  for (int t = 0; t < ntiles; ++t) {
-    const int s = t % kStages, n0 = n_begin + t * kTok;
-    const bool ok = mbar_wait(smem_u32(&full[s]), (t / kStages) & 1, wc);
-    // tile t landed; every warp is done with tile t - 1 (its stage may be refilled)
-    if (__syncthreads_or(!ok)) break;
-    consumed = t + 1;
-    if (tid == 0 && issued < ntiles) {
+        for (int p = 0; p < HR / 2; ++p) {
+          const int a = a0 + 2 * p;
+          uint8_t* ih = smem + G::offF;
+          *reinterpret_cast<uint16_t*>(ih + img_off(a, row)) = (uint16_t)(hi[p] & 0xffffu);
+          *reinterpret_cast<uint16_t*>(ih + img_off(a + 1, row)) = (uint16_t)(hi[p] >> 16);
+          *reinterpret_cast<uint16_t*>(ih + RK * 128 + img_off(a, row)) = (uint16_t)(lo[p] & 0xffffu);
+          *reinterpret_cast<uint16_t*>(ih + RK * 128 + img_off(a + 1, row)) = (uint16_t)(lo[p] >> 16);
+        }
+      }
       fence_proxy_async_smem();
-      load_tile(issued++);
+      tc_fence_before();
+      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      if (issuer) {
+        tc_fence_after();
+        const uint32_t tv = sbase + G::offV + s * kTileBytes;
+        const uint64_t da = sdesc_sw128(tv, 8192, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kTok / 16; ++kk) {
+          const uint64_t dh = sdesc_sw128(sbase + G::offF + kk * 32, 16, 1024);
+          const uint64_t dl = sdesc_sw128(sbase + G::offF + RK * 128 + kk * 32, 16, 1024);
+          mma_f16_ss(tmem + kColS, da + 128 * kk, dh, idesc_s, t > 0 || kk > 0);
+          mma_f16_ss(tmem + kColS, da + 128 * kk, dl, idesc_s, true);
+        }
+        mma_commit(bar(ctl->freed[s]));
+        mma_commit(bar(ctl->img_free));
+      }
+      done = t + 1;
     }
-    const int cnt = min(kTok, n_end - n0);
-    const uint32_t tK = sbase + (uint32_t)(L::offK + s * kTileBytes);
-    const uint32_t tV = sbase + (uint32_t)(L::offV + s * kTileBytes);
-    const uint8_t* pK = smem + L::offK + s * kTileBytes;
-    const uint8_t* pV = smem + L::offV + s * kTileBytes;
-
-    if (warp < 4) {
-      // ---- F = K Wk for tokens 16*warp .. +15, all r; phi, z, rotation -> sF (hi, lo)
-      float f[NT_F][4];
+    // ---- chunk end: S^T (lane = channel) and z
+    if (issuer) {
+      mma_commit(bar(ctl->drain));             // every MMA of this CTA has completed
+      mbar_wait(bar(ctl->drain), 0, wc, false);
+    }
+    named_sync(1, 128);
+    tc_fence_after();
+    float* Sp = S_part + ((size_t)bh * dm.nchunk + chunk) * RK * kD;
+    if (ok && done == ntiles && ntiles > 0) {
+      float sv_[RK];
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+      tmem_ld32x32_x16(lane_addr + kColS, sv_);
+      if constexpr (RK == 32) tmem_ld32x32_x16(lane_addr + kColS + 16, sv_ + 16);
+      tmem_wait_ld();
 #pragma unroll
-      for (int a = 0; a < NT_F; ++a)
+      for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * warp + lane] = sv_[a];
+    } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) f[a][e] = 0.f;
+      for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * warp + lane] = 0.f;
+    }
+    // z: the 16 token lanes of each half-warp hold the same rank values
 #pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        uint32_t af[4];
-        ldsm_x4(tK + swz(16 * warp + (lane & 15), 2 * kk + (lane >> 4)), af[0], af[1], af[2], af[3]);
-#pragma unroll
-        for (int nt = 0; nt < NT_F; nt += 2) {
-          uint32_t bf[4];
-          const int row = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          ldsm_x4_t(smem_u32(sW + row * L::WP + nt * 8 + (lane >> 4) * 8), bf[0], bf[1], bf[2], bf[3]);
-          mma_bf16(f[nt], af, bf);
-          mma_bf16(f[nt + 1], af, bf + 2);
-        }
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int row = 16 * warp + g8 + 8 * half;
-        const int n = n0 + row;
-        const bool valid = n < n_end;
-        const TokPos pos = token_pos(dm, valid ? n : 0);
-#pragma unroll
-        for (int nt = 0; nt < NT_F; ++nt) {
-          const float x0 = valid ? phi_fast(f[nt][2 * half]) : 0.f;
-          const float x1 = valid ? phi_fast(f[nt][2 * half + 1]) : 0.f;
-          zacc[nt][0] += x0;
-          zacc[nt][1] += x1;
-          const float2 cs = valid ? rope_at(dm, rope, pos, nt * 4 + t4) : make_float2(1.f, 0.f);
-          const float y0 = cs.x * x0 - cs.y * x1;
-          const float y1 = cs.y * x0 + cs.x * x1;
-          uint32_t hi, lo;
-          split_bf16(y0, y1, hi, lo);
-          *reinterpret_cast<uint32_t*>(sF + row * L::RP + nt * 8 + 2 * t4) = hi;
-          *reinterpret_cast<uint32_t*>(sFl + row * L::RP + nt * 8 + 2 * t4) = lo;
-        }
-      }
-    } else if (warp < 6) {
-      // ---- pooling of k: thread = two adjacent channels, tokens added in order
-      const int cp = tid - 128;                     // channel pair 0..63
-      const int blk = n0 / kTok;
+    for (int a = 0; a < HR; ++a) {
+      float x = zacc[a];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      x += __shfl_xor_sync(0xffffffffu, x, 4);
+      x += __shfl_xor_sync(0xffffffffu, x, 8);
+      if ((lane & 15) == 0) ctl->zred[warp][a0 + a] = x;
+    }
+    named_sync(1, 128);
+    if (tid < RK)
+      z_part[((size_t)bh * dm.nchunk + chunk) * RK + tid] =
+          ((ctl->zred[0][tid] + ctl->zred[1][tid]) + ctl->zred[2][tid]) + ctl->zred[3][tid];
+    tc_fence_before();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ k means (+ e4m3 k)
+    const int cp = tid - 128;                     // channel pair 0..63
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages, n0 = n_begin + t * kTok;
+      const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
+      if (named_vote_or(2, 64, !ok)) break;
+      const uint8_t* pK = smem + G::offK + s * kTileBytes;
+      const int cnt = min(kTok, n_end - n0), blk = n0 / kTok;
       float a0 = 0.f, a1 = 0.f, am = 0.f;
       const uint8_t* col = pK + (cp >> 5) * 8192 + (cp & 3) * 4;   // box, word in chunk
       const int ch = (cp >> 2) & 7;                                 // chunk within the box
@@ -230,9 +359,9 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
         // e4m3 copy of the k tile: block scale from the max over the two warps
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        if (lane == 0) sRed[warp - 4] = am;
-        asm volatile("bar.sync 1, 64;" ::: "memory");
-        am = fmaxf(sRed[0], sRed[1]);
+        if (lane == 0) ctl->red[warp - 4] = am;
+        named_sync(2, 64);
+        am = fmaxf(ctl->red[0], ctl->red[1]);
         const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;
         if (cp == 0) sk[(size_t)bh * dm.nb + blk] = sc;
         for (int e = cp; e < cnt * 16; e += 64) {
@@ -240,13 +369,38 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
           *reinterpret_cast<uint2*>(k8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
               e4m3x8(*reinterpret_cast<const uint4*>(pK + swz(r, cv)), inv);
         }
-        asm volatile("bar.sync 1, 64;" ::: "memory");   // sRed is rewritten next tile
+        named_sync(2, 64);                         // red is rewritten next tile
       }
-    } else {
-      // ---- copy of v: fp16 (bf16 configuration) or e4m3 with its block scale (fp8)
-      const int tv = tid - 192;                     // 0..63
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ctl->freed[s]));
+    }
+  } else {
+    // ------------------------------------------------------------ copy of v
+    const int tv = tid - 192;                     // 0..63
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages, n0 = n_begin + t * kTok;
+      const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
+      if (named_vote_or(3, 64, !ok)) break;
+      const uint8_t* pV = smem + G::offV + s * kTileBytes;
+      const int cnt = min(kTok, n_end - n0), blk = n0 / kTok;
+      float am = 0.f;
+      bool finite = true;
+      for (int e = tv; e < cnt * 16; e += 64) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(e >> 4, e & 15));
+        const float m = absmax8(raw);
+        finite &= m <= 3.402823466e38f;             // false for inf and nan
+        am = fmaxf(am, m);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) ctl->red[4 + warp - 6] = am;
+      finite = !named_vote_or(3, 64, !finite);     // also orders the red writes
+      am = fmaxf(ctl->red[4], ctl->red[5]);
+      if (!finite && tv == 0) record_status(status, kDevRange);
       if constexpr (!FP8) {
-        bool bad = false;
+        // the block's exponent: v is carried as v * 2^-e in fp16
+        const int ex = v16_exponent(am);
+        if (tv == 0) vexp[(size_t)bh * dm.nb + blk] = ex;
         for (int e = tv; e < cnt * 16; e += 64) {
           const int r = e >> 4, cv = e & 15;
           const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(r, cv));
@@ -254,103 +408,43 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
           uint32_t o[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            // |x| >= 65536 (bf16 0x4780 and up, inf, nan) does not fit fp16; below that
-            // every bf16 value rounds to fp16 within its range
-            bad |= ((w[u] & 0x7fffu) >= 0x4780u) || (((w[u] >> 16) & 0x7fffu) >= 0x4780u);
-            const __half2 hv = __floats2half2_rn(__uint_as_float(w[u] << 16), __uint_as_float(w[u] & 0xffff0000u));
+            float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+            if (ex != 0) {
+              x0 = ldexpf(x0, -ex);
+              x1 = ldexpf(x1, -ex);
+            }
+            const __half2 hv = __floats2half2_rn(x0, x1);
             o[u] = *reinterpret_cast<const uint32_t*>(&hv);
           }
           *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
               make_uint4(o[0], o[1], o[2], o[3]);
         }
-        if (bad) record_status(status, kDevRange);
       } else {
-        float am = 0.f;
-        for (int e = tv; e < cnt * 16; e += 64) {
-          const int r = e >> 4, cv = e & 15;
-          am = fmaxf(am, absmax8(*reinterpret_cast<const uint4*>(pV + swz(r, cv))));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        if (lane == 0) sRed[4 + warp - 6] = am;
-        asm volatile("bar.sync 2, 64;" ::: "memory");
-        am = fmaxf(sRed[4], sRed[5]);
         const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;
-        const int blk = n0 / kTok;
         if (tv == 0) sv[(size_t)bh * dm.nb + blk] = sc;
         for (int e = tv; e < cnt * 16; e += 64) {
           const int r = e >> 4, cv = e & 15;
           *reinterpret_cast<uint2*>(v8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
               e4m3x8(*reinterpret_cast<const uint4*>(pV + swz(r, cv)), inv);
         }
-        asm volatile("bar.sync 2, 64;" ::: "memory");
       }
-    }
-    __syncthreads();                 // sF complete
-
-    // ---- S += F^T V: warp w owns channels 16w .. 16w + 15
-#pragma unroll
-    for (int kk = 0; kk < kTok / 16; ++kk) {
-      const int q = lane >> 3;
-      uint32_t af[MT_S][4], al[MT_S][4];
-#pragma unroll
-      for (int mt = 0; mt < MT_S; ++mt) {
-        const int off = (kk * 16 + (q >> 1) * 8 + (lane & 7)) * L::RP + mt * 16 + (q & 1) * 8;
-        ldsm_x4_t(smem_u32(sF + off), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-        ldsm_x4_t(smem_u32(sFl + off), al[mt][0], al[mt][1], al[mt][2], al[mt][3]);
-      }
-      uint32_t bf[4];
-      ldsm_x4_t(tV + swz(kk * 16 + (q & 1) * 8 + (lane & 7), 2 * warp + (q >> 1)), bf[0], bf[1], bf[2], bf[3]);
-#pragma unroll
-      for (int mt = 0; mt < MT_S; ++mt) {
-        mma_bf16(sacc[mt][0], af[mt], bf);
-        mma_bf16(sacc[mt][1], af[mt], bf + 2);
-        mma_bf16(sacc[mt][0], al[mt], bf);
-        mma_bf16(sacc[mt][1], al[mt], bf + 2);
-      }
+      named_sync(3, 64);                           // red is rewritten next tile
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ctl->freed[s]));
     }
   }
-  // every issued copy must land before the CTA leaves (only a failed wait leaves some)
-  if (tid == 0)
-    for (int t = consumed; t < issued; ++t) mbar_wait(smem_u32(&full[t % kStages]), (t / kStages) & 1, wc, false);
 
-  // ---- partials of this chunk (zeros for an empty chunk)
-  float* Sp = S_part + ((size_t)bh * dm.nchunk + chunk) * RK * kD;
-#pragma unroll
-  for (int mt = 0; mt < MT_S; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int row = mt * 16 + g8 + 8 * hh;
-        const int col = 16 * warp + nt * 8 + 2 * t4;
-        *reinterpret_cast<float2*>(Sp + (size_t)row * kD + col) =
-            make_float2(sacc[mt][nt][2 * hh], sacc[mt][nt][2 * hh + 1]);
-      }
   __syncthreads();
-  if (warp < 4) {
-    // lanes with equal t4 hold the same columns: add over the 8 row groups
-#pragma unroll
-    for (int nt = 0; nt < NT_F; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float x = zacc[nt][e];
-        x += __shfl_xor_sync(0xffffffffu, x, 4);
-        x += __shfl_xor_sync(0xffffffffu, x, 8);
-        x += __shfl_xor_sync(0xffffffffu, x, 16);
-        if (g8 == 0) sZ[warp * RK + nt * 8 + 2 * t4 + e] = x;
-      }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
-  __syncthreads();
-  if (tid < RK)
-    z_part[((size_t)bh * dm.nchunk + chunk) * RK + tid] =
-        ((sZ[tid] + sZ[RK + tid]) + sZ[2 * RK + tid]) + sZ[3 * RK + tid];
 }
 
 template <int RK, bool FP8>
 cudaError_t launch_variant(const Dims& dm, const void* k, const void* v, const void* Wk, const Workspace& ws,
                            cudaStream_t st) {
-  constexpr size_t smem = KVSmem<RK>::bytes;
+  constexpr size_t smem = kv_smem_bytes<RK>();
   cudaError_t e = cudaFuncSetAttribute(kv_pass_kernel<RK, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -360,8 +454,8 @@ cudaError_t launch_variant(const Dims& dm, const void* k, const void* v, const v
     return cudaErrorInvalidValue;
   dim3 grid(dm.nchunk, dm.B * dm.H);
   kv_pass_kernel<RK, FP8><<<grid, kThreads, smem, st>>>(
-      tk, tv, static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.kbar, ws.v16, ws.k8, ws.v8,
-      ws.sk, ws.sv, ws.status);
+      tk, tv, static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.kbar, ws.v16, ws.vexp,
+      ws.k8, ws.v8, ws.sk, ws.sv, ws.status);
   return cudaGetLastError();
 }
 

@@ -53,7 +53,7 @@ struct LSSmem {
   static constexpr int kTileElems = kLSTile * DP;
   static constexpr int kF = kLSTile * RP;     // rotated features [tok][r] (hi and lo parts)
   static constexpr size_t bytes = sizeof(__nv_bfloat16) * (kW + 4 * kTileElems + 2 * kF) +
-                                  sizeof(float) * 4 * RK;
+                                  sizeof(float) * (4 * RK + 4);   // z partials, v block maxima
 };
 
 // grid: x = chunk, y = b*H + h; 128 threads (4 warps).
@@ -62,13 +62,14 @@ struct LSSmem {
 //      the rotated features are split into bf16 hi + lo parts (F = hi + lo to ~2^-17)
 //   C: S += R(F)^T V_tile  (warp w: d columns [w*D/4, (w+1)*D/4))    2 x mma m16n8k16
 // The kernel also writes the fp16 copy of v that the attention kernel multiplies the
-// fp16 softmax weights with, and flags values outside the fp16 range.
+// fp16 softmax weights with (one power-of-two exponent per block, see v16_exponent), and
+// flags non-finite values.
 template <int D, int RK, bool FP8>
 __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin,
     const __nv_bfloat16* __restrict__ Wk, Dims dm, const float2* __restrict__ rope,
     float* __restrict__ S_part, float* __restrict__ z_part, __half* __restrict__ v16,
-    uint8_t* __restrict__ v8, float* __restrict__ sv, int* __restrict__ status) {
+    int* __restrict__ vexp, uint8_t* __restrict__ v8, float* __restrict__ sv, int* __restrict__ status) {
   using L = LSSmem<D, RK>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem_raw);
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
   __nv_bfloat16* sV = sK + 2 * L::kTileElems;         // [2][tile]
   __nv_bfloat16* sF = sV + 2 * L::kTileElems;       // hi part
   __nv_bfloat16* sFl = sF + L::kF;                    // lo part
-  float* sZ = reinterpret_cast<float*>(sFl + L::kF);  // [4][RK]
+  float* sZ = reinterpret_cast<float*>(sFl + L::kF);  // [4][RK] z partials, then 4 maxima of v
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
@@ -137,10 +138,32 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
     const __nv_bfloat16* tV = sV + stage * L::kTileElems;
 
     if constexpr (!FP8) {
-      // fp16 copy of the V tile (+ range check)
+      // fp16 copy of the V tile (one 64-token block) as v * 2^-e, e from the block's
+      // largest |v| (v16_exponent); non-finite values set ROLA_ERR_RANGE
       constexpr int kVecPerRow = D / 8;
       const int n0 = n_begin + tile * kLSTile;
-      bool bad = false;
+      float amax = 0.f;
+      bool finite = true;
+      for (int e = tid; e < kLSTile * kVecPerRow; e += 128) {
+        const int rr = e / kVecPerRow, cv = e % kVecPerRow;
+        if (n0 + rr >= n_end) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(tV + rr * L::DP + cv * 8);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float m = fmaxf(fabsf(__uint_as_float(w[t] << 16)), fabsf(__uint_as_float(w[t] & 0xffff0000u)));
+          finite &= m <= 3.402823466e38f;
+          amax = fmaxf(amax, m);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) sZ[4 * RK + warp] = amax;
+      finite = __syncthreads_and(finite);
+      amax = fmaxf(fmaxf(sZ[4 * RK], sZ[4 * RK + 1]), fmaxf(sZ[4 * RK + 2], sZ[4 * RK + 3]));
+      if (!finite && tid == 0) record_status(status, kDevRange);
+      const int ex = finite ? v16_exponent(amax) : 0;
+      if (tid == 0) vexp[(size_t)bh * dm.nb + n0 / kLSTile] = ex;
       for (int e = tid; e < kLSTile * kVecPerRow; e += 128) {
         const int rr = e / kVecPerRow, cv = e % kVecPerRow, n = n0 + rr;
         if (n >= n_end) continue;
@@ -150,14 +173,17 @@ __global__ void __launch_bounds__(128) linear_state_bf16_kernel(
         __half2* dst = reinterpret_cast<__half2*>(&packed);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float2 f = __bfloat1622float2(src[t]);
-          bad |= !(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f);
+          float2 f = __bfloat1622float2(src[t]);
+          if (ex != 0) {
+            f.x = ldexpf(f.x, -ex);
+            f.y = ldexpf(f.y, -ex);
+          }
           dst[t] = __floats2half2_rn(f.x, f.y);
         }
         *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n) * row_stride + (size_t)h * D + cv * 8) =
             packed;
       }
-      if (bad) record_status(status, kDevRange);
+      __syncthreads();                             // sZ's maxima are rewritten next tile
     } else {
       // e4m3 copy of the V tile: the tile is one 64-token block; scale = absmax / 448.
       constexpr int kVecPerRow = D / 8;
@@ -426,7 +452,7 @@ cudaError_t launch_ls(const Dims& dm, rola_dtype dt, const void* k, const void* 
       if (e != cudaSuccess) return e;
       linear_state_bf16_kernel<D, RK, true><<<grid, 128, smem, st>>>(
           static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, nullptr, ws.v8,
+          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, nullptr, nullptr, ws.v8,
           ws.sv, ws.status);
     } else {
       cudaError_t e = cudaFuncSetAttribute(linear_state_bf16_kernel<D, RK, false>,
@@ -434,7 +460,7 @@ cudaError_t launch_ls(const Dims& dm, rola_dtype dt, const void* k, const void* 
       if (e != cudaSuccess) return e;
       linear_state_bf16_kernel<D, RK, false><<<grid, 128, smem, st>>>(
           static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.v16, nullptr,
+          static_cast<const __nv_bfloat16*>(Wk), dm, ws.rope, ws.S_part, ws.z_part, ws.v16, ws.vexp, nullptr,
           nullptr, ws.status);
     }
   }

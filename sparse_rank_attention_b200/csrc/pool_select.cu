@@ -460,10 +460,18 @@ cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // The array's device address is looked up with this device current: on the first call
+  // on a device, and again on every call made outside stream capture (so that a device
+  // reset, which reloads the module, cannot leave a stale address behind).  A call made
+  // while `st` is being captured uses the address of the last uncaptured call.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return e;
   char* base = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (g_scratch_addr[dev] == nullptr || cap == cudaStreamCaptureStatusNone) {
+      if (cap != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
       void* ptr = nullptr;
       e = cudaGetSymbolAddress(&ptr, g_select_scratch);
       if (e != cudaSuccess) return e;

@@ -54,7 +54,8 @@ rola_status check_params(const rola_params* p) {
   if (p->dtype != ROLA_F32 && p->dtype != ROLA_BF16 && p->dtype != ROLA_FP8_E4M3)
     return ROLA_ERR_INVALID_ARG;
   if (p->dtype == ROLA_FP8_E4M3 && p->d != 128) return ROLA_ERR_UNSUPPORTED;  // tcgen05 tile only
-  if (p->gate_per_token != 0 && p->gate_per_token != 1) return ROLA_ERR_INVALID_ARG;
+  if (p->gate != ROLA_GATE_HEAD && p->gate != ROLA_GATE_TOKEN && p->gate != ROLA_GATE_QPROJ)
+    return ROLA_ERR_INVALID_ARG;
   const int nb = (p->N + rola::kBlock - 1) / rola::kBlock;
   if (nb > kMaxBlocks) return ROLA_ERR_UNSUPPORTED;
   if ((long long)p->B * p->H * nb > (1ll << 31) / 64) return ROLA_ERR_UNSUPPORTED;
@@ -100,7 +101,7 @@ Dims make_dims(const rola_params& p) {
   dm.nchunk = (p.N + dm.chunk_tok - 1) / dm.chunk_tok;
   dm.scale = p.softmax_scale > 0.f ? p.softmax_scale : (float)(1.0 / std::sqrt((double)p.d));
   dm.rope_base = p.rope_base;
-  dm.gate_per_token = p.gate_per_token;
+  dm.gate_mode = p.gate;
   return dm;
 }
 
@@ -126,8 +127,10 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   w.z = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r));
   w.S_hi = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
   w.S_lo = reinterpret_cast<__nv_bfloat16*>(take(sizeof(__nv_bfloat16) * BH * dm.r * dm.d));
-  if (p.dtype == ROLA_BF16)
+  if (p.dtype == ROLA_BF16) {
     w.v16 = reinterpret_cast<__half*>(take(sizeof(__half) * (size_t)dm.B * dm.N * dm.H * dm.d));
+    w.vexp = reinterpret_cast<int*>(take(sizeof(int) * BH * dm.nb));
+  }
   if (p.dtype != ROLA_F32 && p.d == 128) {
     w.redo = reinterpret_cast<int*>(take(sizeof(int) * (1 + 2 * BH * dm.nb)));
     w.simg = reinterpret_cast<uint8_t*>(take(BH * 4 * dm.r * 128));
@@ -179,7 +182,7 @@ rola_status rola_params_default(rola_params* p) {
   p->rope_base = 10000.0;
   p->softmax_scale = 0.f;
   p->dtype = ROLA_BF16;
-  p->gate_per_token = 0;
+  p->gate = ROLA_GATE_HEAD;
   return ROLA_OK;
 }
 
@@ -389,6 +392,9 @@ rola_status rola_select_blocks_noalloc(const rola_params* p, const void* q, cons
     return ROLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*p);
   if (rola::select_noalloc_bytes(dm) > rola::select_noalloc_capacity()) return ROLA_ERR_WORKSPACE;
+  const size_t act = (size_t)p->B * p->N * p->H * p->d * elem_size(p->dtype);
+  const size_t lists = sizeof(int32_t) * (size_t)dm.B * dm.H * dm.nb * dm.k;
+  if (overlaps(col_idx, lists, q, act) || overlaps(col_idx, lists, k, act)) return ROLA_ERR_INVALID_ARG;
   return cuda_status(rola::select_blocks_noalloc(dm, p->dtype, q, k, col_idx,
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }

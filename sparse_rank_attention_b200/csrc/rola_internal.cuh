@@ -31,12 +31,40 @@ struct Dims {
   int nchunk;                 // linear-state partial sums per (b, h)
   float scale;                // softmax logit scale
   double rope_base;
-  int gate_per_token;         // gain g per token and head [B, N, H] (else per head [H])
+  int gate_mode;              // rola_gate: gain per head g[H], per token g[B, N, H], or
+                              // computed from the query (g = gate_proj [H, d], gate_bias [H])
 };
 
-// The gain of token n of (b, h): g[H], or g[B, N, H] for a per-token gate.
+// The gain of token n of (b, h) for the gates that are read: g[H] (ROLA_GATE_HEAD) or
+// g[B, N, H] (ROLA_GATE_TOKEN).
 __host__ __device__ inline size_t gain_index(const Dims& dm, int b, int n, int h) {
-  return dm.gate_per_token ? ((size_t)b * dm.N + n) * dm.H + h : (size_t)h;
+  return dm.gate_mode == ROLA_GATE_TOKEN ? ((size_t)b * dm.N + n) * dm.H + h : (size_t)h;
+}
+
+// Partial dot product of channels [c0, c1) of a query row with the gate projection of
+// head h (ROLA_GATE_QPROJ; g holds gate_proj [H, d] and then gate_bias [H]).
+template <typename T>
+__device__ __forceinline__ float gate_dot(const Dims& dm, const float* __restrict__ g, const T* q_row, int h,
+                                          int c0, int c1) {
+  const float* wg = g + (size_t)h * dm.d;
+  float a = 0.f;
+  for (int c = c0; c < c1; ++c) a = fmaf(static_cast<float>(q_row[c]), __ldg(wg + c), a);
+  return a;
+}
+
+// sigmoid(dot + gate_bias_h): the gain of ROLA_GATE_QPROJ from the finished dot product.
+__device__ __forceinline__ float gate_sigmoid(const Dims& dm, const float* __restrict__ g, int h, float dot) {
+  const float a = dot + __ldg(g + (size_t)dm.H * dm.d + h);
+  return 1.f / (1.f + __expf(-a));
+}
+
+// The gain of token n of (b, h) for any gate: read, or computed from the whole query row
+// q_row (d channels) for ROLA_GATE_QPROJ.
+template <typename T>
+__device__ __forceinline__ float gate_value(const Dims& dm, const float* __restrict__ g, const T* q_row, int b,
+                                            int n, int h) {
+  if (dm.gate_mode == ROLA_GATE_QPROJ) return gate_sigmoid(dm, g, h, gate_dot(dm, g, q_row, h, 0, dm.d));
+  return g[gain_index(dm, b, n, h)];
 }
 
 // Device pointers carved out of the caller's workspace.
@@ -53,7 +81,8 @@ struct Workspace {
   float* z;           // [B, H, r]
   __nv_bfloat16* S_hi;  // [B, H, r, d] bf16(S)            } S = S_hi + S_lo to ~2^-17:
   __nv_bfloat16* S_lo;  // [B, H, r, d] bf16(S - S_hi)     } tensor-core operands of the epilogue
-  __half* v16;          // [B, N, H, d] fp16 copy of v (bf16 and fp8-free paths: PV operand)
+  __half* v16;          // [B, N, H, d] fp16 copy of v, each (b, h, block) as v * 2^-vexp
+  int* vexp;            // [B, H, nb] the fp16 copy's power-of-two exponent per block
   uint8_t* simg;        // [B, H] S_h^T hi|lo as 128-byte-swizzled MN-major operand images
   uint8_t* uimg;        // [B, H, nb] (R u)^T hi|lo images ([r rows][64 tokens], swizzled)
   float* gden;          // [B, H, nb, 64] g_h / (u . z_h) per query token
@@ -120,6 +149,17 @@ cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, 
 // ---- device helpers ----
 __device__ __forceinline__ void record_status(int* status, int code) {
   atomicCAS(status, kDevOk, code);
+}
+
+// Exponent e of the fp16 copy of a 64-token block of v (v is carried as v * 2^-e) from
+// the block's largest |v|: 0 while that lies in [2^-6, 2^15) (every element then keeps
+// fp16's precision down to 2^-8 of the largest), else the exponent that brings it into
+// [2^14, 2^15).  Blocks of zeros, or with a non-finite value, take 0.
+__device__ __forceinline__ int v16_exponent(float absmax) {
+  if (!(absmax > 0.f) || !(absmax <= 3.402823466e38f) || (absmax >= 0x1p-6f && absmax < 32768.f)) return 0;
+  int e2;
+  frexpf(absmax, &e2);                 // absmax = m * 2^e2, m in [0.5, 1)
+  return (e2 - 1) - 14;
 }
 
 // Rotary cos/sin of pair c for token n.

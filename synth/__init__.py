@@ -77,6 +77,22 @@ WORKLOADS["wan21_14b_480p_cfg_b2"] = replace(WORKLOADS["wan21_14b_480p"], name="
 WORKLOADS["wan21_14b_480p_dense_g0"] = replace(WORKLOADS["wan21_14b_480p"],
                                                name="wan21_14b_480p_dense_g0", topk=1.0,
                                                g_const=0.0)
+# Image-to-video at 480P (the pages' I2V example keeps 0.05): the latent grid follows the
+# input image's aspect ratio and the frame count (NUM_FRAMES, ASPECT_RATIO,
+# FIXED_RESOLUTION), so the sequence length and the 3D grid change with them.
+#   portrait 480x832: 21 x 52 x 30 (same N as landscape, transposed grid);
+#   square 624x624:   21 x 39 x 39 = 31941 tokens (a 5-token last block);
+#   49 frames:        13 x 30 x 52 = 20280 tokens.
+WORKLOADS["wan21_14b_i2v_480p_portrait"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_i2v_480p_portrait",
+                                                   grid=(21, 52, 30))
+WORKLOADS["wan21_14b_i2v_480p_square"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_i2v_480p_square",
+                                                 N=31941, grid=(21, 39, 39))
+WORKLOADS["wan21_14b_i2v_480p_49f"] = replace(WORKLOADS["wan21_14b_480p"], name="wan21_14b_i2v_480p_49f",
+                                              N=20280, grid=(13, 30, 52))
+# Wan2.2-A14B (two experts of the 14B attention shape, high- and low-noise) with the keep
+# ratio of the pages' Wan 2.2 example, 0.1, at 480P and 720P.
+WORKLOADS["wan22_a14b_480p"] = replace(WORKLOADS["wan21_14b_480p"], name="wan22_a14b_480p", topk=0.10)
+WORKLOADS["wan22_a14b_720p"] = replace(WORKLOADS["wan21_14b_720p"], name="wan22_a14b_720p", topk=0.10)
 
 
 def custom(name="custom", B=1, H=2, N=1024, d=64, r=16, topk=0.25, grid=None, dtype="bf16",
@@ -149,4 +165,15 @@ def make_gate(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     return torch.rand((w.B, w.N, w.H), generator=gen, device=device, dtype=torch.float32)
 
 
-__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs", "make_gate"]
+def make_gate_proj(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Parameters of a gate computed from the query (the gate_proj / gate_bias pair): one
+    fp32 buffer of H*(d+1) values, gate_proj [H, d] ~ N(0, 1/d) followed by gate_bias [H]
+    ~ U(-0.5, 0.5), from its own seeded stream."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    wg = torch.randn((w.H, w.d), generator=gen, device=device, dtype=torch.float32) / math.sqrt(w.d)
+    bg = torch.rand((w.H,), generator=gen, device=device, dtype=torch.float32) - 0.5
+    return torch.cat([wg.reshape(-1), bg]).contiguous()
+
+
+__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs", "make_gate", "make_gate_proj"]

@@ -9,7 +9,10 @@ Tolerances (stated by the operator's specification, tied to the input type):
   * fp8 configuration:  RMS(out - oracle) <= 6e-2 * RMS(oracle out), over the compared
     elements (a normwise bound: an elementwise one is out of reach of e4m3 V, whose 3
     mantissa bits alone move an output dominated by one value by up to 2^-4 of it), plus
-    a guard on every 64-token query block: RMS of its error <= 0.25 * RMS(oracle out).
+    a guard on every 64-token query block: RMS of its error <= 0.08 * RMS(oracle out)
+    (a CPU emulation of the exact quantisation gives at most 0.047 per block on these
+    inputs; the GPU cases measured up to 0.060 on the smallest ragged problems, where a
+    block's few valid rows weigh most).
 The oracle's double-precision output (before its own final rounding) is the reference.
 The operator's last step rounds out once to bf16; that rounding alone moves an element
 by up to half a bf16 ulp (2^-8 of its magnitude), which on these outputs (max/RMS of
@@ -28,7 +31,7 @@ import synth
 import sparse_rank_attention_b200 as rola
 
 TOL_REL = {"bf16": 2e-2, "fp8": 6e-2}
-FP8_BLOCK_GUARD = 0.25
+FP8_BLOCK_GUARD = 0.08
 TOL_ABS_F32 = 1e-4
 
 

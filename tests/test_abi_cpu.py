@@ -59,18 +59,20 @@ def test_invalid_params_rejected(kw, code):
     assert rola.load().rola_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code
 
 
-def test_gate_per_token_flag():
+def test_gate_modes():
     lib = rola.load()
     p = rola.RolaParams()
     assert lib.rola_params_default(ctypes.byref(p)) == 0
-    assert p.gate_per_token == 0                       # per-head gain by default
+    assert p.gate == 0                                 # ROLA_GATE_HEAD by default
     n = ctypes.c_size_t()
-    for flag, code in ((0, 0), (1, 0), (2, 1), (-1, 1)):
+    for mode, code in ((0, 0), (1, 0), (2, 0), (3, 1), (-1, 1)):
         q = _params()
-        q.gate_per_token = flag
+        q.gate = mode
         assert lib.rola_workspace_size(ctypes.byref(q), ctypes.byref(n)) == code
-    # the flag does not change the workspace (the gains are an input, read in place)
-    assert rola.workspace_size(_params(gate_per_token=True)) == rola.workspace_size(_params())
+    # the gate does not change the workspace (gains or gate parameters are read in place)
+    base = rola.workspace_size(_params())
+    assert rola.workspace_size(_params(gate_per_token=True)) == base
+    assert rola.workspace_size(_params(gate="proj")) == base
 
 
 def test_block_size_must_be_64():

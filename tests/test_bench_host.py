@@ -93,3 +93,14 @@ def test_reference_arm_prints_one_contract_line():
 def test_reference_arm_other_ranks_exit_without_work():
     assert _run_bench(["--impl", "reference", "--workload", "tiny_f32_h2_n1024", "--steps", "1",
                        "--warmup", "1"], {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_clock_summary_from_nvml_samples():
+    """The clock record names each throttle reason whose NVML bit was seen and reports the
+    median SM clock over the samples taken during the timed region."""
+    c = bench.ClockSampler(0)
+    c.samples = [(1965.0, 1965.0, 0), (1800.0, 1965.0, 0x4), (1950.0, 1965.0, 0x4 | 0x8)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert s["source"].startswith("nvml")

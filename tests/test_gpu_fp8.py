@@ -83,6 +83,9 @@ SMALL = [
                  dtype="fp8"),
     synth.custom("fp8_block_offsets", B=1, H=2, N=2048, d=128, r=32, topk=0.125, dist="block_offset",
                  dtype="fp8"),
+    # more than 3 x 148 tiles: each persistent CTA runs several tiles, across heads and batches
+    synth.custom("fp8_multitile_b2_tail54", B=2, H=4, N=7990, d=128, r=32, topk=0.1, grid=(2, 17, 235),
+                 dtype="fp8"),
 ]
 
 
@@ -107,7 +110,7 @@ def test_fp8_zero_block_scale_is_one():
 
 def test_fp8_wan_720p_sampled():
     w = synth.WORKLOADS["wan21_14b_720p_fp8"]
-    _check(w, seed=0, blocks=sample_blocks(w, 3, 12, 0))
+    _check(w, seed=0, blocks=sample_blocks(w, 4, 64, 0))
 
 
 def test_fp8_careful_pass_recomputes_overflowing_tiles():

@@ -1,9 +1,13 @@
 """GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
 
 Small cases are compared in full (every output element, every block list, the
-pooled means and the linear state).  The Wan-shaped workloads are compared at full
-size on every block list, pooled mean and state entry, and on a seeded sample of
-query blocks (always including the ragged tail block) for the outputs.
+pooled means and the linear state).  Two of them have more than three query-block
+tiles per SM (1024 and 1000 tiles over 148 persistent CTAs), so every CTA of the
+tcgen05 attention kernel walks several tiles and crosses head (and batch) boundaries
+while compared element by element.  The Wan-shaped workloads, including every point of
+the 14B-480P sparsity sweep, are compared at full size on every block list, pooled mean
+and state entry, and on a seeded sample of at least 4 heads x 64 query blocks (always
+including the first and the ragged tail block) for the outputs.
 """
 import numpy as np
 import pytest
@@ -69,6 +73,10 @@ SMALL = [
     synth.custom("f32_d128_r32_3d", B=1, H=2, N=900, d=128, r=32, topk=0.3, grid=(3, 5, 60),
                  dtype="f32"),
     synth.custom("f32_tail1", B=2, H=1, N=129, d=64, r=16, topk=0.6, dtype="f32"),
+    # more than 3 x 148 tiles: each persistent CTA runs several tiles, across heads
+    synth.custom("bf16_multitile_h8", B=1, H=8, N=8192, d=128, r=32, topk=0.1, grid=(2, 64, 64)),
+    synth.custom("bf16_multitile_b2_tail54", B=2, H=4, N=7990, d=128, r=32, topk=0.1,
+                 grid=(2, 17, 235)),
 ]
 
 
@@ -104,7 +112,7 @@ def test_run_to_run_bitwise_identical():
     assert torch.equal(a, b) and torch.equal(Sa, Sb) and torch.equal(za, zb)
 
 
-def _compare_sampled(w, n_heads=3, n_blocks=12, seed=0):
+def _compare_sampled(w, n_heads=4, n_blocks=64, seed=0):
     inp = synth.make_inputs(w, seed=seed, device="cuda")
     res = run_gpu(w, inp)
     assert res["status"] == 0
@@ -128,9 +136,15 @@ def _compare_sampled(w, n_heads=3, n_blocks=12, seed=0):
     return r
 
 
+# every Wan shape, the whole 14B-480P sparsity sweep (topk 0.03 / 0.05 / 0.1 / 0.25 / 1 with
+# per-head gains, and 1 with g = 0), the B = 2 classifier-free-guidance batch, the I2V
+# grids (portrait, square with a 5-token last block, 49 frames) and Wan2.2-A14B at topk 0.1
 @pytest.mark.parametrize("name", ["wan21_1p3b_480p", "wan21_14b_480p", "wan21_14b_720p",
-                                  "wan21_14b_480p_dense_g0", "wan21_14b_480p_topk0.25",
-                                  "wan21_14b_480p_cfg_b2"])
+                                  "wan21_14b_480p_topk0.03", "wan21_14b_480p_topk0.1",
+                                  "wan21_14b_480p_topk0.25", "wan21_14b_480p_topk1",
+                                  "wan21_14b_480p_dense_g0", "wan21_14b_480p_cfg_b2",
+                                  "wan21_14b_i2v_480p_portrait", "wan21_14b_i2v_480p_square",
+                                  "wan21_14b_i2v_480p_49f", "wan22_a14b_480p", "wan22_a14b_720p"])
 def test_wan_shapes_sampled(name):
     _compare_sampled(synth.WORKLOADS[name])
 
@@ -170,3 +184,41 @@ def test_fast_pass_alone_on_wan_like_inputs():
     w = synth.custom("bf16_wan_like", B=1, H=2, N=4152, d=128, r=32, topk=0.1, grid=(2, 4, 519))
     res = run_gpu(w, synth.make_inputs(w, seed=1, device="cuda"))
     assert res["status"] == 0 and res["plan"].attend_redo_count() == 0
+
+
+def _wide_range_v(inp, w):
+    """v spread over the whole bf16 range: blocks scaled by 1e6, 1e-6 and 1e30 (values
+    outside fp16's range both ways), the rest left as drawn."""
+    v = inp["v"].float()
+    for blk, f in ((1, 1e6), (3, 1e-6), (6, 1e30), (9, 1e-30), (12, 3e4)):
+        v[:, 64 * blk:64 * blk + 64] *= f
+    inp["v"] = v.to(inp["v"].dtype)
+    return inp
+
+
+@pytest.mark.parametrize("g_const", [0.0, None], ids=["sparse_only", "with_linear"])
+@pytest.mark.parametrize("d", [128, 64])
+def test_v_over_the_whole_bf16_range(d, g_const):
+    """Every finite bf16 v is accepted: the fp16 copy of v carries one power-of-two exponent
+    per block, applied back inside the attention (in the careful pass where a row's kept
+    blocks differ).  Compared in full with the oracle; with g = 0 the output is the sparse
+    branch alone, so each query block's check sees its own kept blocks' scale (the linear
+    branch, over all keys, would otherwise carry the 1e30 blocks into every row)."""
+    w = synth.custom(f"bf16_wide_v_d{d}", B=1, H=2, N=1000, d=d, r=32, topk=0.5, grid=(1, 8, 125),
+                     g_const=g_const)
+    inp = _wide_range_v(synth.make_inputs(w, seed=8, device="cuda"), w)
+    res = run_gpu(w, inp)
+    assert res["status"] == 0
+    if d == 128:
+        assert res["plan"].attend_redo_count() > 0   # rows mixing exponents took the careful pass
+    h = host_inputs(inp)
+    out, col = O.forward(shape_of(w), h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"])
+    np.testing.assert_array_equal(res["col"], col)
+    got = np32(res["out"]).astype(np.float64)
+    # rows differ by up to 1e60 in magnitude here: the tolerance is taken per query block
+    # (2e-2 of the block's own RMS plus half an ulp), so small rows are held to their scale
+    for b in range(w.B):
+        for hh in range(w.H):
+            for i in range(w.nb):
+                n0, n1 = 64 * i, min(w.N, 64 * i + 64)
+                check_out(got[b, n0:n1, hh], out[b, n0:n1, hh], "bf16", f"{w.name} h{hh} block {i}")

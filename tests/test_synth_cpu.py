@@ -32,3 +32,14 @@ def test_cfg_batch_workload_is_the_480p_shape_with_two_entries():
     w, base = synth.WORKLOADS["wan21_14b_480p_cfg_b2"], synth.WORKLOADS["wan21_14b_480p"]
     assert (w.B, w.H, w.N, w.d, w.r, w.topk, w.grid) == (2, base.H, base.N, base.d, base.r, base.topk,
                                                           base.grid)
+
+
+def test_gate_projection_parameters_are_reproducible_and_shaped():
+    w = synth.custom("gp", B=1, H=3, N=100, d=64, r=16)
+    a = synth.make_gate_proj(w, seed=2)
+    b = synth.make_gate_proj(w, seed=2)
+    assert a.shape == (w.H * (w.d + 1),) and a.dtype == torch.float32
+    assert torch.equal(a, b)
+    bias = a[w.H * w.d:]
+    assert torch.all(bias.abs() <= 0.5)
+    assert 0.5 / w.d ** 0.5 < a[:w.H * w.d].std() < 2.0 / w.d ** 0.5
