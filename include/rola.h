@@ -70,8 +70,8 @@ typedef enum {
   ROLA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed                */
   ROLA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out (see poll)       */
   ROLA_ERR_DEVICE_BOUNDS = 6,   /* a device-side index check failed (see poll)         */
-  ROLA_ERR_RANGE = 7            /* an input value is non-finite or, for v in ROLA_BF16, */
-                                /* outside +-65504 (v is carried in fp16; see poll)     */
+  ROLA_ERR_RANGE = 7            /* v holds a non-finite value (ROLA_BF16; reported by  */
+                                /* poll: the kernels that copy v check every element)  */
 } rola_status;
 
 typedef enum {
@@ -229,6 +229,18 @@ ROLA_API rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us);
 ROLA_API rola_status rola_profile_stages(rola_plan_t plan, int enable);
 ROLA_API rola_status rola_get_stage_times(rola_plan_t plan, float* ms, int max_stages, int* nstages,
                                           int* ncalls);
+
+/* Self-test of the softmax exponentials of the head-dim-128 attention kernels (a
+ * measurement aid; the pages fix only P = exp(s - m)): y[i] = 2^x[i] for the n device
+ * floats at x, computed by the same device functions the kernels call.  mode 0: the
+ * special-function unit's ex2.approx (relative error about 2^-22; 2^-inf = 0).  mode 1: the
+ * polynomial on the FMA pipe that the e4m3 path uses for a quarter of its exponentials
+ * (x = n + f, n = round(x), a cubic in f, n added into the exponent field; relative error
+ * below 7.8e-5 for -125 <= x <= 0; x below -125, -inf and NaN give 2^-125).  x and y are
+ * device pointers of n floats (equal or disjoint); n >= 0.  Asynchronous on `stream`.
+ * Returns ROLA_ERR_INVALID_ARG for a null pointer with n > 0, a negative n or another mode,
+ * ROLA_ERR_CUDA if the launch fails. */
+ROLA_API rola_status rola_eval_exp2(const float* x, float* y, int64_t n, int mode, rola_stream_t stream);
 
 ROLA_API const char* rola_status_string(rola_status s);
 

@@ -37,7 +37,7 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
            "rola_select_blocks_noalloc", "rola_get_fp8_copies", "rola_profile_stages",
-           "rola_get_stage_times", "rola_get_attend_redo_count")
+           "rola_get_stage_times", "rola_get_attend_redo_count", "rola_eval_exp2")
 
 
 class RolaError(RuntimeError):
@@ -93,6 +93,7 @@ def load() -> ctypes.CDLL:
         "rola_get_fp8_copies": [P, P, P, P, P, P, P, P],
         "rola_profile_stages": [P, i32],
         "rola_get_attend_redo_count": [P, ctypes.POINTER(i32), P],
+        "rola_eval_exp2": [P, P, ctypes.c_int64, i32, P],
         "rola_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32),
                                  ctypes.POINTER(i32)],
     }.items():
@@ -105,6 +106,16 @@ def load() -> ctypes.CDLL:
     lib.rola_status_string.restype = ctypes.c_char_p
     _lib = lib
     return lib
+
+
+def eval_exp2(x, mode: int):
+    """2^x of a contiguous fp32 CUDA tensor through rola_eval_exp2 (mode 0: ex2.approx, 1: the
+    polynomial on the FMA pipe), the device functions of the attention kernels' softmax."""
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    y = torch.empty_like(x)
+    _check(load().rola_eval_exp2(x.data_ptr(), y.data_ptr(), x.numel(), mode,
+                                 torch.cuda.current_stream().cuda_stream), "rola_eval_exp2")
+    return y
 
 
 def _lib_status_string(code: int) -> str:

@@ -46,15 +46,22 @@
 
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "softmax_exp.cuh"
 
 namespace rola {
 namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
-constexpr int kSoftmaxWarp0 = 4;  // warps 4-7: query columns 0-31, warps 8-11: columns 32-63
-constexpr int kSoftmaxWarps = 8;
+#ifndef ROLA_ATTEND_GROUPS
+#define ROLA_ATTEND_GROUPS 2
+#endif
+constexpr int kGroups = ROLA_ATTEND_GROUPS;   // softmax groups of four warps
+constexpr int kCols = 64 / kGroups;            // query columns of a group
+constexpr int kThreads = 128 + 128 * kGroups;
+constexpr int kSoftmaxWarp0 = 4;  // group g = warps 4 + 4g .. 7 + 4g: query columns [kCols g, kCols (g + 1))
+constexpr int kSoftmaxWarps = 4 * kGroups;
+static_assert(kGroups == 2 || kGroups == 4, "softmax groups");
 constexpr unsigned kGroupOffsetNs = 400;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;         // S^T buffers at columns 0, 64, 128
@@ -100,36 +107,14 @@ struct Ctl {
   uint32_t tmem_base;
   int abort;
   alignas(16) float fac[64];
-  alignas(16) float red[2][4][32];   // per query group: per-warp partial reductions
+  alignas(16) float red[kGroups][4][32];   // per query group: per-warp partial reductions
   alignas(16) float linv[64];
-  float vref[2][4];  // fp8: per-warp partial max of the kept blocks' V scales
-  int emax[2][4], emin[2][4];  // 16-bit path: per-warp range of the kept blocks' v exponents
+  float vref[kGroups][4];  // fp8: per-warp partial max of the kept blocks' V scales
+  int emax[kGroups][4], emin[kGroups][4];  // 16-bit path: per-warp range of the kept blocks' v exponents
 };
 template <bool FP8>
 constexpr size_t smem_bytes() { return Geo<FP8>::kOffCtl + sizeof(Ctl) + 1024; }
 
-
-// 2^x on the special-function unit (ex2.approx: relative error ~2^-22, 2^-inf = 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^x on the FMA and integer pipes, leaving the special-function unit to the other
-// exponentials: x = n + f with n = round(x) (1.5 * 2^23 added and taken away), f in
-// [-0.5, 0.5]; 2^f from a cubic least-squares fit at Chebyshev nodes (relative error
-// below 7.8e-5, under half an fp16 ulp); 2^n added into the exponent field.  x is clamped
-// to -125 (results below 2^-125 are not needed: P is e4m3 where this is used).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float n = t - 12582912.f;
-  const float fr = x - n;
-  const float p = fmaf(fmaf(fmaf(0.05508868f, fr, 0.24260405f), fr, 0.69327623f), fr, 0.99992895f);
-  // t's low mantissa bits hold n; shifting by 23 drops the rest of t's bits
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
 
 // Reduce 32 per-lane values over the warp; lane l receives entry l (31 shuffles).
 template <bool kMax>
@@ -162,11 +147,6 @@ __device__ __forceinline__ float reduce_scatter32(const float* x, int lane) {
   return op(mine, __shfl_xor_sync(full, send, 1));
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 // Writes NC 16-byte chunks (4 packed words each), logical chunks c0 .. c0 + NC - 1 of
 // row `row` of a SW128 tile (128-byte rows): chunk c goes to position c ^ (row % 8).
 template <int NC>
@@ -188,11 +168,46 @@ __device__ __forceinline__ void st_chunks_sw64(uint8_t* tile, int row, int c0, c
   }
 }
 
-// Four floats to four e4m3 bytes (round to nearest even, saturating to +-448).
-__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
-  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-  return lo | (hi << 16);
+// kCols consecutive fp32 columns of this thread's TMEM lane (warp-wide).
+__device__ __forceinline__ void tmem_ldc(uint32_t taddr, float* v) {
+  if constexpr (kCols == 32) tmem_ld32(taddr, v); else tmem_ld16(taddr, v);
+}
+__device__ __forceinline__ void tmem_stc(uint32_t taddr, const float* v) {
+  if constexpr (kCols == 32) tmem_st32(taddr, v); else tmem_st16(taddr, v);
+}
+
+// Reduce kCols per-lane values over the warp into red[0 .. kCols): 32 columns with lane l
+// writing entry l (31 shuffles); 16 columns by four halving steps and a last exchange,
+// lane l then holding entry l / 2 (16 shuffles).
+template <bool kMax>
+__device__ __forceinline__ void reduce_cols(float* red, const float* x, int lane) {
+  if constexpr (kCols == 32) {
+    red[lane] = reduce_scatter32<kMax>(x, lane);
+  } else {
+    const unsigned full = 0xffffffffu;
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+    float b[8], c[4], d[2];
+    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float mine = h16 ? x[8 + e] : x[e], send = h16 ? x[e] : x[8 + e];
+      b[e] = op(mine, __shfl_xor_sync(full, send, 16));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mine = h8 ? b[4 + e] : b[e], send = h8 ? b[e] : b[4 + e];
+      c[e] = op(mine, __shfl_xor_sync(full, send, 8));
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float mine = h4 ? c[2 + e] : c[e], send = h4 ? c[e] : c[2 + e];
+      d[e] = op(mine, __shfl_xor_sync(full, send, 4));
+    }
+    const float mine = h2 ? d[1] : d[0], send = h2 ? d[0] : d[1];
+    float r = op(mine, __shfl_xor_sync(full, send, 2));
+    r = op(r, __shfl_xor_sync(full, r, 1));
+    if (!(lane & 1)) red[lane >> 1] = r;
+  }
 }
 
 template <int RK, bool FP8, bool CAREFUL>
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(ctl->q_full[s]), 1);
-      mbar_init(bar(ctl->q_free[s]), 2);                 // one arrive per softmax group
+      mbar_init(bar(ctl->q_free[s]), kGroups);           // one arrive per softmax group
     }
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(ctl->k_full[s]), 1);
@@ -473,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const int g = (warp - kSoftmaxWarp0) >> 2;
     const int wq = warp & 3;                       // TMEM lane quadrant of this warp
     const int t = 32 * wq + lane;                  // TMEM lane: key of the pair / channel d
-    const int c0 = 32 * g;                         // first query column of the group
+    const int c0 = kCols * g;                      // first query column of the group
     const uint32_t gbar = 1 + g;                   // the group's named barrier
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
     const float sl2 = dm.scale * 1.4426950408889634f;
@@ -493,9 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     const int bh = tile_bh(tau), i = tau - bh * dm.nb, h = bh % dm.H;
     const int b = bh / dm.H;
     const int32_t* L = list_of(tau);
-    float lp[32];
+    float lp[kCols];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) lp[q] = 0.f;
+    for (int q = 0; q < kCols; ++q) lp[q] = 0.f;
 
     // fp8: the scores carry sq_i * sk_j, P carries sv_j / vref and the output vref, where
     // vref = the largest V scale of this row's kept blocks (so P * sv_j / vref <= 256).
@@ -573,23 +588,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     auto key_block = [&](int it) {
       return (t < 64) ? __ldg(L + 2 * it) : ((2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : -1);
     };
-    int jb_next = FP8 ? -1 : key_block(0);
 
     // fp8: the second group starts each tile a little later, so that the two groups'
     // phases (exponentials and e4m3 packing on the special-function unit, the rest on the
     // other pipes) interleave; this measured faster for fp8 only.
-    if (FP8 && g == 1) __nanosleep(kGroupOffsetNs);
+    if (FP8 && (g & 1)) __nanosleep(kGroupOffsetNs);
     bool s_seen = false;                           // the next pair's S was seen complete early
+    // the queries' negated exponent offsets -m: set on a tile's first pair and kept in
+    // registers by the fast pass (the careful pass moves them and reads its TMEM copy)
+    float mn_tile[kCols];
     for (int it = 0; it < npairs; ++it, ++gp) {
+      float mn_pair[kCols];
+      float(&mn)[kCols] = CAREFUL ? mn_pair : mn_tile;
       const int sb = gp % kSBufs;
       const bool ok = !fail && (s_seen || mbar_wait(bar(ctl->s_full[sb]), (gp / kSBufs) & 1, wc));
       fail |= !ok;
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads; invalid keys are masked after.
-      // mn = the queries' negated exponent offsets (the first pair of a tile: none yet).
-      float x[32], mn[32];
-      tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
-      if (it > 0) tmem_ld32(lane_addr + kColM + c0, mn);
+      float x[kCols];
+      tmem_ldc(lane_addr + kColS + 64 * sb + c0, x);
+      if (CAREFUL && it > 0) tmem_ldc(lane_addr + kColM + c0, mn);
       // The P buffer was last read by the P V two pairs back (maybe in the previous tile):
       // its barrier is tested now and waited for only if that P V was not done yet.
       const bool p_free = gp < 2 || mbar_test_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1);
@@ -605,28 +623,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         slt = __shfl_sync(0xffffffffu, lane_slt, it & 31);
         pf = __shfl_sync(0xffffffffu, lane_pf, it & 31);
       } else {
-        jb = jb_next;
-        if (it + 1 < npairs) jb_next = key_block(it + 1);
+        // the fast pass needs the key block only on the last pair (below)
+        jb = (CAREFUL || it + 1 == npairs) ? key_block(it) : 0;
       }
       // x = score * scale * log2(e) - m   (m = the query's exponent offset)
       if (it > 0) {
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) fma2(x[q], x[q + 1], x[q], x[q + 1], slt, slt, mn[q], mn[q + 1]);
+        for (int q = 0; q < kCols; q += 2) fma2(x[q], x[q + 1], x[q], x[q + 1], slt, slt, mn[q], mn[q + 1]);
       } else {
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) mul2(x[q], x[q + 1], slt, slt);
+        for (int q = 0; q < kCols; q += 2) mul2(x[q], x[q + 1], slt, slt);
       }
-      // keys past the end of the sequence and the padding half of an odd list (rare pairs)
-      const bool valid = ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
+      // keys past the end of the sequence and the padding half of an odd list: block lists
+      // are ascending (the top-k writes them so), so only a tile's last pair can hold
+      // either, and the fast pass checks only there (an out-of-range index is recorded by
+      // the producers, ROLA_ERR_DEVICE_BOUNDS)
+      const bool check = FP8 || CAREFUL || it + 1 == npairs;
+      const bool valid = !check ? ok : (ok && jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N);
       bool any_invalid;
       if constexpr (FP8)   // the test is uniform over the warp but for a failed wait
         any_invalid = !ok || jb < 0 || jb >= dm.nb || (ragged_tail && jb == dm.nb - 1);
       else
-        any_invalid = __any_sync(0xffffffffu, !valid);
+        any_invalid = check ? __any_sync(0xffffffffu, !valid) : !ok;
       if (any_invalid) {
         if (!valid) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
+          for (int q = 0; q < kCols; ++q) x[q] = -INFINITY;
         }
       }
       // The first pair of a tile sets the offsets (its exact column maxima).  Careful pass:
@@ -639,16 +661,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       if constexpr (CAREFUL) {
         float dmax = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) dmax = max3f(dmax, x[q], x[q + 1]);
+        for (int q = 0; q < kCols; q += 2) dmax = max3f(dmax, x[q], x[q + 1]);
         slow = named_vote_or(gbar, 128, fail || it == 0 || dmax > 8.f);
       } else {
         slow = it == 0;
       }
       if (slow) {
         if (named_vote_or(gbar, 128, fail)) break;
-        ctl->red[g][wq][lane] = reduce_scatter32<true>(x, lane);
+        reduce_cols<true>(ctl->red[g][wq], x, lane);
         named_sync(gbar, 128);
-        if (wq == 0) {                               // lane = query column c0 + lane
+        if (wq == 0 && lane < kCols) {               // lane = query column c0 + lane
           const float bm = fmaxf(fmaxf(ctl->red[g][0][lane], ctl->red[g][1][lane]),
                                  fmaxf(ctl->red[g][2][lane], ctl->red[g][3][lane]));
           const float delta = it == 0 ? bm : fmaxf(bm, 0.f);
@@ -657,11 +679,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         }
         named_sync(gbar, 128);
         // new negated offsets -(m + delta) (m = 0 on a tile's first pair) into this lane's copy
-        if (it > 0) tmem_ld32(lane_addr + kColM + c0, mn);
+        if (it > 0) tmem_ldc(lane_addr + kColM + c0, mn);
         const float4* d4 = reinterpret_cast<const float4*>(ctl->red[g][0]);
         tmem_wait_ld();
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
+        for (int q4 = 0; q4 < kCols / 4; ++q4) {
           const float4 dd = d4[q4];
           const float d[4] = {dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
@@ -671,12 +693,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
             mn[q] = it > 0 ? mn[q] - d[e] : -d[e];
           }
         }
-        tmem_st32(lane_addr + kColM + c0, mn);
+        tmem_stc(lane_addr + kColM + c0, mn);
         tmem_wait_st();
         if (it > 0) {
           const float4* f4 = reinterpret_cast<const float4*>(ctl->fac + c0);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
+          for (int q4 = 0; q4 < kCols / 4; ++q4) {
             const float4 ff = f4[q4];
             lp[4 * q4 + 0] *= ff.x;
             lp[4 * q4 + 1] *= ff.y;
@@ -685,27 +707,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           }
           fail |= !mbar_wait(bar(ctl->pv_done[(gp - 1) & 1]), ((gp - 1) >> 1) & 1, wc);
           tc_fence_after();
-          float o[32];
-          tmem_ld32(lane_addr + kColO + c0, o);
+          float o[kCols];
+          tmem_ldc(lane_addr + kColO + c0, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
+          for (int q4 = 0; q4 < kCols / 4; ++q4) {
             const float4 ff = f4[q4];
             o[4 * q4 + 0] *= ff.x;
             o[4 * q4 + 1] *= ff.y;
             o[4 * q4 + 2] *= ff.z;
             o[4 * q4 + 3] *= ff.w;
           }
-          tmem_st32(lane_addr + kColO + c0, o);
+          tmem_stc(lane_addr + kColO + c0, o);
           tmem_wait_st();
         }
         named_sync(gbar, 128);                       // red[g][0] is rewritten next time
       }
       // P = 2^x (fp16, or e4m3 times sv_j / vref) and the per-thread partial row sums
-      uint32_t pw[16];
+      uint32_t pw[kCols / 2];
       if constexpr (FP8) {
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
+        for (int q = 0; q < kCols; q += 4) {
           // a quarter of the exponentials on the FMA pipe (see ex2_poly)
           const bool poly = (q & 12) == 12;
           float p0 = poly ? ex2_poly(x[q]) : ex2_approx(x[q]);
@@ -726,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
           if (jb >= 0 && jb < dm.nb) vf = ldexpf(1.f, __ldg(vexp + sbase_idx + jb) - eref);
         }
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) {
+        for (int q = 0; q < kCols; q += 2) {
           float p0 = ex2_approx(x[q]);
           float p1 = ex2_approx(x[q + 1]);
           add2(lp[q], lp[q + 1], p0, p1);
@@ -740,9 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
                mbar_test_wait(bar(ctl->s_full[(gp + 1) % kSBufs]), ((gp + 1) / kSBufs) & 1);
       if (!p_free && !fail) fail |= !mbar_wait(bar(ctl->pv_done[gp & 1]), ((gp - 2) >> 1) & 1, wc);
       if constexpr (FP8)
-        st_chunks_sw64<2>(sP + (gp & 1) * G::kPBytes, t, 2 * g, pw);
+        st_chunks_sw64<kCols / 16>(sP + (gp & 1) * G::kPBytes, t, (kCols / 16) * g, pw);
       else
-        st_chunks_sw128<4>(sP + (gp & 1) * G::kPBytes, t, 4 * g, pw);
+        st_chunks_sw128<kCols / 8>(sP + (gp & 1) * G::kPBytes, t, (kCols / 8) * g, pw);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();                                  // the warp's P rows and O^T rescale are done
@@ -754,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
       // each P of the tile is at most its thread's partial row sum
       bool overflow = false;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) overflow |= !(lp[q] <= kOverflow);   // (NaN counts too)
+      for (int q = 0; q < kCols; ++q) overflow |= !(lp[q] <= kOverflow);   // (NaN counts too)
       const bool listed = named_vote_or(gbar, 128, overflow);
       bool mixed = false;                  // 16-bit path: the kept blocks' v exponents differ
       if constexpr (!FP8) {
@@ -771,9 +793,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
     }
     if (!named_vote_or(gbar, 128, fail)) {
       // per-query sums l over the group's 128 threads (final once the last P is made)
-      ctl->red[g][wq][lane] = reduce_scatter32<false>(lp, lane);
+      reduce_cols<false>(ctl->red[g][wq], lp, lane);
       named_sync(gbar, 128);
-      if (wq == 0)
+      if (wq == 0 && lane < kCols)
         ctl->linv[c0 + lane] = vref / (ctl->red[g][0][lane] + ctl->red[g][1][lane] +
                                        ctl->red[g][2][lane] + ctl->red[g][3][lane]);
       // the tile's last P V (it also proves both groups are done with its S buffers), and
@@ -788,12 +810,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_sm100_kernel(
         const float* gd = reinterpret_cast<const float*>(base + kOffGden);
         uint8_t* stg = base + kOffQ + (j & 1) * 16384;   // the tile's Q slot
         __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(stg + (t >> 6) * 8192) + (t & 63);
-        float o[32], nm[32];
-        tmem_ld32(lane_addr + kColO + c0, o);
-        tmem_ld32(lane_addr + kColNum + c0, nm);
+        float o[kCols], nm[kCols];
+        tmem_ldc(lane_addr + kColO + c0, o);
+        tmem_ldc(lane_addr + kColNum + c0, nm);
         tmem_wait_ld();
 #pragma unroll
-        for (int qq4 = 0; qq4 < 8; ++qq4) {
+        for (int qq4 = 0; qq4 < kCols / 4; ++qq4) {
           const float4 li = reinterpret_cast<const float4*>(ctl->linv + c0)[qq4];
           const float4 gg = reinterpret_cast<const float4*>(gd + c0)[qq4];
           const int q0 = c0 + 4 * qq4, e = 4 * qq4;
@@ -879,8 +901,8 @@ cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, co
     ok = make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws.v16, dm, CU_TENSOR_MAP_SWIZZLE_128B);
-  // output: [32 tokens x 64 channels] boxes, one per query group and channel half
-  ok = ok && make_act_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE, 32);
+  // output: [kCols tokens x 64 channels] boxes, one per query group and channel half
+  ok = ok && make_act_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dm, CU_TENSOR_MAP_SWIZZLE_NONE, kCols);
   if (!ok) return cudaErrorInvalidValue;
   if (fp8)
     return dm.r == 32 ? launch_variant<32, true>(tq, tk, tv, to, dm, ws, debug_flags, debug_limit_us, st)

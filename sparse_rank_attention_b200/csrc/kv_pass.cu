@@ -23,9 +23,10 @@
 // 128-byte swizzle) flow through a 2-stage ring filled by a producer warp; rows past N
 // arrive as zeros.  Per tile:
 //   F = K Wk           one tcgen05 MMA chain, M = 64 tokens, N = r, K = 128 channels
-//                      (A = the k tile, B = Wk_h^T staged once per CTA), fp32 in TMEM;
+//                      (A = the k tile, B = Wk_h^T staged once per CTA), fp32 in TMEM,
+//                      issued a tile ahead into one of two TMEM buffers;
 //   F~ = R(p) phi(F)   warps 0-3, one token and half of the r values per thread, stored
-//                      as bf16 hi + lo into a K-major operand image;
+//                      as bf16 hi + lo into one of two K-major operand images;
 //   S^T += V^T F~      M = 128 channels, N = r, K = 64 tokens (A = the v tile read
 //                      MN-major, B = the hi and lo images), accumulated in TMEM over the
 //                      whole chunk and read out once at its end;
@@ -46,9 +47,9 @@ constexpr int kTok = 64;                     // tokens per tile = one block
 constexpr int kStages = 2;
 constexpr int kThreads = 288;                // warps 0-3 features, 4-5 k means, 6-7 v copy, 8 TMA
 constexpr uint32_t kTileBytes = kTok * kD * 2;   // 16 KB: two boxes of 64 rows x 128 bytes
-constexpr uint32_t kTmemCols = 64;
-constexpr uint32_t kColF = 0;                // F [64 tokens x r] (M = 64 layout)
-constexpr uint32_t kColS = 32;               // S^T [128 channels x r]
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kColF = 0;                // F [64 tokens x r] (M = 64 layout), two buffers
+constexpr uint32_t kColS = 64;               // S^T [128 channels x r]
 
 // Byte offset of 16-byte chunk c (channels 8c .. 8c + 7, c = 0..15) of token row r in a
 // tile: box c / 8 (8 KB each), 128-byte rows, chunk position (c % 8) ^ (r % 8).
@@ -67,12 +68,13 @@ struct KVGeo {
   static constexpr uint32_t offK = 0;                                // kStages k tiles
   static constexpr uint32_t offV = offK + kStages * kTileBytes;      // kStages v tiles
   static constexpr uint32_t offW = offV + kStages * kTileBytes;      // Wk_h^T: 2 boxes [r][64 ch]
-  static constexpr uint32_t offF = offW + 2 * RK * 128;              // F~ hi [r][64 tok], then lo
-  static constexpr uint32_t offCtl = offF + 2 * RK * 128;
+  static constexpr uint32_t kImg = 2 * RK * 128;                     // F~ hi [r][64 tok], then lo
+  static constexpr uint32_t offF = offW + 2 * RK * 128;              // two F~ images
+  static constexpr uint32_t offCtl = offF + 2 * kImg;
 };
 
 struct KVCtl {
-  uint64_t full[kStages], freed[kStages], f_full, img_free, drain;
+  uint64_t full[kStages], freed[kStages], f_full[2], img_free[2], drain;
   uint32_t tmem_base;
   int abort;
   float zred[4][32];
@@ -173,8 +175,10 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       mbar_init(bar(ctl->full[s]), 1);
       mbar_init(bar(ctl->freed[s]), 5);   // the S^T MMAs' commit + warps 4-7
     }
-    mbar_init(bar(ctl->f_full), 1);
-    mbar_init(bar(ctl->img_free), 1);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(bar(ctl->f_full[b2]), 1);
+      mbar_init(bar(ctl->img_free[b2]), 1);
+    }
     mbar_init(bar(ctl->drain), 1);
     ctl->abort = 0;
     fence_barrier_init();
@@ -229,29 +233,42 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
     for (int a = 0; a < HR; ++a) zacc[a] = 0.f;
     bool ok = true;
     int done = 0;
-    for (int t = 0; t < ntiles && ok; ++t) {
-      const int s = t % kStages, n = n_begin + t * kTok + row;
-      if (issuer) {
-        ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t tk = sbase + G::offK + s * kTileBytes;
+    // F of tile t goes to TMEM buffer t & 1 and is issued one tile ahead, so that the
+    // MMA's latency overlaps the features of the tile before; the F~ images alternate too.
+    auto issue_f = [&](int t) {
+      const int s = t % kStages;
+      if (!mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc)) return false;
+      tc_fence_after();
+      const uint32_t tk = sbase + G::offK + s * kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk)
-            mma_f16_ss(tmem + kColF, sdesc_sw128(tk + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                       sdesc_sw128(sbase + G::offW + (kk >> 2) * (RK * 128) + (kk & 3) * 32, 16, 1024), idesc_f,
-                       kk > 0);
-          mma_commit(bar(ctl->f_full));
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_f16_ss(tmem + kColF + 32 * (t & 1), sdesc_sw128(tk + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sbase + G::offW + (kk >> 2) * (RK * 128) + (kk & 3) * 32, 16, 1024), idesc_f,
+                   kk > 0);
+      mma_commit(bar(ctl->f_full[t & 1]));
+      return true;
+    };
+    // (the MMA of tile t + 1 is issued early only if its tile has already landed: waiting
+    // for it here would hold the current tile back)
+    int nf = 0;                                   // F MMAs issued (issuer thread)
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages, n = n_begin + t * kTok + row;
+      if (issuer && ok) {
+        if (nf == t) { ok = issue_f(t); ++nf; }
+        if (ok && nf == t + 1 && t + 1 < ntiles &&
+            mbar_test_wait(bar(ctl->full[(t + 1) % kStages]), ((t + 1) / kStages) & 1)) {
+          ok = issue_f(t + 1);
+          ++nf;
         }
       }
       if (named_vote_or(1, 128, !ok)) { ok = false; break; }
-      ok = mbar_wait(bar(ctl->f_full), t & 1, wc);
+      ok = mbar_wait(bar(ctl->f_full[t & 1]), (t >> 1) & 1, wc);
       if (named_vote_or(1, 128, !ok)) { ok = false; break; }
       tc_fence_after();
       float f[HR];
-      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-      if constexpr (RK == 32) tmem_ld16x2_x16(lane_addr + kColF, f);
-      else tmem_ld16x2_x8(lane_addr + kColF, f);
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16) + kColF + 32 * (t & 1);
+      if constexpr (RK == 32) tmem_ld16x2_x16(lane_addr, f);
+      else tmem_ld16x2_x8(lane_addr, f);
       tmem_wait_ld();
       // phi, z, rotation (pairs a0/2 ..) and the hi / lo split; tokens past the chunk
       // (or N) contribute nothing
@@ -267,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
         const float2 cs = valid ? rope_at(dm, rope, pos, a0 / 2 + p) : make_float2(1.f, 0.f);
         split_bf16x2(cs.x * x0 - cs.y * x1, cs.y * x0 + cs.x * x1, hi[p], lo[p]);
       }
-      // the previous tile's S^T MMAs read the images: wait for them before rewriting
-      if (t > 0) ok = mbar_wait(bar(ctl->img_free), (t - 1) & 1, wc);
+      // the S^T MMAs of tile t - 2 read this image: wait for them before rewriting it
+      if (t >= 2) ok = mbar_wait(bar(ctl->img_free[t & 1]), ((t - 2) >> 1) & 1, wc);
+      uint8_t* ih = smem + G::offF + (t & 1) * G::kImg;
       if (ok) {
 #pragma unroll
         for (int p = 0; p < HR / 2; ++p) {
           const int a = a0 + 2 * p;
-          uint8_t* ih = smem + G::offF;
           *reinterpret_cast<uint16_t*>(ih + img_off(a, row)) = (uint16_t)(hi[p] & 0xffffu);
           *reinterpret_cast<uint16_t*>(ih + img_off(a + 1, row)) = (uint16_t)(hi[p] >> 16);
           *reinterpret_cast<uint16_t*>(ih + RK * 128 + img_off(a, row)) = (uint16_t)(lo[p] & 0xffffu);
@@ -286,16 +303,17 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       if (issuer) {
         tc_fence_after();
         const uint32_t tv = sbase + G::offV + s * kTileBytes;
+        const uint32_t fi = sbase + G::offF + (t & 1) * G::kImg;
         const uint64_t da = sdesc_sw128(tv, 8192, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTok / 16; ++kk) {
-          const uint64_t dh = sdesc_sw128(sbase + G::offF + kk * 32, 16, 1024);
-          const uint64_t dl = sdesc_sw128(sbase + G::offF + RK * 128 + kk * 32, 16, 1024);
+          const uint64_t dh = sdesc_sw128(fi + kk * 32, 16, 1024);
+          const uint64_t dl = sdesc_sw128(fi + RK * 128 + kk * 32, 16, 1024);
           mma_f16_ss(tmem + kColS, da + 128 * kk, dh, idesc_s, t > 0 || kk > 0);
           mma_f16_ss(tmem + kColS, da + 128 * kk, dl, idesc_s, true);
         }
         mma_commit(bar(ctl->freed[s]));
-        mma_commit(bar(ctl->img_free));
+        mma_commit(bar(ctl->img_free[t & 1]));
       }
       done = t + 1;
     }
@@ -385,11 +403,31 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       const int cnt = min(kTok, n_end - n0), blk = n0 / kTok;
       float am = 0.f;
       bool finite = true;
-      for (int e = tv; e < cnt * 16; e += 64) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(e >> 4, e & 15));
-        const float m = absmax8(raw);
-        finite &= m <= 3.402823466e38f;             // false for inf and nan
-        am = fmaxf(am, m);
+      if constexpr (!FP8) {
+        // one pass with the block exponent 0 (the common case): fp16 copy and the block's
+        // largest |v| together; a block that needs another exponent is rewritten below
+        for (int e = tv; e < cnt * 16; e += 64) {
+          const int r = e >> 4, cv = e & 15;
+          const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(r, cv));
+          const float m = absmax8(raw);
+          finite &= m <= 3.402823466e38f;           // false for inf and nan
+          am = fmaxf(am, m);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const __half2 hv = __floats2half2_rn(__uint_as_float(w[u] << 16), __uint_as_float(w[u] & 0xffff0000u));
+            o[u] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+              make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        for (int e = tv; e < cnt * 16; e += 64) {
+          const float m = absmax8(*reinterpret_cast<const uint4*>(pV + swz(e >> 4, e & 15)));
+          finite &= m <= 3.402823466e38f;
+          am = fmaxf(am, m);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
@@ -401,23 +439,21 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
         // the block's exponent: v is carried as v * 2^-e in fp16
         const int ex = v16_exponent(am);
         if (tv == 0) vexp[(size_t)bh * dm.nb + blk] = ex;
-        for (int e = tv; e < cnt * 16; e += 64) {
-          const int r = e >> 4, cv = e & 15;
-          const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(r, cv));
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t o[4];
+        if (ex != 0) {
+          for (int e = tv; e < cnt * 16; e += 64) {
+            const int r = e >> 4, cv = e & 15;
+            const uint4 raw = *reinterpret_cast<const uint4*>(pV + swz(r, cv));
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            uint32_t o[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
-            if (ex != 0) {
-              x0 = ldexpf(x0, -ex);
-              x1 = ldexpf(x1, -ex);
+            for (int u = 0; u < 4; ++u) {
+              const __half2 hv = __floats2half2_rn(ldexpf(__uint_as_float(w[u] << 16), -ex),
+                                                   ldexpf(__uint_as_float(w[u] & 0xffff0000u), -ex));
+              o[u] = *reinterpret_cast<const uint32_t*>(&hv);
             }
-            const __half2 hv = __floats2half2_rn(x0, x1);
-            o[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+                make_uint4(o[0], o[1], o[2], o[3]);
           }
-          *reinterpret_cast<uint4*>(v16 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
-              make_uint4(o[0], o[1], o[2], o[3]);
         }
       } else {
         const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;

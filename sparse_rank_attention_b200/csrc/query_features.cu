@@ -20,10 +20,11 @@
 //
 // Layout of the work (as the key/value pass): a CTA owns one (b, h) and a chunk of whole
 // query blocks; q tiles (two TMA boxes of 64 tokens x 64 channels, 128-byte swizzle) flow
-// through a ring filled by a producer warp, two CTAs per SM.  Per tile one thread issues
+// through a ring filled by a producer warp, two CTAs per SM.  One thread issues, a tile
+// ahead and into one of two TMEM buffers,
 //   U = Q [Wq_h | wg_h hi | wg_h lo]   tcgen05, M = 64 tokens, N = r (+ 8), K = 128
-// into tensor memory (the gate's projection rides along as two extra B rows, gate_proj
-// split into bf16 hi + lo, so q . wg comes out of the same MMA to ~2^-16); warps 0-3 then
+// (the gate's projection rides along as two extra B rows, gate_proj split into bf16 hi +
+// lo, so q . wg comes out of the same MMA to ~2^-16); warps 0-3 then
 // take one token and half of the r values each (phi, den, rotation, the image, g/den),
 // while warps 4-5 take the block mean (and the e4m3 copy).  Every wait is bounded.
 #include "rola_internal.cuh"
@@ -40,7 +41,7 @@ constexpr int kD = 128;
 constexpr int kStages = 3;
 constexpr int kThreads = 288;                 // warps 0-3 features, 4-5 means, 6-7 idle, 8 TMA
 constexpr uint32_t kTileBytes = kBlock * kD * 2;
-constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kTmemCols = 128;           // two U buffers of up to 40 columns, 64 apart
 
 __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)((c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
@@ -65,7 +66,7 @@ struct QGeo {
 };
 
 struct QCtl {
-  uint64_t full[kStages], freed[kStages], u_full, drain;
+  uint64_t full[kStages], freed[kStages], u_full[2], drain;
   uint32_t tmem_base;
   int abort;
   float red[4];
@@ -141,7 +142,8 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
       mbar_init(bar(ctl->full[s]), 1);
       mbar_init(bar(ctl->freed[s]), 3);   // the U MMAs' commit + warps 4-5
     }
-    mbar_init(bar(ctl->u_full), 1);
+    mbar_init(bar(ctl->u_full[0]), 1);
+    mbar_init(bar(ctl->u_full[1]), 1);
     mbar_init(bar(ctl->drain), 1);
     ctl->abort = 0;
     fence_barrier_init();
@@ -199,31 +201,44 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
     for (int a = 0; a < HR; ++a) zr[a] = __ldg(z + (size_t)bh * RK + a0 + a);
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
-      const int s = t % kStages, i = n_begin / kBlock + t, n = i * kBlock + row;
-      if (issuer) {
-        ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t tq = sbase + G::offQ + s * kTileBytes;
+    // U of tile t goes to TMEM buffer t & 1 and is issued one tile ahead, so that the
+    // MMA's latency overlaps the features of the tile before
+    auto issue_u = [&](int t) {
+      const int s = t % kStages;
+      if (!mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc)) return false;
+      tc_fence_after();
+      const uint32_t tq = sbase + G::offQ + s * kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk)
-            mma_f16_ss(tmem, sdesc_sw128(tq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                       sdesc_sw128(sbase + G::offW + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), idesc_u, kk > 0);
-          mma_commit(bar(ctl->u_full));
-          mma_commit(bar(ctl->freed[s]));
+      for (int kk = 0; kk < kD / 16; ++kk)
+        mma_f16_ss(tmem + 64 * (t & 1), sdesc_sw128(tq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sbase + G::offW + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), idesc_u, kk > 0);
+      mma_commit(bar(ctl->u_full[t & 1]));
+      mma_commit(bar(ctl->freed[s]));
+      return true;
+    };
+    // (the MMA of tile t + 1 is issued early only if its tile has already landed)
+    int nu = 0;                                   // U MMAs issued (issuer thread)
+    for (int t = 0; t < ntiles; ++t) {
+      const int i = n_begin / kBlock + t, n = i * kBlock + row;
+      if (issuer && ok) {
+        if (nu == t) { ok = issue_u(t); ++nu; }
+        if (ok && nu == t + 1 && t + 1 < ntiles &&
+            mbar_test_wait(bar(ctl->full[(t + 1) % kStages]), ((t + 1) / kStages) & 1)) {
+          ok = issue_u(t + 1);
+          ++nu;
         }
       }
       if (named_vote_or(1, 128, !ok)) { ok = false; break; }
-      ok = mbar_wait(bar(ctl->u_full), t & 1, wc);
+      ok = mbar_wait(bar(ctl->u_full[t & 1]), (t >> 1) & 1, wc);
       if (named_vote_or(1, 128, !ok)) { ok = false; break; }
       tc_fence_after();
       float u[HR], gl = 0.f;
-      tmem_ld16x2<HR>(lane_addr, u);
-      if constexpr (QG) tmem_ld16x2<1>(lane_addr + RK, &gl);   // q . wg hi (threads 0-15), lo (16-31)
+      const uint32_t ub = lane_addr + 64 * (t & 1);
+      tmem_ld16x2<HR>(ub, u);
+      if constexpr (QG) tmem_ld16x2<1>(ub + RK, &gl);   // q . wg hi (threads 0-15), lo (16-31)
       tmem_wait_ld();
-      tc_fence_before();
-      named_sync(1, 128);                       // U is in registers: the next MMA may overwrite it
+      tc_fence_before();       // U(t)'s buffer is next written by the MMA of tile t + 2, issued
+                               // after this tile's closing barrier
       const bool valid = n < dm.N;
       // gain of the token: read, or sigmoid(q . wg + bg)
       float gh;

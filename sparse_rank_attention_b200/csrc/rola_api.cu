@@ -12,6 +12,8 @@ using rola::Dims;
 using rola::Workspace;
 
 constexpr size_t kAlign = 256;
+
+// The sparse-attention kernel of the head-dim-128 tensor-core path.
 constexpr int kMaxBlocks = 6000;  // one score row per warp must fit shared memory
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -330,8 +332,8 @@ rola_status rola_attend(rola_plan_t plan, const void* q, const void* k, const vo
   else if (p.d == 128) {
     e = rola::launch_query_features(plan->dm, p.dtype == ROLA_FP8_E4M3, q, Wq, g, plan->ws, st);
     if (e == cudaSuccess)
-      e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, p.dtype == ROLA_FP8_E4M3,
-                                    plan->debug_flags, plan->debug_limit_us, st);
+      e = rola::launch_attend_sm100(plan->dm, q, k, plan->ws, out, p.dtype == ROLA_FP8_E4M3, plan->debug_flags,
+                      plan->debug_limit_us, st);
   }
   else  // head dim 64: the transposed tcgen05 tile needs d = 128 rows
     e = rola::launch_attend_bf16_warpmma(plan->dm, q, k, v, Wq, g, out, plan->ws, st);
@@ -476,6 +478,11 @@ rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us) {
   plan->debug_flags = flags;
   plan->debug_limit_us = limit_us;
   return ROLA_OK;
+}
+
+rola_status rola_eval_exp2(const float* x, float* y, int64_t n, int mode, rola_stream_t stream) {
+  if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (!x || !y))) return ROLA_ERR_INVALID_ARG;
+  return rola::launch_eval_exp2(x, y, n, mode, (cudaStream_t)stream) == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 
 const char* rola_status_string(rola_status s) {

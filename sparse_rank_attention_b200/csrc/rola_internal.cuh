@@ -130,6 +130,7 @@ cudaError_t launch_attend_bf16_warpmma(const Dims& dm, const void* q, const void
                                        const Workspace& ws, cudaStream_t st);
 cudaError_t launch_attend_sm100(const Dims& dm, const void* q, const void* k, const Workspace& ws,
                                 void* out, bool fp8, int debug_flags, int debug_limit_us, cudaStream_t st);
+cudaError_t launch_eval_exp2(const float* x, float* y, int64_t n, int mode, cudaStream_t st);
 cudaError_t launch_query_features(const Dims& dm, bool fp8, const void* q, const void* Wq, const float* g,
                                   const Workspace& ws, cudaStream_t st);
 cudaError_t launch_kv_pass(const Dims& dm, bool fp8, const void* k, const void* v, const void* Wk,
