@@ -73,6 +73,7 @@ def _load():
             lib.rola_oracle_e4m3_encode.argtypes = [P, P, ctypes.c_size_t]
             lib.rola_oracle_e4m3_decode.argtypes = [P, P, ctypes.c_size_t]
             lib.rola_oracle_quantize_blocks.argtypes = [sp, P, P, P]
+            lib.rola_oracle_backward.argtypes = [sp] + [P] * 14
             _lib = lib
     return _lib
 
@@ -241,3 +242,24 @@ def forward(s: Shape, q, k, v, Wq, Wk, g):
     col = np.zeros((s.B, s.H, nb, kk), dtype=np.int32)
     _load().rola_oracle_forward(ctypes.byref(s), _p(q), _p(k), _p(v), _p(Wq), _p(Wk), _p(g), _p(out), _p(col))
     return out, col
+
+
+def backward(s: Shape, q, k, v, Wq, Wk, g, dout, col_idx):
+    """Gradients of sum(dout * out) with the kept-block lists col_idx held fixed.
+
+    Returns a dict of float64 arrays: dq, dk, dv [B, N, H, d]; dWq, dWk [H, d, r]; dg
+    with the layout of g ([H], [B, N, H], or gate_proj [H, d] then gate_bias [H]).
+    """
+    q, k, v, Wq, Wk = _f32(q), _f32(k), _f32(v), _f32(Wq), _f32(Wk)
+    g = _gain(s, g)
+    dout = _f64(dout)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    act = (s.B, s.N, s.H, s.d)
+    res = {n: np.zeros(act) for n in ("dq", "dk", "dv")}
+    res["dWq"] = np.zeros((s.H, s.d, s.r))
+    res["dWk"] = np.zeros((s.H, s.d, s.r))
+    res["dg"] = np.zeros(g.size)
+    _load().rola_oracle_backward(ctypes.byref(s), _p(q), _p(k), _p(v), _p(Wq), _p(Wk), _p(g), _p(dout),
+                                 _p(col_idx), _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dWq"]),
+                                 _p(res["dWk"]), _p(res["dg"]))
+    return res

@@ -428,6 +428,218 @@ void rola_oracle_quantize_blocks(const rola_oracle_shape* s, const float* x, uin
       }
 }
 
+// ------------------------------------------------------------------ backward (next row f2)
+//
+// Gradients of L = sum_n dout_n . out_n with respect to q, k, v, Wq, Wk and the gain
+// parameters, the kept-block lists held fixed (the selection is a discrete choice; its
+// gradient is zero almost everywhere).  Derived by the chain rule from steps 4-6 above:
+//   sparse (each query token n, kept keys m):  P_nm = softmax_m(scale q_n . k_m),
+//     O_n = sum_m P_nm v_m;  D_n = dout_n . O_n;  dA_nm = P_nm (dout_n . v_m - D_n);
+//     dv_m += P_nm dout_n;  dq_n += scale sum_m dA_nm k_m;  dk_m += scale sum_n dA_nm q_n;
+//   combination: out_n = O_n + g_n L_n;  dg_n = dout_n . L_n; with gG_n = g_n dout_n
+//   linear, query side (x_n = q_n Wq, u_n = phi(x_n), y_n = R(p_n) u_n, den_n = u_n . z,
+//     L_n = y_n^T S / den_n):  dS += y_n gG_n^T / den_n;  dy_n = S gG_n / den_n;
+//     dden_n = -(gG_n . L_n) / den_n;  du_n = R(p_n)^T dy_n + dden_n z;  dz += dden_n u_n;
+//     dx_n = phi'(x_n) du_n (phi'(x) = 1 for x > 0, e^x otherwise);  dq_n += Wq dx_n;
+//     dWq += q_n dx_n^T;
+//   linear, key side (w_m = k_m Wk, f_m = phi(w_m), S = sum_m R(p_m) f_m v_m^T,
+//     z = sum_m f_m):  dv_m += dS^T R(p_m) f_m;  df_m = R(p_m)^T (dS v_m) + dz;
+//     dw_m = phi'(w_m) df_m;  dk_m += Wk dw_m;  dWk += k_m dw_m^T;
+//   gain from the query (gate_mode 2, g_n = sigmoid(q_n . wg + bg)): dlogit_n =
+//     dg_n g_n (1 - g_n);  dq_n += dlogit_n wg;  dwg += dlogit_n q_n;  dbg += dlogit_n.
+// Inputs as for the forward; dout [B,N,H,d] (double); col_idx the forward's lists.
+// Outputs (double, overwritten): dq, dk, dv [B,N,H,d]; dWq, dWk [H,d,r]; dg with the
+// layout of g ([H], [B,N,H], or gate_proj [H][d] then gate_bias [H]).
+static double phi_grad(double x) { return x > 0.0 ? 1.0 : std::exp(x); }
+
+// y = R(p)^T x: pair (2c, 2c+1) turned clockwise by theta_c.
+static void rotate_back(const rola_oracle_shape* s, const double* p, const double* x, double* y) {
+  for (int c = 0; c < s->r / 2; ++c) {
+    int axis, cp, cnt;
+    pair_axis(s, c, &axis, &cp, &cnt);
+    double theta = p[axis] * std::pow(s->rope_base, -(double)cp / (double)cnt);
+    double cs = std::cos(theta), sn = std::sin(theta);
+    y[2 * c] = cs * x[2 * c] + sn * x[2 * c + 1];
+    y[2 * c + 1] = -sn * x[2 * c] + cs * x[2 * c + 1];
+  }
+}
+
+void rola_oracle_backward(const rola_oracle_shape* s, const float* q, const float* k,
+                          const float* v, const float* Wq, const float* Wk, const double* g,
+                          const double* dout, const int32_t* col_idx, double* dq, double* dk,
+                          double* dv, double* dWq, double* dWk, double* dg) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d, r = s->r;
+  const int nb = rola_oracle_num_blocks(N);
+  const int kk = rola_oracle_keep_count(nb, s->topk);
+  std::vector<double> pos((size_t)N * 3);
+  rola_oracle_positions(s, pos.data());
+  const size_t nact = (size_t)B * N * H * d;
+  std::fill(dq, dq + nact, 0.0);
+  std::fill(dk, dk + nact, 0.0);
+  std::fill(dv, dv + nact, 0.0);
+  std::fill(dWq, dWq + (size_t)H * d * r, 0.0);
+  std::fill(dWk, dWk + (size_t)H * d * r, 0.0);
+  const size_t ng = s->gate_mode == 0 ? (size_t)H : s->gate_mode == 1 ? (size_t)B * N * H : (size_t)H * (d + 1);
+  std::fill(dg, dg + ng, 0.0);
+  auto at = [&](int b, int n, int h) { return (((size_t)b * N + n) * H + h) * d; };
+  // heads are independent, and dWq, dWk and a per-head dg sum over the batch inside one head
+#pragma omp parallel for schedule(dynamic)
+  for (int h = 0; h < H; ++h)
+    for (int b = 0; b < B; ++b) {
+      // key-side features and the state (as the forward computes them, in double)
+      std::vector<double> w((size_t)N * r), f((size_t)N * r), yk((size_t)N * r);
+      std::vector<double> S((size_t)r * d, 0.0), z(r, 0.0);
+      for (int m = 0; m < N; ++m) {
+        const float* km = k + at(b, m, h);
+        const float* vm = v + at(b, m, h);
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += (double)km[c] * (double)Wk[((size_t)h * d + c) * r + a];
+          w[(size_t)m * r + a] = acc;
+          f[(size_t)m * r + a] = phi(acc);
+        }
+        rotate(s, &pos[3 * (size_t)m], &f[(size_t)m * r], &yk[(size_t)m * r]);
+        for (int a = 0; a < r; ++a) {
+          z[a] += f[(size_t)m * r + a];
+          for (int c = 0; c < d; ++c) S[(size_t)a * d + c] += yk[(size_t)m * r + a] * (double)vm[c];
+        }
+      }
+      std::vector<double> dS((size_t)r * d, 0.0), dz(r, 0.0);
+      std::vector<double> x(r), u(r), yq(r), L(d), O(d), gG(d), dy(r), du(r), dx(r);
+      std::vector<int> keys;
+      std::vector<double> P;
+      for (int i = 0; i < nb; ++i) {
+        const int32_t* Li = col_idx + (((size_t)b * H + h) * nb + i) * kk;
+        keys.clear();
+        for (int a = 0; a < kk; ++a)
+          for (int m = Li[a] * kBlock; m < std::min(N, (Li[a] + 1) * kBlock); ++m) keys.push_back(m);
+        P.resize(keys.size());
+        for (int n = i * kBlock; n < std::min(N, (i + 1) * kBlock); ++n) {
+          const float* qn = q + at(b, n, h);
+          const double* G = dout + at(b, n, h);
+          // sparse branch: P and O
+          double mx = -std::numeric_limits<double>::infinity();
+          for (size_t a = 0; a < keys.size(); ++a) {
+            const float* km = k + at(b, keys[a], h);
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += (double)qn[c] * (double)km[c];
+            P[a] = acc * s->scale;
+            mx = std::max(mx, P[a]);
+          }
+          double sum = 0.0;
+          for (size_t a = 0; a < keys.size(); ++a) {
+            P[a] = std::exp(P[a] - mx);
+            sum += P[a];
+          }
+          for (int c = 0; c < d; ++c) O[c] = 0.0;
+          for (size_t a = 0; a < keys.size(); ++a) {
+            P[a] /= sum;
+            const float* vm = v + at(b, keys[a], h);
+            for (int c = 0; c < d; ++c) O[c] += P[a] * (double)vm[c];
+          }
+          double Dn = 0.0;
+          for (int c = 0; c < d; ++c) Dn += G[c] * O[c];
+          for (size_t a = 0; a < keys.size(); ++a) {
+            const int m = keys[a];
+            const float* km = k + at(b, m, h);
+            const float* vm = v + at(b, m, h);
+            double dP = 0.0;
+            for (int c = 0; c < d; ++c) dP += G[c] * (double)vm[c];
+            const double dA = P[a] * (dP - Dn);
+            for (int c = 0; c < d; ++c) {
+              dv[at(b, m, h) + c] += P[a] * G[c];
+              dq[at(b, n, h) + c] += s->scale * dA * (double)km[c];
+              dk[at(b, m, h) + c] += s->scale * dA * (double)qn[c];
+            }
+          }
+          // linear branch, query side
+          for (int a = 0; a < r; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += (double)qn[c] * (double)Wq[((size_t)h * d + c) * r + a];
+            x[a] = acc;
+            u[a] = phi(acc);
+          }
+          rotate(s, &pos[3 * (size_t)n], u.data(), yq.data());
+          double den = 0.0;
+          for (int a = 0; a < r; ++a) den += u[a] * z[a];
+          for (int c = 0; c < d; ++c) {
+            double num = 0.0;
+            for (int a = 0; a < r; ++a) num += yq[a] * S[(size_t)a * d + c];
+            L[c] = num / den;
+          }
+          const double gn = gain(s, g, qn, b, n, h);
+          double dgn = 0.0;
+          for (int c = 0; c < d; ++c) dgn += G[c] * L[c];
+          if (s->gate_mode == 0) {
+            dg[h] += dgn;
+          } else if (s->gate_mode == 1) {
+            dg[((size_t)b * N + n) * H + h] = dgn;
+          } else {
+            const double dlogit = dgn * gn * (1.0 - gn);
+            const double* wg = g + (size_t)h * d;
+            for (int c = 0; c < d; ++c) {
+              dq[at(b, n, h) + c] += dlogit * wg[c];
+              dg[(size_t)h * d + c] += dlogit * (double)qn[c];
+            }
+            dg[(size_t)H * d + h] += dlogit;
+          }
+          for (int c = 0; c < d; ++c) gG[c] = gn * G[c];
+          double gGL = 0.0;
+          for (int c = 0; c < d; ++c) gGL += gG[c] * L[c];
+          const double dden = -gGL / den;
+          for (int a = 0; a < r; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) {
+              dS[(size_t)a * d + c] += yq[a] * gG[c] / den;
+              acc += S[(size_t)a * d + c] * gG[c];
+            }
+            dy[a] = acc / den;
+          }
+          rotate_back(s, &pos[3 * (size_t)n], dy.data(), du.data());
+          for (int a = 0; a < r; ++a) {
+            du[a] += dden * z[a];
+            dz[a] += dden * u[a];
+            dx[a] = phi_grad(x[a]) * du[a];
+          }
+          for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < r; ++a) {
+              acc += (double)Wq[((size_t)h * d + c) * r + a] * dx[a];
+              dWq[((size_t)h * d + c) * r + a] += (double)qn[c] * dx[a];
+            }
+            dq[at(b, n, h) + c] += acc;
+          }
+        }
+      }
+      // linear branch, key side
+      std::vector<double> dyk(r), df(r);
+      for (int m = 0; m < N; ++m) {
+        const float* km = k + at(b, m, h);
+        const float* vm = v + at(b, m, h);
+        for (int c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int a = 0; a < r; ++a) acc += dS[(size_t)a * d + c] * yk[(size_t)m * r + a];
+          dv[at(b, m, h) + c] += acc;
+        }
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += dS[(size_t)a * d + c] * (double)vm[c];
+          dyk[a] = acc;
+        }
+        rotate_back(s, &pos[3 * (size_t)m], dyk.data(), df.data());
+        for (int a = 0; a < r; ++a) df[a] = phi_grad(w[(size_t)m * r + a]) * (df[a] + dz[a]);
+        for (int c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int a = 0; a < r; ++a) {
+            acc += (double)Wk[((size_t)h * d + c) * r + a] * df[a];
+            dWk[((size_t)h * d + c) * r + a] += (double)km[c] * df[a];
+          }
+          dk[at(b, m, h) + c] += acc;
+        }
+      }
+    }
+}
+
 int rola_oracle_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -53,10 +53,10 @@ namespace {
 
 using namespace sm100;
 
-#ifndef ROLA_ATTEND_GROUPS
-#define ROLA_ATTEND_GROUPS 2
-#endif
-constexpr int kGroups = ROLA_ATTEND_GROUPS;   // softmax groups of four warps
+// Softmax groups of four warps.  Four groups of 16 columns (640 threads, 96 registers)
+// measured no faster than two of 32: a warp's per-pair chain, not the issue rate, sets
+// the softmax side's pace.
+constexpr int kGroups = 2;
 constexpr int kCols = 64 / kGroups;            // query columns of a group
 constexpr int kThreads = 128 + 128 * kGroups;
 constexpr int kSoftmaxWarp0 = 4;  // group g = warps 4 + 4g .. 7 + 4g: query columns [kCols g, kCols (g + 1))

@@ -25,12 +25,13 @@
 //   F = K Wk           one tcgen05 MMA chain, M = 64 tokens, N = r, K = 128 channels
 //                      (A = the k tile, B = Wk_h^T staged once per CTA), fp32 in TMEM,
 //                      issued a tile ahead into one of two TMEM buffers;
-//   F~ = R(p) phi(F)   warps 0-3, one token and half of the r values per thread, stored
-//                      as bf16 hi + lo into one of two K-major operand images;
+//   F~ = R(p) phi(F)   warps 0-7 (two per TMEM lane quadrant), one token and a quarter
+//                      of the r values per thread, stored as bf16 hi + lo into one of
+//                      two K-major operand images;
 //   S^T += V^T F~      M = 128 channels, N = r, K = 64 tokens (A = the v tile read
 //                      MN-major, B = the hi and lo images), accumulated in TMEM over the
 //                      whole chunk and read out once at its end;
-// while warps 4-5 pool k (and write its e4m3 copy) and warps 6-7 write the copy of v.
+// while warps 8-9 pool k (and write its e4m3 copy) and warps 10-11 write the copy of v.
 // Every wait is bounded (ROLA_ERR_DEVICE_TIMEOUT).
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -45,7 +46,7 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kTok = 64;                     // tokens per tile = one block
 constexpr int kStages = 2;
-constexpr int kThreads = 288;                // warps 0-3 features, 4-5 k means, 6-7 v copy, 8 TMA
+constexpr int kThreads = 416;                // warps 0-7 features, 8-9 k means, 10-11 v copy, 12 TMA
 constexpr uint32_t kTileBytes = kTok * kD * 2;   // 16 KB: two boxes of 64 rows x 128 bytes
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kColF = 0;                // F [64 tokens x r] (M = 64 layout), two buffers
@@ -114,18 +115,14 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// 16 consecutive fp32 columns of TMEM lanes 0-15 of this warp's quadrant for threads
-// 0-15 and the next 16 columns of the same lanes for threads 16-31 (the M = 64 layout).
-__device__ __forceinline__ void tmem_ld16x2_x16(uint32_t taddr, float* v) {
+// TMEM lanes 0-15 of this warp's quadrant (the M = 64 layout): threads 0-15 read n
+// consecutive fp32 columns, threads 16-31 the n columns after them.
+__device__ __forceinline__ void tmem_ld16x2_x4(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16], 16;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0, %1, %2, %3}, [%4], 4;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
 }
 __device__ __forceinline__ void tmem_ld16x2_x8(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -173,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(ctl->full[s]), 1);
-      mbar_init(bar(ctl->freed[s]), 5);   // the S^T MMAs' commit + warps 4-7
+      mbar_init(bar(ctl->freed[s]), 5);   // the S^T MMAs' commit + warps 8-11
     }
     for (int b2 = 0; b2 < 2; ++b2) {
       mbar_init(bar(ctl->f_full[b2]), 1);
@@ -199,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtl wc{&ctl->abort, status, 2000000000ull};
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
@@ -220,14 +217,15 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
         mbar_wait(bar(ctl->full[t % kStages]), (t / kStages) & 1, wc, false);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ features and the MMAs
     const bool issuer = warp == 0 && lane == 0;
     constexpr uint32_t idesc_f = idesc_f16(1, 64, RK, 0, 0);    // F = K Wk
     constexpr uint32_t idesc_s = idesc_f16(1, 128, RK, 1, 0);   // S^T += V^T F~
-    constexpr int HR = RK / 2;                  // rank values per thread
-    const int row = 16 * warp + (lane & 15);    // token of the tile
-    const int a0 = (lane >> 4) * HR;            // first rank value of this thread
+    constexpr int HR = RK / 4;                  // rank values per thread
+    const int qd = warp & 3, hf = warp >> 2;    // TMEM lane quadrant; half of the ranks
+    const int row = 16 * qd + (lane & 15);      // token of the tile
+    const int a0 = hf * (RK / 2) + (lane >> 4) * HR;   // first rank value of this thread
     float zacc[HR];
 #pragma unroll
     for (int a = 0; a < HR; ++a) zacc[a] = 0.f;
@@ -261,14 +259,15 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
           ++nf;
         }
       }
-      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
-      ok = mbar_wait(bar(ctl->f_full[t & 1]), (t >> 1) & 1, wc);
-      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      // one barrier per tile (before the S^T MMAs): a failed wait is carried to it, and
+      // tcgen05.ld runs on the whole converged warp whatever its lanes' waits returned
+      if (ok) ok = mbar_wait(bar(ctl->f_full[t & 1]), (t >> 1) & 1, wc);
+      __syncwarp();
       tc_fence_after();
       float f[HR];
-      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16) + kColF + 32 * (t & 1);
-      if constexpr (RK == 32) tmem_ld16x2_x16(lane_addr, f);
-      else tmem_ld16x2_x8(lane_addr, f);
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * qd) << 16) + kColF + 32 * (t & 1) + hf * (RK / 2);
+      if constexpr (RK == 32) tmem_ld16x2_x8(lane_addr, f);
+      else tmem_ld16x2_x4(lane_addr, f);
       tmem_wait_ld();
       // phi, z, rotation (pairs a0/2 ..) and the hi / lo split; tokens past the chunk
       // (or N) contribute nothing
@@ -285,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
         split_bf16x2(cs.x * x0 - cs.y * x1, cs.y * x0 + cs.x * x1, hi[p], lo[p]);
       }
       // the S^T MMAs of tile t - 2 read this image: wait for them before rewriting it
-      if (t >= 2) ok = mbar_wait(bar(ctl->img_free[t & 1]), ((t - 2) >> 1) & 1, wc);
+      if (ok && t >= 2) ok = mbar_wait(bar(ctl->img_free[t & 1]), ((t - 2) >> 1) & 1, wc);
       uint8_t* ih = smem + G::offF + (t & 1) * G::kImg;
       if (ok) {
 #pragma unroll
@@ -299,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      if (named_vote_or(1, 256, !ok)) { ok = false; break; }
       if (issuer) {
         tc_fence_after();
         const uint32_t tv = sbase + G::offV + s * kTileBytes;
@@ -322,20 +321,22 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       mma_commit(bar(ctl->drain));             // every MMA of this CTA has completed
       mbar_wait(bar(ctl->drain), 0, wc, false);
     }
-    named_sync(1, 128);
+    named_sync(1, 256);
     tc_fence_after();
     float* Sp = S_part + ((size_t)bh * dm.nchunk + chunk) * RK * kD;
-    if (ok && done == ntiles && ntiles > 0) {
-      float sv_[RK];
-      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-      tmem_ld32x32_x16(lane_addr + kColS, sv_);
-      if constexpr (RK == 32) tmem_ld32x32_x16(lane_addr + kColS + 16, sv_ + 16);
-      tmem_wait_ld();
+    if (hf == 0) {                               // S^T spans the 128 lanes: warps 0-3 read it
+      if (ok && done == ntiles && ntiles > 0) {
+        float sv_[RK];
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * qd) << 16);
+        tmem_ld32x32_x16(lane_addr + kColS, sv_);
+        if constexpr (RK == 32) tmem_ld32x32_x16(lane_addr + kColS + 16, sv_ + 16);
+        tmem_wait_ld();
 #pragma unroll
-      for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * warp + lane] = sv_[a];
-    } else {
+        for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * qd + lane] = sv_[a];
+      } else {
 #pragma unroll
-      for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * warp + lane] = 0.f;
+        for (int a = 0; a < RK; ++a) Sp[(size_t)a * kD + 32 * qd + lane] = 0.f;
+      }
     }
     // z: the 16 token lanes of each half-warp hold the same rank values
 #pragma unroll
@@ -345,16 +346,16 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       x += __shfl_xor_sync(0xffffffffu, x, 2);
       x += __shfl_xor_sync(0xffffffffu, x, 4);
       x += __shfl_xor_sync(0xffffffffu, x, 8);
-      if ((lane & 15) == 0) ctl->zred[warp][a0 + a] = x;
+      if ((lane & 15) == 0) ctl->zred[qd][a0 + a] = x;
     }
-    named_sync(1, 128);
+    named_sync(1, 256);
     if (tid < RK)
       z_part[((size_t)bh * dm.nchunk + chunk) * RK + tid] =
           ((ctl->zred[0][tid] + ctl->zred[1][tid]) + ctl->zred[2][tid]) + ctl->zred[3][tid];
     tc_fence_before();
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ k means (+ e4m3 k)
-    const int cp = tid - 128;                     // channel pair 0..63
+    const int cp = tid - 256;                     // channel pair 0..63
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % kStages, n0 = n_begin + t * kTok;
       const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
         // e4m3 copy of the k tile: block scale from the max over the two warps
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        if (lane == 0) ctl->red[warp - 4] = am;
+        if (lane == 0) ctl->red[warp - 8] = am;
         named_sync(2, 64);
         am = fmaxf(ctl->red[0], ctl->red[1]);
         const float sc = am > 0.f ? am / 448.f : 1.f, inv = 1.f / sc;
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
     }
   } else {
     // ------------------------------------------------------------ copy of v
-    const int tv = tid - 192;                     // 0..63
+    const int tv = tid - 320;                     // 0..63
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % kStages, n0 = n_begin + t * kTok;
       const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_pass_kernel(
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      if (lane == 0) ctl->red[4 + warp - 6] = am;
+      if (lane == 0) ctl->red[4 + warp - 10] = am;
       finite = !named_vote_or(3, 64, !finite);     // also orders the red writes
       am = fmaxf(ctl->red[4], ctl->red[5]);
       if (!finite && tv == 0) record_status(status, kDevRange);

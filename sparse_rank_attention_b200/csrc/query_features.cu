@@ -24,9 +24,11 @@
 // ahead and into one of two TMEM buffers,
 //   U = Q [Wq_h | wg_h hi | wg_h lo]   tcgen05, M = 64 tokens, N = r (+ 8), K = 128
 // (the gate's projection rides along as two extra B rows, gate_proj split into bf16 hi +
-// lo, so q . wg comes out of the same MMA to ~2^-16); warps 0-3 then
-// take one token and half of the r values each (phi, den, rotation, the image, g/den),
-// while warps 4-5 take the block mean (and the e4m3 copy).  Every wait is bounded.
+// lo, so q . wg comes out of the same MMA to ~2^-16); warps 0-7 then take one token
+// and a quarter of the r values each (phi, den, rotation, the image, g/den: two warps
+// per TMEM lane quadrant, so that twice as many warps hide the latencies of the per-token
+// work), while warps 8-9 take the block mean and, fp8, warps 10-11 the block's absmax
+// and the e4m3 copy.  Every wait is bounded.
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -39,7 +41,12 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kStages = 3;
-constexpr int kThreads = 288;                 // warps 0-3 features, 4-5 means, 6-7 idle, 8 TMA
+// warps 0-7 features, 8-9 means, (fp8: 10-11 the e4m3 copy), then the TMA producer
+template <bool FP8>
+struct QRoles {
+  static constexpr int kTmaWarp = FP8 ? 12 : 10;
+  static constexpr int kThreads = 32 * (kTmaWarp + 1);
+};
 constexpr uint32_t kTileBytes = kBlock * kD * 2;
 constexpr uint32_t kTmemCols = 128;           // two U buffers of up to 40 columns, 64 apart
 
@@ -70,6 +77,7 @@ struct QCtl {
   uint32_t tmem_base;
   int abort;
   float red[4];
+  float dpart[4][16];     // per quadrant and row: den over the upper half of the ranks
 };
 
 template <int RK, bool QG>
@@ -109,13 +117,21 @@ __device__ __forceinline__ void tmem_ld16x2<8>(uint32_t taddr, float* v) {
                : "memory");
 }
 template <>
+__device__ __forceinline__ void tmem_ld16x2<4>(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0, %1, %2, %3}, [%4], 4;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+}
+template <>
 __device__ __forceinline__ void tmem_ld16x2<1>(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
   asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x1.b32 {%0}, [%1], 1;" : "=r"(r[0]) : "r"(taddr) : "memory");
 }
 
 template <int RK, bool FP8, bool QG>
-__global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
+__global__ void __launch_bounds__(QRoles<FP8>::kThreads, 2) query_features_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ Wq, const float* __restrict__ g,
     Dims dm, const float* __restrict__ z, const float2* __restrict__ rope, float* __restrict__ qbar,
     uint8_t* __restrict__ uimg, float* __restrict__ gden, uint8_t* __restrict__ q8, float* __restrict__ sq,
@@ -140,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(ctl->full[s]), 1);
-      mbar_init(bar(ctl->freed[s]), 3);   // the U MMAs' commit + warps 4-5
+      mbar_init(bar(ctl->freed[s]), FP8 ? 5 : 3);   // the U MMAs' commit + warps 8-9 (10-11)
     }
     mbar_init(bar(ctl->u_full[0]), 1);
     mbar_init(bar(ctl->u_full[1]), 1);
@@ -149,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
     fence_barrier_init();
   }
   // B = [Wq_h^T; wg hi; wg lo; 0]: row a, channel c in box c / 64 (K-major, 128-byte swizzle)
-  for (int e = tid; e < kD * NB; e += kThreads) {
+  for (int e = tid; e < kD * NB; e += QRoles<FP8>::kThreads) {
     const int c = e / NB, a = e % NB;
     __nv_bfloat16 val;
     if (a < RK) {
@@ -171,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtl wc{&ctl->abort, status, 2000000000ull};
 
-  if (warp == 8) {
+  if (warp == QRoles<FP8>::kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -189,17 +205,18 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
       for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
         mbar_wait(bar(ctl->full[t % kStages]), (t / kStages) & 1, wc, false);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ U and the features
     const bool issuer = warp == 0 && lane == 0;
     constexpr uint32_t idesc_u = idesc_f16(1, 64, NB, 0, 0);
-    constexpr int HR = RK / 2;
-    const int row = 16 * warp + (lane & 15);    // token of the tile
-    const int a0 = (lane >> 4) * HR;            // first rank value of this thread
+    constexpr int HR = RK / 4;                  // rank values of a thread
+    const int qd = warp & 3, hf = warp >> 2;    // TMEM lane quadrant; half of the ranks
+    const int row = 16 * qd + (lane & 15);      // token of the tile
+    const int a0 = hf * (RK / 2) + (lane >> 4) * HR;   // first rank value of this thread
     float zr[HR];
 #pragma unroll
     for (int a = 0; a < HR; ++a) zr[a] = __ldg(z + (size_t)bh * RK + a0 + a);
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * qd) << 16);
     bool ok = true;
     // U of tile t goes to TMEM buffer t & 1 and is issued one tile ahead, so that the
     // MMA's latency overlaps the features of the tile before
@@ -228,26 +245,21 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
           ++nu;
         }
       }
-      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
-      ok = mbar_wait(bar(ctl->u_full[t & 1]), (t >> 1) & 1, wc);
-      if (named_vote_or(1, 128, !ok)) { ok = false; break; }
+      // one barrier per tile (after the image): a failed wait is carried to it, and
+      // tcgen05.ld runs on the whole converged warp whatever its lanes' waits returned
+      if (ok) ok = mbar_wait(bar(ctl->u_full[t & 1]), (t >> 1) & 1, wc);
+      __syncwarp();
       tc_fence_after();
       float u[HR], gl = 0.f;
       const uint32_t ub = lane_addr + 64 * (t & 1);
-      tmem_ld16x2<HR>(ub, u);
-      if constexpr (QG) tmem_ld16x2<1>(ub + RK, &gl);   // q . wg hi (threads 0-15), lo (16-31)
+      tmem_ld16x2<HR>(ub + hf * (RK / 2), u);
+      // q . wg hi (threads 0-15), lo (16-31): read by the warps that write g/den
+      if (QG && hf == 0) tmem_ld16x2<1>(ub + RK, &gl);
       tmem_wait_ld();
       tc_fence_before();       // U(t)'s buffer is next written by the MMA of tile t + 2, issued
                                // after this tile's closing barrier
       const bool valid = n < dm.N;
-      // gain of the token: read, or sigmoid(q . wg + bg)
-      float gh;
-      if constexpr (QG) {
-        gl += __shfl_xor_sync(0xffffffffu, gl, 16);
-        gh = gate_sigmoid(dm, g, h, gl);
-      } else {
-        gh = valid ? g[gain_index(dm, b, n, h)] : 0.f;
-      }
+      if constexpr (QG) gl += __shfl_xor_sync(0xffffffffu, gl, 16);
       const TokPos pos = token_pos(dm, valid ? n : 0);
       uint8_t* img = smem + G::offImg + (t & 1) * G::kImg;
       float den = 0.f;
@@ -265,61 +277,86 @@ __global__ void __launch_bounds__(kThreads, 2) query_features_kernel(
         *reinterpret_cast<uint16_t*>(img + RK * 128 + img_off(a + 1, row)) = (uint16_t)(lo >> 16);
       }
       den += __shfl_xor_sync(0xffffffffu, den, 16);
-      if (lane < 16) gden[((size_t)bh * dm.nb + i) * kBlock + row] = valid ? gh / den : 0.f;
-      named_sync(1, 128);                       // the image is complete
+      if (hf == 1 && lane < 16) ctl->dpart[qd][lane] = den;
+      // the image and the partial dens are complete (and U(t) is read: its buffer may be
+      // refilled)
+      if (named_vote_or(1, 256, !ok)) { ok = false; break; }
+      if (hf == 0 && lane < 16) {
+        // gain of the token: read, or sigmoid(q . wg + bg)
+        const float gh = QG ? gate_sigmoid(dm, g, h, gl) : (valid ? g[gain_index(dm, b, n, h)] : 0.f);
+        den += ctl->dpart[qd][lane];
+        gden[((size_t)bh * dm.nb + i) * kBlock + row] = valid ? gh / den : 0.f;
+      }
       uint4* dst = reinterpret_cast<uint4*>(uimg + ((size_t)bh * dm.nb + i) * G::kImg);
       const uint4* src = reinterpret_cast<const uint4*>(img);
-      for (int e = tid; e < (int)(G::kImg / 16); e += 128) dst[e] = src[e];
+      for (int e = tid; e < (int)(G::kImg / 16); e += 256) dst[e] = src[e];
     }
     if (issuer) {
       mma_commit(bar(ctl->drain));             // no MMA may run when TMEM is freed
       mbar_wait(bar(ctl->drain), 0, wc, false);
     }
     tc_fence_before();
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ block mean (+ e4m3 q)
-    const int cp = tid - 128;                     // channel pair 0..63
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ block mean
+    const int cp = tid - 256;                     // channel pair 0..63
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % kStages, n0 = n_begin + t * kBlock, i = n0 / kBlock;
       const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
       if (named_vote_or(2, 64, !ok)) break;
       const uint8_t* pQ = smem + G::offQ + s * kTileBytes;
       const int cnt = min(kBlock, dm.N - n0);
-      float a0 = 0.f, a1 = 0.f, am = 0.f;
+      float a0 = 0.f, a1 = 0.f;
       const uint8_t* col = pQ + (cp >> 5) * 8192 + (cp & 3) * 4;   // box, word in chunk
       const int ch = (cp >> 2) & 7;                                 // chunk within the box
       for (int r = 0; r < cnt; ++r) {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(col + r * 128 + ((ch ^ (r & 7)) << 4));
-        const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
-        a0 = a0 + x0;
-        a1 = a1 + x1;
-        if (FP8) am = fmaxf(am, fmaxf(fabsf(x0), fabsf(x1)));
+        a0 = a0 + __uint_as_float(w << 16);
+        a1 = a1 + __uint_as_float(w & 0xffff0000u);
       }
       *reinterpret_cast<float2*>(qbar + ((size_t)bh * dm.nb + i) * kD + 2 * cp) =
           make_float2(__fdiv_rn(a0, (float)cnt), __fdiv_rn(a1, (float)cnt));
-      if constexpr (FP8) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ctl->freed[s]));
+    }
+  } else if (FP8) {
+    // ------------------------------------------------------------ e4m3 copy of q
+    // (its own warps, beside the means: the block's absmax, then every code)
+    const int tq = tid - 320;                     // 0..63
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages, n0 = n_begin + t * kBlock, i = n0 / kBlock;
+      const bool ok = mbar_wait(bar(ctl->full[s]), (t / kStages) & 1, wc);
+      if (named_vote_or(3, 64, !ok)) break;
+      const uint8_t* pQ = smem + G::offQ + s * kTileBytes;
+      const int cnt = min(kBlock, dm.N - n0);
+      float am = 0.f;
+      for (int e = tq; e < cnt * 16; e += 64) {
+        const uint4 v = *reinterpret_cast<const uint4*>(pQ + swz(e >> 4, e & 15));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        if (lane == 0) ctl->red[warp - 4] = am;
-        named_sync(2, 64);
-        am = fmaxf(ctl->red[0], ctl->red[1]);
-        const float scale = am > 0.f ? am / 448.f : 1.f, inv = 1.f / scale;
-        if (cp == 0) sq[(size_t)bh * dm.nb + i] = scale;
-        for (int e = cp; e < cnt * 16; e += 64) {
-          const int r = e >> 4, cv = e & 15;
-          const uint4 v = *reinterpret_cast<const uint4*>(pQ + swz(r, cv));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[2] = {0, 0};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 f = make_float2(__uint_as_float(w[u] << 16) * inv, __uint_as_float(w[u] & 0xffff0000u) * inv);
-            o[u >> 1] |= (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3) << (16 * (u & 1));
-          }
-          *reinterpret_cast<uint2*>(q8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
-              make_uint2(o[0], o[1]);
-        }
-        named_sync(2, 64);                         // red is rewritten next tile
+        for (int u = 0; u < 4; ++u)
+          am = fmaxf(am, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xffff0000u))));
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) ctl->red[warp - 10] = am;
+      named_sync(3, 64);
+      am = fmaxf(ctl->red[0], ctl->red[1]);
+      const float scale = am > 0.f ? am / 448.f : 1.f, inv = 1.f / scale;
+      if (tq == 0) sq[(size_t)bh * dm.nb + i] = scale;
+      for (int e = tq; e < cnt * 16; e += 64) {
+        const int r = e >> 4, cv = e & 15;
+        const uint4 v = *reinterpret_cast<const uint4*>(pQ + swz(r, cv));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[2] = {0, 0};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = make_float2(__uint_as_float(w[u] << 16) * inv, __uint_as_float(w[u] & 0xffff0000u) * inv);
+          o[u >> 1] |= (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3) << (16 * (u & 1));
+        }
+        *reinterpret_cast<uint2*>(q8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
+            make_uint2(o[0], o[1]);
+      }
+      named_sync(3, 64);                           // red is rewritten next tile
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(ctl->freed[s]));
     }
@@ -343,7 +380,7 @@ cudaError_t launch_variant(const Dims& dm, const void* q, const void* Wq, const 
   if (!make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   dim3 grid(dm.nchunk, dm.B * dm.H);
-  query_features_kernel<RK, FP8, QG><<<grid, kThreads, smem, st>>>(
+  query_features_kernel<RK, FP8, QG><<<grid, QRoles<FP8>::kThreads, smem, st>>>(
       tq, static_cast<const __nv_bfloat16*>(Wq), g, dm, ws.z, ws.rope, ws.qbar, ws.uimg, ws.gden,
       FP8 ? ws.q8 : nullptr, FP8 ? ws.sq : nullptr, ws.status);
   return cudaGetLastError();
