@@ -230,6 +230,30 @@ ROLA_API rola_status rola_profile_stages(rola_plan_t plan, int enable);
 ROLA_API rola_status rola_get_stage_times(rola_plan_t plan, float* ms, int max_stages, int* nstages,
                                           int* ncalls);
 
+/* Backward of rola_forward (gradients for training; the pages' sparse-finetuning section
+ * trains proj_q, proj_k, gate_proj and gate_bias with the attention).  Computes the
+ * gradients of L = sum(dout * out) with the kept-block lists held fixed (the selection is
+ * a discrete choice, so its gradient is zero almost everywhere):
+ *   dq, dk, dv  [B, N, H, d] fp32      dWq, dWk  [H, d, r] fp32
+ *   dg          the layout of g: [H] (ROLA_GATE_HEAD), [B, N, H] (ROLA_GATE_TOKEN), or
+ *               d gate_proj [H, d] then d gate_bias [H] (ROLA_GATE_QPROJ), fp32.
+ * q, k, v, Wq, Wk, g are the forward's inputs and dout [B, N, H, d] has the input dtype.
+ * The call recomputes what it needs (block selection, the linear state, the softmax row
+ * statistics) on the plan's workspace, so it needs no saved forward state; it overwrites
+ * the plan's workspace as rola_forward does.  Configurations: ROLA_F32 and ROLA_BF16 (fp8
+ * is a forward-only configuration: ROLA_ERR_UNSUPPORTED), every d, r and gate of the
+ * forward.  Arithmetic: fp32 on the inputs' values.  Scratch: bwd_workspace, at least
+ * rola_backward_workspace_size bytes, 16-byte aligned, caller-owned.  Every pointer is a
+ * device pointer, 16-byte aligned; the gradients must not overlap each other or the
+ * inputs (ROLA_ERR_INVALID_ARG).  Asynchronous on `stream`; deterministic (partial sums
+ * are reduced in a fixed order). */
+ROLA_API rola_status rola_backward_workspace_size(const rola_params* p, size_t* bytes);
+ROLA_API rola_status rola_backward(rola_plan_t plan, const void* q, const void* k, const void* v,
+                                   const void* Wq, const void* Wk, const float* g, const void* dout,
+                                   float* dq, float* dk, float* dv, float* dWq, float* dWk, float* dg,
+                                   void* bwd_workspace, size_t bwd_workspace_bytes,
+                                   rola_stream_t stream);
+
 /* Self-test of the softmax exponentials of the head-dim-128 attention kernels (a
  * measurement aid; the pages fix only P = exp(s - m)): y[i] = 2^x[i] for the n device
  * floats at x, computed by the same device functions the kernels call.  mode 0: the

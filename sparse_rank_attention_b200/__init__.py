@@ -37,7 +37,8 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_forward", "rola_get_block_lists", "rola_get_pooled", "rola_get_linear_state",
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
            "rola_select_blocks_noalloc", "rola_get_fp8_copies", "rola_profile_stages",
-           "rola_get_stage_times", "rola_get_attend_redo_count", "rola_eval_exp2")
+           "rola_get_stage_times", "rola_get_attend_redo_count", "rola_eval_exp2",
+           "rola_backward_workspace_size", "rola_backward")
 
 
 class RolaError(RuntimeError):
@@ -94,6 +95,8 @@ def load() -> ctypes.CDLL:
         "rola_profile_stages": [P, i32],
         "rola_get_attend_redo_count": [P, ctypes.POINTER(i32), P],
         "rola_eval_exp2": [P, P, ctypes.c_int64, i32, P],
+        "rola_backward_workspace_size": [pp, ctypes.POINTER(ctypes.c_size_t)],
+        "rola_backward": [P] * 15 + [ctypes.c_size_t, P],
         "rola_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), i32, ctypes.POINTER(i32),
                                  ctypes.POINTER(i32)],
     }.items():
@@ -228,6 +231,29 @@ class Plan:
         _check(load().rola_forward(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(Wq), _ptr(Wk),
                                    _ptr(g), _ptr(out), _stream(stream)), "rola_forward")
         return out
+
+    def backward(self, q, k, v, Wq, Wk, g, dout, stream=None):
+        """Gradients of sum(dout * out) through rola_backward (kept-block lists fixed).
+
+        Returns a dict of fp32 tensors: dq, dk, dv [B, N, H, d]; dWq, dWk [H, d, r]; dg with
+        the layout of g.  The backward scratch is allocated once per plan and kept."""
+        p = self.params
+        dev = self.workspace.device
+        if getattr(self, "bwd_workspace", None) is None:
+            n = ctypes.c_size_t()
+            _check(load().rola_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)),
+                   "rola_backward_workspace_size")
+            self.bwd_workspace = torch.empty(n.value, dtype=torch.uint8, device=dev)
+        act = (p.B, p.N, p.H, p.d)
+        res = {n: torch.empty(act, dtype=torch.float32, device=dev) for n in ("dq", "dk", "dv")}
+        res["dWq"] = torch.empty((p.H, p.d, p.r), dtype=torch.float32, device=dev)
+        res["dWk"] = torch.empty((p.H, p.d, p.r), dtype=torch.float32, device=dev)
+        res["dg"] = torch.empty(g.numel(), dtype=torch.float32, device=dev)
+        _check(load().rola_backward(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(Wq), _ptr(Wk), _ptr(g),
+                                    _ptr(dout), *[_ptr(res[n]) for n in ("dq", "dk", "dv", "dWq", "dWk", "dg")],
+                                    _ptr(self.bwd_workspace), self.bwd_workspace.numel(), _stream(stream)),
+               "rola_backward")
+        return res
 
     # ---- inspection
     def block_lists(self, stream=None) -> torch.Tensor:

@@ -480,6 +480,63 @@ rola_status rola_set_debug(rola_plan_t plan, int flags, int limit_us) {
   return ROLA_OK;
 }
 
+rola_status rola_backward_workspace_size(const rola_params* p, size_t* bytes) {
+  if (!bytes) return ROLA_ERR_INVALID_ARG;
+  const rola_status s = check_params(p);
+  if (s != ROLA_OK) return s;
+  if (p->dtype != ROLA_F32 && p->dtype != ROLA_BF16) return ROLA_ERR_UNSUPPORTED;
+  *bytes = rola::backward_workspace_bytes(make_dims(*p), nullptr, nullptr);
+  return ROLA_OK;
+}
+
+rola_status rola_backward(rola_plan_t plan, const void* q, const void* k, const void* v, const void* Wq,
+                          const void* Wk, const float* g, const void* dout, float* dq, float* dk, float* dv,
+                          float* dWq, float* dWk, float* dg, void* bwd_workspace, size_t bwd_workspace_bytes,
+                          rola_stream_t stream) {
+  if (!plan) return ROLA_ERR_INVALID_ARG;
+  const rola_params& p = plan->p;
+  if (p.dtype != ROLA_F32 && p.dtype != ROLA_BF16) return ROLA_ERR_UNSUPPORTED;
+  const void* in[] = {q, k, v, Wq, Wk, g, dout};
+  const void* outp[] = {dq, dk, dv, dWq, dWk, dg, bwd_workspace};
+  for (const void* x : in)
+    if (!x || !aligned16(x)) return ROLA_ERR_INVALID_ARG;
+  for (const void* x : outp)
+    if (!x || !aligned16(x)) return ROLA_ERR_INVALID_ARG;
+  const rola::Dims& dm = plan->dm;
+  rola::BwdWorkspace bw;
+  if (bwd_workspace_bytes < rola::backward_workspace_bytes(dm, nullptr, nullptr)) return ROLA_ERR_WORKSPACE;
+  rola::backward_workspace_bytes(dm, &bw, static_cast<char*>(bwd_workspace));
+  const size_t es = elem_size(p.dtype);
+  const size_t act = (size_t)p.B * p.N * p.H * p.d;
+  const size_t wsz = (size_t)p.H * p.d * p.r;
+  const size_t gsz = p.gate == ROLA_GATE_HEAD ? (size_t)p.H
+                     : p.gate == ROLA_GATE_TOKEN ? (size_t)p.B * p.N * p.H
+                                                 : (size_t)p.H * (p.d + 1);
+  // the gradients (and the scratch) overlap neither each other nor any input
+  const void* ob[] = {dq, dk, dv, dWq, dWk, dg, bwd_workspace};
+  const size_t on[] = {act * 4, act * 4, act * 4, wsz * 4, wsz * 4, gsz * 4, bwd_workspace_bytes};
+  const size_t inn[] = {act * es, act * es, act * es, wsz * es, wsz * es, gsz * 4, act * es};
+  for (int a = 0; a < 7; ++a) {
+    for (int c = 0; c < 7; ++c)
+      if (overlaps(ob[a], on[a], in[c], inn[c])) return ROLA_ERR_INVALID_ARG;
+    for (int c = a + 1; c < 7; ++c)
+      if (overlaps(ob[a], on[a], ob[c], on[c])) return ROLA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  rola_status s = ensure_status_word(plan, st);
+  if (s != ROLA_OK) return s;
+  if (!plan->rope_ready) {
+    if (rola::launch_rope_table(dm, plan->ws, st) != cudaSuccess) return ROLA_ERR_CUDA;
+    plan->rope_ready = true;
+  }
+  cudaError_t e = rola::launch_pool(dm, p.dtype, q, k, plan->ws, st);
+  if (e == cudaSuccess) e = rola::launch_select(dm, plan->ws, st);
+  if (e == cudaSuccess) e = rola::launch_linear_state(dm, p.dtype, k, v, Wk, plan->ws, st);
+  if (e == cudaSuccess)
+    e = rola::launch_backward(dm, p.dtype, q, k, v, Wq, Wk, g, dout, dq, dk, dv, dWq, dWk, dg, plan->ws, bw, st);
+  return cuda_status(e);
+}
+
 rola_status rola_eval_exp2(const float* x, float* y, int64_t n, int mode, rola_stream_t stream) {
   if (n < 0 || (mode != 0 && mode != 1) || (n > 0 && (!x || !y))) return ROLA_ERR_INVALID_ARG;
   return rola::launch_eval_exp2(x, y, n, mode, (cudaStream_t)stream) == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;

@@ -95,6 +95,27 @@ struct Workspace {
   float* sv;
 };
 
+// Scratch of the backward (rola_backward), carved from the caller's second workspace.
+struct BwdWorkspace {
+  float* lse;       // [B, H, nb, 64] log-sum-exp of each query row's scaled logits (+inf past N)
+  float* Drow;      // [B, H, nb, 64] dout . O_sparse per query row
+  int* inv_off;     // [B, H, nb + 1] start of each key block's list of query blocks
+  int* inv_idx;     // [B, H, nb * k] the query blocks that kept each key block, ascending
+  float* dS_part;   // [B, H, nchunk, r, d] partial gradients of the state
+  float* dz_part;   // [B, H, nchunk, r]
+  float* dWq_part;  // [B, H, nchunk, d, r]
+  float* dWk_part;  // [B, H, nchunk, d, r]
+  float* dg_part;   // [B, H, nchunk, d + 1] gain: per head (entry 0), or gate_proj then gate_bias
+  float* dS;        // [B, H, r, d]
+  float* dz;        // [B, H, r]
+};
+
+size_t backward_workspace_bytes(const Dims& dm, BwdWorkspace* bw, char* base);
+cudaError_t launch_backward(const Dims& dm, rola_dtype dt, const void* q, const void* k, const void* v,
+                            const void* Wq, const void* Wk, const float* g, const void* dout, float* dq, float* dk,
+                            float* dv, float* dWq, float* dWk, float* dg, const Workspace& ws,
+                            const BwdWorkspace& bw, cudaStream_t st);
+
 }  // namespace rola
 
 struct rola_plan_s {

@@ -176,4 +176,13 @@ def make_gate_proj(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     return torch.cat([wg.reshape(-1), bg]).contiguous()
 
 
-__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs", "make_gate", "make_gate_proj"]
+def make_dout(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """An upstream gradient dout [B, N, H, d] ~ N(0, 1) in the workload's input dtype (bf16,
+    or fp32), from its own seeded stream: the cotangent a backward call consumes."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randn((w.B, w.N, w.H, w.d), generator=gen, device=device).to(_torch_dtype(w))
+
+
+__all__ = ["Workload", "WORKLOADS", "BLOCK", "custom", "make_inputs", "make_gate", "make_gate_proj",
+           "make_dout"]

@@ -1,0 +1,112 @@
+"""GPU parity of the backward (the next row f2: gradients of the RoLA forward) against the
+oracle's backward, through the C ABI (rola_backward).
+
+The oracle's backward is pinned against central differences of the forward oracle
+(tests/test_oracle_backward.py).  Both sides take the kept-block lists of the forward as
+fixed and differentiate the same function of the same input values (bf16 inputs enter both
+as their exact values); the kernels compute in fp32 and the oracle in double, so the bound
+is fp32 rounding over sums of up to k*64 terms, plus, at head dim 128 with bf16 inputs,
+the state S from the tensor-core key/value pass (its feature operand as a bf16 hi + lo
+pair, ~2^-16 relative): every element within 5e-4 of its tensor's RMS, and the whole
+tensor within 5e-5 of it normwise.  The lists themselves are compared
+bit for bit, and two calls must give identical bits (partial sums in a fixed order).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+import sparse_rank_attention_b200 as rola
+from rola_testlib import host_inputs, np32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    rola.load()
+
+
+CASES = [
+    # the tiny fp32 configuration (1D grid)
+    (synth.custom("bwd_tiny_f32", B=1, H=2, N=1024, d=64, r=16, topk=0.25, dtype="f32"), "head"),
+    # bf16 at head dim 128: a ragged 40-token tail, a 3D grid, two batch entries
+    (synth.custom("bwd_bf16_d128_b2", B=2, H=2, N=1000, d=128, r=32, topk=0.3, grid=(2, 4, 125)), "head"),
+    (synth.custom("bwd_bf16_d128_token", B=1, H=3, N=777, d=128, r=32, topk=0.25, grid=(3, 7, 37)), "token"),
+    (synth.custom("bwd_bf16_d128_proj", B=1, H=2, N=1000, d=128, r=16, topk=0.2), "proj"),
+    (synth.custom("bwd_bf16_d64_r32", B=1, H=2, N=700, d=64, r=32, topk=0.4, grid=(7, 10, 10)), "head"),
+    (synth.custom("bwd_f32_d128_tail1", B=2, H=1, N=129, d=128, r=32, topk=0.6, dtype="f32"), "token"),
+    # several key-major passes per CTA wave: 128 blocks per head, 13 kept
+    (synth.custom("bwd_bf16_d128_n8192", B=1, H=2, N=8192, d=128, r=32, topk=0.1, grid=(8, 32, 32)), "head"),
+]
+
+
+def _gain(w, gate, inp):
+    if gate == "head":
+        return inp["g"]
+    if gate == "token":
+        return synth.make_gate(w, seed=9, device="cuda")
+    return synth.make_gate_proj(w, seed=9, device="cuda")
+
+
+def _compare(name, got, want):
+    got = got.astype(np.float64).reshape(-1)
+    want = want.reshape(-1)
+    rms = float(np.sqrt(np.mean(want ** 2))) or 1.0
+    err = np.abs(got - want)
+    worst = int(np.argmax(err))
+    assert err[worst] <= 5e-4 * rms, f"{name}: |err| {err[worst]:.3e} at {worst} vs rms {rms:.3e}"
+    nerr = float(np.sqrt(np.mean(err ** 2)))
+    assert nerr <= 5e-5 * rms, f"{name}: normwise {nerr / rms:.3e}"
+
+
+@pytest.mark.parametrize("w,gate", CASES, ids=[f"{w.name}-{g}" for w, g in CASES])
+def test_backward_matches_oracle(w, gate):
+    inp = synth.make_inputs(w, seed=5, device="cuda")
+    g = _gain(w, gate, inp)
+    dout = synth.make_dout(w, seed=6, device="cuda")
+    plan = rola.Plan.for_workload(w, gate=gate)
+    got = plan.backward(inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], g, dout)
+    assert plan.poll_status() == 0
+    again = plan.backward(inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], g, dout)
+    torch.cuda.synchronize()
+    for key in got:
+        assert torch.equal(got[key], again[key]), f"{key} differs between two calls"
+    h = host_inputs(inp)
+    s = O.make_shape(w.B, w.H, w.N, w.d, w.r, w.topk, grid=w.grid, pairs=w.pairs, gate=gate)
+    _, col = O.forward(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], np32(g))
+    np.testing.assert_array_equal(plan.block_lists().cpu().numpy(), col)
+    want = O.backward(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], np32(g), np32(dout).astype(np.float64), col)
+    for key in ("dq", "dk", "dv", "dWq", "dWk", "dg"):
+        _compare(f"{w.name}/{key}", np32(got[key]), want[key].reshape(np32(got[key]).shape))
+
+
+def test_backward_rejects_bad_calls():
+    w = synth.custom("bwd_args", B=1, H=2, N=256, d=128, r=32, topk=0.5)
+    inp = synth.make_inputs(w, seed=1, device="cuda")
+    dout = synth.make_dout(w, seed=2, device="cuda")
+    plan = rola.Plan.for_workload(w)
+    lib = rola.load()
+    grads = plan.backward(inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], inp["g"], dout)
+    ws = plan.bwd_workspace
+    p = lambda t: rola._ptr(t)  # noqa: E731
+    args = [p(inp[n]) for n in ("q", "k", "v", "Wq", "Wk", "g")] + [p(dout)]
+    outs = [p(grads[n]) for n in ("dq", "dk", "dv", "dWq", "dWk", "dg")]
+    st = rola._stream(None)
+    assert lib.rola_backward(plan._h, *args, *outs, p(ws), ws.numel(), st) == 0
+    assert lib.rola_backward(plan._h, *args, *outs, p(ws), ws.numel() - 256, st) == 3   # scratch too small
+    bad = list(outs)
+    bad[0] = p(inp["q"])                                                             # dq over q
+    assert lib.rola_backward(plan._h, *args, *bad, p(ws), ws.numel(), st) == 1
+    bad = list(outs)
+    bad[1] = outs[0]                                                                 # dk over dq
+    assert lib.rola_backward(plan._h, *args, *bad, p(ws), ws.numel(), st) == 1
+    assert lib.rola_backward(plan._h, *args[:6], rola._ptr(None), *outs, p(ws), ws.numel(), st) == 1
+    w8 = synth.custom("bwd_fp8", B=1, H=2, N=256, d=128, r=32, topk=0.5, dtype="fp8")
+    n = rola.ctypes.c_size_t()
+    assert lib.rola_backward_workspace_size(rola.ctypes.byref(rola.Plan.for_workload(w8).params),
+                                            rola.ctypes.byref(n)) == 2
+    assert plan.poll_status() == 0
