@@ -8,13 +8,15 @@ the sparse branch, 4*d*c_i*c_j summed over every kept (query block i, key block 
 pair (c = valid tokens of a block), divided by the step time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rola|reference]
-                  [--gate head|token] [--no-e2e] [--no-cpu-baseline] [--no-fp8]
+                  [--gate head|token] [--no-e2e] [--no-cpu-baseline] [--no-fp8] [--no-backward]
 
 ``--gate token`` feeds a gain per token and head (g [B, N, H]) instead of per head;
 ``--gate proj`` has the library compute it from the query (gate_proj, gate_bias).
 For a bf16 workload that has an fp8-e4m3 twin (the 720P and 480P 14B shapes), the same
 line also carries ``fp8``: the twin timed the same way on the same inputs (``--no-fp8``
-skips it).
+skips it).  ``backward`` times rola_backward (the gradients of the same forward, fp32
+arithmetic) on the same workload: a few calls, the same timing rules; its TFLOP/s counts the
+five kept-block products of an attention backward (2.5 x the forward's kept-block FLOPs).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs an independent forward of the
 same workload (different seed), no collective on the data path ("scaling": "weak");
@@ -296,7 +298,8 @@ def measure(w, plan, step, steps, warmup, ws, dev):
     stage_sum, ncalls = plan.stage_times()
     plan.profile_stages(False)
     assert plan.poll_status() == 0
-    return {"flops": flops, "ms_step": ms_total / steps, "stage_ms": [x / ncalls for x in stage_sum],
+    return {"flops": flops, "ms_step": ms_total / steps,
+            "stage_ms": [x / ncalls for x in stage_sum] if ncalls else None,
             "clocks": clk.summary()}
 
 
@@ -330,6 +333,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the fp8-e4m3 twin of a bf16 workload")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--gate", default="head", choices=["head", "token", "proj"],
                     help="gain of the linear branch per head (default), per token and head, or "
                          "computed from the query (sigmoid of q . gate_proj + gate_bias)")
@@ -487,6 +491,23 @@ def main():
         plan8.close()
         del out8
 
+    bwd = None
+    if not args.no_backward and w.dtype in ("bf16", "f32"):
+        # the backward on the same inputs and gain: dout drawn once; a short timed region
+        # (each call is long), the same barriers and max over ranks
+        dout = synth.make_dout(w, seed=7 + rank, device=dev)
+        bwd_warm, bwd_steps = 2, 5
+
+        def bstep():
+            plan.backward(q, k, v, Wq, Wk, g, dout)
+
+        mb = measure(w, plan, bstep, bwd_steps, bwd_warm, ws, dev)
+        bflops = int(2.5 * mb["flops"])
+        bwd = {"ms_per_call": mb["ms_step"], "steps": bwd_steps, "warmup": bwd_warm,
+               "value": aggregate_tflops(bflops, mb["ms_step"], ws), "unit": "kept-block TFLOP/s (backward)",
+               "flops_per_call": bflops, "arithmetic": "fp32 (CUDA cores)", "clocks": mb["clocks"]}
+        del dout
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not per_token:
         r = oracle_sample(w, seconds_hint=15.0)
@@ -506,6 +527,7 @@ def main():
                            "l2": "inputs (3 x 774 MB) larger than L2 (126 MB); no flush",
                            "parallelism": f"replicas x{ws} (independent forward per GPU)"},
                 "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "fp8": fp8,
+                "backward": bwd,
                 "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk}
         print(json.dumps(line))
     if ws > 1:
