@@ -27,7 +27,10 @@
 // products thread (ty, tx) = (tid / 16, tid % 16) holds rows 4 ty .. 4 ty + 3 and columns
 // tx + 16 j.  Partial sums over token chunks are reduced in a fixed order, so the result
 // is the same from run to run.  Every wait is a __syncthreads; no kernel spins.
+#include <type_traits>
+
 #include "rola_internal.cuh"
+#include "warp_mma.cuh"
 
 namespace rola {
 namespace {
@@ -332,6 +335,306 @@ __global__ void __launch_bounds__(kT) bwd_dkv_kernel(const T* __restrict__ q, co
   }
 }
 
+// ------------------------------------------------------------------ sparse branch, bf16
+// The same three kernels for bf16 inputs on the warp-level tensor cores (mma.sync
+// m16n8k16, fp32 accumulation): 128 threads, warp w owning rows 16 w .. 16 w + 15 of its
+// tile, tiles in shared memory as bf16 [64][D + 8].  Q, K, V and dout enter exactly; P and
+// dA enter the second products as bf16 hi + lo pairs (two products each, ~2^-16 relative),
+// so the gradients keep fp32-level accuracy.
+template <int D>
+struct MmaTiles {
+  static constexpr int DP = D + 8;
+  static constexpr int kTile = 64 * DP;
+  static constexpr size_t bytes = sizeof(__nv_bfloat16) * 4 * kTile + sizeof(float) * 128;
+};
+
+// rows [n0, n0 + 64) of head h of a [B, N, H, D] bf16 tensor -> s[64][D + 8] (cp.async;
+// rows at or past N zero-filled)
+template <int D>
+__device__ __forceinline__ void load_tile_bf16(__nv_bfloat16* s, const __nv_bfloat16* __restrict__ x, const Dims& dm,
+                                               int b, int h, int n0) {
+  constexpr int VPR = D / 8;
+  for (int e = threadIdx.x; e < 64 * VPR; e += 128) {
+    const int r = e / VPR, cv = e % VPR, n = n0 + r;
+    const bool ok = n < dm.N;
+    cp_async16(smem_u32(s + r * (D + 8) + cv * 8), x + (((size_t)b * dm.N + (ok ? n : 0)) * dm.H + h) * D + cv * 8,
+               ok ? 16 : 0);
+  }
+}
+
+// acc[nt] (16 x 64 per warp) = A (rows 16 w.. of sA) times B^T (rows of sB), K = D
+template <int D>
+__device__ __forceinline__ void mma_rows_abt(float (&acc)[8][4], const __nv_bfloat16* sA, const __nv_bfloat16* sB,
+                                             int warp, int lane) {
+  constexpr int DP = D + 8;
+  const int quad = lane >> 3;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t af[4];
+    ldsm_x4(smem_u32(sA + (16 * warp + (lane & 15)) * DP + kk * 16 + (lane >> 4) * 8), af[0], af[1], af[2], af[3]);
+#pragma unroll
+    for (int nt = 0; nt < 8; nt += 2) {
+      uint32_t bf[4];
+      ldsm_x4(smem_u32(sB + ((nt + (quad >> 1)) * 8 + (lane & 7)) * DP + kk * 16 + (quad & 1) * 8), bf[0], bf[1],
+              bf[2], bf[3]);
+      mma_bf16(acc[nt], af, bf);
+      mma_bf16(acc[nt + 1], af, bf + 2);
+    }
+  }
+}
+
+// acc (16 x D per warp) += X (16 x 64, accumulator layout, as bf16 hi + lo) times sB (64 x D)
+template <int D>
+__device__ __forceinline__ void mma_rows_xb(float (&acc)[D / 8][4], const float (&x)[8][4], const __nv_bfloat16* sB,
+                                            int lane) {
+  constexpr int DP = D + 8;
+  const int quad = lane >> 3;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t hi[4], lo[4];
+    split_bf16(x[2 * kk][0], x[2 * kk][1], hi[0], lo[0]);
+    split_bf16(x[2 * kk][2], x[2 * kk][3], hi[1], lo[1]);
+    split_bf16(x[2 * kk + 1][0], x[2 * kk + 1][1], hi[2], lo[2]);
+    split_bf16(x[2 * kk + 1][2], x[2 * kk + 1][3], hi[3], lo[3]);
+#pragma unroll
+    for (int nt = 0; nt < D / 8; nt += 2) {
+      uint32_t bf[4];
+      ldsm_x4_t(smem_u32(sB + (kk * 16 + (quad & 1) * 8 + (lane & 7)) * DP + (nt + (quad >> 1)) * 8), bf[0], bf[1],
+                bf[2], bf[3]);
+      mma_bf16(acc[nt], hi, bf);
+      mma_bf16(acc[nt + 1], hi, bf + 2);
+      mma_bf16(acc[nt], lo, bf);
+      mma_bf16(acc[nt + 1], lo, bf + 2);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const __nv_bfloat16* __restrict__ dout, Dims dm, const int32_t* __restrict__ col_idx, float* __restrict__ lse,
+    float* __restrict__ Drow, int* __restrict__ status) {
+  using L = MmaTiles<D>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smb);
+  __nv_bfloat16* sG = sQ + L::kTile;
+  __nv_bfloat16* sK = sG + L::kTile;
+  __nv_bfloat16* sV = sK + L::kTile;
+  const int i = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
+  const int32_t* Lst = col_idx + ((size_t)bh * dm.nb + i) * dm.k;
+  const float sl2 = dm.scale * 1.4426950408889634f;
+  load_tile_bf16<D>(sQ, q, dm, b, h, i * 64);
+  load_tile_bf16<D>(sG, dout, dm, b, h, i * 64);
+  cp_async_commit();
+  float o[D / 8][4], m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  for (int jj = 0; jj < dm.k; ++jj) {
+    const int j = checked_block(dm, Lst[jj], status);
+    __syncthreads();
+    load_tile_bf16<D>(sK, k, dm, b, h, j * 64);
+    load_tile_bf16<D>(sV, v, dm, b, h, j * 64);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    float s[8][4];
+    mma_rows_abt<D>(s, sQ, sK, warp, lane);
+    const int nvalid = min(64, dm.N - j * 64);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 2 * hh; e < 2 * hh + 2; ++e) {
+          s[nt][e] = nt * 8 + 2 * t4 + (e & 1) < nvalid ? s[nt][e] * sl2 : -INFINITY;
+          mx = fmaxf(mx, s[nt][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mnew = fmaxf(m[hh], mx);
+      const float corr = m[hh] == -INFINITY ? 0.f : exp2f(m[hh] - mnew);
+      float rs = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 2 * hh; e < 2 * hh + 2; ++e) {
+          s[nt][e] = exp2f(s[nt][e] - mnew);
+          rs += s[nt][e];
+        }
+      l[hh] = l[hh] * corr + rs;
+      m[hh] = mnew;
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt) {
+        o[nt][2 * hh] *= corr;
+        o[nt][2 * hh + 1] *= corr;
+      }
+    }
+    mma_rows_xb<D>(o, s, sV, lane);
+  }
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float lt = l[hh];
+    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+    const int row = 16 * warp + g8 + 8 * hh, n = i * 64 + row;
+    float dsum = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+      for (int e = 2 * hh; e < 2 * hh + 2; ++e)
+        dsum = fmaf(__bfloat162float(sG[row * (D + 8) + nt * 8 + 2 * t4 + (e & 1)]), o[nt][e] / lt, dsum);
+    dsum += __shfl_xor_sync(0xffffffffu, dsum, 1);
+    dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
+    if (t4 == 0) {
+      const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + row;
+      lse[at] = n < dm.N ? m[hh] + log2f(lt) : INFINITY;   // log2 units of scale * log2(e) * q.k
+      Drow[at] = n < dm.N ? dsum : 0.f;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_dq_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const __nv_bfloat16* __restrict__ dout, Dims dm, const int32_t* __restrict__ col_idx,
+    const float* __restrict__ lse, const float* __restrict__ Drow, float* __restrict__ dq, int* __restrict__ status) {
+  using L = MmaTiles<D>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smb);
+  __nv_bfloat16* sG = sQ + L::kTile;
+  __nv_bfloat16* sK = sG + L::kTile;
+  __nv_bfloat16* sV = sK + L::kTile;
+  const int i = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
+  const int32_t* Lst = col_idx + ((size_t)bh * dm.nb + i) * dm.k;
+  const float sl2 = dm.scale * 1.4426950408889634f;
+  load_tile_bf16<D>(sQ, q, dm, b, h, i * 64);
+  load_tile_bf16<D>(sG, dout, dm, b, h, i * 64);
+  cp_async_commit();
+  float ls[2], dd[2], acc[D / 8][4];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + 16 * warp + g8 + 8 * hh;
+    ls[hh] = lse[at];
+    dd[hh] = Drow[at];
+  }
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  for (int jj = 0; jj < dm.k; ++jj) {
+    const int j = checked_block(dm, Lst[jj], status);
+    __syncthreads();
+    load_tile_bf16<D>(sK, k, dm, b, h, j * 64);
+    load_tile_bf16<D>(sV, v, dm, b, h, j * 64);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    float s[8][4], dp[8][4];
+    mma_rows_abt<D>(s, sQ, sK, warp, lane);
+    mma_rows_abt<D>(dp, sG, sV, warp, lane);
+    const int nvalid = min(64, dm.N - j * 64);
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hh = e >> 1;
+        const float p = nt * 8 + 2 * t4 + (e & 1) < nvalid ? exp2f(s[nt][e] * sl2 - ls[hh]) : 0.f;
+        s[nt][e] = p * (dp[nt][e] - dd[hh]);
+      }
+    mma_rows_xb<D>(acc, s, sK, lane);
+  }
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int n = i * 64 + 16 * warp + g8 + 8 * hh;
+    if (n >= dm.N) continue;
+    float* row = dq + (((size_t)b * dm.N + n) * dm.H + h) * D;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+      row[nt * 8 + 2 * t4] += dm.scale * acc[nt][2 * hh];
+      row[nt * 8 + 2 * t4 + 1] += dm.scale * acc[nt][2 * hh + 1];
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_dkv_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const __nv_bfloat16* __restrict__ dout, Dims dm, const int* __restrict__ inv_off, const int* __restrict__ inv_idx,
+    const float* __restrict__ lse, const float* __restrict__ Drow, float* __restrict__ dk, float* __restrict__ dv) {
+  using L = MmaTiles<D>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smb);
+  __nv_bfloat16* sV = sK + L::kTile;
+  __nv_bfloat16* sQ = sV + L::kTile;
+  __nv_bfloat16* sG = sQ + L::kTile;
+  float* sL = reinterpret_cast<float*>(sG + L::kTile);   // [64] lse of the query tile
+  float* sD = sL + 64;                                     // [64] D of the query tile
+  const int j = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
+  const float sl2 = dm.scale * 1.4426950408889634f;
+  load_tile_bf16<D>(sK, k, dm, b, h, j * 64);
+  load_tile_bf16<D>(sV, v, dm, b, h, j * 64);
+  cp_async_commit();
+  float ak[D / 8][4], av[D / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ak[nt][e] = av[nt][e] = 0.f;
+  const int* lst = inv_idx + (size_t)bh * dm.nb * dm.k;
+  const int e0 = inv_off[(size_t)bh * (dm.nb + 1) + j], e1 = inv_off[(size_t)bh * (dm.nb + 1) + j + 1];
+  for (int e = e0; e < e1; ++e) {
+    const int i = lst[e];
+    __syncthreads();
+    load_tile_bf16<D>(sQ, q, dm, b, h, i * 64);
+    load_tile_bf16<D>(sG, dout, dm, b, h, i * 64);
+    cp_async_commit();
+    if (threadIdx.x < 64) {
+      const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + threadIdx.x;
+      sL[threadIdx.x] = lse[at];
+      sD[threadIdx.x] = Drow[at];
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    float st[8][4], dpt[8][4];          // rows: keys 16 w + g8 (+ 8); columns: queries
+    mma_rows_abt<D>(st, sK, sQ, warp, lane);
+    mma_rows_abt<D>(dpt, sV, sG, warp, lane);
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int qc = nt * 8 + 2 * t4 + (x & 1);
+        const float p = exp2f(st[nt][x] * sl2 - sL[qc]);   // 0 for queries past N (lse = +inf)
+        st[nt][x] = p;
+        dpt[nt][x] = p * (dpt[nt][x] - sD[qc]);
+      }
+    mma_rows_xb<D>(av, st, sG, lane);
+    mma_rows_xb<D>(ak, dpt, sQ, lane);
+  }
+  const int nvalid = min(64, dm.N - j * 64);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int r = 16 * warp + g8 + 8 * hh;
+    if (r >= nvalid) continue;
+    const size_t at = (((size_t)b * dm.N + j * 64 + r) * dm.H + h) * D;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+      dk[at + nt * 8 + 2 * t4] += dm.scale * ak[nt][2 * hh];
+      dk[at + nt * 8 + 2 * t4 + 1] += dm.scale * ak[nt][2 * hh + 1];
+      dv[at + nt * 8 + 2 * t4] += av[nt][2 * hh];
+      dv[at + nt * 8 + 2 * t4 + 1] += av[nt][2 * hh + 1];
+    }
+  }
+}
+
 // For each (b, h): the query blocks that kept each key block, ascending (the key-major
 // view of the lists).  Counts, an exclusive scan, a scatter, then each list sorted.
 __global__ void __launch_bounds__(kT) bwd_inverse_lists_kernel(Dims dm, const int32_t* __restrict__ col_idx,
@@ -381,32 +684,82 @@ __global__ void __launch_bounds__(kT) bwd_inverse_lists_kernel(Dims dm, const in
 }
 
 // ------------------------------------------------------------------ linear branch
+// Per chunk of tokens, 64-token tiles; the small products (64 x r x d) run as 4 x 4
+// register tiles per thread over shared-memory operands (tile t = tid + 256 s: rows
+// 4 (t / NT) .. + 3, columns t % NT + NT j), the per-row steps (phi, the rotation, the
+// normaliser, the gain) one row or one rank pair per thread.
 template <int D, int RK>
 struct LinSmem {
   static constexpr int kTile = 64 * (D + 1);
   static constexpr int kW = D * (RK + 1);      // Wq or Wk [D][RK]
   static constexpr int kS = RK * (D + 1);      // S or dS [RK][D]
   static constexpr int kR = 64 * (RK + 1);     // [64][RK] row vectors
-  static constexpr size_t bytes = sizeof(float) * (2 * kTile + kW + kS + 3 * kR + RK + 3 * 64);
+  static constexpr size_t bytes = sizeof(float) * (2 * kTile + kW + kS + 4 * kR + RK + 6 * 64);
 };
 
-// Rotation of the rank pairs of row `n` (this thread's RK / 4 ranks from a0): y = R x, or
-// R^T x when back is set.
-template <int Q>
-__device__ __forceinline__ void rotate_q(const Dims& dm, const float2* __restrict__ rope, int n, int a0,
-                                         const float (&x)[Q], float (&y)[Q], bool back) {
-  const TokPos pos = token_pos(dm, n < dm.N ? n : 0);
+// acc[s][i][j] += sum_k a(m, k) b(k, n) for the tiles of this thread of an M x N product
+// (m = 4 (t / NT) + i, n = t % NT + NT j).
+template <int M, int N, int K, int S_, class FA, class FB>
+__device__ __forceinline__ void tile_gemm(float (&acc)[S_][4][4], FA a, FB b) {
+  constexpr int NT = N / 4, TILES = (M / 4) * NT;
 #pragma unroll
-  for (int p = 0; p < Q / 2; ++p) {
-    const float2 cs = n < dm.N ? rope_at(dm, rope, pos, a0 / 2 + p) : make_float2(1.f, 0.f);
-    const float sn = back ? -cs.y : cs.y;
-    y[2 * p] = cs.x * x[2 * p] - sn * x[2 * p + 1];
-    y[2 * p + 1] = sn * x[2 * p] + cs.x * x[2 * p + 1];
+  for (int s = 0; s < S_; ++s) {
+    const int t = threadIdx.x + kT * s;
+    if (t >= TILES) break;
+    const int m0 = 4 * (t / NT), n0 = t % NT;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = a(m0 + i, k);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = b(k, n0 + NT * j);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[s][i][j] = fmaf(av[i], bv[j], acc[s][i][j]);
+    }
   }
 }
 
-// Query side: per chunk of query tokens, the linear branch's dq (written, the sparse part
-// is added later), the chunk's partial dS, dz, dWq and gain gradients.
+template <int M, int N>
+constexpr int tiles_per_thread() { return ((M / 4) * (N / 4) + kT - 1) / kT; }
+
+template <int S_>
+__device__ __forceinline__ void zero_acc(float (&acc)[S_][4][4]) {
+#pragma unroll
+  for (int s = 0; s < S_; ++s)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[s][i][j] = 0.f;
+}
+
+// Visits the elements of this thread's tiles: f(m, n, value).
+template <int M, int N, int S_, class F>
+__device__ __forceinline__ void tile_each(const float (&acc)[S_][4][4], F f) {
+  constexpr int NT = N / 4, TILES = (M / 4) * NT;
+#pragma unroll
+  for (int s = 0; s < S_; ++s) {
+    const int t = threadIdx.x + kT * s;
+    if (t >= TILES) break;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f(4 * (t / NT) + i, t % NT + NT * j, acc[s][i][j]);
+  }
+}
+
+// (cos, sin) of rank pair p at token n (identity past N)
+__device__ __forceinline__ float2 pair_cs(const Dims& dm, const float2* __restrict__ rope, int n, int p) {
+  if (n >= dm.N) return make_float2(1.f, 0.f);
+  return rope_at(dm, rope, token_pos(dm, n), p);
+}
+
+// Query side: per chunk of query tokens, the linear branch's dq (written; the sparse part
+// is added later), the chunk's partial dS, dz, dWq and gain gradients.  With T = G S^T
+// (the row's dout against each rank of the state), dg = y . T / den and dy = g T / den, so
+// the linear output itself is never formed.
 template <typename T, int D, int RK>
 __global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
     const T* __restrict__ q, const T* __restrict__ dout, const T* __restrict__ Wq, const float* __restrict__ g,
@@ -414,163 +767,136 @@ __global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
     float* __restrict__ dq, float* __restrict__ dg, float* __restrict__ dS_part, float* __restrict__ dz_part,
     float* __restrict__ dWq_part, float* __restrict__ dg_part) {
   using Lsm = LinSmem<D, RK>;
-  constexpr int QR = RK / 4, QC = D / 4, PT = D * RK / kT;
+  constexpr int WS = RK + 1, TS = D + 1;
   extern __shared__ float sm[];
   float* sQ = sm;
   float* sG = sQ + Lsm::kTile;
   float* sW = sG + Lsm::kTile;        // Wq [D][RK + 1]
   float* sS = sW + Lsm::kW;           // S [RK][D + 1]
-  float* sY = sS + Lsm::kS;           // R u [64][RK + 1]
-  float* sX = sY + Lsm::kR;           // dx [64][RK + 1]
-  float* sZr = sX + Lsm::kR;          // dz partials of the last tile [64][RK + 1]
-  float* sz = sZr + Lsm::kR;          // z [RK]
+  float* sX = sS + Lsm::kS;           // x, then dx [64][RK + 1]
+  float* sU = sX + Lsm::kR;           // u
+  float* sY = sU + Lsm::kR;           // R u
+  float* sT = sY + Lsm::kR;           // G S^T
+  float* sz = sT + Lsm::kR;           // z [RK]
   float* sgd = sz + RK;               // g / den per row [64]
-  float* sdl = sgd + 64;              // dlogit per row (gate from the query) [64]
-  float* sdg = sdl + 64;              // dg per row [64]
+  float* sdd = sgd + 64;              // dden per row
+  float* sdl = sdd + 64;              // dlogit per row (gate from the query)
+  float* sdg = sdl + 64;              // dg per row
+  float* sdot = sdg + 64;             // q . wg per row
+  float* sden = sdot + 64;            // den per row
   const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
-  const int tid = threadIdx.x, row = tid >> 2, qt = tid & 3, a0 = qt * QR, c0 = qt * QC;
+  const int tid = threadIdx.x;
   const int n_begin = chunk * dm.chunk_tok, n_end = min(dm.N, n_begin + dm.chunk_tok);
-  for (int e = tid; e < D * RK; e += kT) sW[(e / RK) * (RK + 1) + e % RK] = to_f(Wq[(size_t)h * D * RK + e]);
-  for (int e = tid; e < RK * D; e += kT) sS[(e / D) * (D + 1) + e % D] = S[(size_t)bh * RK * D + e];
+  const bool qproj = dm.gate_mode == ROLA_GATE_QPROJ;
+  for (int e = tid; e < D * RK; e += kT) sW[(e / RK) * WS + e % RK] = to_f(Wq[(size_t)h * D * RK + e]);
+  for (int e = tid; e < RK * D; e += kT) sS[(e / D) * TS + e % D] = S[(size_t)bh * RK * D + e];
   if (tid < RK) sz[tid] = z[(size_t)bh * RK + tid];
-  // per-thread accumulators: dS[a][c] and dWq[c][a] for c = tid % D, a in the thread's
-  // block of PT ranks; dz over this thread's rows; the gain's parts
-  const int pc = tid % D, pa = (tid / D) * PT;
-  float aS[PT], aW[PT], aZ[QR], adg = 0.f, awg = 0.f, abg = 0.f;
-#pragma unroll
-  for (int x = 0; x < PT; ++x) aS[x] = aW[x] = 0.f;
-#pragma unroll
-  for (int x = 0; x < QR; ++x) aZ[x] = 0.f;
+  constexpr int SP = tiles_per_thread<RK, D>(), WP = tiles_per_thread<D, RK>();
+  constexpr int XP = tiles_per_thread<64, RK>(), QP = tiles_per_thread<64, D>();
+  float aS[SP][4][4], aW[WP][4][4];
+  zero_acc(aS);
+  zero_acc(aW);
+  float az = 0.f, awg = 0.f, adg = 0.f, abg = 0.f;   // rank tid (dz), channel tid (dwg), sums
   for (int n0 = n_begin; n0 < n_end; n0 += 64) {
     __syncthreads();
     load_tile<T, D>(sQ, q, dm, b, h, n0);
     load_tile<T, D>(sG, dout, dm, b, h, n0);
     __syncthreads();
-    const int n = n0 + row;
-    const bool valid = n < n_end;
-    // x = q Wq (this thread's ranks), u = phi(x), y = R u, den = u . z
-    float x[QR], u[QR], y[QR];
-#pragma unroll
-    for (int a = 0; a < QR; ++a) x[a] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float qv = sQ[row * (D + 1) + c];
-#pragma unroll
-      for (int a = 0; a < QR; ++a) x[a] = fmaf(qv, sW[c * (RK + 1) + a0 + a], x[a]);
+    // x = q Wq and T = G S^T
+    {
+      float ax[XP][4][4], at[XP][4][4];
+      zero_acc(ax);
+      zero_acc(at);
+      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return sQ[m * TS + c]; }, [&](int c, int a) { return sW[c * WS + a]; });
+      tile_gemm<64, RK, D>(at, [&](int m, int c) { return sG[m * TS + c]; }, [&](int c, int a) { return sS[a * TS + c]; });
+      tile_each<64, RK>(ax, [&](int m, int a, float x) {
+        sX[m * WS + a] = x;
+        sU[m * WS + a] = phi_f(x);
+      });
+      tile_each<64, RK>(at, [&](int m, int a, float x) { sT[m * WS + a] = x; });
     }
-    float den = 0.f;
-#pragma unroll
-    for (int a = 0; a < QR; ++a) {
-      u[a] = phi_f(x[a]);
-      den = fmaf(u[a], sz[a0 + a], den);
-    }
-    den += __shfl_xor_sync(0xffffffffu, den, 1);
-    den += __shfl_xor_sync(0xffffffffu, den, 2);
-    rotate_q<QR>(dm, rope, n, a0, u, y, false);
-#pragma unroll
-    for (int a = 0; a < QR; ++a) sY[row * (RK + 1) + a0 + a] = y[a];
-    // the gain of the token
-    float gn;
-    if (dm.gate_mode == ROLA_GATE_QPROJ) {
+    if (qproj && tid < 64) {
       float dot = 0.f;
-      for (int c = c0; c < c0 + QC; ++c) dot = fmaf(sQ[row * (D + 1) + c], __ldg(g + (size_t)h * D + c), dot);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-      gn = gate_sigmoid(dm, g, h, dot);
-    } else {
-      gn = g[gain_index(dm, b, valid ? n : n_begin, h)];
+      for (int c = 0; c < D; ++c) dot = fmaf(sQ[tid * TS + c], __ldg(g + (size_t)h * D + c), dot);
+      sdot[tid] = dot;
     }
     __syncthreads();
-    // L = y^T S / den on this thread's columns; dg = dout . L
-    float dgn = 0.f;
-    float Lc[QC];
-#pragma unroll
-    for (int c = 0; c < QC; ++c) Lc[c] = 0.f;
-    for (int a = 0; a < RK; ++a) {
-      const float ya = sY[row * (RK + 1) + a];
-#pragma unroll
-      for (int c = 0; c < QC; ++c) Lc[c] = fmaf(ya, sS[a * (D + 1) + c0 + c], Lc[c]);
+    // y = R u (one rank pair per item) and the row's den = u . z
+    for (int e = tid; e < 64 * (RK / 2); e += kT) {
+      const int m = e / (RK / 2), p = e % (RK / 2);
+      const float2 cs = pair_cs(dm, rope, n0 + m, p);
+      const float x0 = sU[m * WS + 2 * p], x1 = sU[m * WS + 2 * p + 1];
+      sY[m * WS + 2 * p] = cs.x * x0 - cs.y * x1;
+      sY[m * WS + 2 * p + 1] = cs.y * x0 + cs.x * x1;
     }
-#pragma unroll
-    for (int c = 0; c < QC; ++c) dgn = fmaf(sG[row * (D + 1) + c0 + c], Lc[c] / den, dgn);
-    dgn += __shfl_xor_sync(0xffffffffu, dgn, 1);
-    dgn += __shfl_xor_sync(0xffffffffu, dgn, 2);
-    if (!valid) dgn = 0.f;
-    // dy = S gG / den on this thread's ranks; dden = -g dg / den
-    const float gd = valid ? gn / den : 0.f;
-    float dy[QR];
-#pragma unroll
-    for (int a = 0; a < QR; ++a) dy[a] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float gv = sG[row * (D + 1) + c];
-#pragma unroll
-      for (int a = 0; a < QR; ++a) dy[a] = fmaf(sS[(a0 + a) * (D + 1) + c], gv, dy[a]);
-    }
-    const float dden = -gn * dgn / den;
-    float du[QR];
-#pragma unroll
-    for (int a = 0; a < QR; ++a) dy[a] *= gd;
-    rotate_q<QR>(dm, rope, n, a0, dy, du, true);
-#pragma unroll
-    for (int a = 0; a < QR; ++a) {
-      du[a] = fmaf(dden, sz[a0 + a], du[a]);
-      aZ[a] = fmaf(dden, u[a], aZ[a]);
-      sX[row * (RK + 1) + a0 + a] = valid ? dphi_f(x[a]) * du[a] : 0.f;
-    }
-    if (qt == 0) {
-      sgd[row] = gd;
-      sdg[row] = dgn;
-      sdl[row] = valid ? dgn * gn * (1.f - gn) : 0.f;
+    if (tid < 64) {
+      float den = 0.f;
+      for (int a = 0; a < RK; ++a) den = fmaf(sU[tid * WS + a], sz[a], den);
+      sden[tid] = den;
     }
     __syncthreads();
-    // dq = Wq dx (+ dlogit wg), this thread's columns; the token's dg
-    if (valid) {
-      float* dqrow = dq + (((size_t)b * dm.N + n) * dm.H + h) * D;
-#pragma unroll 4
-      for (int c = 0; c < QC; ++c) {
-        float acc = 0.f;
-#pragma unroll
-        for (int a = 0; a < RK; ++a) acc = fmaf(sW[(c0 + c) * (RK + 1) + a], sX[row * (RK + 1) + a], acc);
-        if (dm.gate_mode == ROLA_GATE_QPROJ) acc = fmaf(sdl[row], __ldg(g + (size_t)h * D + c0 + c), acc);
-        dqrow[c0 + c] = acc;
-      }
-      if (dm.gate_mode == ROLA_GATE_TOKEN && qt == 0) dg[((size_t)b * dm.N + n) * dm.H + h] = dgn;
+    // per row: dg = y . T / den, the gain, g / den, dden = -g dg / den, dlogit
+    if (tid < 64) {
+      const int n = n0 + tid;
+      const bool valid = n < n_end;
+      const float den = sden[tid];
+      float dgn = 0.f;
+      for (int a = 0; a < RK; ++a) dgn = fmaf(sY[tid * WS + a], sT[tid * WS + a], dgn);
+      dgn = valid ? dgn / den : 0.f;
+      const float gn = qproj ? gate_sigmoid(dm, g, h, sdot[tid]) : g[gain_index(dm, b, valid ? n : n_begin, h)];
+      sdg[tid] = dgn;
+      sgd[tid] = valid ? gn / den : 0.f;
+      sdd[tid] = -gn * dgn / den;
+      sdl[tid] = valid ? dgn * gn * (1.f - gn) : 0.f;
+      if (valid && dm.gate_mode == ROLA_GATE_TOKEN) dg[((size_t)b * dm.N + n) * dm.H + h] = dgn;
     }
-    // dS[a][c] += sum_rows y gG / den;  dWq[c][a] += sum_rows q dx  (c = pc, a from pa)
-    for (int rr = 0; rr < 64; ++rr) {
-      const float gq = sG[rr * (D + 1) + pc] * sgd[rr];
-      const float qv = sQ[rr * (D + 1) + pc];
-#pragma unroll
-      for (int x2 = 0; x2 < PT; ++x2) {
-        aS[x2] = fmaf(sY[rr * (RK + 1) + pa + x2], gq, aS[x2]);
-        aW[x2] = fmaf(qv, sX[rr * (RK + 1) + pa + x2], aW[x2]);
-      }
+    __syncthreads();
+    // dy = (g / den) T, du = R^T dy + dden z, dx = phi'(x) du (one rank pair per item)
+    for (int e = tid; e < 64 * (RK / 2); e += kT) {
+      const int m = e / (RK / 2), p = e % (RK / 2);
+      const float2 cs = pair_cs(dm, rope, n0 + m, p);
+      const float gd = sgd[m], dd = sdd[m];
+      const float y0 = gd * sT[m * WS + 2 * p], y1 = gd * sT[m * WS + 2 * p + 1];
+      const float u0 = cs.x * y0 + cs.y * y1 + dd * sz[2 * p];
+      const float u1 = -cs.y * y0 + cs.x * y1 + dd * sz[2 * p + 1];
+      const bool valid = n0 + m < n_end;
+      sX[m * WS + 2 * p] = valid ? dphi_f(sX[m * WS + 2 * p]) * u0 : 0.f;
+      sX[m * WS + 2 * p + 1] = valid ? dphi_f(sX[m * WS + 2 * p + 1]) * u1 : 0.f;
     }
-    if (tid < D)
-      for (int rr = 0; rr < 64; ++rr) awg = fmaf(sdl[rr], sQ[rr * (D + 1) + tid], awg);
+    __syncthreads();
+    // dq = dx Wq^T (+ dlogit wg) for the valid rows
+    {
+      float aq[QP][4][4];
+      zero_acc(aq);
+      tile_gemm<64, D, RK>(aq, [&](int m, int a) { return sX[m * WS + a]; }, [&](int a, int c) { return sW[c * WS + a]; });
+      tile_each<64, D>(aq, [&](int m, int c, float x) {
+        const int n = n0 + m;
+        if (n < n_end) {
+          if (qproj) x = fmaf(sdl[m], __ldg(g + (size_t)h * D + c), x);
+          dq[(((size_t)b * dm.N + n) * dm.H + h) * D + c] = x;
+        }
+      });
+    }
+    // dS += y^T (G g / den), dWq += Q^T dx, dz += dden u, the gains' sums (rows in order)
+    tile_gemm<RK, D, 64>(aS, [&](int a, int m) { return sY[m * WS + a]; },
+                         [&](int m, int c) { return sG[m * TS + c] * sgd[m]; });
+    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return sQ[m * TS + c]; }, [&](int m, int a) { return sX[m * WS + a]; });
+    if (tid < RK)
+      for (int m = 0; m < 64; ++m) az = fmaf(sdd[m], sU[m * WS + tid], az);
+    if (qproj && tid < D)
+      for (int m = 0; m < 64; ++m) awg = fmaf(sdl[m], sQ[m * TS + tid], awg);
     if (tid == 0)
-      for (int rr = 0; rr < 64; ++rr) {
-        adg += sdg[rr];
-        abg += sdl[rr];
+      for (int m = 0; m < 64; ++m) {
+        adg += sdg[m];
+        abg += sdl[m];
       }
   }
-  // the chunk's partials: dS, dWq (fixed per thread), dz (rows summed in order), gain
   const size_t pbase = (size_t)bh * dm.nchunk + chunk;
-#pragma unroll
-  for (int x2 = 0; x2 < PT; ++x2) {
-    dS_part[pbase * RK * D + (size_t)(pa + x2) * D + pc] = aS[x2];
-    dWq_part[pbase * D * RK + (size_t)pc * RK + pa + x2] = aW[x2];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int a = 0; a < QR; ++a) sZr[row * (RK + 1) + a0 + a] = aZ[a];
-  __syncthreads();
-  if (tid < RK) {
-    float acc = 0.f;
-    for (int rr = 0; rr < 64; ++rr) acc += sZr[rr * (RK + 1) + tid];
-    dz_part[pbase * RK + tid] = acc;
-  }
+  tile_each<RK, D>(aS, [&](int a, int c, float x) { dS_part[pbase * RK * D + (size_t)a * D + c] = x; });
+  tile_each<D, RK>(aW, [&](int c, int a, float x) { dWq_part[pbase * D * RK + (size_t)c * RK + a] = x; });
+  if (tid < RK) dz_part[pbase * RK + tid] = az;
   float* gp = dg_part + pbase * (D + 1);
-  if (dm.gate_mode == ROLA_GATE_QPROJ) {
+  if (qproj) {
     if (tid < D) gp[tid] = awg;
     if (tid == 0) gp[D] = abg;
   } else if (tid == 0) {
@@ -598,7 +924,8 @@ __global__ void __launch_bounds__(kT) bwd_state_grad_reduce_kernel(Dims dm, cons
 }
 
 // Key side: per chunk of key tokens, the linear branch's dk and dv (written; the sparse
-// parts are added later) and the chunk's partial dWk.
+// parts are added later) and the chunk's partial dWk.  With Tk = V dS^T:
+// dv = (R f) dS, df = R^T Tk + dz, dw = phi'(w) df, dk = dw Wk^T, dWk += K^T dw.
 template <typename T, int D, int RK>
 __global__ void __launch_bounds__(kT) bwd_linear_key_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                                             const T* __restrict__ Wk, Dims dm,
@@ -606,82 +933,71 @@ __global__ void __launch_bounds__(kT) bwd_linear_key_kernel(const T* __restrict_
                                                             const float2* __restrict__ rope, float* __restrict__ dk,
                                                             float* __restrict__ dv, float* __restrict__ dWk_part) {
   using Lsm = LinSmem<D, RK>;
-  constexpr int QR = RK / 4, QC = D / 4, PT = D * RK / kT;
+  constexpr int WS = RK + 1, TS = D + 1;
   extern __shared__ float sm[];
   float* sK = sm;
   float* sV = sK + Lsm::kTile;
   float* sW = sV + Lsm::kTile;        // Wk [D][RK + 1]
   float* sS = sW + Lsm::kW;           // dS [RK][D + 1]
-  float* sY = sS + Lsm::kS;           // R f [64][RK + 1]
-  float* sX = sY + Lsm::kR;           // dw [64][RK + 1]
-  float* sz = sX + 2 * Lsm::kR;       // dz [RK]
+  float* sX = sS + Lsm::kS;           // w, then dw [64][RK + 1]
+  float* sY = sX + Lsm::kR;           // R f
+  float* sT = sY + Lsm::kR;           // V dS^T
+  float* sz = sT + 2 * Lsm::kR;       // dz [RK]
   const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
-  const int tid = threadIdx.x, row = tid >> 2, qt = tid & 3, a0 = qt * QR, c0 = qt * QC;
+  const int tid = threadIdx.x;
   const int n_begin = chunk * dm.chunk_tok, n_end = min(dm.N, n_begin + dm.chunk_tok);
-  for (int e = tid; e < D * RK; e += kT) sW[(e / RK) * (RK + 1) + e % RK] = to_f(Wk[(size_t)h * D * RK + e]);
-  for (int e = tid; e < RK * D; e += kT) sS[(e / D) * (D + 1) + e % D] = dS[(size_t)bh * RK * D + e];
+  for (int e = tid; e < D * RK; e += kT) sW[(e / RK) * WS + e % RK] = to_f(Wk[(size_t)h * D * RK + e]);
+  for (int e = tid; e < RK * D; e += kT) sS[(e / D) * TS + e % D] = dS[(size_t)bh * RK * D + e];
   if (tid < RK) sz[tid] = dz[(size_t)bh * RK + tid];
-  const int pc = tid % D, pa = (tid / D) * PT;
-  float aW[PT];
-#pragma unroll
-  for (int x2 = 0; x2 < PT; ++x2) aW[x2] = 0.f;
+  constexpr int WP = tiles_per_thread<D, RK>(), XP = tiles_per_thread<64, RK>(), QP = tiles_per_thread<64, D>();
+  float aW[WP][4][4];
+  zero_acc(aW);
   for (int n0 = n_begin; n0 < n_end; n0 += 64) {
     __syncthreads();
     load_tile<T, D>(sK, k, dm, b, h, n0);
     load_tile<T, D>(sV, v, dm, b, h, n0);
     __syncthreads();
-    const int n = n0 + row;
-    const bool valid = n < n_end;
-    float w[QR], f[QR], y[QR];
-#pragma unroll
-    for (int a = 0; a < QR; ++a) w[a] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float kv = sK[row * (D + 1) + c];
-#pragma unroll
-      for (int a = 0; a < QR; ++a) w[a] = fmaf(kv, sW[c * (RK + 1) + a0 + a], w[a]);
+    {
+      float ax[XP][4][4], at[XP][4][4];
+      zero_acc(ax);
+      zero_acc(at);
+      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return sK[m * TS + c]; }, [&](int c, int a) { return sW[c * WS + a]; });
+      tile_gemm<64, RK, D>(at, [&](int m, int c) { return sV[m * TS + c]; }, [&](int c, int a) { return sS[a * TS + c]; });
+      tile_each<64, RK>(ax, [&](int m, int a, float x) { sX[m * WS + a] = x; });
+      tile_each<64, RK>(at, [&](int m, int a, float x) { sT[m * WS + a] = x; });
     }
-#pragma unroll
-    for (int a = 0; a < QR; ++a) f[a] = phi_f(w[a]);
-    rotate_q<QR>(dm, rope, n, a0, f, y, false);
-#pragma unroll
-    for (int a = 0; a < QR; ++a) sY[row * (RK + 1) + a0 + a] = y[a];
-    // R^T (dS v) + dz on this thread's ranks
-    float dyk[QR];
-#pragma unroll
-    for (int a = 0; a < QR; ++a) dyk[a] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float vv = sV[row * (D + 1) + c];
-#pragma unroll
-      for (int a = 0; a < QR; ++a) dyk[a] = fmaf(sS[(a0 + a) * (D + 1) + c], vv, dyk[a]);
-    }
-    float df[QR];
-    rotate_q<QR>(dm, rope, n, a0, dyk, df, true);
-#pragma unroll
-    for (int a = 0; a < QR; ++a) sX[row * (RK + 1) + a0 + a] = valid ? dphi_f(w[a]) * (df[a] + sz[a0 + a]) : 0.f;
     __syncthreads();
-    if (valid) {
-      const size_t at = (((size_t)b * dm.N + n) * dm.H + h) * D;
-#pragma unroll 4
-      for (int c = 0; c < QC; ++c) {
-        float av = 0.f, ak = 0.f;
-#pragma unroll
-        for (int a = 0; a < RK; ++a) {
-          av = fmaf(sY[row * (RK + 1) + a], sS[a * (D + 1) + c0 + c], av);
-          ak = fmaf(sW[(c0 + c) * (RK + 1) + a], sX[row * (RK + 1) + a], ak);
-        }
-        dv[at + c0 + c] = av;
-        dk[at + c0 + c] = ak;
-      }
+    // R f and dw = phi'(w) (R^T Tk + dz), one rank pair per item
+    for (int e = tid; e < 64 * (RK / 2); e += kT) {
+      const int m = e / (RK / 2), p = e % (RK / 2);
+      const float2 cs = pair_cs(dm, rope, n0 + m, p);
+      const float w0 = sX[m * WS + 2 * p], w1 = sX[m * WS + 2 * p + 1];
+      const float f0 = phi_f(w0), f1 = phi_f(w1);
+      sY[m * WS + 2 * p] = cs.x * f0 - cs.y * f1;
+      sY[m * WS + 2 * p + 1] = cs.y * f0 + cs.x * f1;
+      const float t0 = sT[m * WS + 2 * p], t1 = sT[m * WS + 2 * p + 1];
+      const bool valid = n0 + m < n_end;
+      sX[m * WS + 2 * p] = valid ? dphi_f(w0) * (cs.x * t0 + cs.y * t1 + sz[2 * p]) : 0.f;
+      sX[m * WS + 2 * p + 1] = valid ? dphi_f(w1) * (-cs.y * t0 + cs.x * t1 + sz[2 * p + 1]) : 0.f;
     }
-    for (int rr = 0; rr < 64; ++rr) {
-      const float kv = sK[rr * (D + 1) + pc];
-#pragma unroll
-      for (int x2 = 0; x2 < PT; ++x2) aW[x2] = fmaf(kv, sX[rr * (RK + 1) + pa + x2], aW[x2]);
+    __syncthreads();
+    {
+      float avv[QP][4][4], akk[QP][4][4];
+      zero_acc(avv);
+      zero_acc(akk);
+      tile_gemm<64, D, RK>(avv, [&](int m, int a) { return sY[m * WS + a]; }, [&](int a, int c) { return sS[a * TS + c]; });
+      tile_gemm<64, D, RK>(akk, [&](int m, int a) { return sX[m * WS + a]; }, [&](int a, int c) { return sW[c * WS + a]; });
+      tile_each<64, D>(avv, [&](int m, int c, float x) {
+        if (n0 + m < n_end) dv[(((size_t)b * dm.N + n0 + m) * dm.H + h) * D + c] = x;
+      });
+      tile_each<64, D>(akk, [&](int m, int c, float x) {
+        if (n0 + m < n_end) dk[(((size_t)b * dm.N + n0 + m) * dm.H + h) * D + c] = x;
+      });
     }
+    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return sK[m * TS + c]; }, [&](int m, int a) { return sX[m * WS + a]; });
   }
   const size_t pbase = (size_t)bh * dm.nchunk + chunk;
-#pragma unroll
-  for (int x2 = 0; x2 < PT; ++x2) dWk_part[pbase * D * RK + (size_t)pc * RK + pa + x2] = aW[x2];
+  tile_each<D, RK>(aW, [&](int c, int a, float x) { dWk_part[pbase * D * RK + (size_t)c * RK + a] = x; });
 }
 
 // Per head: dWq, dWk and the per-head gain gradients summed over the batch and the chunks
@@ -737,12 +1053,6 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
                                 (int)lin_smem)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(bwd_linear_key_kernel<T, D, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)lin_smem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(bwd_rowstats_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)rs_smem)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(bwd_dq_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem)) !=
-          cudaSuccess ||
-      (e = cudaFuncSetAttribute(bwd_dkv_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)dkv_smem)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(bwd_inverse_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(sizeof(int) * (dm.nb + 1)))) != cudaSuccess)
     return e;
@@ -759,16 +1069,43 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_head_reduce_kernel<D, RK><<<dm.H, kT, 0, st>>>(dm, bw.dWq_part, bw.dWk_part, bw.dg_part, dWq, dWk, dg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // sparse branch
-  bwd_rowstats_kernel<T, D><<<gtile, kT, rs_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, ws.status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // sparse branch: row statistics, the key-major lists, dq, then dk and dv
   bwd_inverse_lists_kernel<<<BH, kT, sizeof(int) * (dm.nb + 1), st>>>(dm, ws.col_idx, bw.inv_off, bw.inv_idx);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_dq_kernel<T, D><<<gtile, kT, dq_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, dq, ws.status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_dkv_kernel<T, D><<<gtile, kT, dkv_smem, st>>>(q, k, v, dout, dm, bw.inv_off, bw.inv_idx, bw.lse, bw.Drow, dk,
-                                                     dv);
-  return cudaGetLastError();
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    constexpr size_t mm_smem = MmaTiles<D>::bytes;
+    if ((e = cudaFuncSetAttribute(bwd_rowstats_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)mm_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_dq_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)mm_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_dkv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)mm_smem)) != cudaSuccess)
+      return e;
+    bwd_rowstats_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow,
+                                                            ws.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_dq_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, dq, ws.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_dkv_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, bw.inv_off, bw.inv_idx, bw.lse, bw.Drow,
+                                                       dk, dv);
+    return cudaGetLastError();
+  } else {
+    if ((e = cudaFuncSetAttribute(bwd_rowstats_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)rs_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_dq_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)dq_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(bwd_dkv_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)dkv_smem)) != cudaSuccess)
+      return e;
+    bwd_rowstats_kernel<T, D><<<gtile, kT, rs_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow,
+                                                          ws.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_dq_kernel<T, D><<<gtile, kT, dq_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, dq, ws.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_dkv_kernel<T, D><<<gtile, kT, dkv_smem, st>>>(q, k, v, dout, dm, bw.inv_off, bw.inv_idx, bw.lse, bw.Drow,
+                                                       dk, dv);
+    return cudaGetLastError();
+  }
 }
 
 template <typename T>
