@@ -413,6 +413,9 @@ __device__ __forceinline__ void mma_rows_xb(float (&acc)[D / 8][4], const float 
   }
 }
 
+// Row statistics on the tensor cores.  D_n = dout_n . O_n = sum_m P_nm (dout_n . v_m), so the
+// row's D is accumulated online like its softmax sum, from dP = dout V^T (one exact bf16
+// product per block) instead of forming O.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -424,18 +427,16 @@ __global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
   __nv_bfloat16* sG = sQ + L::kTile;
   __nv_bfloat16* sK = sG + L::kTile;
   __nv_bfloat16* sV = sK + L::kTile;
-  const int i = blockIdx.x, bh = blockIdx.y, b = bh / dm.H, h = bh % dm.H;
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / dm.H, h = bh % dm.H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int32_t* Lst = col_idx + ((size_t)bh * dm.nb + i) * dm.k;
   const float sl2 = dm.scale * 1.4426950408889634f;
   load_tile_bf16<D>(sQ, q, dm, b, h, i * 64);
   load_tile_bf16<D>(sG, dout, dm, b, h, i * 64);
   cp_async_commit();
-  float o[D / 8][4], m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-#pragma unroll
-  for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  // per row half hh: running max m (log2 units), sum l and sum of p dP (this thread's columns)
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, pd[2] = {0.f, 0.f};
   for (int jj = 0; jj < dm.k; ++jj) {
     const int j = checked_block(dm, Lst[jj], status);
     __syncthreads();
@@ -444,8 +445,9 @@ __global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    float s[8][4];
+    float s[8][4], dp[8][4];
     mma_rows_abt<D>(s, sQ, sK, warp, lane);
+    mma_rows_abt<D>(dp, sG, sV, warp, lane);
     const int nvalid = min(64, dm.N - j * 64);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -461,42 +463,32 @@ __global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float mnew = fmaxf(m[hh], mx);
       const float corr = m[hh] == -INFINITY ? 0.f : exp2f(m[hh] - mnew);
-      float rs = 0.f;
+      float rs = 0.f, rd = 0.f;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e = 2 * hh; e < 2 * hh + 2; ++e) {
-          s[nt][e] = exp2f(s[nt][e] - mnew);
-          rs += s[nt][e];
+          const float p = exp2f(s[nt][e] - mnew);
+          rs += p;
+          rd = fmaf(p, dp[nt][e], rd);
         }
       l[hh] = l[hh] * corr + rs;
+      pd[hh] = pd[hh] * corr + rd;
       m[hh] = mnew;
-#pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        o[nt][2 * hh] *= corr;
-        o[nt][2 * hh + 1] *= corr;
-      }
     }
-    mma_rows_xb<D>(o, s, sV, lane);
   }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
-    float lt = l[hh];
+    float lt = l[hh], dt = pd[hh];
     lt += __shfl_xor_sync(0xffffffffu, lt, 1);
     lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+    dt += __shfl_xor_sync(0xffffffffu, dt, 1);
+    dt += __shfl_xor_sync(0xffffffffu, dt, 2);
     const int row = 16 * warp + g8 + 8 * hh, n = i * 64 + row;
-    float dsum = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-      for (int e = 2 * hh; e < 2 * hh + 2; ++e)
-        dsum = fmaf(__bfloat162float(sG[row * (D + 8) + nt * 8 + 2 * t4 + (e & 1)]), o[nt][e] / lt, dsum);
-    dsum += __shfl_xor_sync(0xffffffffu, dsum, 1);
-    dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
     if (t4 == 0) {
       const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + row;
       lse[at] = n < dm.N ? m[hh] + log2f(lt) : INFINITY;   // log2 units of scale * log2(e) * q.k
-      Drow[at] = n < dm.N ? dsum : 0.f;
+      Drow[at] = n < dm.N ? dt / lt : 0.f;
     }
   }
 }
@@ -688,14 +680,33 @@ __global__ void __launch_bounds__(kT) bwd_inverse_lists_kernel(Dims dm, const in
 // register tiles per thread over shared-memory operands (tile t = tid + 256 s: rows
 // 4 (t / NT) .. + 3, columns t % NT + NT j), the per-row steps (phi, the rotation, the
 // normaliser, the gain) one row or one rank pair per thread.
-template <int D, int RK>
+// The two token tiles stay in the inputs' type (bf16 rows padded by 2 elements, fp32 by 1),
+// so that two CTAs fit an SM; everything else is fp32.
+template <typename T, int D, int RK>
 struct LinSmem {
-  static constexpr int kTile = 64 * (D + 1);
+  static constexpr int TT = D + (sizeof(T) == 2 ? 2 : 1);                       // tile row stride
+  static constexpr size_t kTileBytes = (sizeof(T) * 64 * TT + 15) / 16 * 16;
   static constexpr int kW = D * (RK + 1);      // Wq or Wk [D][RK]
   static constexpr int kS = RK * (D + 1);      // S or dS [RK][D]
   static constexpr int kR = 64 * (RK + 1);     // [64][RK] row vectors
-  static constexpr size_t bytes = sizeof(float) * (2 * kTile + kW + kS + 4 * kR + RK + 6 * 64);
+  static constexpr size_t bytes = 2 * kTileBytes + sizeof(float) * (kW + kS + 4 * kR + RK + 6 * 64);
 };
+
+// rows [n0, n0 + 64) of head h of a [B, N, H, D] tensor into s[64][TT] in its own type, by
+// 16-byte loads; rows at or past N are zero
+template <typename T, int D, int TT>
+__device__ __forceinline__ void load_tile_t(T* s, const T* __restrict__ x, const Dims& dm, int b, int h, int n0) {
+  constexpr int EV = 16 / sizeof(T);           // elements per 16-byte load
+  for (int e = threadIdx.x; e < 64 * (D / EV); e += kT) {
+    const int r = e / (D / EV), c = (e % (D / EV)) * EV, n = n0 + r;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (n < dm.N) val = *reinterpret_cast<const uint4*>(x + (((size_t)b * dm.N + n) * dm.H + h) * D + c);
+    const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+    uint32_t* dst = reinterpret_cast<uint32_t*>(s + r * TT + c);   // 4-byte aligned for both types
+#pragma unroll
+    for (int u = 0; u < 4; ++u) dst[u] = w[u];
+  }
+}
 
 // acc[s][i][j] += sum_k a(m, k) b(k, n) for the tiles of this thread of an M x N product
 // (m = 4 (t / NT) + i, n = t % NT + NT j).
@@ -761,17 +772,17 @@ __device__ __forceinline__ float2 pair_cs(const Dims& dm, const float2* __restri
 // (the row's dout against each rank of the state), dg = y . T / den and dy = g T / den, so
 // the linear output itself is never formed.
 template <typename T, int D, int RK>
-__global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
+__global__ void __launch_bounds__(kT, 2) bwd_linear_query_kernel(
     const T* __restrict__ q, const T* __restrict__ dout, const T* __restrict__ Wq, const float* __restrict__ g,
     Dims dm, const float* __restrict__ S, const float* __restrict__ z, const float2* __restrict__ rope,
     float* __restrict__ dq, float* __restrict__ dg, float* __restrict__ dS_part, float* __restrict__ dz_part,
     float* __restrict__ dWq_part, float* __restrict__ dg_part) {
-  using Lsm = LinSmem<D, RK>;
-  constexpr int WS = RK + 1, TS = D + 1;
-  extern __shared__ float sm[];
-  float* sQ = sm;
-  float* sG = sQ + Lsm::kTile;
-  float* sW = sG + Lsm::kTile;        // Wq [D][RK + 1]
+  using Lsm = LinSmem<T, D, RK>;
+  constexpr int WS = RK + 1, TS = D + 1, TT = Lsm::TT;
+  extern __shared__ __align__(16) unsigned char smraw[];
+  T* sQ = reinterpret_cast<T*>(smraw);
+  T* sG = reinterpret_cast<T*>(smraw + Lsm::kTileBytes);
+  float* sW = reinterpret_cast<float*>(smraw + 2 * Lsm::kTileBytes);   // Wq [D][RK + 1]
   float* sS = sW + Lsm::kW;           // S [RK][D + 1]
   float* sX = sS + Lsm::kS;           // x, then dx [64][RK + 1]
   float* sU = sX + Lsm::kR;           // u
@@ -799,16 +810,16 @@ __global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
   float az = 0.f, awg = 0.f, adg = 0.f, abg = 0.f;   // rank tid (dz), channel tid (dwg), sums
   for (int n0 = n_begin; n0 < n_end; n0 += 64) {
     __syncthreads();
-    load_tile<T, D>(sQ, q, dm, b, h, n0);
-    load_tile<T, D>(sG, dout, dm, b, h, n0);
+    load_tile_t<T, D, TT>(sQ, q, dm, b, h, n0);
+    load_tile_t<T, D, TT>(sG, dout, dm, b, h, n0);
     __syncthreads();
     // x = q Wq and T = G S^T
     {
       float ax[XP][4][4], at[XP][4][4];
       zero_acc(ax);
       zero_acc(at);
-      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return sQ[m * TS + c]; }, [&](int c, int a) { return sW[c * WS + a]; });
-      tile_gemm<64, RK, D>(at, [&](int m, int c) { return sG[m * TS + c]; }, [&](int c, int a) { return sS[a * TS + c]; });
+      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return to_f(sQ[m * TT + c]); }, [&](int c, int a) { return sW[c * WS + a]; });
+      tile_gemm<64, RK, D>(at, [&](int m, int c) { return to_f(sG[m * TT + c]); }, [&](int c, int a) { return sS[a * TS + c]; });
       tile_each<64, RK>(ax, [&](int m, int a, float x) {
         sX[m * WS + a] = x;
         sU[m * WS + a] = phi_f(x);
@@ -817,7 +828,7 @@ __global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
     }
     if (qproj && tid < 64) {
       float dot = 0.f;
-      for (int c = 0; c < D; ++c) dot = fmaf(sQ[tid * TS + c], __ldg(g + (size_t)h * D + c), dot);
+      for (int c = 0; c < D; ++c) dot = fmaf(to_f(sQ[tid * TT + c]), __ldg(g + (size_t)h * D + c), dot);
       sdot[tid] = dot;
     }
     __syncthreads();
@@ -879,12 +890,12 @@ __global__ void __launch_bounds__(kT) bwd_linear_query_kernel(
     }
     // dS += y^T (G g / den), dWq += Q^T dx, dz += dden u, the gains' sums (rows in order)
     tile_gemm<RK, D, 64>(aS, [&](int a, int m) { return sY[m * WS + a]; },
-                         [&](int m, int c) { return sG[m * TS + c] * sgd[m]; });
-    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return sQ[m * TS + c]; }, [&](int m, int a) { return sX[m * WS + a]; });
+                         [&](int m, int c) { return to_f(sG[m * TT + c]) * sgd[m]; });
+    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return to_f(sQ[m * TT + c]); }, [&](int m, int a) { return sX[m * WS + a]; });
     if (tid < RK)
       for (int m = 0; m < 64; ++m) az = fmaf(sdd[m], sU[m * WS + tid], az);
     if (qproj && tid < D)
-      for (int m = 0; m < 64; ++m) awg = fmaf(sdl[m], sQ[m * TS + tid], awg);
+      for (int m = 0; m < 64; ++m) awg = fmaf(sdl[m], to_f(sQ[m * TT + tid]), awg);
     if (tid == 0)
       for (int m = 0; m < 64; ++m) {
         adg += sdg[m];
@@ -927,17 +938,17 @@ __global__ void __launch_bounds__(kT) bwd_state_grad_reduce_kernel(Dims dm, cons
 // parts are added later) and the chunk's partial dWk.  With Tk = V dS^T:
 // dv = (R f) dS, df = R^T Tk + dz, dw = phi'(w) df, dk = dw Wk^T, dWk += K^T dw.
 template <typename T, int D, int RK>
-__global__ void __launch_bounds__(kT) bwd_linear_key_kernel(const T* __restrict__ k, const T* __restrict__ v,
+__global__ void __launch_bounds__(kT, 2) bwd_linear_key_kernel(const T* __restrict__ k, const T* __restrict__ v,
                                                             const T* __restrict__ Wk, Dims dm,
                                                             const float* __restrict__ dS, const float* __restrict__ dz,
                                                             const float2* __restrict__ rope, float* __restrict__ dk,
                                                             float* __restrict__ dv, float* __restrict__ dWk_part) {
-  using Lsm = LinSmem<D, RK>;
-  constexpr int WS = RK + 1, TS = D + 1;
-  extern __shared__ float sm[];
-  float* sK = sm;
-  float* sV = sK + Lsm::kTile;
-  float* sW = sV + Lsm::kTile;        // Wk [D][RK + 1]
+  using Lsm = LinSmem<T, D, RK>;
+  constexpr int WS = RK + 1, TS = D + 1, TT = Lsm::TT;
+  extern __shared__ __align__(16) unsigned char smraw[];
+  T* sK = reinterpret_cast<T*>(smraw);
+  T* sV = reinterpret_cast<T*>(smraw + Lsm::kTileBytes);
+  float* sW = reinterpret_cast<float*>(smraw + 2 * Lsm::kTileBytes);   // Wk [D][RK + 1]
   float* sS = sW + Lsm::kW;           // dS [RK][D + 1]
   float* sX = sS + Lsm::kS;           // w, then dw [64][RK + 1]
   float* sY = sX + Lsm::kR;           // R f
@@ -954,15 +965,15 @@ __global__ void __launch_bounds__(kT) bwd_linear_key_kernel(const T* __restrict_
   zero_acc(aW);
   for (int n0 = n_begin; n0 < n_end; n0 += 64) {
     __syncthreads();
-    load_tile<T, D>(sK, k, dm, b, h, n0);
-    load_tile<T, D>(sV, v, dm, b, h, n0);
+    load_tile_t<T, D, TT>(sK, k, dm, b, h, n0);
+    load_tile_t<T, D, TT>(sV, v, dm, b, h, n0);
     __syncthreads();
     {
       float ax[XP][4][4], at[XP][4][4];
       zero_acc(ax);
       zero_acc(at);
-      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return sK[m * TS + c]; }, [&](int c, int a) { return sW[c * WS + a]; });
-      tile_gemm<64, RK, D>(at, [&](int m, int c) { return sV[m * TS + c]; }, [&](int c, int a) { return sS[a * TS + c]; });
+      tile_gemm<64, RK, D>(ax, [&](int m, int c) { return to_f(sK[m * TT + c]); }, [&](int c, int a) { return sW[c * WS + a]; });
+      tile_gemm<64, RK, D>(at, [&](int m, int c) { return to_f(sV[m * TT + c]); }, [&](int c, int a) { return sS[a * TS + c]; });
       tile_each<64, RK>(ax, [&](int m, int a, float x) { sX[m * WS + a] = x; });
       tile_each<64, RK>(at, [&](int m, int a, float x) { sT[m * WS + a] = x; });
     }
@@ -994,7 +1005,7 @@ __global__ void __launch_bounds__(kT) bwd_linear_key_kernel(const T* __restrict_
         if (n0 + m < n_end) dk[(((size_t)b * dm.N + n0 + m) * dm.H + h) * D + c] = x;
       });
     }
-    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return sK[m * TS + c]; }, [&](int m, int a) { return sX[m * WS + a]; });
+    tile_gemm<D, RK, 64>(aW, [&](int c, int m) { return to_f(sK[m * TT + c]); }, [&](int m, int a) { return sX[m * WS + a]; });
   }
   const size_t pbase = (size_t)bh * dm.nchunk + chunk;
   tile_each<D, RK>(aW, [&](int c, int a, float x) { dWk_part[pbase * D * RK + (size_t)c * RK + a] = x; });
@@ -1046,7 +1057,7 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
   const T* dout = static_cast<const T*>(dout_);
   const int BH = dm.B * dm.H;
   cudaError_t e;
-  constexpr size_t lin_smem = LinSmem<D, RK>::bytes;
+  constexpr size_t lin_smem = LinSmem<T, D, RK>::bytes;
   constexpr size_t tile = sizeof(float) * 64 * (D + 1), ptile = sizeof(float) * 64 * 65;
   constexpr size_t rs_smem = 3 * tile + ptile, dq_smem = 4 * tile + ptile, dkv_smem = 4 * tile + 2 * ptile + 128 * 4;
   if ((e = cudaFuncSetAttribute(bwd_linear_query_kernel<T, D, RK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
