@@ -74,6 +74,8 @@ def _load():
             lib.rola_oracle_e4m3_decode.argtypes = [P, P, ctypes.c_size_t]
             lib.rola_oracle_quantize_blocks.argtypes = [sp, P, P, P]
             lib.rola_oracle_backward.argtypes = [sp] + [P] * 14
+            lib.rola_oracle_backward_sample.argtypes = ([sp] + [P] * 8 + [ctypes.c_int, P, ctypes.c_int, P,
+                                                        ctypes.c_int, P] + [P] * 6)
             _lib = lib
     return _lib
 
@@ -262,4 +264,29 @@ def backward(s: Shape, q, k, v, Wq, Wk, g, dout, col_idx):
     _load().rola_oracle_backward(ctypes.byref(s), _p(q), _p(k), _p(v), _p(Wq), _p(Wk), _p(g), _p(dout),
                                  _p(col_idx), _p(res["dq"]), _p(res["dk"]), _p(res["dv"]), _p(res["dWq"]),
                                  _p(res["dWk"]), _p(res["dg"]))
+    return res
+
+
+def backward_sample(s: Shape, q, k, v, Wq, Wk, g, dout, col_idx, heads, qblocks, kblocks):
+    """The backward on a sample (per-head gain only): for the listed heads their dWq, dWk, dg
+    (summed over the batch), and for the listed (b, h, i) blocks the 64 rows of dq (qblocks)
+    or of dk, dv (kblocks); every listed block's head must be in ``heads``.
+
+    Returns a dict of float64 arrays: dq [nq, 64, d]; dk, dv [nk, 64, d]; dWq, dWk [nh, d, r];
+    dg [nh]."""
+    assert s.gate_mode == 0
+    q, k, v, Wq, Wk = _f32(q), _f32(k), _f32(v), _f32(Wq), _f32(Wk)
+    g = _gain(s, g)
+    dout = _f64(dout)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    heads = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    qb = np.ascontiguousarray(np.asarray(qblocks, dtype=np.int32).reshape(-1, 3))
+    kb = np.ascontiguousarray(np.asarray(kblocks, dtype=np.int32).reshape(-1, 3))
+    assert set(qb[:, 1]) | set(kb[:, 1]) <= set(heads.tolist())
+    nh, nq, nk = heads.size, qb.shape[0], kb.shape[0]
+    res = {"dq": np.zeros((nq, BLOCK, s.d)), "dk": np.zeros((nk, BLOCK, s.d)), "dv": np.zeros((nk, BLOCK, s.d)),
+           "dWq": np.zeros((nh, s.d, s.r)), "dWk": np.zeros((nh, s.d, s.r)), "dg": np.zeros(nh)}
+    _load().rola_oracle_backward_sample(ctypes.byref(s), _p(q), _p(k), _p(v), _p(Wq), _p(Wk), _p(g), _p(dout),
+                                        _p(col_idx), nh, _p(heads), nq, _p(qb), nk, _p(kb), _p(res["dq"]),
+                                        _p(res["dk"]), _p(res["dv"]), _p(res["dWq"]), _p(res["dWk"]), _p(res["dg"]))
     return res

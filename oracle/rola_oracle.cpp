@@ -640,6 +640,210 @@ void rola_oracle_backward(const rola_oracle_shape* s, const float* q, const floa
     }
 }
 
+// The same gradients on a sample, for problems too large for the whole backward: for the
+// listed heads h (all batch entries) the per-head dWq[h], dWk[h] and dg[h] (gate_mode 0
+// only), and for the listed blocks (b, h, i) the 64 rows of dq (qblocks) or of dk, dv
+// (kblocks).  Every listed block's head must be listed.  Same definition and arithmetic as
+// rola_oracle_backward, restricted to what the sample needs: the linear branch over all
+// tokens of the listed heads, the softmax of every query row that touches a listed block.
+// Outputs: dq [nq][64][d], dk, dv [nk][64][d] (rows past N zero), dWq, dWk [nh][d][r],
+// dg [nh].
+void rola_oracle_backward_sample(const rola_oracle_shape* s, const float* q, const float* k,
+                                 const float* v, const float* Wq, const float* Wk, const double* g,
+                                 const double* dout, const int32_t* col_idx, int nh, const int32_t* heads,
+                                 int nq, const int32_t* qblocks, int nk, const int32_t* kblocks,
+                                 double* dq, double* dk, double* dv, double* dWq, double* dWk, double* dg) {
+  const int B = s->B, H = s->H, N = s->N, d = s->d, r = s->r;
+  const int nb = rola_oracle_num_blocks(N);
+  const int kk = rola_oracle_keep_count(nb, s->topk);
+  std::vector<double> pos((size_t)N * 3);
+  rola_oracle_positions(s, pos.data());
+  std::fill(dq, dq + (size_t)nq * kBlock * d, 0.0);
+  std::fill(dk, dk + (size_t)nk * kBlock * d, 0.0);
+  std::fill(dv, dv + (size_t)nk * kBlock * d, 0.0);
+  std::fill(dWq, dWq + (size_t)nh * d * r, 0.0);
+  std::fill(dWk, dWk + (size_t)nh * d * r, 0.0);
+  std::fill(dg, dg + nh, 0.0);
+  auto at = [&](int b, int n, int h) { return (((size_t)b * N + n) * H + h) * d; };
+  // softmax row of query token n of (b, h): probabilities over its kept keys, and D_n
+  auto softmax_row = [&](int b, int h, int n, std::vector<int>& keys, std::vector<double>& P, double& Dn) {
+    const int i = n / kBlock;
+    const int32_t* Li = col_idx + (((size_t)b * H + h) * nb + i) * kk;
+    keys.clear();
+    for (int a = 0; a < kk; ++a)
+      for (int m = Li[a] * kBlock; m < std::min(N, (Li[a] + 1) * kBlock); ++m) keys.push_back(m);
+    P.resize(keys.size());
+    const float* qn = q + at(b, n, h);
+    double mx = -std::numeric_limits<double>::infinity();
+    for (size_t a = 0; a < keys.size(); ++a) {
+      const float* km = k + at(b, keys[a], h);
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += (double)qn[c] * (double)km[c];
+      P[a] = acc * s->scale;
+      mx = std::max(mx, P[a]);
+    }
+    double sum = 0.0;
+    for (size_t a = 0; a < keys.size(); ++a) {
+      P[a] = std::exp(P[a] - mx);
+      sum += P[a];
+    }
+    Dn = 0.0;
+    const double* G = dout + at(b, n, h);
+    for (size_t a = 0; a < keys.size(); ++a) {
+      P[a] /= sum;
+      const float* vm = v + at(b, keys[a], h);
+      double gv = 0.0;
+      for (int c = 0; c < d; ++c) gv += G[c] * (double)vm[c];
+      Dn += P[a] * gv;
+    }
+  };
+#pragma omp parallel for schedule(dynamic)
+  for (int t = 0; t < nh; ++t) {
+    const int h = heads[t];
+    std::vector<int> keys;
+    std::vector<double> P;
+    for (int b = 0; b < B; ++b) {
+      std::vector<double> w((size_t)N * r), yk((size_t)N * r), f(r);
+      std::vector<double> S((size_t)r * d, 0.0), z(r, 0.0), dS((size_t)r * d, 0.0), dz(r, 0.0);
+      for (int m = 0; m < N; ++m) {
+        const float* km = k + at(b, m, h);
+        const float* vm = v + at(b, m, h);
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += (double)km[c] * (double)Wk[((size_t)h * d + c) * r + a];
+          w[(size_t)m * r + a] = acc;
+          f[a] = phi(acc);
+        }
+        rotate(s, &pos[3 * (size_t)m], f.data(), &yk[(size_t)m * r]);
+        for (int a = 0; a < r; ++a) {
+          z[a] += f[a];
+          for (int c = 0; c < d; ++c) S[(size_t)a * d + c] += yk[(size_t)m * r + a] * (double)vm[c];
+        }
+      }
+      // linear branch, query side, every token of (b, h)
+      std::vector<double> x(r), u(r), yq(r), L(d), dy(r), du(r), dx(r);
+      for (int n = 0; n < N; ++n) {
+        const float* qn = q + at(b, n, h);
+        const double* G = dout + at(b, n, h);
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += (double)qn[c] * (double)Wq[((size_t)h * d + c) * r + a];
+          x[a] = acc;
+          u[a] = phi(acc);
+        }
+        rotate(s, &pos[3 * (size_t)n], u.data(), yq.data());
+        double den = 0.0;
+        for (int a = 0; a < r; ++a) den += u[a] * z[a];
+        double dgn = 0.0;
+        for (int c = 0; c < d; ++c) {
+          double num = 0.0;
+          for (int a = 0; a < r; ++a) num += yq[a] * S[(size_t)a * d + c];
+          L[c] = num / den;
+          dgn += G[c] * L[c];
+        }
+        const double gn = g[h];
+        dg[t] += dgn;
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) {
+            dS[(size_t)a * d + c] += yq[a] * gn * G[c] / den;
+            acc += S[(size_t)a * d + c] * gn * G[c];
+          }
+          dy[a] = acc / den;
+        }
+        const double dden = -gn * dgn / den;
+        rotate_back(s, &pos[3 * (size_t)n], dy.data(), du.data());
+        for (int a = 0; a < r; ++a) {
+          du[a] += dden * z[a];
+          dz[a] += dden * u[a];
+          dx[a] = phi_grad(x[a]) * du[a];
+        }
+        for (int c = 0; c < d; ++c)
+          for (int a = 0; a < r; ++a) dWq[((size_t)t * d + c) * r + a] += (double)qn[c] * dx[a];
+        for (int e = 0; e < nq; ++e)   // the listed query blocks' linear part of dq
+          if (qblocks[3 * e] == b && qblocks[3 * e + 1] == h && qblocks[3 * e + 2] == n / kBlock)
+            for (int c = 0; c < d; ++c) {
+              double acc = 0.0;
+              for (int a = 0; a < r; ++a) acc += (double)Wq[((size_t)h * d + c) * r + a] * dx[a];
+              dq[((size_t)e * kBlock + n % kBlock) * d + c] += acc;
+            }
+      }
+      // linear branch, key side, every key of (b, h)
+      std::vector<double> dyk(r), df(r);
+      for (int m = 0; m < N; ++m) {
+        const float* km = k + at(b, m, h);
+        const float* vm = v + at(b, m, h);
+        for (int a = 0; a < r; ++a) {
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += dS[(size_t)a * d + c] * (double)vm[c];
+          dyk[a] = acc;
+        }
+        rotate_back(s, &pos[3 * (size_t)m], dyk.data(), df.data());
+        for (int a = 0; a < r; ++a) df[a] = phi_grad(w[(size_t)m * r + a]) * (df[a] + dz[a]);
+        for (int c = 0; c < d; ++c)
+          for (int a = 0; a < r; ++a) dWk[((size_t)t * d + c) * r + a] += (double)km[c] * df[a];
+        for (int e = 0; e < nk; ++e)
+          if (kblocks[3 * e] == b && kblocks[3 * e + 1] == h && kblocks[3 * e + 2] == m / kBlock)
+            for (int c = 0; c < d; ++c) {
+              double ak = 0.0, av = 0.0;
+              for (int a = 0; a < r; ++a) {
+                ak += (double)Wk[((size_t)h * d + c) * r + a] * df[a];
+                av += dS[(size_t)a * d + c] * yk[(size_t)m * r + a];
+              }
+              dk[((size_t)e * kBlock + m % kBlock) * d + c] += ak;
+              dv[((size_t)e * kBlock + m % kBlock) * d + c] += av;
+            }
+      }
+      // sparse branch: dq of the listed query blocks
+      double Dn;
+      for (int e = 0; e < nq; ++e) {
+        if (qblocks[3 * e] != b || qblocks[3 * e + 1] != h) continue;
+        const int i = qblocks[3 * e + 2];
+        for (int n = i * kBlock; n < std::min(N, (i + 1) * kBlock); ++n) {
+          softmax_row(b, h, n, keys, P, Dn);
+          const double* G = dout + at(b, n, h);
+          for (size_t a = 0; a < keys.size(); ++a) {
+            const float* km = k + at(b, keys[a], h);
+            const float* vm = v + at(b, keys[a], h);
+            double dP = 0.0;
+            for (int c = 0; c < d; ++c) dP += G[c] * (double)vm[c];
+            const double dA = P[a] * (dP - Dn);
+            for (int c = 0; c < d; ++c) dq[((size_t)e * kBlock + n % kBlock) * d + c] += s->scale * dA * (double)km[c];
+          }
+        }
+      }
+      // sparse branch: dk, dv of the listed key blocks, over the query blocks that kept them
+      for (int e = 0; e < nk; ++e) {
+        if (kblocks[3 * e] != b || kblocks[3 * e + 1] != h) continue;
+        const int j = kblocks[3 * e + 2];
+        for (int i = 0; i < nb; ++i) {
+          const int32_t* Li = col_idx + (((size_t)b * H + h) * nb + i) * kk;
+          bool kept = false;
+          for (int a = 0; a < kk; ++a) kept |= Li[a] == j;
+          if (!kept) continue;
+          for (int n = i * kBlock; n < std::min(N, (i + 1) * kBlock); ++n) {
+            softmax_row(b, h, n, keys, P, Dn);
+            const float* qn = q + at(b, n, h);
+            const double* G = dout + at(b, n, h);
+            for (size_t a = 0; a < keys.size(); ++a) {
+              if (keys[a] / kBlock != j) continue;
+              const float* vm = v + at(b, keys[a], h);
+              double dP = 0.0;
+              for (int c = 0; c < d; ++c) dP += G[c] * (double)vm[c];
+              const double dA = P[a] * (dP - Dn);
+              const size_t row = (size_t)e * kBlock + keys[a] % kBlock;
+              for (int c = 0; c < d; ++c) {
+                dk[row * d + c] += s->scale * dA * (double)qn[c];
+                dv[row * d + c] += P[a] * G[c];
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 int rola_oracle_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -110,3 +110,39 @@ def test_backward_rejects_bad_calls():
     assert lib.rola_backward_workspace_size(rola.ctypes.byref(rola.Plan.for_workload(w8).params),
                                             rola.ctypes.byref(n)) == 2
     assert plan.poll_status() == 0
+
+
+@pytest.mark.parametrize("wname", ["wan21_14b_480p"])
+def test_backward_at_full_size_on_sampled_heads_and_blocks(wname):
+    """The whole backward at a Wan shape, checked on two heads: their dWq, dWk, dg (summed
+    over every token) and, on seeded query and key blocks including the ragged tail, dq and
+    dk, dv, against the oracle's sampled backward (pinned to its whole backward)."""
+    w = synth.WORKLOADS[wname]
+    inp = synth.make_inputs(w, seed=11, device="cuda")
+    dout = synth.make_dout(w, seed=12, device="cuda")
+    plan = rola.Plan.for_workload(w)
+    got = plan.backward(inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], inp["g"], dout)
+    assert plan.poll_status() == 0
+    col = plan.block_lists().cpu().numpy()
+    rng = np.random.default_rng(3)
+    heads = sorted(rng.choice(w.H, size=2, replace=False).tolist())
+    nb = plan.nb
+    blocks = lambda: [0, nb - 1] + rng.choice(np.arange(1, nb - 1), size=2, replace=False).tolist()  # noqa: E731
+    qb = [(0, h, i) for h in heads for i in blocks()]
+    kb = [(0, h, j) for h in heads for j in blocks()]
+    h = host_inputs(inp)
+    s = O.make_shape(w.B, w.H, w.N, w.d, w.r, w.topk, grid=w.grid, pairs=w.pairs)
+    smp = O.backward_sample(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"],
+                            np32(dout).astype(np.float64), col, heads, qb, kb)
+    def rows(t, blist):
+        out = np.zeros((len(blist), 64, w.d))
+        for e, (b, hh, i) in enumerate(blist):
+            n = min(w.N, i * 64 + 64) - i * 64
+            out[e, :n] = np32(t[b, i * 64:i * 64 + n, hh])
+        return out
+    _compare("dq", rows(got["dq"], qb), smp["dq"])
+    _compare("dk", rows(got["dk"], kb), smp["dk"])
+    _compare("dv", rows(got["dv"], kb), smp["dv"])
+    _compare("dWq", np32(got["dWq"])[heads], smp["dWq"])
+    _compare("dWk", np32(got["dWk"])[heads], smp["dWk"])
+    _compare("dg", np32(got["dg"])[heads], smp["dg"])

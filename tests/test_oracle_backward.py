@@ -89,3 +89,35 @@ def test_backward_is_linear_in_dout():
     b = oracle.backward(s, inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], inp["g"], 3.0 * dout, col)
     for key in a:
         np.testing.assert_allclose(b[key], 3.0 * a[key], rtol=1e-12, atol=1e-12)
+
+
+def test_sampled_backward_equals_the_whole_one():
+    """The sampled form (for problems too large for the whole backward) gives, on the listed
+    heads and blocks, what the whole backward gives (B = 2: dWq, dWk, dg sum over the batch)."""
+    rng = np.random.default_rng(7)
+    B, H, N, d, r = 2, 3, 300, 16, 8
+    s = oracle.make_shape(B, H, N, d, r, 0.4, grid=(3, 10, 10))
+    q, k, v = (rng.normal(0, 1, (B, N, H, d)).astype(np.float32) for _ in range(3))
+    Wq, Wk = (rng.normal(0, 1 / np.sqrt(d), (H, d, r)).astype(np.float32) for _ in range(2))
+    g = rng.uniform(0.1, 1.0, H)
+    dout = rng.normal(0, 1, (B, N, H, d))
+    _, col = oracle.forward(s, q, k, v, Wq, Wk, g)
+    full = oracle.backward(s, q, k, v, Wq, Wk, g, dout, col)
+    heads = [0, 2]
+    qb = [(0, 0, 1), (1, 2, 4), (1, 0, 0)]          # block 4 is the 44-token tail
+    kb = [(1, 2, 2), (0, 0, 4), (0, 2, 0)]
+    smp = oracle.backward_sample(s, q, k, v, Wq, Wk, g, dout, col, heads, qb, kb)
+    for e, (b, h, i) in enumerate(qb):
+        rows = slice(i * 64, min(N, i * 64 + 64))
+        n = rows.stop - rows.start
+        np.testing.assert_allclose(smp["dq"][e, :n], full["dq"][b, rows, h], rtol=1e-10, atol=1e-12)
+        assert np.all(smp["dq"][e, n:] == 0)
+    for e, (b, h, j) in enumerate(kb):
+        rows = slice(j * 64, min(N, j * 64 + 64))
+        n = rows.stop - rows.start
+        np.testing.assert_allclose(smp["dk"][e, :n], full["dk"][b, rows, h], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(smp["dv"][e, :n], full["dv"][b, rows, h], rtol=1e-10, atol=1e-12)
+    for t, h in enumerate(heads):
+        np.testing.assert_allclose(smp["dWq"][t], full["dWq"][h], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(smp["dWk"][t], full["dWk"][h], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(smp["dg"][t], full["dg"][h], rtol=1e-10, atol=1e-12)
