@@ -548,12 +548,14 @@ __global__ void __launch_bounds__(128) bwd_dq_mma_kernel(
   for (int hh = 0; hh < 2; ++hh) {
     const int n = i * 64 + 16 * warp + g8 + 8 * hh;
     if (n >= dm.N) continue;
-    float* row = dq + (((size_t)b * dm.N + n) * dm.H + h) * D;
+    float2* row = reinterpret_cast<float2*>(dq + (((size_t)b * dm.N + n) * dm.H + h) * D);
+    float2 cur[D / 8];               // all loads first, then the stores
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      row[nt * 8 + 2 * t4] += dm.scale * acc[nt][2 * hh];
-      row[nt * 8 + 2 * t4 + 1] += dm.scale * acc[nt][2 * hh + 1];
-    }
+    for (int nt = 0; nt < D / 8; ++nt) cur[nt] = row[nt * 4 + t4];
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt)
+      row[nt * 4 + t4] = make_float2(fmaf(dm.scale, acc[nt][2 * hh], cur[nt].x),
+                                     fmaf(dm.scale, acc[nt][2 * hh + 1], cur[nt].y));
   }
 }
 
@@ -617,12 +619,18 @@ __global__ void __launch_bounds__(128) bwd_dkv_mma_kernel(
     const int r = 16 * warp + g8 + 8 * hh;
     if (r >= nvalid) continue;
     const size_t at = (((size_t)b * dm.N + j * 64 + r) * dm.H + h) * D;
+    float2* rk = reinterpret_cast<float2*>(dk + at);
+    float2* rv = reinterpret_cast<float2*>(dv + at);
+    float2 ck[D / 8], cv[D / 8];     // all loads first, then the stores
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
-      dk[at + nt * 8 + 2 * t4] += dm.scale * ak[nt][2 * hh];
-      dk[at + nt * 8 + 2 * t4 + 1] += dm.scale * ak[nt][2 * hh + 1];
-      dv[at + nt * 8 + 2 * t4] += av[nt][2 * hh];
-      dv[at + nt * 8 + 2 * t4 + 1] += av[nt][2 * hh + 1];
+      ck[nt] = rk[nt * 4 + t4];
+      cv[nt] = rv[nt * 4 + t4];
+    }
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+      rk[nt * 4 + t4] = make_float2(fmaf(dm.scale, ak[nt][2 * hh], ck[nt].x), fmaf(dm.scale, ak[nt][2 * hh + 1], ck[nt].y));
+      rv[nt * 4 + t4] = make_float2(cv[nt].x + av[nt][2 * hh], cv[nt].y + av[nt][2 * hh + 1]);
     }
   }
 }
@@ -1095,8 +1103,13 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
     bwd_rowstats_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow,
                                                             ws.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_dq_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, dq, ws.status);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if constexpr (D == 128) {   // the forward's transposed tcgen05 tile
+      if ((e = launch_bwd_dq_sm100(dm, q, k, v, dout, ws, bw, dq, st)) != cudaSuccess) return e;
+    } else {
+      bwd_dq_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, dq,
+                                                        ws.status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     bwd_dkv_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, bw.inv_off, bw.inv_idx, bw.lse, bw.Drow,
                                                        dk, dv);
     return cudaGetLastError();

@@ -1,0 +1,400 @@
+// The backward's dq over the kept blocks on the sm_100a tensor cores (tcgen05 + TMEM + TMA),
+// bf16 inputs, head dim 128: the same transposed tile as the forward's attention kernel.
+//
+// Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
+// Preserving Global Context at Extreme Sparsity" (the block-sparse softmax branch whose
+// gradient this is); README sparse-finetuning section (the attention is trained).
+//
+// With the softmax row statistics known (lse of each query row and D = dout . O, from the
+// row-statistics kernel), each (query block i, pair of its kept key blocks j1, j2) needs
+//   S^T  [128 keys x 64 q] = [K_j1; K_j2] Q_i^T            (bf16, K-major A and B)
+//   dP^T [128 keys x 64 q] = [V_j1; V_j2] G_i^T            (G = dout; the same shape)
+//   dA^T = P^T (dP^T - D_q),  P^T = 2^(S^T scale log2(e) - lse_q)    (elementwise: every
+//          constant belongs to a column, so no reduction crosses the TMEM lanes)
+//   dQ^T [128 d x 64 q]   += [K_j1; K_j2]^T dA^T             (A = the K pair read MN-major,
+//          as the forward reads V; B = dA^T as bf16 hi + lo, two products)
+// and dq += scale dQ at the tile's end (added to the linear part already in dq).
+//
+// Roles (384 threads): warp 0 = TMA producer of the tile's Q and dout (one slot) and of the
+// K ring; warp 1 = issuer of S^T and dP^T (and TMEM owner); warp 2 = issuer of dQ^T;
+// warp 3 = producer of the V ring; warps 4-11 = two groups of four, group g owning query
+// columns [32 g, 32 g + 32): thread t of a group owns TMEM lane t (key t of the pair for
+// S^T, dP^T; channel t for dQ^T).  K stages are freed after their dQ^T products (three of
+// them), V stages after their dP^T products (two); S^T/dP^T are double-buffered in TMEM.
+// Persistent: one CTA per SM walks the tiles tau = blockIdx.x + n * gridDim.x.
+//
+// Every mbarrier wait is bounded (ROLA_ERR_DEVICE_TIMEOUT); on a timeout all roles leave
+// their loops, in-flight MMAs and TMA copies are drained and TMEM is freed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "rola_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace rola {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kSoftmaxWarps = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;      // S^T, two buffers (0, 64)
+constexpr uint32_t kColDP = 128;   // dP^T, two buffers (128, 192)
+constexpr uint32_t kColQ = 256;    // dQ^T
+constexpr int kKStages = 3;   // K is held until its dQ^T products: one more stage than V
+constexpr int kVStages = 2;
+constexpr int kABufs = 1;     // dA^T staging buffers (hi + lo each)
+
+constexpr uint32_t kPairBytes = 128 * 128 * 2;   // K or V pair (two 64-channel boxes of 16 KB)
+constexpr uint32_t kBoxKV = 16384;
+constexpr uint32_t kStgBytes = 128 * 128;        // one dA^T half: 128 keys x 64 q bf16
+constexpr uint32_t kOffQG = 0;                   // Q (16 KB) then dout (16 KB)
+constexpr uint32_t kOffK = 32768;
+constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;
+constexpr uint32_t kOffA = kOffV + kVStages * kPairBytes;   // [kABufs][hi, lo] dA^T
+constexpr uint32_t kOffCtl = kOffA + 2 * kABufs * kStgBytes;
+
+struct Ctl {
+  uint64_t qg_full, qg_free, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], a_full[kABufs], a_free[kABufs], dq_done, dq_free, drain_s, drain_q;
+  uint32_t tmem_base;
+  int abort;
+  alignas(16) float lse[2][64];   // per group: the tile's lse (log2 units) and D per query
+  alignas(16) float dd[2][64];
+};
+constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x0, x1);
+  const float2 bf = __bfloat1622float2(b);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - bf.x, x1 - bf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&b);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Dims dm,
+    const int32_t* __restrict__ col_idx, const float* __restrict__ lse, const float* __restrict__ Drow,
+    float* __restrict__ dq, int* __restrict__ status, unsigned long long limit_cycles) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + kOffCtl);
+  const uint32_t sbase = smem_addr(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = dm.nb * dm.B * dm.H;
+  const int kk_list = dm.k, npairs = (kk_list + 1) >> 1;
+  const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto bar = [&](uint64_t& m) { return smem_addr(&m); };
+  auto tile_of = [&](int jt) { return (int)blockIdx.x + jt * (int)gridDim.x; };
+  auto list_of = [&](int tau) { return col_idx + (size_t)tau * kk_list; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(ctl->qg_full), 1);
+    mbar_init(bar(ctl->qg_free), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(ctl->k_full[s]), 1);
+      mbar_init(bar(ctl->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(ctl->v_full[s]), 1);
+      mbar_init(bar(ctl->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ctl->s_full[s]), 1);
+      mbar_init(bar(ctl->s_free[s]), kSoftmaxWarps);
+    }
+    for (int s = 0; s < kABufs; ++s) {
+      mbar_init(bar(ctl->a_full[s]), kSoftmaxWarps);
+      mbar_init(bar(ctl->a_free[s]), 1);
+    }
+    mbar_init(bar(ctl->dq_done), 1);
+    mbar_init(bar(ctl->dq_free), kSoftmaxWarps);
+    mbar_init(bar(ctl->drain_s), 1);
+    mbar_init(bar(ctl->drain_q), 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtl wc{&ctl->abort, status, limit_cycles};
+  auto pair_blocks = [&](const int32_t* L, int it, int& j1, int& j2) {
+    j1 = __ldg(L + 2 * it);
+    j2 = (2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : j1;
+    if (j1 < 0 || j1 >= dm.nb || j2 < 0 || j2 >= dm.nb) {
+      atomicCAS(status, 0, kDevBounds);
+      j1 = j2 = 0;
+    }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q, dout and the K ring
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_g);
+      tma_prefetch_desc(&tm_k);
+      int gp = 0, nqg = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        const int tau = tile_of(jt);
+        const int bh = tau / dm.nb, i = tau - bh * dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        // one slot: the previous tile's S^T and dP^T products must be done with it
+        if (jt > 0 && !mbar_wait(bar(ctl->qg_free), (jt - 1) & 1, wc)) break;
+        mbar_expect_tx(bar(ctl->qg_full), 32768);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + kOffQG + c * 8192, &tm_q, xh + 64 * c, i * 64, b, bar(ctl->qg_full));
+          tma_load_3d(sbase + kOffQG + 16384 + c * 8192, &tm_g, xh + 64 * c, i * 64, b, bar(ctl->qg_full));
+        }
+        ++nqg;
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int s = gp % kKStages;
+          if (gp >= kKStages && !mbar_wait(bar(ctl->k_empty[s]), ((gp / kKStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + kOffK + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_k, xh + 64 * c, j1 * 64, b, bar(ctl->k_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_k, xh + 64 * c, j2 * 64, b, bar(ctl->k_full[s]));
+          }
+        }
+      }
+      if (nqg > 0) mbar_wait(bar(ctl->qg_full), (nqg - 1) & 1, wc, false);
+      for (int x = (gp > kKStages ? gp - kKStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->k_full[x % kKStages]), (x / kKStages) & 1, wc, false);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ the V ring
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_v);
+      int gp = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        const int tau = tile_of(jt);
+        const int bh = tau / dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int s = gp % kVStages;
+          if (gp >= kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((gp / kVStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + kOffV + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
+          }
+        }
+      }
+      for (int x = (gp > kVStages ? gp - kVStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->v_full[x % kVStages]), (x / kVStages) & 1, wc, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S^T and dP^T
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(1, 128, 64, 0, 0);
+      int gp = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        if (!mbar_wait(bar(ctl->qg_full), jt & 1, wc)) break;
+        const uint64_t dqd = sdesc_sw128(sbase + kOffQG, 16, 1024);
+        const uint64_t dgd = sdesc_sw128(sbase + kOffQG + 16384, 16, 1024);
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int ks = gp % kKStages, vs = gp % kVStages, sb = gp & 1;
+          if (!mbar_wait(bar(ctl->k_full[ks]), (gp / kKStages) & 1, wc) ||
+              !mbar_wait(bar(ctl->v_full[vs]), (gp / kVStages) & 1, wc) ||
+              (gp >= 2 && !mbar_wait(bar(ctl->s_free[sb]), ((gp - 2) >> 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dk = sdesc_sw128(sbase + kOffK + ks * kPairBytes, 16, 1024);
+          const uint64_t dv = sdesc_sw128(sbase + kOffV + vs * kPairBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
+            const uint32_t ab = ((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4, bb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tmem + kColS + 64 * sb, dk + ab, dqd + bb, idesc, kk > 0);
+            mma_f16_ss(tmem + kColDP + 64 * sb, dv + ab, dgd + bb, idesc, kk > 0);
+          }
+          mma_commit(bar(ctl->s_full[sb]));
+          mma_commit(bar(ctl->v_empty[vs]));
+        }
+        if (ok) mma_commit(bar(ctl->qg_free));   // this tile's Q and dout are read
+      }
+      mma_commit(bar(ctl->drain_s));
+      mbar_wait(bar(ctl->drain_s), 0, wc, false);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ dQ^T += K^T dA^T
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(1, 128, 64, 1, 1);
+      int gp = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int s = gp % kKStages, ab = gp % kABufs;
+          if (!mbar_wait(bar(ctl->a_full[ab]), (gp / kABufs) & 1, wc) ||
+              (it == 0 && jt > 0 && !mbar_wait(bar(ctl->dq_free), (jt - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = sdesc_sw128(sbase + kOffK + s * kPairBytes, kBoxKV, 1024);
+          const uint64_t dh = sdesc_sw128(sbase + kOffA + ab * 2 * kStgBytes, 8192, 1024);
+          const uint64_t dl = sdesc_sw128(sbase + kOffA + ab * 2 * kStgBytes + kStgBytes, 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step: +2048 bytes in both operands
+            mma_f16_ss(tmem + kColQ, da + 128 * kk, dh + 128 * kk, idesc, (it > 0) || (kk > 0));
+            mma_f16_ss(tmem + kColQ, da + 128 * kk, dl + 128 * kk, idesc, true);
+          }
+          mma_commit(bar(ctl->a_free[ab]));
+          mma_commit(bar(ctl->k_empty[s]));
+          if (it == npairs - 1) mma_commit(bar(ctl->dq_done));
+        }
+      }
+      mma_commit(bar(ctl->drain_q));
+      mbar_wait(bar(ctl->drain_q), 0, wc, false);
+    }
+  } else {
+    // ------------------------------------------------------------ dA^T and the tile's dq
+    const int g = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;
+    const int t = 32 * wq + lane;                  // TMEM lane: key of the pair / channel
+    const int c0 = 32 * g;
+    const uint32_t gbar = 1 + g;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
+    const float sl2 = dm.scale * 1.4426950408889634f;
+    bool fail = false;
+    int gp = 0;
+    for (int jt = 0; jt < my_tiles; ++jt) {
+      const int tau = tile_of(jt);
+      if (named_vote_or(gbar, 128, fail)) break;
+      const int bh = tau / dm.nb, i = tau - bh * dm.nb, b = bh / dm.H, h = bh % dm.H;
+      const int32_t* L = list_of(tau);
+      // the group's 32 columns of lse and D (rows past N: lse = +inf, so P = 0)
+      if (wq == 0) {
+        const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + c0 + lane;
+        ctl->lse[g][c0 + lane] = __ldg(lse + at);
+        ctl->dd[g][c0 + lane] = __ldg(Drow + at);
+      }
+      named_sync(gbar, 128);
+      const float4* l4 = reinterpret_cast<const float4*>(&ctl->lse[g][c0]);
+      const float4* d4 = reinterpret_cast<const float4*>(&ctl->dd[g][c0]);
+      for (int it = 0; it < npairs; ++it, ++gp) {
+        const int sb = gp & 1;
+        const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (gp >> 1) & 1, wc);
+        fail |= !ok;
+        tc_fence_after();
+        float x[32], dp[32];
+        tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
+        tmem_ld32(lane_addr + kColDP + 64 * sb + c0, dp);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(bar(ctl->s_free[sb]));
+        // this thread's key: block j1 (t < 64) or j2 (the padding half of an odd list is a
+        // repeat of j1 and contributes nothing), valid below N
+        const int e = 2 * it + (t >> 6);
+        const int jb = e < kk_list ? __ldg(L + e) : -1;
+        const bool valid = jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
+        // the staging buffer was last read by the dQ^T products kABufs pairs back
+        const int ab = gp % kABufs;
+        if (gp >= kABufs && !fail) fail |= !mbar_wait(bar(ctl->a_free[ab]), ((gp - kABufs) / kABufs) & 1, wc);
+        uint8_t* stg = base + kOffA + ab * 2 * kStgBytes;
+        // eight columns at a time: one 16-byte chunk of dA^T hi and one of lo
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const float4 lv = l4[2 * c8 + h2], dv = d4[2 * c8 + h2];
+            const int q0 = 8 * c8 + 4 * h2;
+            const float p0 = valid ? exp2f(fmaf(x[q0], sl2, -lv.x)) : 0.f;
+            const float p1 = valid ? exp2f(fmaf(x[q0 + 1], sl2, -lv.y)) : 0.f;
+            const float p2 = valid ? exp2f(fmaf(x[q0 + 2], sl2, -lv.z)) : 0.f;
+            const float p3 = valid ? exp2f(fmaf(x[q0 + 3], sl2, -lv.w)) : 0.f;
+            split_bf16x2(p0 * (dp[q0] - dv.x), p1 * (dp[q0 + 1] - dv.y), hw[2 * h2], lw[2 * h2]);
+            split_bf16x2(p2 * (dp[q0 + 2] - dv.z), p3 * (dp[q0 + 3] - dv.w), hw[2 * h2 + 1], lw[2 * h2 + 1]);
+          }
+          const uint32_t off = t * 128 + (((4 * g + c8) ^ (t & 7)) << 4);
+          *reinterpret_cast<uint4*>(stg + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(stg + kStgBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ctl->a_full[ab]));
+      }
+      // the tile's dQ^T: lane = channel t, this group's 32 query columns
+      fail |= !mbar_wait(bar(ctl->dq_done), jt & 1, wc);
+      if (!named_vote_or(gbar, 128, fail)) {
+        tc_fence_after();
+        float o[32];
+        tmem_ld32(lane_addr + kColQ + c0, o);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ctl->dq_free));
+        // all 32 loads first (the compiler cannot tell the rows apart), then the stores
+        float* col = dq + (((size_t)b * dm.N + i * 64 + c0) * dm.H + h) * 128 + t;
+        const size_t rs = (size_t)dm.H * 128;
+        const int nv = min(32, dm.N - (i * 64 + c0));
+        float cur[32];
+#pragma unroll
+        for (int qq = 0; qq < 32; ++qq) cur[qq] = qq < nv ? col[qq * rs] : 0.f;
+#pragma unroll
+        for (int qq = 0; qq < 32; ++qq)
+          if (qq < nv) col[qq * rs] = fmaf(dm.scale, o[qq], cur[qq]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                                const Workspace& ws, const BwdWorkspace& bw, float* dq, cudaStream_t st) {
+  CUtensorMap tq, tg, tk, tv;
+  if (!make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dm, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long ntiles = (long long)dm.nb * dm.B * dm.H;
+  dim3 grid((unsigned)(ntiles < sms ? ntiles : sms));
+  // Wait limit in SM clock cycles: 2e9 cycles is 1 s at 2 GHz.
+  bwd_dq_sm100_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tg, tk, tv, dm, ws.col_idx, bw.lse, bw.Drow, dq,
+                                                          ws.status, 2000000000ull);
+  return cudaGetLastError();
+}
+
+}  // namespace rola
