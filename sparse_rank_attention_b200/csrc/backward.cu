@@ -1110,6 +1110,7 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
                                                         ws.status);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if constexpr (D == 128) return launch_bwd_dkv_sm100(dm, q, k, v, dout, ws, bw, dk, dv, st);
     bwd_dkv_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, bw.inv_off, bw.inv_idx, bw.lse, bw.Drow,
                                                        dk, dv);
     return cudaGetLastError();

@@ -373,6 +373,321 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100_kernel(
   }
 }
 
+// ------------------------------------------------------------------ dk, dv
+// Key-major: a tile is one key block j, walked over the query blocks that kept it (the
+// key-major lists), two at a time on the M side:
+//   S  [128 q x 64 keys] = [Q_i1; Q_i2] K_j^T,   dP = [G_i1; G_i2] V_j^T     (K-major)
+//   P = 2^(S scale log2(e) - lse_row),  dA = P (dP - D_row)  (a constant per TMEM lane)
+//   dV^T [128 d x 64 keys] += [G_i1; G_i2]^T P,  dK^T += [Q_i1; Q_i2]^T dA   (the query
+//   pairs read MN-major, P and dA as bf16 hi + lo), and dk += scale dK, dv += dV at the end.
+// Roles: warp 0 = producer of K_j, V_j (one slot) and of the ring of query pairs (Q and
+// dout); warp 1 = issuer of S and dP (and TMEM owner); warp 2 = issuer of dV^T, dK^T;
+// warps 4-11 = two groups of four (thread t: query row t of the pair for S, dP; channel t
+// for dK^T, dV^T; group g: key columns [32 g, 32 g + 32)).  An odd list's last pair repeats
+// its first block with every row masked (lse = +inf).
+namespace kv {
+constexpr uint32_t kKVBytes = 2 * 128 * 64 * 2;             // K_j then V_j, 16 KB each
+constexpr uint32_t kQGBytes = 2 * kPairBytes;               // a query pair of Q, then of dout
+constexpr int kStages = 2;
+constexpr uint32_t kOffKV = 0;
+constexpr uint32_t kOffQG = kKVBytes;
+constexpr uint32_t kOffStg = kOffQG + kStages * kQGBytes;   // P hi, P lo, dA hi, dA lo
+constexpr uint32_t kOffCtl = kOffStg + 4 * kStgBytes;
+constexpr uint32_t kColS = 0, kColDP = 128, kColK = 256, kColV = 320;
+struct Ctl {
+  uint64_t kv_full, kv_free, qg_full[kStages], qg_empty[kStages], s_full[2], s_free[2], a_full, a_free;
+  uint64_t dkv_done, dkv_free, drain_s, drain_d;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
+}  // namespace kv
+
+__global__ void __launch_bounds__(kThreads, 1) bwd_dkv_sm100_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Dims dm,
+    const int* __restrict__ inv_off, const int* __restrict__ inv_idx, const float* __restrict__ lse,
+    const float* __restrict__ Drow, float* __restrict__ dk, float* __restrict__ dv, int* __restrict__ status,
+    unsigned long long limit_cycles) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  kv::Ctl* ctl = reinterpret_cast<kv::Ctl*>(base + kv::kOffCtl);
+  const uint32_t sbase = smem_addr(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = dm.nb * dm.B * dm.H;
+  const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto bar = [&](uint64_t& m) { return smem_addr(&m); };
+  auto tile_of = [&](int jt) { return (int)blockIdx.x + jt * (int)gridDim.x; };
+  // the tile's list of query blocks: [e0, e1) of the (b, h) row of inv_idx
+  auto list_of = [&](int tau, int& e0, int& e1) {
+    const int bh = tau / dm.nb, j = tau - bh * dm.nb;
+    e0 = __ldg(inv_off + (size_t)bh * (dm.nb + 1) + j);
+    e1 = __ldg(inv_off + (size_t)bh * (dm.nb + 1) + j + 1);
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(ctl->kv_full), 1);
+    mbar_init(bar(ctl->kv_free), 1);
+    for (int s = 0; s < kv::kStages; ++s) {
+      mbar_init(bar(ctl->qg_full[s]), 1);
+      mbar_init(bar(ctl->qg_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ctl->s_full[s]), 1);
+      mbar_init(bar(ctl->s_free[s]), kSoftmaxWarps);
+    }
+    mbar_init(bar(ctl->a_full), kSoftmaxWarps);
+    mbar_init(bar(ctl->a_free), 1);
+    mbar_init(bar(ctl->dkv_done), 1);
+    mbar_init(bar(ctl->dkv_free), kSoftmaxWarps);
+    mbar_init(bar(ctl->drain_s), 1);
+    mbar_init(bar(ctl->drain_d), 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtl wc{&ctl->abort, status, limit_cycles};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ K_j, V_j and the query pairs
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_g);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int gp = 0, nt = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        const int tau = tile_of(jt);
+        int e0, e1;
+        list_of(tau, e0, e1);
+        if (e1 <= e0) continue;   // a key block no query block kept: nothing to add
+        const int bh = tau / dm.nb, j = tau - bh * dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        if (nt > 0 && !mbar_wait(bar(ctl->kv_free), (nt - 1) & 1, wc)) break;
+        mbar_expect_tx(bar(ctl->kv_full), kv::kKVBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + kv::kOffKV + c * 8192, &tm_k, xh + 64 * c, j * 64, b, bar(ctl->kv_full));
+          tma_load_3d(sbase + kv::kOffKV + 16384 + c * 8192, &tm_v, xh + 64 * c, j * 64, b, bar(ctl->kv_full));
+        }
+        ++nt;
+        const int* lst = inv_idx + (size_t)bh * dm.nb * dm.k;
+        for (int e = e0; e < e1; e += 2, ++gp) {
+          const int s = gp % kv::kStages;
+          if (gp >= kv::kStages && !mbar_wait(bar(ctl->qg_empty[s]), ((gp / kv::kStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int i1 = __ldg(lst + e), i2 = e + 1 < e1 ? __ldg(lst + e + 1) : i1;
+          if (i1 < 0 || i1 >= dm.nb || i2 < 0 || i2 >= dm.nb) {
+            atomicCAS(status, 0, kDevBounds);
+            i1 = i2 = 0;
+          }
+          const uint32_t st = sbase + kv::kOffQG + s * kv::kQGBytes;
+          mbar_expect_tx(bar(ctl->qg_full[s]), kv::kQGBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_q, xh + 64 * c, i1 * 64, b, bar(ctl->qg_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_q, xh + 64 * c, i2 * 64, b, bar(ctl->qg_full[s]));
+            tma_load_3d(st + kPairBytes + c * kBoxKV, &tm_g, xh + 64 * c, i1 * 64, b, bar(ctl->qg_full[s]));
+            tma_load_3d(st + kPairBytes + c * kBoxKV + 8192, &tm_g, xh + 64 * c, i2 * 64, b, bar(ctl->qg_full[s]));
+          }
+        }
+      }
+      if (nt > 0) mbar_wait(bar(ctl->kv_full), (nt - 1) & 1, wc, false);
+      for (int x = (gp > kv::kStages ? gp - kv::kStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->qg_full[x % kv::kStages]), (x / kv::kStages) & 1, wc, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S and dP
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(1, 128, 64, 0, 0);
+      int gp = 0, nt = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        int e0, e1;
+        list_of(tile_of(jt), e0, e1);
+        if (e1 <= e0) continue;
+        if (!mbar_wait(bar(ctl->kv_full), nt & 1, wc)) break;
+        ++nt;
+        const uint64_t dkd = sdesc_sw128(sbase + kv::kOffKV, 16, 1024);
+        const uint64_t dvd = sdesc_sw128(sbase + kv::kOffKV + 16384, 16, 1024);
+        for (int e = e0; e < e1; e += 2, ++gp) {
+          const int s = gp % kv::kStages, sb = gp & 1;
+          if (!mbar_wait(bar(ctl->qg_full[s]), (gp / kv::kStages) & 1, wc) ||
+              (gp >= 2 && !mbar_wait(bar(ctl->s_free[sb]), ((gp - 2) >> 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dq = sdesc_sw128(sbase + kv::kOffQG + s * kv::kQGBytes, 16, 1024);
+          const uint64_t dg = sdesc_sw128(sbase + kv::kOffQG + s * kv::kQGBytes + kPairBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t ab = ((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4, bb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tmem + kv::kColS + 64 * sb, dq + ab, dkd + bb, idesc, kk > 0);
+            mma_f16_ss(tmem + kv::kColDP + 64 * sb, dg + ab, dvd + bb, idesc, kk > 0);
+          }
+          mma_commit(bar(ctl->s_full[sb]));
+        }
+        if (ok) mma_commit(bar(ctl->kv_free));   // K_j and V_j are read
+      }
+      mma_commit(bar(ctl->drain_s));
+      mbar_wait(bar(ctl->drain_s), 0, wc, false);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ dV^T, dK^T
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(1, 128, 64, 1, 1);
+      int gp = 0, nt = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        int e0, e1;
+        list_of(tile_of(jt), e0, e1);
+        if (e1 <= e0) continue;
+        for (int e = e0; e < e1; e += 2, ++gp) {
+          const int s = gp % kv::kStages;
+          const bool first = e == e0;
+          if (!mbar_wait(bar(ctl->a_full), gp & 1, wc) ||
+              (first && nt > 0 && !mbar_wait(bar(ctl->dkv_free), (nt - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dq = sdesc_sw128(sbase + kv::kOffQG + s * kv::kQGBytes, kBoxKV, 1024);
+          const uint64_t dg = sdesc_sw128(sbase + kv::kOffQG + s * kv::kQGBytes + kPairBytes, kBoxKV, 1024);
+          const uint32_t stg = sbase + kv::kOffStg;
+          const uint64_t ph = sdesc_sw128(stg, 8192, 1024), pl = sdesc_sw128(stg + kStgBytes, 8192, 1024);
+          const uint64_t ah = sdesc_sw128(stg + 2 * kStgBytes, 8192, 1024);
+          const uint64_t al = sdesc_sw128(stg + 3 * kStgBytes, 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {   // 16 queries per step: +2048 bytes in every operand
+            mma_f16_ss(tmem + kv::kColV, dg + 128 * kk, ph + 128 * kk, idesc, !first || kk > 0);
+            mma_f16_ss(tmem + kv::kColV, dg + 128 * kk, pl + 128 * kk, idesc, true);
+            mma_f16_ss(tmem + kv::kColK, dq + 128 * kk, ah + 128 * kk, idesc, !first || kk > 0);
+            mma_f16_ss(tmem + kv::kColK, dq + 128 * kk, al + 128 * kk, idesc, true);
+          }
+          mma_commit(bar(ctl->a_free));
+          mma_commit(bar(ctl->qg_empty[s]));
+          if (e + 2 >= e1) mma_commit(bar(ctl->dkv_done));
+        }
+        ++nt;
+      }
+      mma_commit(bar(ctl->drain_d));
+      mbar_wait(bar(ctl->drain_d), 0, wc, false);
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ P, dA and the tile's dk, dv
+    const int g = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;
+    const int t = 32 * wq + lane;                  // TMEM lane: query row of the pair / channel
+    const int c0 = 32 * g;
+    const uint32_t gbar = 1 + g;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
+    const float sl2 = dm.scale * 1.4426950408889634f;
+    bool fail = false;
+    int gp = 0, nt = 0;
+    for (int jt = 0; jt < my_tiles; ++jt) {
+      const int tau = tile_of(jt);
+      int e0, e1;
+      list_of(tau, e0, e1);
+      if (e1 <= e0) continue;
+      if (named_vote_or(gbar, 128, fail)) break;
+      const int bh = tau / dm.nb, j = tau - bh * dm.nb, b = bh / dm.H, h = bh % dm.H;
+      const int* lst = inv_idx + (size_t)bh * dm.nb * dm.k;
+      const int kvalid = min(64, dm.N - j * 64) - c0;   // this group's valid key columns
+      for (int e = e0; e < e1; e += 2, ++gp) {
+        const int sb = gp & 1;
+        // this thread's query row: block i1 (t < 64) or i2 (the padding half of an odd
+        // list is masked), its lse and D
+        const int ee = e + (t >> 6);
+        float lr = INFINITY, dr = 0.f;
+        if (ee < e1) {
+          const int ib = __ldg(lst + ee);
+          if (ib >= 0 && ib < dm.nb) {
+            const size_t at = (size_t)bh * dm.nb * 64 + (size_t)ib * 64 + (t & 63);
+            lr = __ldg(lse + at);
+            dr = __ldg(Drow + at);
+          }
+        }
+        const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (gp >> 1) & 1, wc);
+        fail |= !ok;
+        tc_fence_after();
+        float x[32], dp[32];
+        tmem_ld32(lane_addr + kv::kColS + 64 * sb + c0, x);
+        tmem_ld32(lane_addr + kv::kColDP + 64 * sb + c0, dp);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(bar(ctl->s_free[sb]));
+        // the staging was last read by the previous step's dV^T, dK^T products
+        if (gp >= 1 && !fail) fail |= !mbar_wait(bar(ctl->a_free), (gp - 1) & 1, wc);
+        uint8_t* stg = base + kv::kOffStg;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t ph[4], pl[4], ah[4], al[4];
+#pragma unroll
+          for (int w2 = 0; w2 < 4; ++w2) {
+            const int k0 = 8 * c8 + 2 * w2;
+            const float p0 = k0 < kvalid ? exp2f(fmaf(x[k0], sl2, -lr)) : 0.f;
+            const float p1 = k0 + 1 < kvalid ? exp2f(fmaf(x[k0 + 1], sl2, -lr)) : 0.f;
+            split_bf16x2(p0, p1, ph[w2], pl[w2]);
+            split_bf16x2(p0 * (dp[k0] - dr), p1 * (dp[k0 + 1] - dr), ah[w2], al[w2]);
+          }
+          const uint32_t off = t * 128 + (((4 * g + c8) ^ (t & 7)) << 4);
+          *reinterpret_cast<uint4*>(stg + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+          *reinterpret_cast<uint4*>(stg + kStgBytes + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+          *reinterpret_cast<uint4*>(stg + 2 * kStgBytes + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+          *reinterpret_cast<uint4*>(stg + 3 * kStgBytes + off) = make_uint4(al[0], al[1], al[2], al[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(ctl->a_full));
+      }
+      // the tile's dK^T, dV^T: lane = channel t, this group's 32 key columns
+      fail |= !mbar_wait(bar(ctl->dkv_done), nt & 1, wc);
+      ++nt;
+      if (!named_vote_or(gbar, 128, fail)) {
+        const size_t rs = (size_t)dm.H * 128;
+        const size_t row0 = (((size_t)b * dm.N + j * 64 + c0) * dm.H + h) * 128 + t;
+        // dK^T then dV^T, each: the TMEM columns, all loads of the rows, then the stores
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          tc_fence_after();
+          float a[32];
+          tmem_ld32(lane_addr + (which ? kv::kColV : kv::kColK) + c0, a);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (which == 1 && lane == 0) mbar_arrive(bar(ctl->dkv_free));
+          float* col = (which ? dv : dk) + row0;
+          const float f = which ? 1.f : dm.scale;
+          float u[32];
+#pragma unroll
+          for (int kq = 0; kq < 32; ++kq) u[kq] = kq < kvalid ? col[kq * rs] : 0.f;
+#pragma unroll
+          for (int kq = 0; kq < 32; ++kq)
+            if (kq < kvalid) col[kq * rs] = fmaf(f, a[kq], u[kq]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
@@ -394,6 +709,27 @@ cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, co
   // Wait limit in SM clock cycles: 2e9 cycles is 1 s at 2 GHz.
   bwd_dq_sm100_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tg, tk, tv, dm, ws.col_idx, bw.lse, bw.Drow, dq,
                                                           ws.status, 2000000000ull);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkv_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                                 const Workspace& ws, const BwdWorkspace& bw, float* dk, float* dv, cudaStream_t st) {
+  CUtensorMap tq, tg, tk, tv;
+  if (!make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dm, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkv_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kv::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long ntiles = (long long)dm.nb * dm.B * dm.H;
+  dim3 grid((unsigned)(ntiles < sms ? ntiles : sms));
+  bwd_dkv_sm100_kernel<<<grid, kThreads, kv::kSmemBytes, st>>>(tq, tg, tk, tv, dm, bw.inv_off, bw.inv_idx, bw.lse,
+                                                               bw.Drow, dk, dv, ws.status, 2000000000ull);
   return cudaGetLastError();
 }
 

@@ -113,6 +113,8 @@ struct BwdWorkspace {
 size_t backward_workspace_bytes(const Dims& dm, BwdWorkspace* bw, char* base);
 cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
                                 const Workspace& ws, const BwdWorkspace& bw, float* dq, cudaStream_t st);
+cudaError_t launch_bwd_dkv_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                                 const Workspace& ws, const BwdWorkspace& bw, float* dk, float* dv, cudaStream_t st);
 cudaError_t launch_backward(const Dims& dm, rola_dtype dt, const void* q, const void* k, const void* v,
                             const void* Wq, const void* Wk, const float* g, const void* dout, float* dq, float* dk,
                             float* dv, float* dWq, float* dWk, float* dg, const Workspace& ws,
