@@ -186,6 +186,12 @@ ROLA_API rola_status rola_get_block_lists(rola_plan_t plan, int32_t* col_idx, ro
 ROLA_API rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_stream_t stream);
 ROLA_API rola_status rola_get_linear_state(rola_plan_t plan, float* S, float* z, rola_stream_t stream);
 
+/* Inspection (tests): copy, on `stream`, the tensor-core block scores of the last selection
+ * [B, H, nb, nb] fp32 (row i of (b, h) at ((b*H + h)*nb + i)*nb; s~_ij = qbar_i . kbar_j from
+ * tf32 operands: they only prune, the kept lists are decided on exact fp32 scores) and the
+ * key-block norms ||kbar_j||_2 [B, H, nb] fp32 into caller device buffers. */
+ROLA_API rola_status rola_get_block_scores(rola_plan_t plan, float* scores, float* knorm, rola_stream_t stream);
+
 /* Inspection (tests), ROLA_FP8_E4M3 plans only (ROLA_ERR_INVALID_ARG otherwise): copy the
  * e4m3 copies q8, k8, v8 [B, N, H, d] (one byte per element, OCP E4M3 encoding) and their
  * scales sq, sk, sv [B, H, nb] fp32 (value = decoded byte * scale of its (b, h, block))

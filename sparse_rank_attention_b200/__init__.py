@@ -38,7 +38,7 @@ EXPORTS = ("rola_params_default", "rola_keep_count", "rola_workspace_size", "rol
            "rola_poll_device_status", "rola_set_debug", "rola_status_string",
            "rola_select_blocks_noalloc", "rola_get_fp8_copies", "rola_profile_stages",
            "rola_get_stage_times", "rola_get_attend_redo_count", "rola_eval_exp2",
-           "rola_backward_workspace_size", "rola_backward")
+           "rola_backward_workspace_size", "rola_backward", "rola_get_block_scores")
 
 
 class RolaError(RuntimeError):
@@ -87,6 +87,7 @@ def load() -> ctypes.CDLL:
         "rola_forward": [P, P, P, P, P, P, P, P, P],
         "rola_get_block_lists": [P, P, P],
         "rola_get_pooled": [P, P, P, P],
+        "rola_get_block_scores": [P, P, P, P],
         "rola_get_linear_state": [P, P, P, P],
         "rola_poll_device_status": [P, P],
         "rola_set_debug": [P, i32, i32],
@@ -268,6 +269,15 @@ class Plan:
         kb = torch.empty_like(qb)
         _check(load().rola_get_pooled(self._h, _ptr(qb), _ptr(kb), _stream(stream)), "rola_get_pooled")
         return qb, kb
+
+    def block_scores(self, stream=None):
+        """The tensor-core block scores [B, H, nb, nb] of the last selection and the key-block
+        norms [B, H, nb] that bound their error."""
+        p = self.params
+        sc = torch.empty((p.B, p.H, self.nb, self.nb), dtype=torch.float32, device=self.workspace.device)
+        kn = torch.empty((p.B, p.H, self.nb), dtype=torch.float32, device=self.workspace.device)
+        _check(load().rola_get_block_scores(self._h, _ptr(sc), _ptr(kn), _stream(stream)), "rola_get_block_scores")
+        return sc, kn
 
     def state(self, stream=None):
         p = self.params

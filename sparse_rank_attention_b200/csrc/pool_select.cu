@@ -1,4 +1,5 @@
-// Block pooling (step 1) and block scores + top-k selection (step 2) of RoLA.
+// Block pooling (step 1) and the top-k selection (step 2) of RoLA; the block scores that
+// prune the selection come from the tensor cores (score_sm100.cu).
 //
 // Sources: "SparkDiffusion: 265x Faster Video Generation ..." page, section "RoLA:
 // Preserving Global Context at Extreme Sparsity" (the sparse branch keeps the high-energy
@@ -9,6 +10,7 @@
 // The kernels reproduce a stated fp32 order exactly, so the block lists are bit-exact:
 //   qbar = (fp32 sum of the block's tokens in token order) / count   (IEEE division)
 //   s_ij = fma chain over channels 0..d-1 starting from 0
+// (s_ij is computed exactly for every block that the tensor-core scores cannot rule out).
 #include <cuda_fp8.h>
 
 #include <mutex>
@@ -133,136 +135,152 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, cons
   }
 }
 
-// ------------------------------------------------------------------ block scores
-
-constexpr int kTS = 128;  // score tile: 128 query blocks x 128 key blocks
-constexpr int kKC = 16;   // channels staged per step
-
-// grid: x = key-block tile, y = query-block tile, z = b*H + h; 256 threads, 8x8 scores each.
-// s_ij accumulates q_i[c] * k_j[c] with fmaf in channel order 0..d-1 (the stated order).
-// The next 16-channel chunk is loaded into registers (float4 per row and channel quad)
-// while the current one is multiplied, then stored transposed into the other buffer.
-constexpr size_t kScoreSmem = sizeof(float) * 2 * 2 * kKC * (kTS + 4);
-
-__global__ void __launch_bounds__(256, 2) score_kernel(Dims dm, const float* __restrict__ qbar,
-                                                       const float* __restrict__ kbar,
-                                                       float* __restrict__ scores, int nbp) {
-  extern __shared__ __align__(16) float ssm[];
-  float (*As)[kKC][kTS + 4] = reinterpret_cast<float (*)[kKC][kTS + 4]>(ssm);
-  float (*Bs)[kKC][kTS + 4] = reinterpret_cast<float (*)[kKC][kTS + 4]>(ssm + 2 * kKC * (kTS + 4));
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int i0 = blockIdx.y * kTS, j0 = blockIdx.x * kTS, bh = blockIdx.z;
-  const int nb = dm.nb, d = dm.d;
-  const float* qb = qbar + (size_t)bh * nb * d;
-  const float* kb = kbar + (size_t)bh * nb * d;
-  constexpr int kQuads = kKC / 4, kPer = kTS * kQuads / 256;   // float4 loads per thread
-  float4 ra[kPer], rb[kPer];
-  auto load = [&](int c0) {
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int e = tid + 256 * u, r = e / kQuads, cq = e % kQuads;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      ra[u] = (i0 + r < nb) ? *reinterpret_cast<const float4*>(qb + (size_t)(i0 + r) * d + c0 + 4 * cq) : z;
-      rb[u] = (j0 + r < nb) ? *reinterpret_cast<const float4*>(kb + (size_t)(j0 + r) * d + c0 + 4 * cq) : z;
-    }
-  };
-  auto store = [&](int buf) {
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int e = tid + 256 * u, r = e / kQuads, c = 4 * (e % kQuads);
-      As[buf][c][r] = ra[u].x; As[buf][c + 1][r] = ra[u].y; As[buf][c + 2][r] = ra[u].z; As[buf][c + 3][r] = ra[u].w;
-      Bs[buf][c][r] = rb[u].x; Bs[buf][c + 1][r] = rb[u].y; Bs[buf][c + 2][r] = rb[u].z; Bs[buf][c + 3][r] = rb[u].w;
-    }
-  };
-  float acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-  const int nch = d / kKC;
-  load(0);
-  store(0);
-  __syncthreads();
-  for (int ch = 0; ch < nch; ++ch) {
-    const int buf = ch & 1;
-    if (ch + 1 < nch) load((ch + 1) * kKC);
-#pragma unroll 1
-    for (int c = 0; c < kKC; ++c) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][c][ty * 8 + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][c][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][c][tx * 8 + 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      // two scores per packed f32x2 FMA (each rounded as fmaf: the chains stay exact)
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int e = 0; e < 8; e += 2)
-          sm100::fma2(acc[a][e], acc[a][e + 1], av[a], av[a], bv[e], bv[e + 1], acc[a][e], acc[a][e + 1]);
-    }
-    if (ch + 1 < nch) store(buf ^ 1);   // the other buffer was last read before the barrier below
-    __syncthreads();
-  }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = i0 + ty * 8 + a;
-    if (i >= nb) continue;
-    float* row = scores + ((size_t)bh * nb + i) * nbp + j0 + tx * 8;
-    if (j0 + tx * 8 + 8 <= nbp) {
-      *reinterpret_cast<float4*>(row) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-      *reinterpret_cast<float4*>(row + 4) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (j0 + tx * 8 + e < nbp) row[e] = acc[a][e];
-    }
-  }
-}
-
 // ------------------------------------------------------------------ top-k per row
 
 constexpr int kTopkWarps = 8;
-constexpr int kTopkCand = 256;   // keys left after the first digit, kept apart (if they fit)
+constexpr int kTopkCand = 256;   // candidate blocks (or keys) kept apart, if they fit
+constexpr int kTopkBatch = 6;    // float4 loads of a score row in flight per lane
 
-__host__ __device__ inline size_t topk_smem(int nbp) {
-  return sizeof(uint32_t) * ((size_t)kTopkWarps * (nbp + 256 + kTopkCand));
+// Bound on |s~ - s| between the tensor-core score s~ and the exact score s of a pair:
+//   kBoundRel |qbar_i| |kbar_j| + kBoundAbs (|qbar_i| + |kbar_j|) + kBoundFloor
+// (split tf32 operands, fp32 accumulation, flushed subnormals; derived where the scores
+// are made).
+constexpr float kBoundRel = 0x1p-14f;
+constexpr float kBoundAbs = 0x1p-122f;
+constexpr float kBoundFloor = 0x1p-116f;
+
+__host__ __device__ inline size_t topk_smem(int nbp, int d) {
+  return sizeof(uint32_t) * ((size_t)kTopkWarps * (nbp + 256 + 2 * kTopkCand + d));
 }
 
-// One warp per row (b, h, i): 4-pass 8-bit radix select of the k-th largest score, then
-// one pass in index order emits the kept block indices (ties -> lower index).  For
-// k <= 64 the select runs over few keys: the k-th largest of the 64 lane top-twos is a
-// lower bound of the answer, and only the keys at or above it (when at most kTopkCand)
-// are gathered and selected from.  Otherwise the first pass reads every key and the keys
-// still matching its digit are gathered for the other three.
-__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const float* __restrict__ scores,
-                                                               int nbp, int32_t* __restrict__ col_idx,
+// Order-preserving map float -> uint32 (both zeros map to the key of +0) and its inverse.
+__device__ __forceinline__ uint32_t float_key(float f) {
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Bitonic sort (ascending) of 64 keys across the warp, two per lane: element i sits in lane
+// i mod 32, register i / 32 (v0 for i < 32).
+__device__ __forceinline__ void warp_sort64(uint32_t& v0, uint32_t& v1, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {   // partners in the same lane; the final merge is ascending
+        const uint32_t a = min(v0, v1), b = max(v0, v1);
+        v0 = a;
+        v1 = b;
+      } else {
+        const uint32_t p0 = __shfl_xor_sync(0xffffffffu, v0, j), p1 = __shfl_xor_sync(0xffffffffu, v1, j);
+        const bool lower = (lane & j) == 0;
+        const bool up0 = (lane & k) == 0, up1 = ((lane + 32) & k) == 0;
+        v0 = (lower == up0) ? min(v0, p0) : max(v0, p0);
+        v1 = (lower == up1) ? min(v1, p1) : max(v1, p1);
+      }
+    }
+  }
+}
+
+// Exact scores of key blocks j1 and j2 against the query block's mean (in shared memory):
+// each a chain of fused multiply-adds over channels 0..d-1 starting from 0.  The key rows
+// are read kExactStep float4 at a time, the next step's loads issued before this step's
+// multiply-adds, so that one L2 round trip is exposed per step rather than per load.
+constexpr int kExactStep = 2;
+__device__ __forceinline__ void exact_scores(const float* qrow, const float* __restrict__ kb, int d, int j1, int j2,
+                                             float& s1, float& s2) {
+  const float4* k1 = reinterpret_cast<const float4*>(kb + (size_t)j1 * d);
+  const float4* k2 = reinterpret_cast<const float4*>(kb + (size_t)j2 * d);
+  const float4* q4 = reinterpret_cast<const float4*>(qrow);
+  const int n4 = d / 4;
+  float a = 0.f, b = 0.f;
+  float4 x[kExactStep], y[kExactStep];
+#pragma unroll
+  for (int u = 0; u < kExactStep; ++u) {
+    x[u] = __ldg(k1 + u);
+    y[u] = __ldg(k2 + u);
+  }
+  for (int c4 = 0; c4 < n4; c4 += kExactStep) {
+    float4 xn[kExactStep], yn[kExactStep];
+    const bool more = c4 + kExactStep < n4;
+#pragma unroll
+    for (int u = 0; u < kExactStep; ++u) {
+      xn[u] = more ? __ldg(k1 + c4 + kExactStep + u) : x[u];
+      yn[u] = more ? __ldg(k2 + c4 + kExactStep + u) : y[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kExactStep; ++u) {
+      const float4 q = q4[c4 + u];
+      a = fmaf(q.x, x[u].x, a);
+      b = fmaf(q.x, y[u].x, b);
+      a = fmaf(q.y, x[u].y, a);
+      b = fmaf(q.y, y[u].y, b);
+      a = fmaf(q.z, x[u].z, a);
+      b = fmaf(q.z, y[u].z, b);
+      a = fmaf(q.w, x[u].w, a);
+      b = fmaf(q.w, y[u].w, b);
+    }
+#pragma unroll
+    for (int u = 0; u < kExactStep; ++u) {
+      x[u] = xn[u];
+      y[u] = yn[u];
+    }
+  }
+  s1 = a;
+  s2 = b;
+}
+
+// One warp per row (b, h, i).  The tensor-core scores s~ and the bound e_j give for every
+// key block an interval [lo_j, hi_j] = [s~_j - e_j, s~_j + e_j] that holds its exact score.
+// L = the k-th largest lo (radix select): at least k blocks score >= L, so a block with
+// hi_j < L is below k others and is not kept.  The others are the candidates: when there
+// are exactly k of them (most rows) they are the kept set; otherwise they get their exact
+// fp32 scores and a radix select over those picks the kept set (ties -> lower index) in
+// index order.  A row with a non-finite score or bound, or with more than kTopkCand
+// candidates, takes the exact score of every block instead.
+__global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const float* __restrict__ scores,
+                                                               int nbp, const float* __restrict__ qbar,
+                                                               const float* __restrict__ kbar,
+                                                               const float* __restrict__ knorm,
+                                                               int32_t* __restrict__ col_idx,
                                                                int* __restrict__ status) {
-  extern __shared__ uint32_t tsm[];
+  extern __shared__ __align__(16) uint32_t tsm[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * kTopkWarps + warp;
   const long long nrows = (long long)dm.B * dm.H * dm.nb;
   if (row >= nrows) return;
-  const int nb = dm.nb, kk = dm.k;
+  const int nb = dm.nb, kk = dm.k, d = dm.d;
+  int32_t* out = col_idx + row * kk;
+  if (kk >= nb) {   // every block is kept
+    for (int j = lane; j < nb; j += 32) out[j] = j;
+    return;
+  }
   uint32_t* key = tsm + warp * nbp;
   uint32_t* hist = tsm + kTopkWarps * nbp + warp * 256;
-  uint32_t* cand = tsm + kTopkWarps * (nbp + 256) + warp * kTopkCand;
-  const float* src = scores + row * nbp;
+  uint32_t* ckey = tsm + kTopkWarps * (nbp + 256) + warp * kTopkCand;
+  int* cidx = reinterpret_cast<int*>(tsm + kTopkWarps * (nbp + 256 + kTopkCand) + warp * kTopkCand);
+  float* qrow = reinterpret_cast<float*>(tsm + kTopkWarps * (nbp + 256 + 2 * kTopkCand) + warp * d);
+  const size_t bh = (size_t)(row / nb);
+  const float* kb = kbar + bh * nb * d;
+  const float* kn = knorm + bh * nbp;
   const unsigned full = 0xffffffffu;
   const unsigned lt_mask = (1u << lane) - 1u;
-  // Order-preserving map float -> uint32 (both zeros map to the key of +0); each lane
-  // also keeps the two largest of its keys.
-  uint32_t top1 = 0, top2 = 0;
-  for (int j = lane; j < nb; j += 32) {
-    float f = src[j];
-    if (f == 0.f) f = 0.f;
-    const uint32_t u = __float_as_uint(f);
-    const uint32_t kj = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    key[j] = kj;
-    top2 = max(top2, min(top1, kj));
-    top1 = max(top1, kj);
+
+  // the query block's mean (to shared memory) and its norm
+  float ss = 0.f;
+  for (int c = 4 * lane; c < d; c += 128) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(qbar + (size_t)row * d + c));
+    *reinterpret_cast<float4*>(qrow + c) = v;
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
   }
-  __syncwarp();
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(full, ss, off);
+  const float qn = sqrtf(ss);
+  const float cq = fmaf(kBoundRel, qn, kBoundAbs);   // e_j = cq |kbar_j| + c0
+  const float c0 = fmaf(kBoundAbs, qn, kBoundFloor);
 
   // One 8-bit radix step over keys[0, n) that match (prefix, pmask): picks the digit at
   // `shift` of the need-th largest and updates prefix, pmask and need (the count still to
@@ -315,53 +333,189 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(Dims dm, const fl
     pmask |= 255u << shift;
     __syncwarp();
   };
-  // Gathers the keys that satisfy `in` into cand (in any order; counts are all the radix
-  // steps take from them).  Returns their number (those past kTopkCand are not stored).
-  auto gather = [&](auto in) {
+  // The kk-th largest of keys[0, n) (prefix) and how many keys equal to it are kept (need):
+  // every key through the first digit; the keys still matching it are gathered into ckey
+  // (when they fit) for the other three.
+  auto select_kth = [&](const uint32_t* keys, int n, uint32_t& prefix, int& need) {
+    uint32_t pmask = 0;
+    prefix = 0;
+    need = kk;
+    radix_step(keys, n, 24, prefix, pmask, need);
     int nc = 0;
-    for (int j0 = 0; j0 < nb; j0 += 32) {
+    for (int j0 = 0; j0 < n; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t u = j < nb ? key[j] : 0u;
-      const bool take = j < nb && in(u);
+      const uint32_t u = j < n ? keys[j] : 0u;
+      const bool take = j < n && (u & pmask) == prefix;
       const unsigned bin = __ballot_sync(full, take);
       const int pos = nc + __popc(bin & lt_mask);
-      if (take && pos < kTopkCand) cand[pos] = u;
+      if (take && pos < kTopkCand) ckey[pos] = u;
       nc += __popc(bin);
     }
     __syncwarp();
-    return nc;
+    const uint32_t* src = nc <= kTopkCand ? ckey : keys;
+    const int ns = nc <= kTopkCand ? nc : n;
+    for (int pass = 1; pass < 4; ++pass) radix_step(src, ns, 24 - 8 * pass, prefix, pmask, need);
   };
 
-  uint32_t prefix = 0, pmask = 0;
-  int need = kk;
-  bool done = false;
-  if (kk <= 64 && nb >= 64) {
-    // Bound from below: T = the kk-th largest of the 64 lane top-twos is a key with at least
-    // kk keys at or above it, so the kk-th largest key is >= T; the keys >= T (usually little
-    // more than kk) are gathered and the exact select runs over them alone.
-    cand[lane] = top1;
-    cand[32 + lane] = top2;
-    __syncwarp();
-    uint32_t tp = 0, tm = 0;
-    int tn = kk;
-    for (int pass = 0; pass < 4; ++pass) radix_step(cand, 64, 24 - 8 * pass, tp, tm, tn);
-    const int nc = gather([&](uint32_t u) { return u >= tp; });
-    if (nc <= kTopkCand) {
-      for (int pass = 0; pass < 4; ++pass) radix_step(cand, nc, 24 - 8 * pass, prefix, pmask, need);
-      done = true;
+  // The kk-th largest (kk <= 64) of 64 keys held two per lane (0 = absent: no finite score
+  // maps to key 0).
+  auto kth_of64 = [&](uint32_t v0, uint32_t v1) -> uint32_t {
+    warp_sort64(v0, v1, lane);
+    const int e = 64 - kk;
+    return __shfl_sync(full, (e >> 5) ? v1 : v0, e & 31);
+  };
+
+  // Lower bounds lo_j as keys in shared memory; each lane keeps the two largest of its lo
+  // and the largest e_j.  The row is read as float4 (rows are nbp floats, nbp a multiple of
+  // 4), kTopkBatch per lane in flight.
+  const float4* src4 = reinterpret_cast<const float4*>(scores + row * nbp);
+  const float4* kn4 = reinterpret_cast<const float4*>(kn);
+  const int n4 = (nb + 3) >> 2;
+  uint32_t top1 = 0, top2 = 0;
+  float emax = 0.f;
+  bool finite = isfinite(qn);
+  for (int t0 = 0; t0 < n4; t0 += 32 * kTopkBatch) {
+    float4 sv[kTopkBatch], kv[kTopkBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int t = t0 + 32 * u + lane;
+      if (t < n4) {
+        sv[u] = __ldcs(src4 + t);
+        kv[u] = __ldg(kn4 + t);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int t = t0 + 32 * u + lane;
+      if (t < n4) {
+        const float s4[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+        const float k4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+        uint32_t l4[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool in = 4 * t + c < nb;
+          const float e = fmaf(cq, in ? k4[c] : 0.f, c0);
+          const float sc = in ? s4[c] : 0.f;
+          const float lo = sc - e;
+          finite = finite && isfinite(lo) && isfinite(sc + e);
+          l4[c] = in ? float_key(lo) : 0u;
+          top2 = max(top2, min(top1, l4[c]));
+          top1 = max(top1, l4[c]);
+          emax = fmaxf(emax, e);
+        }
+        *reinterpret_cast<uint4*>(key + 4 * t) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+      }
     }
   }
-  if (!done) {
-    // every key through the first digit; then the keys still matching it are gathered
-    // (when they fit) for the other three
-    radix_step(key, nb, 24, prefix, pmask, need);
-    const int nc = gather([&](uint32_t u) { return (u & pmask) == prefix; });
-    const uint32_t* src_keys = nc <= kTopkCand ? cand : key;
-    const int nsrc = nc <= kTopkCand ? nc : nb;
-    for (int pass = 1; pass < 4; ++pass) radix_step(src_keys, nsrc, 24 - 8 * pass, prefix, pmask, need);
+  __syncwarp();
+  uint32_t prefix = 0;
+  int need = kk;
+  if (__all_sync(full, finite)) {
+    // L = the kk-th largest lo.  T0 = the kk-th largest of the 64 lane top-twos is at most L
+    // (kk keys reach it); the lo at or above it (usually little more than kk) are gathered
+    // and L is the kk-th largest of those.  Both selections sort 64 keys in registers.
+    bool have_l = false;
+    if (kk <= 64) {
+      const uint32_t t0 = kth_of64(top1, top2);
+      int ng = 0;
+#pragma unroll 4
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t u = j < nb ? key[j] : 0u;
+        const bool take = j < nb && u >= t0;
+        const unsigned bin = __ballot_sync(full, take);
+        const int pos = ng + __popc(bin & lt_mask);
+        if (take && pos < kTopkCand) ckey[pos] = u;
+        ng += __popc(bin);
+      }
+      __syncwarp();
+      if (ng <= 64) {
+        prefix = kth_of64(lane < ng ? ckey[lane] : 0u, lane + 32 < ng ? ckey[lane + 32] : 0u);
+        have_l = true;
+      } else if (ng <= kTopkCand) {
+        uint32_t pmask = 0;
+        for (int pass = 0; pass < 4; ++pass) radix_step(ckey, ng, 24 - 8 * pass, prefix, pmask, need);
+        have_l = true;
+      }
+    }
+    if (!have_l) select_kth(key, nb, prefix, need);
+    // Candidates: hi_j >= L for some j is only possible if lo_j + 2 emax >= L.  Every other
+    // block scores below the kk blocks whose lo >= L.
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) emax = fmaxf(emax, __shfl_xor_sync(full, emax, off));
+    const uint32_t TL = float_key(key_float(prefix) - 2.f * emax);
+    int nc = 0;
+#pragma unroll 4
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      const bool take = j < nb && key[j] >= TL;
+      const unsigned bin = __ballot_sync(full, take);
+      const int pos = nc + __popc(bin & lt_mask);
+      if (take && pos < kTopkCand) cidx[pos] = j;
+      nc += __popc(bin);
+    }
+    __syncwarp();
+    if (nc == kk) {
+      // no block outside the kk can reach them: the boundary is settled without exact scores
+      for (int e = lane; e < kk; e += 32) out[e] = cidx[e];
+      return;
+    }
+    if (nc <= kTopkCand) {
+      for (int e0 = 0; e0 < nc; e0 += 64) {
+        const int a = e0 + lane, b = e0 + 32 + lane;
+        const int ja = a < nc ? cidx[a] : cidx[0];
+        const int jb = b < nc ? cidx[b] : ja;
+        float sa, sb;
+        exact_scores(qrow, kb, d, ja, jb, sa, sb);
+        if (a < nc) ckey[a] = float_key(sa);
+        if (b < nc) ckey[b] = float_key(sb);
+      }
+      __syncwarp();
+      if (kk <= 64 && nc <= 64) {
+        // the kk-th largest exact key, and how many equal to it are kept
+        prefix = kth_of64(lane < nc ? ckey[lane] : 0u, lane + 32 < nc ? ckey[lane + 32] : 0u);
+        const int above = __popc(__ballot_sync(full, lane < nc && ckey[lane] > prefix)) +
+                          __popc(__ballot_sync(full, lane + 32 < nc && ckey[lane + 32] > prefix));
+        need = kk - above;
+      } else {
+        uint32_t pmask = 0;
+        prefix = 0;
+        need = kk;
+        for (int pass = 0; pass < 4; ++pass) radix_step(ckey, nc, 24 - 8 * pass, prefix, pmask, need);
+      }
+      // the kept candidates in index order: above the k-th largest, or equal to it and
+      // among the first `need` such
+      int written = 0, eqseen = 0;
+      for (int e0 = 0; e0 < nc; e0 += 32) {
+        const int e = e0 + lane;
+        const uint32_t u = e < nc ? ckey[e] : 0u;
+        const bool gt = e < nc && u > prefix;
+        const bool eq = e < nc && u == prefix;
+        const unsigned beq = __ballot_sync(full, eq);
+        const bool keep = gt || (eq && eqseen + __popc(beq & lt_mask) < need);
+        const unsigned bk = __ballot_sync(full, keep);
+        const int pos = written + __popc(bk & lt_mask);
+        if (keep && pos < kk) out[pos] = cidx[e];
+        written += __popc(bk);
+        eqseen += __popc(beq);
+      }
+      if (lane == 0 && written != kk) record_status(status, kDevBounds);
+      return;
+    }
   }
-  // prefix is the k-th largest key; `need` elements equal to it are kept.
-  int32_t* out = col_idx + row * kk;
+
+  // every block's exact score, then the same select over the whole row
+  for (int j0 = 0; j0 < nb; j0 += 64) {
+    const int a = j0 + lane, b = j0 + 32 + lane;
+    const int ja = a < nb ? a : 0;
+    const int jb = b < nb ? b : ja;
+    float sa, sb;
+    exact_scores(qrow, kb, d, ja, jb, sa, sb);
+    if (a < nb) key[a] = float_key(sa);
+    if (b < nb) key[b] = float_key(sb);
+  }
+  __syncwarp();
+  select_kth(key, nb, prefix, need);
   int written = 0, eqseen = 0;
   for (int j0 = 0; j0 < nb; j0 += 32) {
     const int j = j0 + lane;
@@ -405,30 +559,26 @@ cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void
 
 int score_row_stride(const Dims& dm) { return (dm.nb + 3) / 4 * 4; }
 
-size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm)); }
+size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm), dm.d); }
 
 cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   const int nbp = score_row_stride(dm);
-  dim3 g1((dm.nb + kTS - 1) / kTS, (dm.nb + kTS - 1) / kTS, dm.B * dm.H);
-  cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+  cudaError_t e = launch_score_sm100(dm, ws, nbp, st);
   if (e != cudaSuccess) return e;
-  score_kernel<<<g1, 256, kScoreSmem, st>>>(dm, ws.qbar, ws.kbar, ws.scores, nbp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const size_t smem = topk_smem(nbp);
+  const size_t smem = topk_smem(nbp, dm.d);
   e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)dm.B * dm.H * dm.nb;
   topk_kernel<<<(unsigned)((rows + kTopkWarps - 1) / kTopkWarps), kTopkWarps * 32, smem, st>>>(
-      dm, ws.scores, nbp, ws.col_idx, ws.status);
+      dm, ws.scores, nbp, ws.qbar, ws.kbar, ws.knorm, ws.col_idx, ws.status);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ allocation-free variant
 //
 // Block selection for callers that cannot allocate device memory and have no workspace
-// to lend.  Its scratch (status word, pooled means, block scores) lives in one file-scope
-// device array of kSelectScratchBytes; every GPU that loads this library holds that array
+// to lend.  Its scratch (status word, pooled means, block scores and key norms) lives in
+// one file-scope device array of kSelectScratchBytes; every GPU that loads this library holds that array
 // until the process exits.  In host code `g_select_scratch` only names a host-side
 // stand-in, so its device address is looked up with cudaGetSymbolAddress, once per device
 // (on the first call made with that device current), and passed to the kernels.
@@ -449,7 +599,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 size_t select_noalloc_bytes(const Dims& dm) {
   const size_t BH = (size_t)dm.B * dm.H;
   return 256 + 2 * align256(sizeof(float) * BH * dm.nb * dm.d) +
-         align256(sizeof(float) * BH * dm.nb * score_row_stride(dm));
+         align256(sizeof(float) * BH * dm.nb * score_row_stride(dm)) + align256(sizeof(float) * BH * score_row_stride(dm));
 }
 
 size_t select_noalloc_capacity() { return kSelectScratchBytes; }
@@ -485,6 +635,8 @@ cudaError_t select_blocks_noalloc(const Dims& dm, rola_dtype dt, const void* q, 
   w.qbar = reinterpret_cast<float*>(base + 256);
   w.kbar = reinterpret_cast<float*>(base + 256 + align256(sizeof(float) * BH * dm.nb * dm.d));
   w.scores = reinterpret_cast<float*>(base + 256 + 2 * align256(sizeof(float) * BH * dm.nb * dm.d));
+  w.knorm = reinterpret_cast<float*>(reinterpret_cast<char*>(w.scores) +
+                                     align256(sizeof(float) * BH * dm.nb * score_row_stride(dm)));
   w.col_idx = col_idx;
   // The array keeps the previous call's contents: the status word must start at zero.
   e = cudaMemsetAsync(w.status, 0, 256, st);

@@ -123,6 +123,7 @@ size_t carve(const rola_params& p, const Dims& dm, char* base, Workspace* ws) {
   w.kbar = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * dm.d));
   w.col_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * BH * dm.nb * dm.k));
   w.scores = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nb * rola::score_row_stride(dm)));
+  w.knorm = reinterpret_cast<float*>(take(sizeof(float) * BH * rola::score_row_stride(dm)));
   w.S_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r * dm.d));
   w.z_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * dm.r));
   w.S = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r * dm.d));
@@ -417,6 +418,18 @@ rola_status rola_get_pooled(rola_plan_t plan, float* qbar, float* kbar, rola_str
   if (cudaMemcpyAsync(qbar, plan->ws.qbar, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return ROLA_ERR_CUDA;
   return cuda_status(cudaMemcpyAsync(kbar, plan->ws.kbar, bytes, cudaMemcpyDeviceToDevice, st));
+}
+
+rola_status rola_get_block_scores(rola_plan_t plan, float* scores, float* knorm, rola_stream_t stream) {
+  if (!plan || !scores || !knorm) return ROLA_ERR_INVALID_ARG;
+  const Dims& dm = plan->dm;
+  const size_t BH = (size_t)dm.B * dm.H, nbp = (size_t)rola::score_row_stride(dm);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpy2DAsync(scores, sizeof(float) * dm.nb, plan->ws.scores, sizeof(float) * nbp, sizeof(float) * dm.nb,
+                        BH * dm.nb, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  return cuda_status(cudaMemcpy2DAsync(knorm, sizeof(float) * dm.nb, plan->ws.knorm, sizeof(float) * nbp,
+                                       sizeof(float) * dm.nb, BH, cudaMemcpyDeviceToDevice, st));
 }
 
 rola_status rola_get_fp8_copies(rola_plan_t plan, uint8_t* q8, uint8_t* k8, uint8_t* v8, float* sq,

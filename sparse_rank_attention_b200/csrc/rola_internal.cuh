@@ -74,7 +74,8 @@ struct Workspace {
   float* qbar;        // [B, H, nb, d]
   float* kbar;        // [B, H, nb, d]
   int32_t* col_idx;   // [B, H, nb, k]
-  float* scores;      // [B, H, nb, nbp] block scores (nbp = nb rounded up to 4)
+  float* scores;      // [B, H, nb, nbp] tensor-core block scores (nbp = nb rounded up to 4)
+  float* knorm;       // [B, H, nbp] ||kbar_j||_2 (bounds the tensor-core scores' error)
   float* S_part;      // [B, H, nchunk, r, d]
   float* z_part;      // [B, H, nchunk, r]
   float* S;           // [B, H, r, d]
@@ -165,7 +166,11 @@ cudaError_t launch_state_reduce(const Dims& dm, const Workspace& ws, cudaStream_
 // bytes (64 channels of a 16-bit type, 128 of an 8-bit one).  False if encoding fails.
 bool make_act_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, const Dims& dm,
                   CUtensorMapSwizzle sw, uint32_t box_rows = 64);
-size_t select_smem_bytes(const Dims& dm);
+bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, uint64_t d0,
+                 uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw);
+// Tensor-core block scores s~ = qbar kbar^T (tf32) into ws.scores and the key-block norms
+// into ws.knorm: the input of the exact top-k (launch_select runs both).
+cudaError_t launch_score_sm100(const Dims& dm, const Workspace& ws, int nbp, cudaStream_t st);
 int score_row_stride(const Dims& dm);
 size_t select_noalloc_bytes(const Dims& dm);
 size_t select_noalloc_capacity();

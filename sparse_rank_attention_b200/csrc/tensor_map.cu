@@ -38,4 +38,18 @@ bool make_act_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, con
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [d2][d1][d0] tensor (d0 contiguous) with [box1 x box0] boxes; rows past d1 read as zeros
+// and are clipped on stores.  The row pitch d0 * el_bytes must be a multiple of 16 bytes.
+bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, uint32_t el_bytes, const void* ptr, uint64_t d0,
+                 uint64_t d1, uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * el_bytes, d0 * el_bytes * d1};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace rola

@@ -146,3 +146,25 @@ def test_backward_at_full_size_on_sampled_heads_and_blocks(wname):
     _compare("dWq", np32(got["dWq"])[heads], smp["dWq"])
     _compare("dWk", np32(got["dWk"])[heads], smp["dWk"])
     _compare("dg", np32(got["dg"])[heads], smp["dg"])
+
+
+def test_backward_with_peaked_softmax_rows():
+    """Key blocks scaled up along the sequence (the inputs that send forward tiles to the
+    careful pass): the softmax rows are peaked and their logits span a wide range; the
+    backward takes each row's exact lse, so it must hold the same bound."""
+    w = synth.custom("bwd_bf16_rising", B=1, H=2, N=4096, d=128, r=32, topk=0.25, grid=(4, 16, 64))
+    inp = synth.make_inputs(w, seed=7, device="cuda")
+    nb = w.nb
+    scale = 1.0 + 1.5 * torch.arange(nb, device="cuda", dtype=torch.float32) / nb
+    inp["k"] = (inp["k"].float() * scale.repeat_interleave(64)[: w.N].view(1, w.N, 1, 1)).to(inp["k"].dtype)
+    dout = synth.make_dout(w, seed=8, device="cuda")
+    plan = rola.Plan.for_workload(w)
+    got = plan.backward(inp["q"], inp["k"], inp["v"], inp["Wq"], inp["Wk"], inp["g"], dout)
+    assert plan.poll_status() == 0
+    h = host_inputs(inp)
+    s = O.make_shape(w.B, w.H, w.N, w.d, w.r, w.topk, grid=w.grid, pairs=w.pairs)
+    _, col = O.forward(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"])
+    np.testing.assert_array_equal(plan.block_lists().cpu().numpy(), col)
+    want = O.backward(s, h["q"], h["k"], h["v"], h["Wq"], h["Wk"], h["g"], np32(dout).astype(np.float64), col)
+    for key in ("dq", "dk", "dv", "dWq", "dWk", "dg"):
+        _compare(f"{w.name}/{key}", np32(got[key]), want[key].reshape(np32(got[key]).shape))
