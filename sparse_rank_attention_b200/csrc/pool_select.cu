@@ -138,8 +138,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const T* __restrict__ q, cons
 // ------------------------------------------------------------------ top-k per row
 
 constexpr int kTopkWarps = 8;
-constexpr int kTopkCand = 256;   // candidate blocks (or keys) kept apart, if they fit
-constexpr int kTopkBatch = 6;    // float4 loads of a score row in flight per lane
+constexpr int kTopkBatch = 3;    // float4 loads of a score row in flight per lane
 
 // Bound on |s~ - s| between the tensor-core score s~ and the exact score s of a pair:
 //   kBoundRel |qbar_i| |kbar_j| + kBoundAbs (|qbar_i| + |kbar_j|) + kBoundFloor
@@ -149,8 +148,14 @@ constexpr float kBoundRel = 0x1p-14f;
 constexpr float kBoundAbs = 0x1p-122f;
 constexpr float kBoundFloor = 0x1p-116f;
 
-__host__ __device__ inline size_t topk_smem(int nbp, int d) {
-  return sizeof(uint32_t) * ((size_t)kTopkWarps * (nbp + 256 + 2 * kTopkCand + d));
+// Candidate blocks (or keys) a warp keeps apart: room for k and a margin, 64 to 256.
+__host__ __device__ inline int topk_cand(int k) {
+  const int c = (k + 32 + 31) / 32 * 32;
+  return c < 64 ? 64 : (c > 256 ? 256 : c);
+}
+
+__host__ __device__ inline size_t topk_smem(int nbp, int d, int cand) {
+  return sizeof(uint32_t) * ((size_t)kTopkWarps * (nbp + 256 + 2 * cand + d));
 }
 
 // Order-preserving map float -> uint32 (both zeros map to the key of +0) and its inverse.
@@ -239,9 +244,9 @@ __device__ __forceinline__ void exact_scores(const float* qrow, const float* __r
 // hi_j < L is below k others and is not kept.  The others are the candidates: when there
 // are exactly k of them (most rows) they are the kept set; otherwise they get their exact
 // fp32 scores and a radix select over those picks the kept set (ties -> lower index) in
-// index order.  A row with a non-finite score or bound, or with more than kTopkCand
+// index order.  A row with a non-finite score or bound, or with more than `cand`
 // candidates, takes the exact score of every block instead.
-__global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const float* __restrict__ scores,
+__global__ void __launch_bounds__(kTopkWarps * 32, 4) topk_kernel(Dims dm, const float* __restrict__ scores,
                                                                int nbp, const float* __restrict__ qbar,
                                                                const float* __restrict__ kbar,
                                                                const float* __restrict__ knorm,
@@ -260,9 +265,10 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const
   }
   uint32_t* key = tsm + warp * nbp;
   uint32_t* hist = tsm + kTopkWarps * nbp + warp * 256;
-  uint32_t* ckey = tsm + kTopkWarps * (nbp + 256) + warp * kTopkCand;
-  int* cidx = reinterpret_cast<int*>(tsm + kTopkWarps * (nbp + 256 + kTopkCand) + warp * kTopkCand);
-  float* qrow = reinterpret_cast<float*>(tsm + kTopkWarps * (nbp + 256 + 2 * kTopkCand) + warp * d);
+  const int cand = topk_cand(kk);
+  uint32_t* ckey = tsm + kTopkWarps * (nbp + 256) + warp * cand;
+  int* cidx = reinterpret_cast<int*>(tsm + kTopkWarps * (nbp + 256 + cand) + warp * cand);
+  float* qrow = reinterpret_cast<float*>(tsm + kTopkWarps * (nbp + 256 + 2 * cand) + warp * d);
   const size_t bh = (size_t)(row / nb);
   const float* kb = kbar + bh * nb * d;
   const float* kn = knorm + bh * nbp;
@@ -348,12 +354,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const
       const bool take = j < n && (u & pmask) == prefix;
       const unsigned bin = __ballot_sync(full, take);
       const int pos = nc + __popc(bin & lt_mask);
-      if (take && pos < kTopkCand) ckey[pos] = u;
+      if (take && pos < cand) ckey[pos] = u;
       nc += __popc(bin);
     }
     __syncwarp();
-    const uint32_t* src = nc <= kTopkCand ? ckey : keys;
-    const int ns = nc <= kTopkCand ? nc : n;
+    const uint32_t* src = nc <= cand ? ckey : keys;
+    const int ns = nc <= cand ? nc : n;
     for (int pass = 1; pass < 4; ++pass) radix_step(src, ns, 24 - 8 * pass, prefix, pmask, need);
   };
 
@@ -366,14 +372,18 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const
   };
 
   // Lower bounds lo_j as keys in shared memory; each lane keeps the two largest of its lo
-  // and the largest e_j.  The row is read as float4 (rows are nbp floats, nbp a multiple of
-  // 4), kTopkBatch per lane in flight.
+  // and the largest e_j and |s~_j| (as bit patterns, so that a NaN is seen as the largest).
+  // lo_j = s~_j - e_j with e_j > 0 is never -0, so its key needs no zero fix-up.  The row
+  // is read as float4 (rows are nbp floats, nbp a multiple of 4), kTopkBatch per lane in
+  // flight.
   const float4* src4 = reinterpret_cast<const float4*>(scores + row * nbp);
   const float4* kn4 = reinterpret_cast<const float4*>(kn);
   const int n4 = (nb + 3) >> 2;
-  uint32_t top1 = 0, top2 = 0;
-  float emax = 0.f;
-  bool finite = isfinite(qn);
+  uint32_t top1 = 0, top2 = 0, ebits = 0, sbits = 0;
+  auto lo_key = [](float lo) {
+    const uint32_t u = __float_as_uint(lo);
+    return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+  };
   for (int t0 = 0; t0 < n4; t0 += 32 * kTopkBatch) {
     float4 sv[kTopkBatch], kv[kTopkBatch];
 #pragma unroll
@@ -390,33 +400,47 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const
       if (t < n4) {
         const float s4[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
         const float k4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+        const int nin = min(4, nb - 4 * t);   // blocks of this float4 below nb
         uint32_t l4[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const bool in = 4 * t + c < nb;
-          const float e = fmaf(cq, in ? k4[c] : 0.f, c0);
-          const float sc = in ? s4[c] : 0.f;
-          const float lo = sc - e;
-          finite = finite && isfinite(lo) && isfinite(sc + e);
-          l4[c] = in ? float_key(lo) : 0u;
-          top2 = max(top2, min(top1, l4[c]));
-          top1 = max(top1, l4[c]);
-          emax = fmaxf(emax, e);
+          if (c < nin) {
+            const float e = fmaf(cq, k4[c], c0);
+            l4[c] = lo_key(s4[c] - e);
+            ebits = max(ebits, __float_as_uint(e) & 0x7fffffffu);
+            sbits = max(sbits, __float_as_uint(s4[c]) & 0x7fffffffu);
+            top2 = max(top2, min(top1, l4[c]));
+            top1 = max(top1, l4[c]);
+          } else {
+            l4[c] = 0u;
+          }
         }
         *reinterpret_cast<uint4*>(key + 4 * t) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
       }
     }
   }
   __syncwarp();
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    ebits = max(ebits, __shfl_xor_sync(full, ebits, off));
+    sbits = max(sbits, __shfl_xor_sync(full, sbits, off));
+  }
+  const float emax = __uint_as_float(ebits);
+  // every lo_j and hi_j is finite (and so is every key) when max |s~| + 2 max e is
+  const bool finite = ebits < 0x7f800000u && sbits < 0x7f800000u && isfinite(__uint_as_float(sbits) + 2.f * emax);
   uint32_t prefix = 0;
   int need = kk;
-  if (__all_sync(full, finite)) {
-    // L = the kk-th largest lo.  T0 = the kk-th largest of the 64 lane top-twos is at most L
-    // (kk keys reach it); the lo at or above it (usually little more than kk) are gathered
-    // and L is the kk-th largest of those.  Both selections sort 64 keys in registers.
-    bool have_l = false;
+  if (finite) {
+    // L = the kk-th largest lo; candidates C = {lo_j >= L - 2 emax}: only they can have
+    // hi_j >= L, every other block scores below the kk blocks whose lo >= L.
+    // T0 = the kk-th largest of the 64 lane top-twos is at most L (kk keys reach it), so
+    // G = {lo_j >= T0 - 2 emax} (usually little more than kk blocks) holds both the top kk
+    // lo and C: L is selected within G and C filtered out of it, in index order.
+    bool have_c = false;
+    int nc = 0;
     if (kk <= 64) {
-      const uint32_t t0 = kth_of64(top1, top2);
+      const uint32_t T0 = kth_of64(top1, top2);   // 0 when fewer than kk blocks: take all
+      const uint32_t t0 = T0 ? lo_key(key_float(T0) - 2.f * emax) : 0u;
       int ng = 0;
 #pragma unroll 4
       for (int j0 = 0; j0 < nb; j0 += 32) {
@@ -425,42 +449,55 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3) topk_kernel(Dims dm, const
         const bool take = j < nb && u >= t0;
         const unsigned bin = __ballot_sync(full, take);
         const int pos = ng + __popc(bin & lt_mask);
-        if (take && pos < kTopkCand) ckey[pos] = u;
+        if (take && pos < cand) {
+          ckey[pos] = u;
+          cidx[pos] = j;
+        }
         ng += __popc(bin);
       }
       __syncwarp();
-      if (ng <= 64) {
-        prefix = kth_of64(lane < ng ? ckey[lane] : 0u, lane + 32 < ng ? ckey[lane + 32] : 0u);
-        have_l = true;
-      } else if (ng <= kTopkCand) {
-        uint32_t pmask = 0;
-        for (int pass = 0; pass < 4; ++pass) radix_step(ckey, ng, 24 - 8 * pass, prefix, pmask, need);
-        have_l = true;
+      if (ng <= cand) {
+        if (ng <= 64) {
+          prefix = kth_of64(lane < ng ? ckey[lane] : 0u, lane + 32 < ng ? ckey[lane + 32] : 0u);
+        } else {
+          uint32_t pmask = 0;
+          for (int pass = 0; pass < 4; ++pass) radix_step(ckey, ng, 24 - 8 * pass, prefix, pmask, need);
+        }
+        const uint32_t TL = lo_key(key_float(prefix) - 2.f * emax);
+        for (int e0 = 0; e0 < ng; e0 += 32) {   // compaction in place: entries are read first
+          const int e = e0 + lane;
+          const bool take = e < ng && ckey[e] >= TL;
+          const int j = take ? cidx[e] : 0;
+          const unsigned bin = __ballot_sync(full, take);
+          const int pos = nc + __popc(bin & lt_mask);
+          __syncwarp();
+          if (take) cidx[pos] = j;
+          nc += __popc(bin);
+        }
+        __syncwarp();
+        have_c = true;
       }
     }
-    if (!have_l) select_kth(key, nb, prefix, need);
-    // Candidates: hi_j >= L for some j is only possible if lo_j + 2 emax >= L.  Every other
-    // block scores below the kk blocks whose lo >= L.
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) emax = fmaxf(emax, __shfl_xor_sync(full, emax, off));
-    const uint32_t TL = float_key(key_float(prefix) - 2.f * emax);
-    int nc = 0;
+    if (!have_c) {
+      select_kth(key, nb, prefix, need);
+      const uint32_t TL = lo_key(key_float(prefix) - 2.f * emax);
 #pragma unroll 4
-    for (int j0 = 0; j0 < nb; j0 += 32) {
-      const int j = j0 + lane;
-      const bool take = j < nb && key[j] >= TL;
-      const unsigned bin = __ballot_sync(full, take);
-      const int pos = nc + __popc(bin & lt_mask);
-      if (take && pos < kTopkCand) cidx[pos] = j;
-      nc += __popc(bin);
+      for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const bool take = j < nb && key[j] >= TL;
+        const unsigned bin = __ballot_sync(full, take);
+        const int pos = nc + __popc(bin & lt_mask);
+        if (take && pos < cand) cidx[pos] = j;
+        nc += __popc(bin);
+      }
+      __syncwarp();
     }
-    __syncwarp();
     if (nc == kk) {
       // no block outside the kk can reach them: the boundary is settled without exact scores
       for (int e = lane; e < kk; e += 32) out[e] = cidx[e];
       return;
     }
-    if (nc <= kTopkCand) {
+    if (nc <= cand) {
       for (int e0 = 0; e0 < nc; e0 += 64) {
         const int a = e0 + lane, b = e0 + 32 + lane;
         const int ja = a < nc ? cidx[a] : cidx[0];
@@ -559,13 +596,13 @@ cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void
 
 int score_row_stride(const Dims& dm) { return (dm.nb + 3) / 4 * 4; }
 
-size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm), dm.d); }
+size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm), dm.d, topk_cand(dm.k)); }
 
 cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   const int nbp = score_row_stride(dm);
   cudaError_t e = launch_score_sm100(dm, ws, nbp, st);
   if (e != cudaSuccess) return e;
-  const size_t smem = topk_smem(nbp, dm.d);
+  const size_t smem = topk_smem(nbp, dm.d, topk_cand(dm.k));
   e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)dm.B * dm.H * dm.nb;
