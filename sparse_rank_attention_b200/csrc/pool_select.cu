@@ -371,15 +371,16 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 4) topk_kernel(Dims dm, const
     return __shfl_sync(full, (e >> 5) ? v1 : v0, e & 31);
   };
 
-  // Lower bounds lo_j as keys in shared memory; each lane keeps the two largest of its lo
-  // and the largest e_j and |s~_j| (as bit patterns, so that a NaN is seen as the largest).
-  // lo_j = s~_j - e_j with e_j > 0 is never -0, so its key needs no zero fix-up.  The row
+  // Lower bounds lo_j as keys in shared memory; each lane keeps the two largest and the
+  // smallest of its keys and the largest e_j.  lo_j = s~_j - e_j with e_j > 0 is never -0, so
+  // its key needs no zero fix-up; a NaN lo has a key above +inf's or below -inf's.  The row
   // is read as float4 (rows are nbp floats, nbp a multiple of 4), kTopkBatch per lane in
   // flight.
   const float4* src4 = reinterpret_cast<const float4*>(scores + row * nbp);
   const float4* kn4 = reinterpret_cast<const float4*>(kn);
   const int n4 = (nb + 3) >> 2;
-  uint32_t top1 = 0, top2 = 0, ebits = 0, sbits = 0;
+  uint32_t top1 = 0, top2 = 0, kmin = 0xffffffffu;
+  float emax = 0.f;
   auto lo_key = [](float lo) {
     const uint32_t u = __float_as_uint(lo);
     return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
@@ -407,8 +408,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 4) topk_kernel(Dims dm, const
           if (c < nin) {
             const float e = fmaf(cq, k4[c], c0);
             l4[c] = lo_key(s4[c] - e);
-            ebits = max(ebits, __float_as_uint(e) & 0x7fffffffu);
-            sbits = max(sbits, __float_as_uint(s4[c]) & 0x7fffffffu);
+            emax = fmaxf(emax, e);
+            kmin = min(kmin, l4[c]);
             top2 = max(top2, min(top1, l4[c]));
             top1 = max(top1, l4[c]);
           } else {
@@ -420,14 +421,16 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 4) topk_kernel(Dims dm, const
     }
   }
   __syncwarp();
+  uint32_t kmax = top1;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    ebits = max(ebits, __shfl_xor_sync(full, ebits, off));
-    sbits = max(sbits, __shfl_xor_sync(full, sbits, off));
+    emax = fmaxf(emax, __shfl_xor_sync(full, emax, off));
+    kmin = min(kmin, __shfl_xor_sync(full, kmin, off));
+    kmax = max(kmax, __shfl_xor_sync(full, kmax, off));
   }
-  const float emax = __uint_as_float(ebits);
-  // every lo_j and hi_j is finite (and so is every key) when max |s~| + 2 max e is
-  const bool finite = ebits < 0x7f800000u && sbits < 0x7f800000u && isfinite(__uint_as_float(sbits) + 2.f * emax);
+  // every lo_j is finite when the keys lie strictly between those of -inf and +inf (a NaN e
+  // or s~ makes lo NaN), and every hi_j <= max lo + 2 max e is finite when that sum is
+  const bool finite = kmin > 0x007fffffu && kmax < 0xff800000u && isfinite(key_float(kmax) + 2.f * emax);
   uint32_t prefix = 0;
   int need = kk;
   if (finite) {

@@ -310,8 +310,7 @@ __global__ void __launch_bounds__(QRoles<FP8>::kThreads, 2) query_features_kerne
       const int ch = (cp >> 2) & 7;                                 // chunk within the box
       for (int r = 0; r < cnt; ++r) {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(col + r * 128 + ((ch ^ (r & 7)) << 4));
-        a0 = a0 + __uint_as_float(w << 16);
-        a1 = a1 + __uint_as_float(w & 0xffff0000u);
+        add2(a0, a1, __uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));   // token order, as fadd
       }
       *reinterpret_cast<float2*>(qbar + ((size_t)bh * dm.nb + i) * kD + 2 * cp) =
           make_float2(__fdiv_rn(a0, (float)cnt), __fdiv_rn(a1, (float)cnt));
@@ -328,14 +327,10 @@ __global__ void __launch_bounds__(QRoles<FP8>::kThreads, 2) query_features_kerne
       if (named_vote_or(3, 64, !ok)) break;
       const uint8_t* pQ = smem + G::offQ + s * kTileBytes;
       const int cnt = min(kBlock, dm.N - n0);
-      float am = 0.f;
-      for (int e = tq; e < cnt * 16; e += 64) {
-        const uint4 v = *reinterpret_cast<const uint4*>(pQ + swz(e >> 4, e & 15));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          am = fmaxf(am, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xffff0000u))));
-      }
+      uint32_t amb = 0;   // largest |q| of the thread's elements, as bf16 patterns
+      for (int e = tq; e < cnt * 16; e += 64)
+        amb = __vmaxu2(amb, bf16x8_absmax_bits(*reinterpret_cast<const uint4*>(pQ + swz(e >> 4, e & 15))));
+      float am = bf16_absmax_value(amb);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
       if (lane == 0) ctl->red[warp - 10] = am;
@@ -349,9 +344,10 @@ __global__ void __launch_bounds__(QRoles<FP8>::kThreads, 2) query_features_kerne
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[2] = {0, 0};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = make_float2(__uint_as_float(w[u] << 16) * inv, __uint_as_float(w[u] & 0xffff0000u) * inv);
-          o[u >> 1] |= (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3) << (16 * (u & 1));
+        for (int u = 0; u < 4; ++u) {   // each product rounded as a scalar multiply, two per f32x2
+          float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+          mul2(x0, x1, inv, inv);
+          o[u >> 1] |= (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3) << (16 * (u & 1));
         }
         *reinterpret_cast<uint2*>(q8 + ((size_t)b * dm.N + n0 + r) * rs + (size_t)h * kD + cv * 8) =
             make_uint2(o[0], o[1]);

@@ -193,6 +193,18 @@ __device__ __forceinline__ int v16_exponent(float absmax) {
   return (e2 - 1) - 14;
 }
 
+// Largest |x| over the bf16 pairs of v, per 16-bit half: with the sign bit cleared, bf16
+// patterns order as unsigned integers by magnitude (NaN above inf above every finite value),
+// so one unsigned max per pair of halves does it.  bf16_absmax_value() folds the two halves
+// into the float value (exact).
+__device__ __forceinline__ uint32_t bf16x8_absmax_bits(const uint4& v) {
+  const uint32_t m = 0x7fff7fffu;
+  return __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+}
+__device__ __forceinline__ float bf16_absmax_value(uint32_t halves) {
+  return __uint_as_float(max(halves & 0xffffu, halves >> 16) << 16);
+}
+
 // Rotary cos/sin of pair c for token n.
 __device__ __forceinline__ float2 rope_cs(const Dims& dm, const float2* __restrict__ rope, int n,
                                           int c) {
