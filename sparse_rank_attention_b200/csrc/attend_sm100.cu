@@ -116,37 +116,6 @@ template <bool FP8>
 constexpr size_t smem_bytes() { return Geo<FP8>::kOffCtl + sizeof(Ctl) + 1024; }
 
 
-// Reduce 32 per-lane values over the warp; lane l receives entry l (31 shuffles).
-template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(const float* x, int lane) {
-  const unsigned full = 0xffffffffu;
-  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
-  float b[16], c[8], d[4], e2[2];
-  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2, h1 = lane & 1;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float mine = h16 ? x[16 + e] : x[e], send = h16 ? x[e] : x[16 + e];
-    b[e] = op(mine, __shfl_xor_sync(full, send, 16));
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float mine = h8 ? b[8 + e] : b[e], send = h8 ? b[e] : b[8 + e];
-    c[e] = op(mine, __shfl_xor_sync(full, send, 8));
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float mine = h4 ? c[4 + e] : c[e], send = h4 ? c[e] : c[4 + e];
-    d[e] = op(mine, __shfl_xor_sync(full, send, 4));
-  }
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float mine = h2 ? d[2 + e] : d[e], send = h2 ? d[e] : d[2 + e];
-    e2[e] = op(mine, __shfl_xor_sync(full, send, 2));
-  }
-  const float mine = h1 ? e2[1] : e2[0], send = h1 ? e2[0] : e2[1];
-  return op(mine, __shfl_xor_sync(full, send, 1));
-}
-
 // Writes NC 16-byte chunks (4 packed words each), logical chunks c0 .. c0 + NC - 1 of
 // row `row` of a SW128 tile (128-byte rows): chunk c goes to position c ^ (row % 8).
 template <int NC>

@@ -417,17 +417,15 @@ __device__ __forceinline__ void mma_rows_xb(float (&acc)[D / 8][4], const float 
 // row's D is accumulated online like its softmax sum, from dP = dout V^T (one exact bf16
 // product per block) instead of forming O.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
+__device__ __forceinline__ void rowstats_mma_tile(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    const __nv_bfloat16* __restrict__ dout, Dims dm, const int32_t* __restrict__ col_idx, float* __restrict__ lse,
-    float* __restrict__ Drow, int* __restrict__ status) {
+    const __nv_bfloat16* __restrict__ dout, const Dims& dm, const int32_t* __restrict__ col_idx,
+    float* __restrict__ lse, float* __restrict__ Drow, int* __restrict__ status, int i, int bh, unsigned char* smb) {
   using L = MmaTiles<D>;
-  extern __shared__ __align__(16) unsigned char smb[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smb);
   __nv_bfloat16* sG = sQ + L::kTile;
   __nv_bfloat16* sK = sG + L::kTile;
   __nv_bfloat16* sV = sK + L::kTile;
-  const int i = blockIdx.x, bh = blockIdx.y;
   const int b = bh / dm.H, h = bh % dm.H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, t4 = lane & 3;
   const int32_t* Lst = col_idx + ((size_t)bh * dm.nb + i) * dm.k;
@@ -490,6 +488,34 @@ __global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
       lse[at] = n < dm.N ? m[hh] + log2f(lt) : INFINITY;   // log2 units of scale * log2(e) * q.k
       Drow[at] = n < dm.N ? dt / lt : 0.f;
     }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_rowstats_mma_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const __nv_bfloat16* __restrict__ dout, Dims dm, const int32_t* __restrict__ col_idx, float* __restrict__ lse,
+    float* __restrict__ Drow, int* __restrict__ status) {
+  extern __shared__ __align__(16) unsigned char smb[];
+  rowstats_mma_tile<D>(q, k, v, dout, dm, col_idx, lse, Drow, status, blockIdx.x, blockIdx.y, smb);
+}
+
+// The query tiles listed in redo (count, then tiles b*H*nb + h*nb + i), grid-strided.
+template <int D>
+__global__ void __launch_bounds__(128) bwd_rowstats_redo_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const __nv_bfloat16* __restrict__ dout, Dims dm, const int32_t* __restrict__ col_idx, float* __restrict__ lse,
+    float* __restrict__ Drow, const int* __restrict__ redo, int* __restrict__ status) {
+  extern __shared__ __align__(16) unsigned char smb[];
+  const int count = min(redo[0], dm.B * dm.H * dm.nb);   // each tile is listed at most once
+  for (int e = blockIdx.x; e < count; e += gridDim.x) {
+    const int tau = redo[1 + e];
+    if (tau < 0 || tau >= dm.B * dm.H * dm.nb) {
+      if (threadIdx.x == 0) record_status(status, kDevBounds);
+      continue;
+    }
+    __syncthreads();   // the previous tile's shared memory is read out
+    rowstats_mma_tile<D>(q, k, v, dout, dm, col_idx, lse, Drow, status, tau % dm.nb, tau / dm.nb, smb);
   }
 }
 
@@ -1100,8 +1126,17 @@ cudaError_t launch_all(const Dims& dm, const void* q_, const void* k_, const voi
         (e = cudaFuncSetAttribute(bwd_dkv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)mm_smem)) != cudaSuccess)
       return e;
-    bwd_rowstats_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow,
-                                                            ws.status);
+    if constexpr (D == 128) {   // tcgen05, with the rare overflowing tiles redone block by block
+      if ((e = cudaFuncSetAttribute(bwd_rowstats_redo_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)mm_smem)) != cudaSuccess)
+        return e;
+      if ((e = launch_bwd_rowstats_sm100(dm, q, k, v, dout, ws, bw, st)) != cudaSuccess) return e;
+      bwd_rowstats_redo_kernel<D><<<296, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow, bw.redo,
+                                                             ws.status);
+    } else {
+      bwd_rowstats_mma_kernel<D><<<gtile, 128, mm_smem, st>>>(q, k, v, dout, dm, ws.col_idx, bw.lse, bw.Drow,
+                                                              ws.status);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if constexpr (D == 128) {   // the forward's transposed tcgen05 tile
       if ((e = launch_bwd_dq_sm100(dm, q, k, v, dout, ws, bw, dq, st)) != cudaSuccess) return e;
@@ -1165,6 +1200,7 @@ size_t backward_workspace_bytes(const Dims& dm, BwdWorkspace* bw, char* base) {
   w.dg_part = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.nchunk * (dm.d + 1)));
   w.dS = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r * dm.d));
   w.dz = reinterpret_cast<float*>(take(sizeof(float) * BH * dm.r));
+  w.redo = reinterpret_cast<int*>(take(sizeof(int) * (1 + BH * dm.nb)));
   if (bw) *bw = w;
   return off;
 }

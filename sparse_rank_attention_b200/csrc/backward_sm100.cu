@@ -688,7 +688,332 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_sm100_kernel(
   }
 }
 
+// ------------------------------------------------------------------ row statistics
+// Per query block i, over the pairs of its kept key blocks (as for dq):
+//   S^T [128 keys x 64 q] = [K_j1; K_j2] Q_i^T,   dP^T = [V_j1; V_j2] dout_i^T
+// and per query column c: m_c = the first pair's column max of s = S^T scale log2(e) over
+// valid keys, p = 2^(s - m_c), l_c = sum p, e_c = sum p dP over every valid key of the list;
+// lse_c = m_c + log2(l_c) (log2 units), D_c = e_c / l_c = dout . O_sparse.  Each thread keeps
+// its TMEM lane's (its key's) partial sums for its group's 32 columns; one reduction per tile
+// (a warp reduce-scatter, then the four warps in a fixed order).  A tile where some p would
+// exceed 2^64 (a key far above the first pair's max) is listed for the warp-level kernel,
+// which rescales block by block.
+// Roles (384 threads): warp 0 = TMA producer of Q and dout (one slot) and the K ring; warp 1 =
+// issuer of S^T and dP^T and TMEM owner; warp 3 = the V ring; warps 4-11 = two groups of four
+// over query columns [32 g, 32 g + 32).
+namespace rsx {
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr uint32_t kTmemCols = 256;   // S^T (0, 64), dP^T (128, 192)
+constexpr uint32_t kOffQG = 0;        // Q (16 KB) then dout (16 KB)
+constexpr uint32_t kOffK = 32768;
+constexpr uint32_t kOffV = kOffK + kKStages * kPairBytes;
+constexpr uint32_t kOffCtl = kOffV + kVStages * kPairBytes;
+
+struct Ctl {
+  uint64_t qg_full, qg_free, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  alignas(16) float red[2][2][4][32];   // per group: l and e (or the max), per warp, per column
+  alignas(16) float mcol[2][32];        // per group: the tile's column offsets
+};
+constexpr size_t kSmemBytes = kOffCtl + sizeof(Ctl) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
+}  // namespace rsx
+
+__global__ void __launch_bounds__(kThreads, 1) bwd_rowstats_sm100_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Dims dm,
+    const int32_t* __restrict__ col_idx, float* __restrict__ lse, float* __restrict__ Drow, int* __restrict__ redo,
+    int* __restrict__ status, unsigned long long limit_cycles) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  rsx::Ctl* ctl = reinterpret_cast<rsx::Ctl*>(base + rsx::kOffCtl);
+  const uint32_t sbase = smem_addr(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = dm.nb * dm.B * dm.H;
+  const int kk_list = dm.k, npairs = (kk_list + 1) >> 1;
+  const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto bar = [&](uint64_t& m) { return smem_addr(&m); };
+  auto tile_of = [&](int jt) { return (int)blockIdx.x + jt * (int)gridDim.x; };
+  auto list_of = [&](int tau) { return col_idx + (size_t)tau * kk_list; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(ctl->qg_full), 1);
+    mbar_init(bar(ctl->qg_free), 1);
+    for (int s = 0; s < rsx::kKStages; ++s) {
+      mbar_init(bar(ctl->k_full[s]), 1);
+      mbar_init(bar(ctl->k_empty[s]), 1);
+    }
+    for (int s = 0; s < rsx::kVStages; ++s) {
+      mbar_init(bar(ctl->v_full[s]), 1);
+      mbar_init(bar(ctl->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(ctl->s_full[s]), 1);
+      mbar_init(bar(ctl->s_free[s]), kSoftmaxWarps);
+    }
+    mbar_init(bar(ctl->drain), 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), rsx::kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtl wc{&ctl->abort, status, limit_cycles};
+  auto pair_blocks = [&](const int32_t* L, int it, int& j1, int& j2) {
+    j1 = __ldg(L + 2 * it);
+    j2 = (2 * it + 1 < kk_list) ? __ldg(L + 2 * it + 1) : j1;
+    if (j1 < 0 || j1 >= dm.nb || j2 < 0 || j2 >= dm.nb) {
+      atomicCAS(status, 0, kDevBounds);
+      j1 = j2 = 0;
+    }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q, dout and the K ring
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_g);
+      tma_prefetch_desc(&tm_k);
+      int gp = 0, nqg = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        const int tau = tile_of(jt);
+        const int bh = tau / dm.nb, i = tau - bh * dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        if (jt > 0 && !mbar_wait(bar(ctl->qg_free), (jt - 1) & 1, wc)) break;
+        mbar_expect_tx(bar(ctl->qg_full), 32768);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + rsx::kOffQG + c * 8192, &tm_q, xh + 64 * c, i * 64, b, bar(ctl->qg_full));
+          tma_load_3d(sbase + rsx::kOffQG + 16384 + c * 8192, &tm_g, xh + 64 * c, i * 64, b, bar(ctl->qg_full));
+        }
+        ++nqg;
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int s = gp % rsx::kKStages;
+          if (gp >= rsx::kKStages && !mbar_wait(bar(ctl->k_empty[s]), ((gp / rsx::kKStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + rsx::kOffK + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->k_full[s]), kPairBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_k, xh + 64 * c, j1 * 64, b, bar(ctl->k_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_k, xh + 64 * c, j2 * 64, b, bar(ctl->k_full[s]));
+          }
+        }
+      }
+      if (nqg > 0) mbar_wait(bar(ctl->qg_full), (nqg - 1) & 1, wc, false);
+      for (int x = (gp > rsx::kKStages ? gp - rsx::kKStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->k_full[x % rsx::kKStages]), (x / rsx::kKStages) & 1, wc, false);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ the V ring
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_v);
+      int gp = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        const int tau = tile_of(jt);
+        const int bh = tau / dm.nb, b = bh / dm.H, xh = (bh % dm.H) * 128;
+        const int32_t* L = list_of(tau);
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int s = gp % rsx::kVStages;
+          if (gp >= rsx::kVStages && !mbar_wait(bar(ctl->v_empty[s]), ((gp / rsx::kVStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          int j1, j2;
+          pair_blocks(L, it, j1, j2);
+          const uint32_t st = sbase + rsx::kOffV + s * kPairBytes;
+          mbar_expect_tx(bar(ctl->v_full[s]), kPairBytes);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(st + c * kBoxKV, &tm_v, xh + 64 * c, j1 * 64, b, bar(ctl->v_full[s]));
+            tma_load_3d(st + c * kBoxKV + 8192, &tm_v, xh + 64 * c, j2 * 64, b, bar(ctl->v_full[s]));
+          }
+        }
+      }
+      for (int x = (gp > rsx::kVStages ? gp - rsx::kVStages : 0); x < gp; ++x)
+        mbar_wait(bar(ctl->v_full[x % rsx::kVStages]), (x / rsx::kVStages) & 1, wc, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S^T and dP^T
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(1, 128, 64, 0, 0);
+      int gp = 0;
+      bool ok = true;
+      for (int jt = 0; ok && jt < my_tiles; ++jt) {
+        if (!mbar_wait(bar(ctl->qg_full), jt & 1, wc)) break;
+        const uint64_t dqd = sdesc_sw128(sbase + rsx::kOffQG, 16, 1024);
+        const uint64_t dgd = sdesc_sw128(sbase + rsx::kOffQG + 16384, 16, 1024);
+        for (int it = 0; it < npairs; ++it, ++gp) {
+          const int ks = gp % rsx::kKStages, vs = gp % rsx::kVStages, sb = gp & 1;
+          if (!mbar_wait(bar(ctl->k_full[ks]), (gp / rsx::kKStages) & 1, wc) ||
+              !mbar_wait(bar(ctl->v_full[vs]), (gp / rsx::kVStages) & 1, wc) ||
+              (gp >= 2 && !mbar_wait(bar(ctl->s_free[sb]), ((gp - 2) >> 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dk = sdesc_sw128(sbase + rsx::kOffK + ks * kPairBytes, 16, 1024);
+          const uint64_t dv = sdesc_sw128(sbase + rsx::kOffV + vs * kPairBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {   // K-step offsets: 32 B inside a box, boxes 16 KB / 8 KB apart
+            const uint32_t ab = ((kk >> 2) * kBoxKV + (kk & 3) * 32) >> 4, bb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tmem + kColS + 64 * sb, dk + ab, dqd + bb, idesc, kk > 0);
+            mma_f16_ss(tmem + kColDP + 64 * sb, dv + ab, dgd + bb, idesc, kk > 0);
+          }
+          mma_commit(bar(ctl->s_full[sb]));
+          mma_commit(bar(ctl->k_empty[ks]));
+          mma_commit(bar(ctl->v_empty[vs]));
+        }
+        if (ok) mma_commit(bar(ctl->qg_free));   // this tile's Q and dout are read
+      }
+      mma_commit(bar(ctl->drain));
+      mbar_wait(bar(ctl->drain), 0, wc, false);
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ the statistics
+    const int g = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;
+    const int t = 32 * wq + lane;                  // TMEM lane: key t of the pair
+    const int c0 = 32 * g;
+    const uint32_t gbar = 1 + g;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * wq) << 16);
+    const float sl2 = dm.scale * 1.4426950408889634f;
+    bool fail = false;
+    int gp = 0;
+    for (int jt = 0; jt < my_tiles; ++jt) {
+      const int tau = tile_of(jt);
+      const int bh = tau / dm.nb, i = tau - bh * dm.nb;
+      const int32_t* L = list_of(tau);
+      float m[32], ls[32], es[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        ls[c] = 0.f;
+        es[c] = 0.f;
+      }
+      bool over = false;
+      for (int it = 0; it < npairs; ++it, ++gp) {
+        const int sb = gp & 1;
+        const bool ok = !fail && mbar_wait(bar(ctl->s_full[sb]), (gp >> 1) & 1, wc);
+        fail |= !ok;
+        tc_fence_after();
+        const int e = 2 * it + (t >> 6);
+        const int jb = e < kk_list ? __ldg(L + e) : -1;
+        const bool valid = jb >= 0 && jb < dm.nb && jb * 64 + (t & 63) < dm.N;
+        if (it == 0) {
+          // the tile's column offsets: the max of s over the first pair's valid keys
+          float x[32];
+          tmem_ld32(lane_addr + kColS + 64 * sb + c0, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = valid ? x[c] * sl2 : -INFINITY;
+          ctl->red[g][0][wq][lane] = reduce_scatter32<true>(x, lane);
+          named_sync(gbar, 128);
+          if (wq == 0)
+            ctl->mcol[g][lane] = fmaxf(fmaxf(ctl->red[g][0][0][lane], ctl->red[g][0][1][lane]),
+                                       fmaxf(ctl->red[g][0][2][lane], ctl->red[g][0][3][lane]));
+          named_sync(gbar, 128);
+          const float4* m4 = reinterpret_cast<const float4*>(ctl->mcol[g]);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 v4 = m4[c4];
+            m[4 * c4] = v4.x;
+            m[4 * c4 + 1] = v4.y;
+            m[4 * c4 + 2] = v4.z;
+            m[4 * c4 + 3] = v4.w;
+          }
+        }
+        // sixteen columns at a time: p = 2^(s - m), l += p, e += p dP
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[16], dp[16];
+          tmem_ld16(lane_addr + kColS + 64 * sb + c0 + 16 * hh, x);
+          tmem_ld16(lane_addr + kColDP + 64 * sb + c0 + 16 * hh, dp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float a = fmaf(x[c], sl2, -m[16 * hh + c]);
+            over |= valid && a > 64.f;
+            const float p = valid ? exp2f(a) : 0.f;
+            ls[16 * hh + c] += p;
+            es[16 * hh + c] = fmaf(p, dp[c], es[16 * hh + c]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(bar(ctl->s_free[sb]));
+      }
+      // the tile's statistics: l and e summed over the 128 keys of every pair, in a fixed order.
+      // Both votes span the two groups: they leave together on a failed wait, and a tile with
+      // an overflowing p in either group is listed once and written by neither.
+      if (named_vote_or(3, 256, fail)) break;
+      const bool bad = named_vote_or(3, 256, over);
+      const float lw = reduce_scatter32<false>(ls, lane), ew = reduce_scatter32<false>(es, lane);
+      ctl->red[g][0][wq][lane] = lw;
+      ctl->red[g][1][wq][lane] = ew;
+      named_sync(gbar, 128);
+      if (wq == 0) {
+        const float lt = ((ctl->red[g][0][0][lane] + ctl->red[g][0][1][lane]) + ctl->red[g][0][2][lane]) +
+                         ctl->red[g][0][3][lane];
+        const float et = ((ctl->red[g][1][0][lane] + ctl->red[g][1][1][lane]) + ctl->red[g][1][2][lane]) +
+                         ctl->red[g][1][3][lane];
+        const int n = i * 64 + c0 + lane;
+        const size_t at = (size_t)bh * dm.nb * 64 + (size_t)i * 64 + c0 + lane;
+        if (!bad) {
+          lse[at] = n < dm.N ? ctl->mcol[g][lane] + log2f(lt) : INFINITY;
+          Drow[at] = n < dm.N ? et / lt : 0.f;
+        } else if (g == 0 && lane == 0) {
+          redo[1 + atomicAdd(redo, 1)] = tau;      // at most once per tile: the list holds every tile
+        }
+      }
+      named_sync(gbar, 128);                         // red and mcol are rewritten next tile
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, rsx::kTmemCols);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_bwd_rowstats_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                                     const Workspace& ws, const BwdWorkspace& bw, cudaStream_t st) {
+  CUtensorMap tq, tg, tk, tv;
+  if (!make_act_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, dm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_act_map(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, dm, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(bw.redo, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_rowstats_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)rsx::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long ntiles = (long long)dm.nb * dm.B * dm.H;
+  dim3 grid((unsigned)(ntiles < sms ? ntiles : sms));
+  // Wait limit in SM clock cycles: 2e9 cycles is 1 s at 2 GHz.
+  bwd_rowstats_sm100_kernel<<<grid, kThreads, rsx::kSmemBytes, st>>>(tq, tg, tk, tv, dm, ws.col_idx, bw.lse, bw.Drow,
+                                                                    bw.redo, ws.status, 2000000000ull);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
                                 const Workspace& ws, const BwdWorkspace& bw, float* dq, cudaStream_t st) {

@@ -109,9 +109,14 @@ struct BwdWorkspace {
   float* dg_part;   // [B, H, nchunk, d + 1] gain: per head (entry 0), or gate_proj then gate_bias
   float* dS;        // [B, H, r, d]
   float* dz;        // [B, H, r]
+  int* redo;        // [1 + B*H*nb]: count, then the query tiles whose row statistics are redone
 };
 
 size_t backward_workspace_bytes(const Dims& dm, BwdWorkspace* bw, char* base);
+// Row statistics (lse, D) of every query tile on tcgen05; tiles it cannot take (a p above
+// 2^64 against the first pair's column max) are listed in bw.redo (count zeroed here).
+cudaError_t launch_bwd_rowstats_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                                     const Workspace& ws, const BwdWorkspace& bw, cudaStream_t st);
 cudaError_t launch_bwd_dq_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
                                 const Workspace& ws, const BwdWorkspace& bw, float* dq, cudaStream_t st);
 cudaError_t launch_bwd_dkv_sm100(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,

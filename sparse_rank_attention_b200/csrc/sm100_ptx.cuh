@@ -139,6 +139,37 @@ __device__ __forceinline__ bool named_vote_or(uint32_t id, uint32_t count, bool 
   return r != 0;
 }
 
+// Reduce 32 per-lane values over the warp; lane l receives entry l (31 shuffles).
+template <bool kMax>
+__device__ __forceinline__ float reduce_scatter32(const float* x, int lane) {
+  const unsigned full = 0xffffffffu;
+  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+  float b[16], c[8], d[4], e2[2];
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4, h2 = lane & 2, h1 = lane & 1;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float mine = h16 ? x[16 + e] : x[e], send = h16 ? x[e] : x[16 + e];
+    b[e] = op(mine, __shfl_xor_sync(full, send, 16));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float mine = h8 ? b[8 + e] : b[e], send = h8 ? b[e] : b[8 + e];
+    c[e] = op(mine, __shfl_xor_sync(full, send, 8));
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float mine = h4 ? c[4 + e] : c[e], send = h4 ? c[e] : c[4 + e];
+    d[e] = op(mine, __shfl_xor_sync(full, send, 4));
+  }
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float mine = h2 ? d[2 + e] : d[e], send = h2 ? d[e] : d[2 + e];
+    e2[e] = op(mine, __shfl_xor_sync(full, send, 2));
+  }
+  const float mine = h1 ? e2[1] : e2[0], send = h1 ? e2[0] : e2[1];
+  return op(mine, __shfl_xor_sync(full, send, 1));
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
