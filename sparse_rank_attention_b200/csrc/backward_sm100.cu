@@ -23,6 +23,9 @@
 // them), V stages after their dP^T products (two); S^T/dP^T are double-buffered in TMEM.
 // Persistent: one CTA per SM walks the tiles tau = blockIdx.x + n * gridDim.x.
 //
+// The exponentials run on ex2.approx (relative error ~2^-22, far inside the gradients'
+// tolerance), as in the forward's softmax.
+//
 // Every mbarrier wait is bounded (ROLA_ERR_DEVICE_TIMEOUT); on a timeout all roles leave
 // their loops, in-flight MMAs and TMA copies are drained and TMEM is freed.
 #include <cuda.h>
@@ -30,6 +33,7 @@
 
 #include "rola_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "softmax_exp.cuh"
 
 namespace rola {
 namespace {
@@ -325,10 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100_kernel(
           for (int h2 = 0; h2 < 2; ++h2) {
             const float4 lv = l4[2 * c8 + h2], dv = d4[2 * c8 + h2];
             const int q0 = 8 * c8 + 4 * h2;
-            const float p0 = valid ? exp2f(fmaf(x[q0], sl2, -lv.x)) : 0.f;
-            const float p1 = valid ? exp2f(fmaf(x[q0 + 1], sl2, -lv.y)) : 0.f;
-            const float p2 = valid ? exp2f(fmaf(x[q0 + 2], sl2, -lv.z)) : 0.f;
-            const float p3 = valid ? exp2f(fmaf(x[q0 + 3], sl2, -lv.w)) : 0.f;
+            const float p0 = valid ? ex2_approx(fmaf(x[q0], sl2, -lv.x)) : 0.f;
+            const float p1 = valid ? ex2_approx(fmaf(x[q0 + 1], sl2, -lv.y)) : 0.f;
+            const float p2 = valid ? ex2_approx(fmaf(x[q0 + 2], sl2, -lv.z)) : 0.f;
+            const float p3 = valid ? ex2_approx(fmaf(x[q0 + 3], sl2, -lv.w)) : 0.f;
             split_bf16x2(p0 * (dp[q0] - dv.x), p1 * (dp[q0 + 1] - dv.y), hw[2 * h2], lw[2 * h2]);
             split_bf16x2(p2 * (dp[q0 + 2] - dv.z), p3 * (dp[q0 + 3] - dv.w), hw[2 * h2 + 1], lw[2 * h2 + 1]);
           }
@@ -635,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_sm100_kernel(
 #pragma unroll
           for (int w2 = 0; w2 < 4; ++w2) {
             const int k0 = 8 * c8 + 2 * w2;
-            const float p0 = k0 < kvalid ? exp2f(fmaf(x[k0], sl2, -lr)) : 0.f;
-            const float p1 = k0 + 1 < kvalid ? exp2f(fmaf(x[k0 + 1], sl2, -lr)) : 0.f;
+            const float p0 = k0 < kvalid ? ex2_approx(fmaf(x[k0], sl2, -lr)) : 0.f;
+            const float p1 = k0 + 1 < kvalid ? ex2_approx(fmaf(x[k0 + 1], sl2, -lr)) : 0.f;
             split_bf16x2(p0, p1, ph[w2], pl[w2]);
             split_bf16x2(p0 * (dp[k0] - dr), p1 * (dp[k0 + 1] - dr), ah[w2], al[w2]);
           }
@@ -944,7 +948,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_rowstats_sm100_kernel(
           for (int c = 0; c < 16; ++c) {
             const float a = fmaf(x[c], sl2, -m[16 * hh + c]);
             over |= valid && a > 64.f;
-            const float p = valid ? exp2f(a) : 0.f;
+            const float p = valid ? ex2_approx(a) : 0.f;
             ls[16 * hh + c] += p;
             es[16 * hh + c] = fmaf(p, dp[c], es[16 * hh + c]);
           }
