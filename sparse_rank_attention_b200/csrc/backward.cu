@@ -30,6 +30,7 @@
 #include <type_traits>
 
 #include "rola_internal.cuh"
+#include "sm100_ptx.cuh"
 #include "warp_mma.cuh"
 
 namespace rola {
@@ -760,9 +761,10 @@ __device__ __forceinline__ void tile_gemm(float (&acc)[S_][4][4], FA a, FB b) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) bv[j] = b(k, n0 + NT * j);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)   // two columns per packed f32x2 FMA, each rounded as fmaf
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[s][i][j] = fmaf(av[i], bv[j], acc[s][i][j]);
+        for (int j = 0; j < 4; j += 2)
+          sm100::fma2(acc[s][i][j], acc[s][i][j + 1], av[i], av[i], bv[j], bv[j + 1], acc[s][i][j], acc[s][i][j + 1]);
     }
   }
 }
