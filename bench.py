@@ -15,7 +15,7 @@ pair (c = valid tokens of a block), divided by the step time.
 For a bf16 workload that has an fp8-e4m3 twin (the 720P and 480P 14B shapes), the same
 line also carries ``fp8``: the twin timed the same way on the same inputs (``--no-fp8``
 skips it).  ``backward`` times rola_backward (the gradients of the same forward, fp32
-arithmetic) on the same workload: a few calls, the same timing rules; its TFLOP/s counts the
+gradients) on the same workload: a few calls, the same timing rules; its TFLOP/s counts the
 five kept-block products of an attention backward (2.5 x the forward's kept-block FLOPs).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs an independent forward of the
@@ -506,7 +506,10 @@ def main():
         bflops = int(2.5 * mb["flops"])
         bwd = {"ms_per_call": mb["ms_step"], "steps": bwd_steps, "warmup": bwd_warm,
                "value": aggregate_tflops(bflops, mb["ms_step"], ws), "unit": "kept-block TFLOP/s (backward)",
-               "flops_per_call": bflops, "arithmetic": "fp32 (CUDA cores)", "clocks": mb["clocks"]}
+               "flops_per_call": bflops,
+               "arithmetic": ("bf16 tensor-core products (tcgen05) with fp32 accumulation; P and dA as bf16 "
+                              "hi + lo; the linear branch in fp32" if w.dtype == "bf16" else "fp32"),
+               "clocks": mb["clocks"]}
         del dout
 
     cpu = None
