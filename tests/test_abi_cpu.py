@@ -103,6 +103,9 @@ def test_plan_checks_workspace_without_touching_device():
     assert lib.rola_select_blocks(h, ctypes.c_void_p(0x2008), ctypes.c_void_p(0x2000), None) == 1
     assert lib.rola_attend(h, *[ctypes.c_void_p(0x4000)] * 6, None) == 1   # out overlaps q
     assert lib.rola_set_debug(h, -1, 0) == 1
+    # inspection calls reject missing buffers (and a missing plan) before any copy
+    assert lib.rola_get_block_scores(h, None, ctypes.c_void_p(0x2000), None) == 1
+    assert lib.rola_get_block_scores(None, ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000), None) == 1
     lib.rola_plan_destroy(h)
 
 
