@@ -599,8 +599,6 @@ cudaError_t launch_pool(const Dims& dm, rola_dtype dt, const void* q, const void
 
 int score_row_stride(const Dims& dm) { return (dm.nb + 3) / 4 * 4; }
 
-size_t select_smem_bytes(const Dims& dm) { return topk_smem(score_row_stride(dm), dm.d, topk_cand(dm.k)); }
-
 cudaError_t launch_select(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   const int nbp = score_row_stride(dm);
   cudaError_t e = launch_score_sm100(dm, ws, nbp, st);
