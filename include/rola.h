@@ -120,8 +120,8 @@ ROLA_API rola_status rola_params_default(rola_params* p);
 /* Number of 64-token blocks nb and kept blocks per query block k for *p. */
 ROLA_API rola_status rola_keep_count(const rola_params* p, int* nb, int* k);
 
-/* Bytes of device workspace a plan for *p needs (pooled means, block lists, linear
- * state, rotary table, fp8 copies, status word). */
+/* Bytes of device workspace a plan for *p needs (pooled means, block scores and key-block
+ * norms, block lists, linear state, rotary table, the fp16 or fp8 copies, status word). */
 ROLA_API rola_status rola_workspace_size(const rola_params* p, size_t* bytes);
 
 /* Validates *p and binds it to `workspace` (device memory of at least
